@@ -1,0 +1,250 @@
+/*
+ * had_oracle.c -- plain, slow CPU oracle for the Hamming Attention
+ * Distillation (HAD) inference forward pass.
+ *
+ * TEST INFRASTRUCTURE ONLY.  Only the test suite, the smoke check and the
+ * benchmark's CPU-baseline leg may load this library.  It shares no code,
+ * header, table or constant with the CUDA library and must never be used as
+ * a fallback for it.
+ *
+ * What it computes follows "Hamming Attention Distillation: Binarizing Keys
+ * and Queries for Efficient Long-Context Transformers" (arXiv 2502.01770) as
+ * described on the pith.science review page, section "What carries the
+ * argument" and the circularity audit (Eqs. 4-7, Eq. 12):
+ *
+ *   1. standardize Q and K by the data-estimated coefficients sigma_Q,
+ *      sigma_K (Eq. 12), then sign-quantize to {-1,+1} (Eqs. 4-5);
+ *   2. the logit of query i and key j is the +/-1 dot product, which the
+ *      pages compute as a Hamming distance (XNOR + popcount) (Eq. 5);
+ *   3. a top-N mask keeps only the N largest logits of each row (Eq. 6);
+ *   4. softmax over the kept logits only (Eq. 7), then the sparse product
+ *      with the full-precision value matrix (the referee report notes that
+ *      values and the attention map stay in full precision).
+ *
+ * Readings where the pages are silent:
+ *   - sigma is one positive fp32 number per head; z = x / sigma is an IEEE
+ *     fp32 round-to-nearest division with subnormals kept;
+ *   - sign(z) = -1 iff z < 0; +0, -0 and NaN give +1;
+ *   - the logit is the dot product s = d - 2*Hamming; a softmax temperature
+ *     tau multiplies it (the caller passes tau; 1/sqrt(d) in the workloads);
+ *   - ties at the N-th largest logit go to the lower key index, so exactly N
+ *     keys are kept; the kept indices are reported in ascending order;
+ *   - softmax and the value product are evaluated in fp64, stored as fp32.
+ *
+ * Nothing here is blocked, fused or reordered beyond those definitions: the
+ * logit is a +/-1 dot-product loop (not a popcount, so the popcount identity
+ * is something the tests check rather than assume), the top-N is a full
+ * sort of the row, and the softmax/value product is a plain double loop.
+ */
+#include <math.h>
+#include <stdint.h>
+#include <stdlib.h>
+#include <string.h>
+#ifdef _OPENMP
+#include <omp.h>
+#endif
+
+/* bf16 is the upper half of an IEEE binary32; widening is exact. */
+static float bf16_to_float(uint16_t b)
+{
+    uint32_t u = ((uint32_t)b) << 16;
+    float f;
+    memcpy(&f, &u, sizeof f);
+    return f;
+}
+
+static float load_elem(const void *x, int is_bf16, long i)
+{
+    return is_bf16 ? bf16_to_float(((const uint16_t *)x)[i])
+                   : ((const float *)x)[i];
+}
+
+/*
+ * Step 1 (Eqs. 4-5, Eq. 12): sign of x / sigma[h] for every element of a
+ * [B,H,n,d] tensor.  Writes +1 or -1 into sign_out (same layout).
+ */
+void had_oracle_binarize(const void *x, int x_is_bf16, const float *sigma,
+                         long B, long H, long n, long d, int8_t *sign_out)
+{
+    for (long b = 0; b < B; ++b)
+        for (long h = 0; h < H; ++h) {
+            float sg = sigma[h];
+            long base = (b * H + h) * n * d;
+            for (long e = 0; e < n * d; ++e) {
+                float z = load_elem(x, x_is_bf16, base + e) / sg;
+                sign_out[base + e] = (z < 0.0f) ? (int8_t)-1 : (int8_t)1;
+            }
+        }
+}
+
+/*
+ * Bit-packed form of the signs (the "binary" Q/K the pages store as bits):
+ * bit k of word w of a row is 1 iff the sign of element 32*w + k is -1.
+ */
+void had_oracle_pack(const int8_t *sign, long rows, long d, uint32_t *bits)
+{
+    long words = d / 32;
+    for (long r = 0; r < rows; ++r)
+        for (long w = 0; w < words; ++w) {
+            uint32_t word = 0;
+            for (int k = 0; k < 32; ++k)
+                if (sign[r * d + 32 * w + k] < 0)
+                    word |= (uint32_t)1 << k;
+            bits[r * words + w] = word;
+        }
+}
+
+/* Step 2 (Eq. 5): logits of one query row against every key of its head. */
+static void row_logits(const int8_t *sq_row, const int8_t *sk_head, long n,
+                       long d, int32_t *s)
+{
+    for (long j = 0; j < n; ++j) {
+        int32_t acc = 0;
+        const int8_t *kr = sk_head + j * d;
+        for (long k = 0; k < d; ++k)
+            acc += (int32_t)sq_row[k] * (int32_t)kr[k];
+        s[j] = acc;
+    }
+}
+
+typedef struct {
+    int32_t s;
+    int32_t j;
+} keyed_t;
+
+/* Larger logit first; equal logits: lower key index first. */
+static int by_logit_then_index(const void *a, const void *b)
+{
+    const keyed_t *x = (const keyed_t *)a, *y = (const keyed_t *)b;
+    if (x->s != y->s)
+        return (x->s > y->s) ? -1 : 1;
+    return (x->j < y->j) ? -1 : (x->j > y->j);
+}
+
+static int by_index(const void *a, const void *b)
+{
+    const keyed_t *x = (const keyed_t *)a, *y = (const keyed_t *)b;
+    return (x->j < y->j) ? -1 : (x->j > y->j);
+}
+
+/*
+ * Logits of a list of query rows.  rows[] holds flat row ids
+ * r = (b*H + h)*n + i; s_out is [nrows, n].
+ */
+void had_oracle_logits_rows(const int8_t *sq, const int8_t *sk, long B,
+                            long H, long n, long d, const int64_t *rows,
+                            long nrows, int32_t *s_out, int nthreads)
+{
+    (void)B;
+    (void)H;
+#ifdef _OPENMP
+    if (nthreads > 0)
+        omp_set_num_threads(nthreads);
+#pragma omp parallel for schedule(dynamic, 4)
+#endif
+    for (long t = 0; t < nrows; ++t) {
+        long r = (long)rows[t];
+        long head = r / n;
+        row_logits(sq + r * d, sk + head * n * d, n, d, s_out + t * n);
+    }
+}
+
+/*
+ * Steps 2-4 for a list of query rows.  Outputs (all [nrows, ...]):
+ *   idx_out  [nrows, N]  kept key indices, ascending;
+ *   s_out    [nrows, N]  their logits;
+ *   p_out    [nrows, N]  softmax probabilities (fp64), or NULL;
+ *   o_out    [nrows, d]  attention output (fp64 sums stored as fp32).
+ * V is [B,H,n,d] fp32 or bf16 bits.  Returns 0, or -1 on a bad argument or
+ * allocation failure.
+ */
+int had_oracle_attention_rows(const int8_t *sq, const int8_t *sk,
+                              const void *v, int v_is_bf16, long B, long H,
+                              long n, long d, long N, float tau,
+                              const int64_t *rows, long nrows,
+                              int32_t *idx_out, int16_t *s_out, double *p_out,
+                              float *o_out, int nthreads)
+{
+    (void)B;
+    (void)H;
+    if (N < 1 || N > n || d < 1 || n < 1)
+        return -1;
+    int failed = 0;
+#ifdef _OPENMP
+    if (nthreads > 0)
+        omp_set_num_threads(nthreads);
+#pragma omp parallel
+#endif
+    {
+        int32_t *s = (int32_t *)malloc(sizeof(int32_t) * (size_t)n);
+        keyed_t *order = (keyed_t *)malloc(sizeof(keyed_t) * (size_t)n);
+        double *e = (double *)malloc(sizeof(double) * (size_t)N);
+#ifdef _OPENMP
+#pragma omp for schedule(dynamic, 4)
+#endif
+        for (long t = 0; t < nrows; ++t) {
+            if (!s || !order || !e) {
+#ifdef _OPENMP
+#pragma omp atomic write
+#endif
+                failed = 1;
+                continue;
+            }
+            {
+                long r = (long)rows[t];
+                long head = r / n;
+                row_logits(sq + r * d, sk + head * n * d, n, d, s);
+
+                /* Eq. 6: the N largest logits, ties to the lower index. */
+                for (long j = 0; j < n; ++j) {
+                    order[j].s = s[j];
+                    order[j].j = (int32_t)j;
+                }
+                qsort(order, (size_t)n, sizeof(keyed_t), by_logit_then_index);
+                qsort(order, (size_t)N, sizeof(keyed_t), by_index);
+
+                /* Eq. 7: softmax over the kept logits only (fp64). */
+                int32_t m = order[0].s;
+                for (long k = 1; k < N; ++k)
+                    if (order[k].s > m)
+                        m = order[k].s;
+                double Z = 0.0;
+                for (long k = 0; k < N; ++k) {
+                    e[k] = exp((double)tau * (double)(order[k].s - m));
+                    Z += e[k];
+                }
+                for (long k = 0; k < N; ++k) {
+                    idx_out[t * N + k] = order[k].j;
+                    s_out[t * N + k] = (int16_t)order[k].s;
+                    if (p_out)
+                        p_out[t * N + k] = e[k] / Z;
+                }
+
+                /* Sparse product with the full-precision values. */
+                const long vbase = head * n * d;
+                for (long c = 0; c < d; ++c) {
+                    double acc = 0.0;
+                    for (long k = 0; k < N; ++k)
+                        acc += (e[k] / Z) *
+                               (double)load_elem(v, v_is_bf16,
+                                                 vbase + (long)order[k].j * d + c);
+                    o_out[t * d + c] = (float)acc;
+                }
+            }
+        }
+        free(s);
+        free(order);
+        free(e);
+    }
+    return failed ? -1 : 0;
+}
+
+/* Number of OpenMP threads a parallel region would use (1 without OpenMP). */
+int had_oracle_max_threads(void)
+{
+#ifdef _OPENMP
+    return omp_get_max_threads();
+#else
+    return 1;
+#endif
+}

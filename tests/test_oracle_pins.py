@@ -1,0 +1,334 @@
+"""Pins for the CPU oracle: checks against what the pages and mathematics fix.
+
+Each test ties one step of the oracle to something other than the oracle
+itself: IEEE edge values, a library routine (numpy float64 matrix product,
+numpy/Python sorts, torch softmax), an independent algorithm (histogram
+threshold selection), a closed form, or the hand-worked fixture under
+tests/golden/.  The steps follow the pith.science review of "Hamming
+Attention Distillation" (arXiv 2502.01770), "What carries the argument":
+standardize by sigma, sign to +/-1 (Eqs. 4-5), Hamming logits (Eq. 5),
+top-N mask (Eq. 6), softmax over the kept logits (Eq. 7), value product.
+"""
+import math
+
+import numpy as np
+import pytest
+import torch
+
+import oracle
+import synth
+from tests import _golden
+
+
+def _signs_np(x, sigma):
+    """Library route to the signs: numpy float32 division, then < 0."""
+    z = np.asarray(x, np.float32) / np.asarray(sigma, np.float32)[None, :, None, None]
+    return np.where(z < 0, -1, 1).astype(np.int8)
+
+
+def _popcount32(a):
+    a = a.astype(np.uint64)
+    return np.array([int(x).bit_count() for x in a.reshape(-1)], np.int64).reshape(a.shape)
+
+
+def _rand_case(B, H, n, d, seed, dist="normal"):
+    g = np.random.default_rng(seed)
+    x = g.standard_normal((B, H, n, d)).astype(np.float32)
+    return x
+
+
+# ----------------------------------------------------------------- step 1
+
+
+SIGN_EDGES = [
+    # (x, sigma, expected sign) -- sign is -1 iff x/sigma < 0 in IEEE fp32
+    (0.0, 1.0, 1),
+    (-0.0, 1.0, 1),                          # -0 is not < 0
+    (float("nan"), 1.0, 1),                  # comparisons with NaN are false
+    (float("inf"), 2.0, 1),
+    (float("-inf"), 2.0, -1),
+    (1e-45, 1.0, 1),                         # smallest subnormal
+    (-1e-45, 1.0, -1),
+    (-1e-45, 3.0, 1),                        # quotient rounds to -0
+    (-1e-45, 0.5, -1),                       # quotient is a subnormal, kept
+    (-1.1754944e-38, 1.0, -1),               # smallest normal
+    (np.nextafter(np.float32(0), np.float32(1)), 1e10, 1),
+    (-np.nextafter(np.float32(0), np.float32(1)), 1e10, 1),   # underflow to -0
+    (-1e-30, 1e9, -1),                       # subnormal quotient, no flush
+    (3.0, 7.0, 1),
+    (-3.0, 7.0, -1),
+]
+
+
+@pytest.mark.parametrize("x,sigma,expected", SIGN_EDGES)
+def test_sign_edge_values(x, sigma, expected):
+    arr = np.full((1, 1, 1, 32), 1.0, np.float32)
+    arr[0, 0, 0, 3] = np.float32(x)
+    s = oracle.binarize(arr, np.asarray([sigma], np.float32))
+    assert s[0, 0, 0, 3] == expected
+    assert (np.delete(s.reshape(-1), 3) == 1).all()
+
+
+def test_sign_bf16_path_matches_widened_fp32():
+    g = torch.Generator().manual_seed(5)
+    x = (torch.randn(2, 3, 16, 64, generator=g) * 1e-3).to(torch.bfloat16)
+    x[0, 0, 0, :4] = torch.tensor([0.0, -0.0, 1e-40, -1e-40]).to(torch.bfloat16)
+    sigma = np.asarray([0.7, 1.3, 2.0], np.float32)
+    a = oracle.binarize(synth.to_oracle_array(x), sigma)
+    b = oracle.binarize(x.float().numpy(), sigma)
+    assert np.array_equal(a, b)
+    assert np.array_equal(a, _signs_np(x.float().numpy(), sigma))
+
+
+def test_sign_matches_numpy_division():
+    g = np.random.default_rng(1)
+    x = g.standard_normal((2, 4, 33, 64)).astype(np.float32)
+    x *= np.float32(10.0) ** g.integers(-40, 5, size=x.shape).astype(np.float32)
+    sigma = np.asarray([0.3, 1.0, 7.5, 1e-3], np.float32)
+    assert np.array_equal(oracle.binarize(x, sigma), _signs_np(x, sigma))
+
+
+def test_sigma_positive_scale_does_not_change_bits():
+    x = _rand_case(2, 3, 40, 64, 2)
+    s1 = oracle.binarize(x, np.asarray([1.0, 2.0, 3.0], np.float32))
+    s2 = oracle.binarize(x, np.asarray([0.01, 50.0, 3e4], np.float32))
+    assert np.array_equal(s1, s2)
+
+
+# ----------------------------------------------------------------- packing
+
+
+def test_pack_bit_order_lsb_first():
+    sg = np.ones((4, 64), np.int8)
+    sg[1, 0] = -1            # word 0, bit 0
+    sg[2, 33] = -1           # word 1, bit 1
+    sg[3, 31] = -1           # word 0, bit 31
+    sg[3, 63] = -1           # word 1, bit 31
+    bits = oracle.pack(sg)
+    assert bits.tolist() == [[0, 0], [1, 0], [0, 2], [1 << 31, 1 << 31]]
+
+
+def test_pack_popcount_counts_negatives():
+    g = np.random.default_rng(3)
+    sg = np.where(g.random((50, 128)) < 0.3, -1, 1).astype(np.int8)
+    bits = oracle.pack(sg)
+    assert np.array_equal(_popcount32(bits).sum(axis=1), (sg < 0).sum(axis=1))
+    # unpack by shifting and compare element by element
+    unpacked = ((bits[:, :, None] >> np.arange(32, dtype=np.uint32)) & 1).reshape(50, 128)
+    assert np.array_equal(unpacked == 1, sg < 0)
+
+
+# ----------------------------------------------------------------- step 2
+
+
+def _head_logits(sq, sk, b, h):
+    B, H, n, d = sq.shape
+    rows = (b * H + h) * n + np.arange(n)
+    return oracle.logits_rows(sq, sk, rows)
+
+
+@pytest.mark.parametrize("d", [64, 128])
+def test_logits_popcount_identity(d):
+    """q.k = d - 2*Hamming(q, k) for +/-1 vectors (the Eq. 5 identity)."""
+    x = _rand_case(1, 2, 37, d, 4)
+    y = _rand_case(1, 2, 37, d, 5)
+    sg = np.asarray([1.0, 1.0], np.float32)
+    sq, sk = oracle.binarize(x, sg), oracle.binarize(y, sg)
+    bq, bk = oracle.pack(sq), oracle.pack(sk)
+    for h in range(2):
+        s = _head_logits(sq, sk, 0, h)
+        xor = bq[0, h][:, None, :] ^ bk[0, h][None, :, :]
+        ham = _popcount32(xor).sum(axis=-1)
+        assert np.array_equal(s, d - 2 * ham)
+
+
+def test_logits_match_float64_matmul():
+    x = _rand_case(2, 3, 29, 64, 6)
+    y = _rand_case(2, 3, 29, 64, 7)
+    sg = np.asarray([0.5, 1.0, 2.0], np.float32)
+    sq, sk = oracle.binarize(x, sg), oracle.binarize(y, sg)
+    for b in range(2):
+        for h in range(3):
+            ref = sq[b, h].astype(np.float64) @ sk[b, h].astype(np.float64).T
+            assert np.array_equal(_head_logits(sq, sk, b, h), ref.astype(np.int32))
+
+
+def test_logits_not_transposed():
+    """Row i of the logits uses query i against all keys (asymmetric case)."""
+    sq = np.ones((1, 1, 3, 64), np.int8)
+    sk = np.ones((1, 1, 3, 64), np.int8)
+    sq[0, 0, 0, :10] = -1          # query 0 differs from every key in 10 places
+    sk[0, 0, 2, :] = -1            # key 2 is the negation of the all-ones key
+    s = _head_logits(sq, sk, 0, 0)
+    assert s.tolist() == [[44, 44, -44], [64, 64, -64], [64, 64, -64]]
+
+
+def test_logits_invariants():
+    x = _rand_case(1, 2, 50, 64, 8)
+    y = _rand_case(1, 2, 50, 64, 9)
+    sg = np.ones(2, np.float32)
+    sq, sk = oracle.binarize(x, sg), oracle.binarize(y, sg)
+    s = _head_logits(sq, sk, 0, 1)
+    assert np.abs(s).max() <= 64 and (s % 2 == 0).all()            # s = d mod 2
+    assert np.array_equal(_head_logits(sq, -sk, 0, 1), -s)         # K -> -K
+    assert np.array_equal(_head_logits(-sq, -sk, 0, 1), s)         # both flipped
+    assert (np.diag(_head_logits(sq, sq, 0, 1)) == 64).all()       # Q == K
+
+
+# ----------------------------------------------------------------- step 3
+
+
+def _binarized(cfg_or_shape, seed=10, offset=0.0):
+    B, H, n, d = cfg_or_shape
+    x = _rand_case(B, H, n, d, seed) + np.float32(offset)
+    y = _rand_case(B, H, n, d, seed + 1) + np.float32(offset)
+    v = _rand_case(B, H, n, d, seed + 2)
+    sg = np.ones(H, np.float32)
+    return oracle.binarize(x, sg), oracle.binarize(y, sg), v
+
+
+def _threshold_select(s_row, N, d):
+    """Histogram-threshold top-N (a different algorithm from a sort).
+
+    Count each logit value; walk values from the largest down until the
+    running count reaches N; keep all larger values and the first q keys
+    (in index order) at the threshold value."""
+    counts = {}
+    for v in s_row.tolist():
+        counts[v] = counts.get(v, 0) + 1
+    above = 0
+    for t in range(d, -d - 1, -2):
+        c = counts.get(t, 0)
+        if above + c >= N:
+            break
+        above += c
+    q = N - above
+    keep = []
+    for j, v in enumerate(s_row.tolist()):
+        if v > t:
+            keep.append(j)
+        elif v == t and q > 0:
+            keep.append(j)
+            q -= 1
+    return keep
+
+
+@pytest.mark.parametrize("shape,N,offset", [((1, 2, 64, 64), 8, 0.0),
+                                            ((1, 2, 197, 64), 32, 0.3),
+                                            ((1, 1, 96, 128), 20, 0.0)])
+def test_topn_against_sorts_and_threshold(shape, N, offset):
+    sq, sk, v = _binarized(shape, offset=offset)
+    B, H, n, d = shape
+    idx, lg, p, out = oracle.attention(sq, sk, v, 0.125, N)
+    for h in range(H):
+        s = _head_logits(sq, sk, 0, h)
+        for i in range(n):
+            py = sorted(sorted(range(n), key=lambda j: (-s[i, j], j))[:N])
+            lx = np.sort(np.lexsort((np.arange(n), -s[i]))[:N])
+            th = _threshold_select(s[i], N, d)
+            assert idx[0, h, i].tolist() == py == lx.tolist() == th
+            assert np.array_equal(lg[0, h, i], s[i, idx[0, h, i]])
+
+
+def test_topn_all_keys_equal_keeps_first_N():
+    sq, sk, v = _binarized((1, 1, 40, 64), seed=20)
+    sk[:] = sk[0, 0, 0]                     # every key identical -> all ties
+    idx, lg, p, out = oracle.attention(sq, sk, v, 0.125, 7)
+    assert (idx == np.arange(7)).all()
+    assert np.allclose(p, 1.0 / 7, rtol=0, atol=1e-15)
+    mean = v[0, 0, :7].astype(np.float64).mean(axis=0)
+    assert np.allclose(out[0, 0], mean[None, :], rtol=0, atol=2e-7)
+
+
+def test_topn_N_equals_n_is_dense_softmax():
+    sq, sk, v = _binarized((1, 2, 48, 64), seed=30)
+    tau = 0.125
+    idx, lg, p, out = oracle.attention(sq, sk, v, tau, 48)
+    for h in range(2):
+        assert (idx[0, h] == np.arange(48)).all()
+        s = torch.from_numpy(_head_logits(sq, sk, 0, h)).double()
+        pd = torch.softmax(tau * s, dim=-1)
+        od = pd @ torch.from_numpy(v[0, h]).double()
+        assert np.allclose(p[0, h], pd.numpy(), rtol=1e-12, atol=1e-15)
+        assert np.allclose(out[0, h], od.numpy(), rtol=0, atol=1e-6)
+
+
+def test_N1_is_first_argmax():
+    sq, sk, v = _binarized((1, 2, 77, 64), seed=40)
+    idx, lg, p, out = oracle.attention(sq, sk, v, 0.125, 1)
+    for h in range(2):
+        s = _head_logits(sq, sk, 0, h)
+        am = np.argmax(s, axis=1)          # numpy returns the first maximum
+        assert np.array_equal(idx[0, h, :, 0], am)
+        assert np.array_equal(out[0, h], v[0, h, am])
+        assert (p == 1.0).all()
+
+
+def test_rows_of_p_sum_to_one_with_N_nonzeros():
+    sq, sk, v = _binarized((2, 2, 130, 128), seed=50)
+    N = 37
+    idx, lg, p, out = oracle.attention(sq, sk, v, 1 / math.sqrt(128), N)
+    assert np.allclose(p.sum(axis=-1), 1.0, rtol=0, atol=1e-12)
+    assert (p > 0).all() and p.shape[-1] == N
+    assert (np.diff(idx, axis=-1) > 0).all()           # ascending, distinct
+
+
+def test_softmax_uses_tau_times_logit_difference():
+    """p_k / p_l = exp(tau * (s_k - s_l)) within a row (Eq. 7)."""
+    sq, sk, v = _binarized((1, 1, 60, 64), seed=60)
+    tau = float(np.float32(0.3))          # tau crosses the C boundary as fp32
+    idx, lg, p, out = oracle.attention(sq, sk, v, tau, 12)
+    r = p[0, 0, 5]
+    s = lg[0, 0, 5].astype(np.float64)
+    assert np.allclose(r / r[0], np.exp(tau * (s - s[0])), rtol=1e-12)
+
+
+# ----------------------------------------------------------------- fixture
+
+
+def test_golden_handworked():
+    case = _golden.load()
+    q, k, v, sgq, sgk = _golden.tensors(case)
+    sq, sk = oracle.binarize(q, sgq), oracle.binarize(k, sgk)
+    exp = case["expected"]
+    assert oracle.pack(sk)[0, 0].tolist() == exp["k_bits"]
+    assert _head_logits(sq, sk, 0, 0)[0].tolist() == exp["logits_row0_all"]
+    idx, lg, p, out = oracle.attention(sq, sk, v, case["tau"], case["N"])
+    for key in ("row0", "row1", "row3"):
+        r = int(key[3:])
+        e = exp[key]
+        assert idx[0, 0, r].tolist() == e["idx"]
+        assert lg[0, 0, r].tolist() == e["logits"]
+        assert np.allclose(p[0, 0, r], [_golden.closed_form(x) for x in e["p"]],
+                           rtol=1e-14, atol=0)
+        want = np.zeros(case["d"])
+        for c, ex in e["out_nonzero"].items():
+            want[int(c)] = _golden.closed_form(ex)
+        assert np.allclose(out[0, 0, r], want, rtol=1e-7, atol=1e-9)
+
+
+# ----------------------------------------------------------------- plumbing
+
+
+def test_threads_deterministic():
+    sq, sk, v = _binarized((2, 2, 100, 64), seed=70)
+    a = oracle.attention(sq, sk, v, 0.125, 10, threads=1)
+    b = oracle.attention(sq, sk, v, 0.125, 10, threads=4)
+    for x, y in zip(a, b):
+        assert np.array_equal(x, y)
+
+
+def test_rows_subset_matches_full():
+    sq, sk, v = _binarized((1, 3, 50, 64), seed=80)
+    full = oracle.attention(sq, sk, v, 0.125, 9)
+    rows = np.array([0, 49, 50, 77, 149])
+    sub = oracle.attention_rows(sq, sk, v, 0.125, 9, rows)
+    for f, s in zip(full, sub):
+        assert np.array_equal(f.reshape(-1, f.shape[-1])[rows], s)
+
+
+@pytest.mark.parametrize("N", [0, 51])
+def test_oracle_rejects_bad_N(N):
+    sq, sk, v = _binarized((1, 1, 50, 64), seed=90)
+    with pytest.raises(ValueError):
+        oracle.attention(sq, sk, v, 0.125, N)
