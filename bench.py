@@ -1,0 +1,415 @@
+#!/usr/bin/env python
+"""Benchmark of the fused HAD attention forward pass (tokens/s).
+
+One step = one ``had_attention_fwd`` call over one batch of the long-context
+workload (B=4, H=16, n=4096, d=64, N=512, bf16; tau = 1/8), inputs resident
+in HBM.  Prints ONE JSON line on rank 0.
+
+    python bench.py [--gpus N] [--steps K] [--warmup W] [--impl had|reference]
+
+N > 1 runs under torchrun, one process per GPU; every rank processes its own
+batch of independent (b, h) problems (weak scaling, no collective on the data
+path) and the timing is the max over ranks.  ``--impl reference`` times the
+CPU oracle (the only reference this method has) on bounded row samples of the
+same workload, on rank 0 only.
+"""
+import argparse
+import json
+import math
+import os
+import statistics
+import subprocess
+import sys
+import threading
+import time
+
+import torch
+
+ROOT = os.path.dirname(os.path.abspath(__file__))
+sys.path.insert(0, ROOT)
+
+import synth  # noqa: E402
+
+WORKLOAD = "long"
+METRIC = "HAD attention tokens/sec at n=4096,d=64,N=512; % of int8-TC/HBM roofline"
+L2_FLUSH_BYTES = 256 << 20
+SM_COUNT = 148
+ALU_LANES_PER_SM = 128
+
+
+def parse():
+    ap = argparse.ArgumentParser()
+    ap.add_argument("--gpus", type=int, default=1)
+    ap.add_argument("--steps", type=int, default=20)
+    ap.add_argument("--warmup", type=int, default=5)
+    ap.add_argument("--impl", choices=["had", "reference"], default="had")
+    ap.add_argument("--config", default=WORKLOAD, choices=sorted(synth.CONFIGS))
+    ap.add_argument("--cpu-seconds", type=float, default=12.0,
+                    help="target CPU time of the oracle baseline sample")
+    ap.add_argument("--no-e2e", action="store_true")
+    ap.add_argument("--no-cpu-baseline", action="store_true")
+    return ap.parse_args()
+
+
+# --------------------------------------------------------------------------- peaks
+
+
+def measured_peaks():
+    path = os.path.join(ROOT, "MEASURED_PEAKS.json")
+    if os.path.exists(path):
+        with open(path) as f:
+            p = json.load(f)
+        return {"hbm_gbs": float(p["hbm_gbs"]), "bf16_tflops": float(p["bf16_tflops"]),
+                "sm_max_mhz": float(p.get("sm_max_mhz", 1965.0)), "source": "measured"}
+    return {"hbm_gbs": 6650.0, "bf16_tflops": 1590.0, "sm_max_mhz": 1965.0,
+            "source": "fallback"}
+
+
+def roofline_model(cfg, peaks):
+    """Algorithmic work of one call and its roofline time.
+
+    work   = 2*B*H*n^2*d (int8 logit ops, counted once) + 2*B*H*n*N*d (AV flops)
+    T_roof = max(T_HBM, T_TC, T_ALU):
+      T_HBM = (3*B*H*n*d*2 + B*H*n*d*4) bytes / HBM bandwidth   (read Q,K,V; write O)
+      T_TC  = logit ops / int8 peak + AV flops / bf16 peak, int8 peak = 2 x bf16 peak
+      T_ALU = B*H*n^2 logits / (SMs * 128 lanes * max SM clock), one op per logit
+    """
+    B, H, n, d, N = cfg.B, cfg.H, cfg.n, cfg.d, cfg.N
+    elt = 2 if cfg.dtype == "bf16" else 4
+    logit_ops = 2.0 * B * H * n * n * d
+    av_flops = 2.0 * B * H * n * N * d
+    hbm_bytes = 3.0 * B * H * n * d * elt + B * H * n * d * 4
+    bf16 = peaks["bf16_tflops"] * 1e12
+    i8 = 2.0 * bf16
+    t_hbm = hbm_bytes / (peaks["hbm_gbs"] * 1e9)
+    t_tc = logit_ops / i8 + av_flops / bf16
+    alu = SM_COUNT * ALU_LANES_PER_SM * peaks["sm_max_mhz"] * 1e6
+    t_alu = B * H * n * n / alu
+    return {"work": logit_ops + av_flops, "hbm_bytes": hbm_bytes, "t_hbm": t_hbm,
+            "t_tc": t_tc, "t_alu": t_alu, "t_roof": max(t_hbm, t_tc, t_alu)}
+
+
+# --------------------------------------------------------------------------- clocks
+
+
+class ClockSampler:
+    """nvidia-smi samples of SM clock and throttle reasons while running."""
+
+    FIELDS = ("index,clocks.sm,clocks.max.sm,power.draw,clocks_event_reasons.active,"
+              "clocks_event_reasons.hw_slowdown,clocks_event_reasons.hw_thermal_slowdown,"
+              "clocks_event_reasons.sw_thermal_slowdown,clocks_event_reasons.sw_power_cap")
+
+    def __init__(self, device_index):
+        self.dev = device_index
+        self.proc = None
+        self.lines = []
+
+    def start(self):
+        try:
+            self.proc = subprocess.Popen(
+                ["nvidia-smi", "-i", str(self.dev), f"--query-gpu={self.FIELDS}",
+                 "--format=csv,noheader,nounits", "-lms", "100"],
+                stdout=subprocess.PIPE, stderr=subprocess.DEVNULL, text=True)
+            self.thread = threading.Thread(target=self._read, daemon=True)
+            self.thread.start()
+        except (OSError, ValueError):
+            self.proc = None
+
+    def _read(self):
+        for line in self.proc.stdout:
+            self.lines.append(line.strip())
+
+    def stop(self):
+        if self.proc is None:
+            return None
+        self.proc.terminate()
+        try:
+            self.proc.wait(timeout=5)
+        except subprocess.TimeoutExpired:
+            self.proc.kill()
+        mhz, maxs, reasons = [], [], set()
+        names = ["hw_slowdown", "hw_thermal_slowdown", "sw_thermal_slowdown", "sw_power_cap"]
+        for line in self.lines:
+            parts = [p.strip() for p in line.split(",")]
+            if len(parts) < 9:
+                continue
+            try:
+                mhz.append(float(parts[1]))
+                maxs.append(float(parts[2]))
+            except ValueError:
+                continue
+            for name, val in zip(names, parts[5:9]):
+                if val.lower() == "active":
+                    reasons.add(name)
+        if not mhz:
+            return None
+        return {"sm_mhz": statistics.median(mhz), "sm_max_mhz": max(maxs),
+                "reasons": sorted(reasons), "samples": len(mhz)}
+
+
+# --------------------------------------------------------------------------- dist
+
+
+def dist_setup(args):
+    world = int(os.environ.get("WORLD_SIZE", "1"))
+    rank = int(os.environ.get("RANK", "0"))
+    local = int(os.environ.get("LOCAL_RANK", "0"))
+    if world > 1:
+        import datetime
+        import torch.distributed as dist
+        backend = "nccl" if args.impl == "had" else "gloo"
+        if args.impl == "had":
+            torch.cuda.set_device(local)
+        dist.init_process_group(backend, timeout=datetime.timedelta(seconds=120))
+    return world, rank, local
+
+
+def max_over_ranks(value, world, device):
+    if world == 1:
+        return value
+    import torch.distributed as dist
+    t = torch.tensor([value], dtype=torch.float64, device=device)
+    dist.all_reduce(t, op=dist.ReduceOp.MAX)
+    return float(t.item())
+
+
+def barrier(world):
+    if world > 1:
+        import torch.distributed as dist
+        dist.barrier()
+
+
+# --------------------------------------------------------------------------- oracle
+
+
+def oracle_baseline(cfg, target_seconds, steps=1):
+    """Time the CPU oracle on bounded row samples; returns (tokens/s, details)."""
+    import numpy as np
+    import oracle
+    q, k, v, sgq, sgk = synth.make_inputs(cfg)
+    t0 = time.time()
+    sq = oracle.binarize(synth.to_oracle_array(q), sgq.numpy())
+    sk = oracle.binarize(synth.to_oracle_array(k), sgk.numpy())
+    t_bin = time.time() - t0
+    vo = synth.to_oracle_array(v)
+    threads = oracle.max_threads()
+    probe = np.arange(0, cfg.rows, max(1, cfg.rows // 64))[:64]
+    t0 = time.time()
+    oracle.attention_rows(sq, sk, vo, cfg.tau, cfg.N, probe, threads=threads)
+    per_row = (time.time() - t0) / len(probe)
+    count = int(max(64, min(cfg.rows, target_seconds / max(per_row, 1e-9))))
+    times, rows_done = [], 0
+    for s in range(steps):
+        rows = synth.sample_rows(cfg, count, seed=100 + s)
+        t0 = time.time()
+        oracle.attention_rows(sq, sk, vo, cfg.tau, cfg.N, rows, threads=threads)
+        times.append(time.time() - t0)
+        rows_done += len(rows)
+    total = sum(times)
+    # binarizing the whole tensors once is part of the work; charge it pro rata
+    total += t_bin * rows_done / cfg.rows
+    tokens = rows_done / cfg.H
+    return tokens / total, {
+        "cores": threads,
+        "sample": (f"{rows_done} query rows (of {cfg.rows}) of the {cfg.name} workload over "
+                   f"{steps} step(s), all heads; plus whole-tensor binarization pro rata; "
+                   f"tokens = rows / H"),
+        "seconds": total,
+    }
+
+
+def run_reference(args, world, rank):
+    cfg = synth.CONFIGS[args.config]
+    if rank != 0:
+        return
+    steps = max(1, args.steps)
+    per_step = max(1.0, min(args.cpu_seconds, 150.0 / (steps + args.warmup)))
+    if args.warmup:
+        oracle_baseline(cfg, per_step * 0.2, steps=1)
+    value, info = oracle_baseline(cfg, per_step, steps=steps)
+    line = {
+        "impl": "reference", "metric": METRIC, "value": value, "unit": "tokens/s",
+        "n_gpus": args.gpus, "steps": steps, "warmup": args.warmup,
+        "ms_per_step": info["seconds"] * 1e3 / steps, "higher_is_better": True,
+        "scaling": "weak", "vs_baseline": None, "dtype": "int32+f64", "data": "synthetic",
+        "config": {"workload": cfg.describe(), "B": cfg.B, "H": cfg.H, "seq_len": cfg.n,
+                   "d": cfg.d, "N": cfg.N, "parallelism": "rank 0 only (CPU oracle)"},
+        "cpu_baseline": {"value": value, "unit": "tokens/s", "cores": info["cores"],
+                         "kind": "oracle", "sample": info["sample"]},
+        "e2e": {"value": value, "unit": "tokens/s", "h2d_bytes_per_step": 0,
+                "d2h_bytes_per_step": 0},
+    }
+    print(json.dumps(line), flush=True)
+
+
+# --------------------------------------------------------------------------- had
+
+
+def run_had(args, world, rank, local):
+    from sparse_attention_sigma_b200 import had
+    cfg = synth.CONFIGS[args.config]
+    dev = torch.device("cuda", local)
+    torch.cuda.set_device(dev)
+    stream = torch.cuda.current_stream()
+    peaks = measured_peaks()
+    model = roofline_model(cfg, peaks)
+
+    q, k, v, sgq, sgk = synth.make_inputs(cfg)
+    gq, gk, gv = q.to(dev), k.to(dev), v.to(dev)
+    gsq, gsk = sgq.to(dev), sgk.to(dev)
+    out = torch.empty((cfg.B, cfg.H, cfg.n, cfg.d), dtype=torch.float32, device=dev)
+    ws = had.workspace(cfg.B, cfg.H, cfg.n, cfg.d, cfg.N, device=dev)
+    flush = torch.empty(L2_FLUSH_BYTES // 4, dtype=torch.float32, device=dev)
+    launches_per_step = had.had_launch_count(had.HAD_OP_ATTENTION_FWD, cfg.B, cfg.H, cfg.n,
+                                             cfg.d, cfg.N)
+
+    def step():
+        had.had_attention_fwd(gq, gk, gv, gsq, gsk, cfg.N, cfg.tau, out=out, ws=ws)
+
+    for _ in range(max(3, args.warmup)):
+        step()
+    torch.cuda.synchronize()
+
+    starts = [torch.cuda.Event(enable_timing=True) for _ in range(args.steps)]
+    ends = [torch.cuda.Event(enable_timing=True) for _ in range(args.steps)]
+    clocks = ClockSampler(local)
+    clocks.start()
+    barrier(world)
+    torch.cuda.synchronize()
+    for i in range(args.steps):
+        flush.fill_(float(i))                 # evict L2 between steps (outside the events)
+        starts[i].record(stream)
+        step()
+        ends[i].record(stream)
+    torch.cuda.synchronize()
+    barrier(world)
+    clock_info = clocks.stop()
+    ms = sum(s.elapsed_time(e) for s, e in zip(starts, ends)) / args.steps
+    ms = max_over_ranks(ms, world, dev)
+
+    tokens_per_rank = cfg.tokens
+    value = tokens_per_rank * world / (ms * 1e-3)
+
+    # per-kernel view: the same work through the unfused entry points, so
+    # each kernel of the step can be bracketed by its own events
+    kernel_ms = per_kernel_times(had, cfg, gq, gk, gv, gsq, gsk, flush, dev)
+    dominant = max(kernel_ms, key=kernel_ms.get)
+    achieved = model["work"] / (ms * 1e-3) / 1e12
+    peak_eff = model["work"] / model["t_roof"] / 1e12
+
+    e2e = None
+    if not args.no_e2e:
+        e2e = end_to_end(had, cfg, q, k, v, gsq, gsk, ws, dev, max(3, args.steps // 2), world)
+
+    cpu = None
+    if rank == 0 and world == 1 and not args.no_cpu_baseline:
+        val, info = oracle_baseline(cfg, args.cpu_seconds)
+        cpu = {"value": val, "unit": "tokens/s", "cores": info["cores"], "kind": "oracle",
+               "sample": info["sample"]}
+
+    if rank != 0:
+        return
+    line = {
+        "metric": METRIC, "value": value, "unit": "tokens/s", "n_gpus": world,
+        "steps": args.steps, "warmup": max(3, args.warmup), "ms_per_step": ms,
+        "higher_is_better": True, "scaling": "weak", "vs_baseline": None, "dtype": "bf16",
+        "data": "synthetic",
+        "config": {"workload": cfg.describe(), "B": cfg.B, "H": cfg.H, "seq_len": cfg.n,
+                   "d": cfg.d, "N": cfg.N, "global_batch": cfg.B * world,
+                   "parallelism": f"weak: {world} rank(s), one batch of independent heads each",
+                   "l2": "flushed between steps (256 MiB write outside the timed events)"},
+        "roofline": {"bound": "tensor", "achieved": achieved, "peak": peak_eff,
+                     "unit": "TFLOP/s", "frac": achieved / peak_eff, "traffic": None,
+                     "kernel": "had_attention_fwd (whole call)",
+                     "t_roof_us": model["t_roof"] * 1e6, "t_hbm_us": model["t_hbm"] * 1e6,
+                     "t_tc_us": model["t_tc"] * 1e6, "t_alu_us": model["t_alu"] * 1e6,
+                     "peaks": peaks["source"]},
+        "kernels_ms": kernel_ms, "dominant_kernel": dominant,
+        "gpu_launches": launches_per_step * args.steps,
+        "clocks": clock_info,
+        "e2e": e2e,
+        "cpu_baseline": cpu,
+    }
+    print(json.dumps(line), flush=True)
+
+
+def per_kernel_times(had, cfg, gq, gk, gv, gsq, gsk, flush, dev, reps=5):
+    qb = had.had_binarize_pack(gq, gsq)
+    kb = had.had_binarize_pack(gk, gsk)
+    idx, lg = had.had_hamming_topn(qb, kb, cfg.d, cfg.N)
+    out, _ = had.had_sparse_softmax_av(idx, lg, gv, cfg.tau)
+    stream = torch.cuda.current_stream()
+    calls = {
+        "pack_bits (Q and K)": lambda: (had.had_binarize_pack(gq, gsq, bits=qb),
+                                        had.had_binarize_pack(gk, gsk, bits=kb)),
+        "topn_simt": lambda: had.had_hamming_topn(qb, kb, cfg.d, cfg.N, idx=idx, logits=lg),
+        "sparse_softmax_av": lambda: had.had_sparse_softmax_av(idx, lg, gv, cfg.tau, out=out),
+    }
+    res = {}
+    for name, fn in calls.items():
+        fn()
+        tot = 0.0
+        for i in range(reps):
+            flush.fill_(float(i))
+            s = torch.cuda.Event(enable_timing=True)
+            e = torch.cuda.Event(enable_timing=True)
+            s.record(stream)
+            fn()
+            e.record(stream)
+            torch.cuda.synchronize()
+            tot += s.elapsed_time(e)
+        res[name] = tot / reps
+    return res
+
+
+def end_to_end(had, cfg, q, k, v, gsq, gsk, ws, dev, steps, world):
+    """Same call with inputs copied from pinned host memory and O copied back."""
+    hq, hk, hv = q.pin_memory(), k.pin_memory(), v.pin_memory()
+    ho = torch.empty((cfg.B, cfg.H, cfg.n, cfg.d), dtype=torch.float32).pin_memory()
+    gq = torch.empty_like(q, device=dev)
+    gk = torch.empty_like(k, device=dev)
+    gv = torch.empty_like(v, device=dev)
+    out = torch.empty(ho.shape, dtype=torch.float32, device=dev)
+    stream = torch.cuda.current_stream()
+
+    def step():
+        gq.copy_(hq, non_blocking=True)
+        gk.copy_(hk, non_blocking=True)
+        gv.copy_(hv, non_blocking=True)
+        had.had_attention_fwd(gq, gk, gv, gsq, gsk, cfg.N, cfg.tau, out=out, ws=ws)
+        ho.copy_(out, non_blocking=True)
+
+    for _ in range(2):
+        step()
+    torch.cuda.synchronize()
+    s = torch.cuda.Event(enable_timing=True)
+    e = torch.cuda.Event(enable_timing=True)
+    barrier(world)
+    s.record(stream)
+    for _ in range(steps):
+        step()
+    e.record(stream)
+    torch.cuda.synchronize()
+    ms = max_over_ranks(s.elapsed_time(e) / steps, world, dev)
+    h2d = (q.numel() + k.numel() + v.numel()) * q.element_size()
+    return {"value": cfg.tokens * world / (ms * 1e-3), "unit": "tokens/s",
+            "h2d_bytes_per_step": h2d, "d2h_bytes_per_step": ho.numel() * 4,
+            "ms_per_step": ms}
+
+
+def main():
+    args = parse()
+    world, rank, local = dist_setup(args)
+    try:
+        if args.impl == "reference":
+            run_reference(args, world, rank)
+        else:
+            run_had(args, world, rank, local)
+    finally:
+        if world > 1:
+            import torch.distributed as dist
+            dist.destroy_process_group()
+
+
+if __name__ == "__main__":
+    main()

@@ -1,0 +1,159 @@
+/*
+ * had.h -- C ABI of the B200 (sm_100a) library for the inference forward pass
+ * of Hamming Attention Distillation (HAD).
+ *
+ * Source of the method: "Hamming Attention Distillation: Binarizing Keys and
+ * Queries for Efficient Long-Context Transformers" (arXiv 2502.01770), as
+ * summarised by its pith.science review page, section "What carries the
+ * argument" and the circularity audit (Eqs. 4-7, Eq. 12), and by the abstract
+ * on the mlsanity.com index page.  Queries and keys are standardized by
+ * per-head coefficients sigma_Q, sigma_K and sign-quantized to {-1,+1}; the
+ * logit of query i and key j is the +/-1 dot product
+ *     s_ij = d - 2 * popcount(q_i XOR k_j)         (an integer in [-d, d]);
+ * each query row keeps its N largest logits (ties go to the lower key index),
+ * a softmax with temperature tau runs over those N only, and the output is
+ *     O_i = sum_{j kept} p_ij V_j,   p_ij = exp(tau (s_ij - m_i)) / Z_i
+ * with V kept in full precision and O returned as fp32.
+ *
+ * Conventions shared by every entry point
+ *   - Tensors are dense, row-major, contiguous, in device memory, 16-byte
+ *     aligned: Q, K, V and O are [B, H, n, d]; packed bits are
+ *     [B, H, n, d/32] uint32; idx / logits / p are [B, H, n, N].
+ *   - Packed bits: bit k of word w of a row is 1 iff element 32*w + k of
+ *     that row has sign -1.  sign(z) = -1 iff z < 0, where z = x / sigma_h is
+ *     an IEEE fp32 round-to-nearest division with subnormals kept; +0, -0 and
+ *     NaN give +1.
+ *   - sigma arrays are device float[H], one coefficient per head.
+ *   - Supported: d in {64, 128}; 1 <= N <= n; n * N < 2^31; B, H, n >= 1.
+ *   - Ownership: the caller allocates and frees every buffer, workspace
+ *     included.  The library allocates nothing and keeps no state between
+ *     calls.
+ *   - Calls are asynchronous on `stream` and never synchronize.  Argument
+ *     errors are returned before anything is launched.  A launch failure
+ *     returns HAD_ERR_CUDA.  Conditions only the device can see are OR-ed
+ *     into *dev_status as bit (1 << code) (for example 1 << HAD_ERR_BAD_SIGMA
+ *     when a sigma is <= 0 or not finite); dev_status is an optional device
+ *     int32 the caller zeroes beforehand and reads after synchronizing.
+ *     Outputs of a call that flagged a device condition are unspecified.
+ */
+#ifndef HAD_H
+#define HAD_H
+
+#include <stddef.h>
+#include <stdint.h>
+#include <cuda_runtime_api.h>
+
+#if defined(__GNUC__)
+#define HAD_API __attribute__((visibility("default")))
+#else
+#define HAD_API
+#endif
+
+#ifdef __cplusplus
+extern "C" {
+#endif
+
+typedef enum {
+    HAD_OK = 0,
+    HAD_ERR_INVALID_ARG = 1,  /* null pointer, bad size, N outside [1, n], misalignment */
+    HAD_ERR_UNSUPPORTED = 2,  /* d not in {64, 128}, or sizes beyond the stated limits */
+    HAD_ERR_WORKSPACE = 3,    /* workspace null or smaller than had_workspace_bytes() */
+    HAD_ERR_CUDA = 4,         /* a CUDA launch or runtime call failed */
+    HAD_ERR_BAD_SIGMA = 5,    /* device flag: a sigma is <= 0, NaN or infinite */
+    HAD_ERR_TIMEOUT = 6       /* device flag: a bounded on-chip wait gave up */
+} had_status_t;
+
+typedef enum {
+    HAD_BF16 = 0,             /* bfloat16 storage */
+    HAD_F32 = 1               /* IEEE binary32 storage */
+} had_dtype_t;
+
+typedef enum {
+    HAD_OP_BINARIZE_PACK = 0,     /* had_binarize_pack */
+    HAD_OP_HAMMING_TOPN = 1,      /* had_hamming_topn */
+    HAD_OP_ATTENTION_FWD = 2,     /* had_attention_fwd */
+    HAD_OP_SPARSE_SOFTMAX_AV = 3  /* had_sparse_softmax_av */
+} had_op_t;
+
+/*
+ * Standardize + sign + bit-pack (Eqs. 4-5 with the Eq. 12 coefficients).
+ *   x      [B,H,n,d] of dtype dt (device)
+ *   sigma  [H] float (device); flags HAD_ERR_BAD_SIGMA if any is <= 0 or
+ *          not finite (the bits are still written from the division)
+ *   bits   [B,H,n,d/32] uint32 out (device)
+ */
+HAD_API had_status_t had_binarize_pack(const void *x, had_dtype_t dt, const float *sigma,
+                               int B, int H, int n, int d, uint32_t *bits,
+                               int32_t *dev_status, cudaStream_t stream);
+
+/*
+ * Hamming logits and top-N selection (Eq. 5 and Eq. 6), unfused.
+ *   qbits, kbits  [B,H,n,d/32] packed as above (device)
+ *   idx     [B,H,n,N] int32 out: kept key indices of each row, ascending
+ *   logits  [B,H,n,N] int16 out, or NULL: s_ij of the kept keys, same order
+ *   ws      workspace of had_workspace_bytes(HAD_OP_HAMMING_TOPN, ...) bytes
+ *           (may be NULL when that size is 0)
+ * The kept set is exact: the N largest s_ij, the lower key index winning at
+ * the threshold.
+ */
+HAD_API had_status_t had_hamming_topn(const uint32_t *qbits, const uint32_t *kbits,
+                              int B, int H, int n, int d, int N,
+                              int32_t *idx, int16_t *logits,
+                              void *ws, size_t ws_bytes,
+                              int32_t *dev_status, cudaStream_t stream);
+
+/*
+ * Softmax over the kept logits and sparse product with V (Eq. 7).
+ *   idx, logits  [B,H,n,N] as produced by had_hamming_topn (device)
+ *   V      [B,H,n,d] of dtype dt (device), full precision
+ *   tau    softmax temperature (1/sqrt(d) in the reference workloads)
+ *   out    [B,H,n,d] float out
+ *   p      [B,H,n,N] float out, or NULL: the probabilities, same order as idx
+ * Every idx entry must lie in [0, n); entries outside it are skipped and
+ * flag HAD_ERR_INVALID_ARG in *dev_status.
+ */
+HAD_API had_status_t had_sparse_softmax_av(const int32_t *idx, const int16_t *logits,
+                                   const void *V, had_dtype_t dt,
+                                   int B, int H, int n, int d, int N, float tau,
+                                   float *out, float *p,
+                                   int32_t *dev_status, cudaStream_t stream);
+
+/*
+ * The whole forward pass, fused: O = sparse_softmax_topN(binarized logits) V.
+ *   Q, K, V   [B,H,n,d] of dtype dt (device)
+ *   sigma_q, sigma_k  [H] float (device)
+ *   out       [B,H,n,d] float out
+ *   dbg_idx, dbg_logits  [B,H,n,N] optional outputs of the kept set (may be
+ *             NULL; when given they hold exactly what had_hamming_topn would)
+ *   ws        workspace of had_workspace_bytes(HAD_OP_ATTENTION_FWD, ...)
+ * The n x n logit matrix never goes to memory.
+ */
+HAD_API had_status_t had_attention_fwd(const void *Q, const void *K, const void *V,
+                               had_dtype_t dt,
+                               const float *sigma_q, const float *sigma_k,
+                               int B, int H, int n, int d, int N, float tau,
+                               float *out, int32_t *dbg_idx, int16_t *dbg_logits,
+                               void *ws, size_t ws_bytes,
+                               int32_t *dev_status, cudaStream_t stream);
+
+/*
+ * Workspace bytes an operation needs for these sizes (0 if none), or
+ * (size_t)-1 for unsupported or invalid sizes.
+ */
+HAD_API size_t had_workspace_bytes(int op, int B, int H, int n, int d, int N);
+
+/* Static, human-readable name of a status code. */
+HAD_API const char *had_status_string(had_status_t status);
+
+/*
+ * Number of kernels one call of `op` enqueues for these sizes (-1 for
+ * unsupported or invalid sizes).  Lets a caller count launches without a
+ * profiler.
+ */
+HAD_API int had_launch_count(int op, int B, int H, int n, int d, int N);
+
+#ifdef __cplusplus
+}
+#endif
+
+#endif /* HAD_H */

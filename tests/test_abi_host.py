@@ -1,0 +1,85 @@
+"""Host-side checks of the C ABI that need no GPU.
+
+The library must load and export every function include/had.h declares;
+argument checks, workspace sizing and status strings run on the host and
+return before anything touches the device.
+"""
+import ctypes
+import os
+import re
+
+import pytest
+
+ROOT = os.path.dirname(os.path.dirname(os.path.abspath(__file__)))
+HEADER = os.path.join(ROOT, "include", "had.h")
+LIB = os.path.join(ROOT, "sparse_attention_sigma_b200", "libhad.so")
+
+
+def declared_functions():
+    text = open(HEADER).read()
+    text = re.sub(r"/\*.*?\*/", "", text, flags=re.S)
+    return sorted(set(re.findall(r"\b(had_[a-z0-9_]+)\s*\(", text)))
+
+
+@pytest.fixture(scope="module")
+def lib():
+    if not os.path.exists(LIB):
+        from sparse_attention_sigma_b200 import build
+        build.build()
+    return ctypes.CDLL(LIB)
+
+
+def test_header_declares_the_entry_points():
+    names = declared_functions()
+    for want in ("had_binarize_pack", "had_hamming_topn", "had_sparse_softmax_av",
+                 "had_attention_fwd", "had_workspace_bytes", "had_status_string"):
+        assert want in names
+
+
+def test_library_exports_every_declared_symbol(lib):
+    missing = [n for n in declared_functions() if not hasattr(lib, n)]
+    assert not missing, missing
+
+
+def test_status_strings(lib):
+    lib.had_status_string.restype = ctypes.c_char_p
+    lib.had_status_string.argtypes = [ctypes.c_int]
+    assert lib.had_status_string(0) == b"HAD_OK"
+    assert lib.had_status_string(5) == b"HAD_ERR_BAD_SIGMA"
+    assert lib.had_status_string(99) == b"HAD_ERR_UNKNOWN"
+
+
+def test_workspace_and_launch_counts(lib):
+    lib.had_workspace_bytes.restype = ctypes.c_size_t
+    lib.had_workspace_bytes.argtypes = [ctypes.c_int] * 6
+    lib.had_launch_count.argtypes = [ctypes.c_int] * 6
+    bad = ctypes.c_size_t(-1).value
+    assert lib.had_workspace_bytes(2, 4, 16, 4096, 64, 512) > 0
+    assert lib.had_workspace_bytes(2, 4, 16, 4096, 96, 512) == bad      # d unsupported
+    assert lib.had_workspace_bytes(2, 4, 16, 4096, 64, 4097) == bad     # N > n
+    assert lib.had_workspace_bytes(0, 1, 1, 8, 64, 1) == 0
+    assert lib.had_launch_count(0, 1, 1, 8, 64, 1) == 1
+    assert lib.had_launch_count(2, 1, 1, 8, 64, 0) == -1
+
+
+def test_argument_errors_return_before_any_cuda_call(lib):
+    f = lib.had_attention_fwd
+    vp, i, sz = ctypes.c_void_p, ctypes.c_int, ctypes.c_size_t
+    f.argtypes = [vp, vp, vp, i, vp, vp, i, i, i, i, i, ctypes.c_float, vp, vp, vp, vp, sz, vp, vp]
+    f.restype = ctypes.c_int
+    fake = vp(4096)        # never dereferenced: the checks fail first
+    # d = 96 is unsupported
+    assert f(fake, fake, fake, 0, fake, fake, 1, 1, 8, 96, 2, 0.1, fake, None, None,
+             fake, 1 << 20, None, None) == 2
+    # N > n
+    assert f(fake, fake, fake, 0, fake, fake, 1, 1, 8, 64, 9, 0.1, fake, None, None,
+             fake, 1 << 20, None, None) == 1
+    # null Q
+    assert f(None, fake, fake, 0, fake, fake, 1, 1, 8, 64, 2, 0.1, fake, None, None,
+             fake, 1 << 20, None, None) == 1
+    # workspace too small
+    assert f(fake, fake, fake, 0, fake, fake, 1, 1, 8, 64, 2, 0.1, fake, None, None,
+             fake, 16, None, None) == 3
+    # misaligned pointer
+    assert f(vp(4097), fake, fake, 0, fake, fake, 1, 1, 8, 64, 2, 0.1, fake, None, None,
+             fake, 1 << 20, None, None) == 1

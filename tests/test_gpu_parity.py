@@ -1,0 +1,245 @@
+"""GPU parity: the CUDA path through the C ABI against the CPU oracle.
+
+Bit-exact for packed bits, kept indices and integer logits; fp32 outputs
+within max |err| <= 2e-3 and ||err||_2 / ||ref||_2 <= 1e-3 (the tolerance
+the forward pass is specified to, on bf16 inputs).  Small cases compare
+every row; the five full-size workloads compare every packed bit and a
+seeded sample of rows, in the launch configuration the benchmark times.
+"""
+import math
+
+import numpy as np
+import pytest
+import torch
+
+import oracle
+import synth
+from tests import _golden
+
+pytestmark = pytest.mark.gpu
+
+MAX_ABS = 2e-3
+REL_L2 = 1e-3
+
+
+@pytest.fixture(scope="module")
+def had():
+    from sparse_attention_sigma_b200 import had as _had
+    return _had
+
+
+def assert_close(got, ref, what=""):
+    got = np.asarray(got, np.float64)
+    ref = np.asarray(ref, np.float64)
+    err = np.abs(got - ref)
+    assert err.max() <= MAX_ABS, f"{what}: max abs err {err.max():.3e}"
+    rel = np.linalg.norm(got - ref) / max(np.linalg.norm(ref), 1e-30)
+    assert rel <= REL_L2, f"{what}: rel L2 err {rel:.3e}"
+
+
+class Case:
+    """Inputs on the CPU and the GPU plus the oracle's signs."""
+
+    def __init__(self, q, k, v, sgq, sgk, N, tau):
+        self.q, self.k, self.v, self.sgq, self.sgk = q, k, v, sgq, sgk
+        self.B, self.H, self.n, self.d = q.shape
+        self.N, self.tau = N, tau
+        self.sq = oracle.binarize(synth.to_oracle_array(q), sgq.numpy())
+        self.sk = oracle.binarize(synth.to_oracle_array(k), sgk.numpy())
+        self.v_or = synth.to_oracle_array(v)
+        self.gq, self.gk, self.gv = q.cuda(), k.cuda(), v.cuda()
+        self.gsq, self.gsk = sgq.cuda(), sgk.cuda()
+
+    def oracle_rows(self, rows):
+        return oracle.attention_rows(self.sq, self.sk, self.v_or, self.tau, self.N, rows)
+
+
+_cases = {}
+
+
+def config_case(name):
+    if name not in _cases:
+        cfg = synth.CONFIGS[name]
+        q, k, v, sgq, sgk = synth.make_inputs(cfg)
+        _cases[name] = Case(q, k, v, sgq, sgk, cfg.N, cfg.tau)
+    return _cases[name]
+
+
+def random_case(B, H, n, d, N, seed, dtype=torch.bfloat16, tau=None):
+    g = torch.Generator().manual_seed(seed)
+    q = torch.randn(B, H, n, d, generator=g).to(dtype)
+    k = torch.randn(B, H, n, d, generator=g).to(dtype)
+    v = torch.randn(B, H, n, d, generator=g).to(dtype)
+    return Case(q, k, v, synth.per_head_sigma(q), synth.per_head_sigma(k), N,
+                1 / math.sqrt(d) if tau is None else tau)
+
+
+def all_rows(c):
+    return np.arange(c.B * c.H * c.n)
+
+
+SMALL = [
+    # (B, H, n, d, N, seed, dtype): several 128-row tiles and ragged tails
+    (1, 2, 128, 64, 16, 1, torch.float32),
+    (2, 3, 300, 64, 40, 2, torch.bfloat16),
+    (1, 2, 700, 64, 90, 3, torch.bfloat16),
+    (1, 2, 260, 128, 33, 4, torch.bfloat16),
+    (2, 1, 129, 128, 129, 5, torch.float32),        # N = n: dense softmax
+    (1, 1, 1, 64, 1, 6, torch.bfloat16),            # a single row and key
+    (1, 3, 97, 64, 1, 7, torch.bfloat16),           # N = 1
+]
+
+
+def _check_bits(had, c):
+    gb = had.had_binarize_pack(c.gq, c.gsq).cpu().numpy().view(np.uint32)
+    assert np.array_equal(gb, oracle.pack(c.sq))
+    kb = had.had_binarize_pack(c.gk, c.gsk)
+    assert np.array_equal(kb.cpu().numpy().view(np.uint32), oracle.pack(c.sk))
+    return had.had_binarize_pack(c.gq, c.gsq), kb
+
+
+def _check_unfused(had, c, rows):
+    qb, kb = _check_bits(had, c)
+    idx, lg = had.had_hamming_topn(qb, kb, c.d, c.N)
+    out, p = had.had_sparse_softmax_av(idx, lg, c.gv, c.tau, want_p=True)
+    torch.cuda.synchronize()
+    o_idx, o_lg, o_p, o_out = c.oracle_rows(rows)
+    flat = lambda t: t.reshape(-1, t.shape[-1]).cpu().numpy()[rows]
+    assert np.array_equal(flat(idx), o_idx)
+    assert np.array_equal(flat(lg), o_lg)
+    assert_close(flat(p), o_p, "p")
+    assert_close(flat(out), o_out, "out")
+
+
+def _check_fused(had, c, rows):
+    dbg_idx = torch.empty((c.B, c.H, c.n, c.N), dtype=torch.int32, device="cuda")
+    dbg_lg = torch.empty((c.B, c.H, c.n, c.N), dtype=torch.int16, device="cuda")
+    status = torch.zeros(1, dtype=torch.int32, device="cuda")
+    out = had.had_attention_fwd(c.gq, c.gk, c.gv, c.gsq, c.gsk, c.N, c.tau,
+                                dbg_idx=dbg_idx, dbg_logits=dbg_lg, dev_status=status)
+    torch.cuda.synchronize()
+    assert status.item() == 0
+    o_idx, o_lg, o_p, o_out = c.oracle_rows(rows)
+    flat = lambda t: t.reshape(-1, t.shape[-1]).cpu().numpy()[rows]
+    assert np.array_equal(flat(dbg_idx), o_idx)
+    assert np.array_equal(flat(dbg_lg), o_lg)
+    assert_close(flat(out), o_out, "fused out")
+    # without the debug outputs the result is the same
+    out2 = had.had_attention_fwd(c.gq, c.gk, c.gv, c.gsq, c.gsk, c.N, c.tau)
+    torch.cuda.synchronize()
+    assert torch.equal(out, out2)
+
+
+@pytest.mark.parametrize("B,H,n,d,N,seed,dtype", SMALL)
+def test_small_unfused_all_rows(had, B, H, n, d, N, seed, dtype):
+    c = random_case(B, H, n, d, N, seed, dtype)
+    _check_unfused(had, c, all_rows(c))
+
+
+@pytest.mark.parametrize("B,H,n,d,N,seed,dtype", SMALL)
+def test_small_fused_all_rows(had, B, H, n, d, N, seed, dtype):
+    c = random_case(B, H, n, d, N, seed, dtype)
+    _check_fused(had, c, all_rows(c))
+
+
+@pytest.mark.parametrize("name", ["tiny", "bert", "vit", "long", "vlong"])
+def test_workload_bits_full(had, name):
+    _check_bits(had, config_case(name))
+
+
+@pytest.mark.parametrize("name,count", [("tiny", 0), ("bert", 384), ("vit", 384),
+                                        ("long", 256), ("vlong", 96)])
+def test_workload_unfused_sampled(had, name, count):
+    c = config_case(name)
+    rows = all_rows(c) if count == 0 else synth.sample_rows(synth.CONFIGS[name], count)
+    _check_unfused(had, c, rows)
+
+
+@pytest.mark.parametrize("name,count", [("tiny", 0), ("bert", 384), ("vit", 384),
+                                        ("long", 256), ("vlong", 96)])
+def test_workload_fused_sampled(had, name, count):
+    c = config_case(name)
+    rows = all_rows(c) if count == 0 else synth.sample_rows(synth.CONFIGS[name], count)
+    _check_fused(had, c, rows)
+
+
+def test_all_keys_equal(had):
+    c = random_case(1, 2, 300, 64, 17, 11)
+    c.k[:] = c.k[:, :, :1]
+    c = Case(c.q, c.k, c.v, c.sgq, synth.per_head_sigma(c.k), c.N, c.tau)
+    dbg = torch.empty((1, 2, 300, 17), dtype=torch.int32, device="cuda")
+    out = had.had_attention_fwd(c.gq, c.gk, c.gv, c.gsq, c.gsk, c.N, c.tau, dbg_idx=dbg)
+    torch.cuda.synchronize()
+    assert (dbg.cpu() == torch.arange(17, dtype=torch.int32)).all()
+    mean = c.v[:, :, :17].double().mean(dim=2, keepdim=True).expand(-1, -1, 300, -1)
+    assert_close(out.cpu().numpy(), mean.numpy(), "mean of first N")
+
+
+def test_golden_handworked(had):
+    case = _golden.load()
+    q, k, v, sgq, sgk = (torch.from_numpy(a) for a in _golden.tensors(case))
+    c = Case(q, k, v, sgq, sgk, case["N"], case["tau"])
+    dbg = torch.empty((1, 1, 4, 2), dtype=torch.int32, device="cuda")
+    out = had.had_attention_fwd(c.gq, c.gk, c.gv, c.gsq, c.gsk, c.N, c.tau, dbg_idx=dbg)
+    torch.cuda.synchronize()
+    exp = case["expected"]
+    kb = had.had_binarize_pack(c.gk, c.gsk).cpu().numpy().view(np.uint32)
+    assert kb[0, 0].tolist() == exp["k_bits"]
+    for key in ("row0", "row1", "row3"):
+        r = int(key[3:])
+        assert dbg[0, 0, r].tolist() == exp[key]["idx"]
+        want = np.zeros(case["d"])
+        for col, ex in exp[key]["out_nonzero"].items():
+            want[int(col)] = _golden.closed_form(ex)
+        assert np.allclose(out[0, 0, r].cpu().numpy(), want, rtol=1e-5, atol=1e-6)
+
+
+def test_sign_edge_values_on_device(had):
+    vals = [0.0, -0.0, float("nan"), float("inf"), float("-inf"), 1e-45, -1e-45,
+            -1.1754944e-38, -1e-30, 3.0, -3.0]
+    x = torch.ones(1, 3, 1, 64)
+    for i, v in enumerate(vals):
+        x[0, :, 0, i] = v
+    sigma = torch.tensor([1.0, 3.0, 1e9])
+    got = had.had_binarize_pack(x.cuda(), sigma.cuda()).cpu().numpy().view(np.uint32)
+    ref = oracle.pack(oracle.binarize(x.numpy(), sigma.numpy()))
+    assert np.array_equal(got, ref)
+
+
+def test_bad_sigma_is_flagged(had):
+    c = random_case(1, 2, 64, 64, 8, 12)
+    status = torch.zeros(1, dtype=torch.int32, device="cuda")
+    had.had_binarize_pack(c.gq, torch.tensor([1.0, -1.0], device="cuda"), dev_status=status)
+    torch.cuda.synchronize()
+    assert status.item() & (1 << had.HAD_ERR_BAD_SIGMA)
+    status.zero_()
+    had.had_attention_fwd(c.gq, c.gk, c.gv, c.gsq, torch.tensor([float("nan"), 1.0], device="cuda"),
+                          c.N, c.tau, dev_status=status)
+    torch.cuda.synchronize()
+    assert status.item() & (1 << had.HAD_ERR_BAD_SIGMA)
+
+
+def test_invalid_arguments_rejected_before_launch(had):
+    c = random_case(1, 1, 64, 64, 8, 13)
+    with pytest.raises(had.HadError) as e:
+        had.had_attention_fwd(c.gq, c.gk, c.gv, c.gsq, c.gsk, 65, c.tau)
+    assert e.value.status == had.HAD_ERR_INVALID_ARG
+    small = torch.empty(16, dtype=torch.uint8, device="cuda")
+    with pytest.raises(had.HadError) as e:
+        had.had_attention_fwd(c.gq, c.gk, c.gv, c.gsq, c.gsk, 8, c.tau, ws=small)
+    assert e.value.status == had.HAD_ERR_WORKSPACE
+    x = torch.randn(1, 1, 8, 96, device="cuda")
+    with pytest.raises(had.HadError) as e:
+        had.had_binarize_pack(x, torch.ones(1, device="cuda"))
+    assert e.value.status == had.HAD_ERR_UNSUPPORTED
+
+
+def test_out_of_range_index_flagged(had):
+    c = random_case(1, 1, 40, 64, 4, 14)
+    idx = torch.zeros((1, 1, 40, 4), dtype=torch.int32, device="cuda")
+    idx[0, 0, 3, 2] = 40
+    lg = torch.zeros((1, 1, 40, 4), dtype=torch.int16, device="cuda")
+    status = torch.zeros(1, dtype=torch.int32, device="cuda")
+    had.had_sparse_softmax_av(idx, lg, c.gv, c.tau, dev_status=status)
+    torch.cuda.synchronize()
+    assert status.item() & (1 << had.HAD_ERR_INVALID_ARG)
