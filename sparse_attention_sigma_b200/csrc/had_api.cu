@@ -76,8 +76,9 @@ had_status_t launch_topn_dw(const uint32_t *qb, const uint32_t *kb, int B, int H
     if (cudaFuncSetAttribute(had::topn_simt_kernel<DW>,
                              cudaFuncAttributeMaxDynamicSharedMemorySize, smem) != cudaSuccess)
         return HAD_ERR_CUDA;
-    dim3 grid((n + had::kTopnRows - 1) / had::kTopnRows, B * H);
-    had::topn_simt_kernel<DW><<<grid, had::kTopnRows, smem, st>>>(qb, kb, n, N, idx, lg);
+    const long long blocks = (long long)((n + had::kTopnRows - 1) / had::kTopnRows) * B * H;
+    if (blocks > INT_MAX) return HAD_ERR_UNSUPPORTED;
+    had::topn_simt_kernel<DW><<<(unsigned)blocks, had::kTopnRows, smem, st>>>(qb, kb, n, N, idx, lg);
     return launched();
 }
 

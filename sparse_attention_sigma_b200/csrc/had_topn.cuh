@@ -42,8 +42,9 @@ topn_simt_kernel(const uint32_t *__restrict__ qbits, const uint32_t *__restrict_
     uint32_t *kch = smem + BINS * kTopnRows;        // [kTopnKeyChunk][DW]
 
     const int tid = threadIdx.x;
-    const long long head = blockIdx.y;
-    const int row = blockIdx.x * kTopnRows + tid;
+    const int tiles = (n + kTopnRows - 1) / kTopnRows;
+    const long long head = blockIdx.x / tiles;
+    const int row = (int)(blockIdx.x % tiles) * kTopnRows + tid;
     const bool active = row < n;
 
     uint32_t q[DW];
