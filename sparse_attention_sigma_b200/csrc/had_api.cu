@@ -10,6 +10,8 @@
 #include "had_pack.cuh"
 #include "had_topn.cuh"
 #include "had_av.cuh"
+#include "had_prep.cuh"
+#include "had_fused.cuh"
 
 namespace {
 
@@ -118,21 +120,96 @@ had_status_t launch_av(const int32_t *idx, const int16_t *lg, const void *V, had
     return launched();
 }
 
-// Workspace of the fused forward: packed Q and K bits, then the kept set.
+// Workspace of the fused forward: tensor-core operand tiles of Q, K and V^T
+// and the per-head V scale.
 struct FwdWorkspace {
-    size_t qbits, kbits, idx, lg, total;
+    size_t qop, kop, vop, vmax, vexp, total;
+    int qtiles, ktiles;
 };
 
 FwdWorkspace fwd_layout(int B, int H, int n, int d, int N)
 {
-    const size_t rows = (size_t)B * H * n;
+    (void)N;
+    const size_t bh = (size_t)B * H;
     FwdWorkspace w;
-    w.qbits = 0;
-    w.kbits = w.qbits + round_up(rows * (d / 32) * 4);
-    w.idx = w.kbits + round_up(rows * (d / 32) * 4);
-    w.lg = w.idx + round_up(rows * (size_t)N * 4);
-    w.total = w.lg + round_up(rows * (size_t)N * 2);
+    const int qt = d == 64 ? had::fused::Cfg<64>::QT : had::fused::Cfg<128>::QT;
+    w.qtiles = (n + had::fused::kRows - 1) / had::fused::kRows;
+    w.qtiles = (w.qtiles + qt - 1) / qt * qt;
+    w.ktiles = (n + had::fused::kKeys - 1) / had::fused::kKeys;
+    w.qop = 0;
+    w.kop = w.qop + round_up(bh * w.qtiles * had::fused::kRows * d);
+    w.vop = w.kop + round_up(bh * w.ktiles * had::fused::kKeys * d);
+    w.vmax = w.vop + round_up(bh * w.ktiles * had::fused::kKeys * d * 2);
+    w.vexp = w.vmax + round_up(bh * 4);
+    w.total = w.vexp + round_up(bh * 4);
     return w;
+}
+
+template <typename T, int D>
+had_status_t launch_fused_typed(const T *Q, const T *K, const T *V, const float *sq,
+                                const float *sk, int B, int H, int n, int N, float tau,
+                                float *out, int32_t *dbg_idx, int16_t *dbg_lg, char *ws,
+                                const FwdWorkspace &w, int32_t *status, cudaStream_t st)
+{
+    using C = had::fused::Cfg<D>;
+    const long long bh = (long long)B * H;
+    auto *qop = reinterpret_cast<int8_t *>(ws + w.qop);
+    auto *kop = reinterpret_cast<int8_t *>(ws + w.kop);
+    auto *vop = reinterpret_cast<__half *>(ws + w.vop);
+    auto *vmax = reinterpret_cast<unsigned int *>(ws + w.vmax);
+    auto *vexp = reinterpret_cast<int *>(ws + w.vexp);
+    if (cudaMemsetAsync(vmax, 0, bh * 4, st) != cudaSuccess) return HAD_ERR_CUDA;
+    const long long qchunks = bh * w.qtiles * had::fused::kRows * (D / 16);
+    const long long kchunks = bh * w.ktiles * had::fused::kKeys * (D / 16);
+    had::prep::sign_operand_kernel<T><<<grid_for(qchunks, 256), 256, 0, st>>>(
+        Q, sq, H, n, D, had::fused::kRows, w.qtiles, qchunks, qop, status);
+    had::prep::sign_operand_kernel<T><<<grid_for(kchunks, 256), 256, 0, st>>>(
+        K, sk, H, n, D, had::fused::kKeys, w.ktiles, kchunks, kop, status);
+    const long long vgroups = bh * n * D / 8;
+    had::prep::vmax_kernel<T><<<grid_for(vgroups, 256), 256, 0, st>>>(
+        V, (long long)n * D / 8, vgroups, vmax);
+    had::prep::v_operand_kernel<T, D><<<(unsigned)(bh * w.ktiles), 256, 0, st>>>(
+        V, n, vmax, vop, vexp);
+    had_status_t s = launched();
+    if (s != HAD_OK) return s;
+    const bool dbg = dbg_idx != nullptr || dbg_lg != nullptr;
+    auto kernel = dbg ? had::fused::attention_fwd_kernel<D, true>
+                      : had::fused::attention_fwd_kernel<D, false>;
+    if (cudaFuncSetAttribute(kernel, cudaFuncAttributeMaxDynamicSharedMemorySize,
+                             C::SMEM_BYTES) != cudaSuccess)
+        return HAD_ERR_CUDA;
+    had::fused::Params p;
+    p.qop = qop;
+    p.kop = kop;
+    p.vop = vop;
+    p.vexp = vexp;
+    p.out = out;
+    p.dbg_idx = dbg_idx;
+    p.dbg_logits = dbg_lg;
+    p.status = status;
+    p.n = n;
+    p.N = N;
+    p.qtiles = w.qtiles;
+    p.ktiles = w.ktiles;
+    p.ctas_per_head = w.qtiles / C::QT;
+    p.c2 = tau * 1.4426950408889634f;
+    const long long blocks = bh * p.ctas_per_head;
+    kernel<<<(unsigned)blocks, C::THREADS, C::SMEM_BYTES, st>>>(p);
+    return launched();
+}
+
+template <typename T>
+had_status_t launch_fused(const void *Q, const void *K, const void *V, const float *sq,
+                          const float *sk, int B, int H, int n, int d, int N, float tau,
+                          float *out, int32_t *dbg_idx, int16_t *dbg_lg, char *ws,
+                          const FwdWorkspace &w, int32_t *status, cudaStream_t st)
+{
+    const T *q = static_cast<const T *>(Q), *k = static_cast<const T *>(K),
+            *v = static_cast<const T *>(V);
+    return d == 64 ? launch_fused_typed<T, 64>(q, k, v, sq, sk, B, H, n, N, tau, out, dbg_idx,
+                                               dbg_lg, ws, w, status, st)
+                   : launch_fused_typed<T, 128>(q, k, v, sq, sk, B, H, n, N, tau, out, dbg_idx,
+                                                dbg_lg, ws, w, status, st);
 }
 
 }  // namespace
@@ -198,15 +275,13 @@ had_status_t had_attention_fwd(const void *Q, const void *K, const void *V, had_
     if (!(tau == tau) || tau > 3.0e38f || tau < -3.0e38f) return HAD_ERR_INVALID_ARG;
     const FwdWorkspace w = fwd_layout(B, H, n, d, N);
     if (!ws || ws_bytes < w.total || !aligned16(ws)) return HAD_ERR_WORKSPACE;
+    if ((long long)B * H * w.qtiles > INT_MAX) return HAD_ERR_UNSUPPORTED;
     char *base = static_cast<char *>(ws);
-    auto *qb = reinterpret_cast<uint32_t *>(base + w.qbits);
-    auto *kb = reinterpret_cast<uint32_t *>(base + w.kbits);
-    int32_t *idx = dbg_idx ? dbg_idx : reinterpret_cast<int32_t *>(base + w.idx);
-    int16_t *lg = dbg_logits ? dbg_logits : reinterpret_cast<int16_t *>(base + w.lg);
-    if ((s = launch_pack(Q, dt, sigma_q, B, H, n, d, qb, dev_status, stream)) != HAD_OK) return s;
-    if ((s = launch_pack(K, dt, sigma_k, B, H, n, d, kb, dev_status, stream)) != HAD_OK) return s;
-    if ((s = launch_topn(qb, kb, B, H, n, d, N, idx, lg, stream)) != HAD_OK) return s;
-    return launch_av(idx, lg, V, dt, B, H, n, d, N, tau, out, nullptr, dev_status, stream);
+    if (dt == HAD_BF16)
+        return launch_fused<__nv_bfloat16>(Q, K, V, sigma_q, sigma_k, B, H, n, d, N, tau, out,
+                                           dbg_idx, dbg_logits, base, w, dev_status, stream);
+    return launch_fused<float>(Q, K, V, sigma_q, sigma_k, B, H, n, d, N, tau, out, dbg_idx,
+                               dbg_logits, base, w, dev_status, stream);
 }
 
 size_t had_workspace_bytes(int op, int B, int H, int n, int d, int N)
@@ -234,7 +309,7 @@ int had_launch_count(int op, int B, int H, int n, int d, int N)
     case HAD_OP_SPARSE_SOFTMAX_AV:
         return check_topn(B, H, n, d, N) == HAD_OK ? 1 : -1;
     case HAD_OP_ATTENTION_FWD:
-        return check_topn(B, H, n, d, N) == HAD_OK ? 4 : -1;
+        return check_topn(B, H, n, d, N) == HAD_OK ? 5 : -1;
     default:
         return -1;
     }

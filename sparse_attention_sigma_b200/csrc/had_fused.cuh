@@ -1,0 +1,465 @@
+// had_fused.cuh -- the fused binarized top-N attention forward on the sm_100a
+// tensor cores ("Hamming Attention Distillation", pith.science review, "What
+// carries the argument": sign-quantized Q/K, Hamming logits, top-N mask,
+// softmax over the kept logits, value product; Eqs. 4-7).
+//
+// A CTA owns QT tiles of 128 query rows of one head (TMEM lane i = row i of
+// a tile) and streams the head's keys in tiles of 64, twice:
+//   pass 1  S = Q K^T on the tensor core (+/-16 int8 operands, so the s32
+//           accumulator holds 256*s); each epilogue thread reads its row of
+//           S and counts the logits in a per-row histogram of d+1 levels in
+//           shared memory (one shared-memory reduction per logit, addressed
+//           straight from the accumulator value).  From the histogram: the
+//           threshold level, the number q of keys kept at it, the row
+//           maximum m and the softmax normaliser Z, all exact.
+//   pass 2  S again; the thread turns its row into P = exp(tau (s - m)) for
+//           logits above the threshold and for the first q logits at it
+//           (ascending key index: the lower index wins the tie), 0 elsewhere,
+//           packs P to fp16 pairs in TMEM, and the tensor core accumulates
+//           O += P V (fp16 operands, f32 accumulate) in TMEM.
+// The n x n logits never leave the SM.
+//
+// Warp roles: warp 0 bulk-copies Q once and K (twice) / V (once) tiles into
+// shared-memory rings; warp 1 issues every MMA from one thread; warps
+// 2 .. 2+4*QT-1 are the epilogue, one query row per thread, four warps per
+// query tile.  The QT tiles share every K and V tile.  Every wait is bounded
+// by a deadline: a CTA that hits it flags HAD_ERR_TIMEOUT, lets its copies
+// and MMAs drain, frees its TMEM and returns.
+#pragma once
+#include <cuda_fp16.h>
+
+#include "had_common.cuh"
+#include "had_prep.cuh"
+#include "had_tc.cuh"
+
+namespace had {
+namespace fused {
+
+constexpr int kRows = 128;
+constexpr int kKeys = 64;
+constexpr int kOperandScale = 16;                   // +/-16 int8: accumulator = 256 s
+constexpr uint64_t kWaitNs = 2000000000ull;         // 2 s: far beyond any real wait
+constexpr int kMagic = 0x4B400000;                  // bits of 1.5 * 2^23
+
+template <int D>
+struct Cfg {
+    static constexpr int QT = D == 64 ? 2 : 1;            // query tiles per CTA
+    static constexpr int THREADS = 32 * (2 + 4 * QT);
+    static constexpr int QBYTES = kRows * D;              // int8 Q tile
+    static constexpr int KBYTES = kKeys * D;              // int8 K tile
+    static constexpr int VBYTES = D * kKeys * 2;          // fp16 V^T tile
+    static constexpr int KSTAGES = 4;
+    static constexpr int VSTAGES = D == 64 ? 3 : 2;
+    static constexpr int BINS = D + 1;
+    static constexpr int HIST_BYTES = BINS * kRows * 4;   // per query tile
+    static constexpr uint32_t TMEM_COLS = 512;
+    static constexpr uint32_t GROUP_COLS = 256;           // TMEM columns per query tile
+    static constexpr uint32_t S_COL = 0;                  // + 64 * buffer: s32, 64 keys
+    static constexpr uint32_t P_COL = 128;                // + 32 * buffer: fp16 pairs
+    static constexpr uint32_t O_COL = 192;                // f32, D columns
+    static_assert(QT * GROUP_COLS <= TMEM_COLS || QT == 1, "TMEM budget");
+    static_assert(O_COL + D <= (QT == 1 ? TMEM_COLS : GROUP_COLS), "TMEM budget");
+    // shared memory layout (offsets from a 1024-aligned base)
+    static constexpr int OFF_Q = 0;
+    static constexpr int OFF_K = OFF_Q + QT * QBYTES;
+    static constexpr int OFF_V = OFF_K + KSTAGES * KBYTES;
+    static constexpr int OFF_HIST = OFF_V + VSTAGES * VBYTES;
+    static constexpr int OFF_BAR = OFF_HIST + QT * HIST_BYTES;
+    static constexpr int NBARS = 1 + 2 * KSTAGES + 2 * VSTAGES + QT * 9 + 1;
+    static constexpr int OFF_MISC = OFF_BAR + NBARS * 8;
+    static constexpr int SMEM_BYTES = OFF_MISC + 16 + 1024;   // + alignment slack
+    static constexpr uint32_t IDESC_QK = tc::idesc(2, 1, 1, kRows, kKeys);   // s32 <- s8 x s8
+    static constexpr uint32_t IDESC_PV = tc::idesc(1, 0, 0, kRows, D);       // f32 <- f16 x f16
+};
+
+struct Params {
+    const int8_t *qop;        // [BH][qtiles] 128 x D int8 tiles (+/-16)
+    const int8_t *kop;        // [BH][ktiles] 64 x D int8 tiles (+/-16)
+    const __half *vop;        // [BH][ktiles] D x 64 fp16 tiles (V^T, scaled)
+    const int *vexp;          // [BH] power of two of the V scale
+    float *out;               // [BH][n][D]
+    int32_t *dbg_idx;         // [BH][n][N] or null
+    int16_t *dbg_logits;      // [BH][n][N] or null
+    int32_t *status;
+    int n, N;
+    int qtiles;               // query tiles per head in qop (a multiple of QT)
+    int ktiles;
+    int ctas_per_head;
+    float c2;                 // tau * log2(e)
+};
+
+struct Bars {
+    uint64_t *q_full;
+    uint64_t *k_full, *k_empty;     // [KSTAGES]
+    uint64_t *v_full, *v_empty;     // [VSTAGES]
+    uint64_t *grp;                  // [QT][9]: s_full[2] s_empty[2] p_full[2] p_empty[2] o_full
+    uint64_t *drain;
+    __device__ uint64_t *s_full(int g, int b) const { return grp + g * 9 + b; }
+    __device__ uint64_t *s_empty(int g, int b) const { return grp + g * 9 + 2 + b; }
+    __device__ uint64_t *p_full(int g, int b) const { return grp + g * 9 + 4 + b; }
+    __device__ uint64_t *p_empty(int g, int b) const { return grp + g * 9 + 6 + b; }
+    __device__ uint64_t *o_full(int g) const { return grp + g * 9 + 8; }
+};
+
+// Bounded wait: false if the deadline passed or another role aborted.
+__device__ __forceinline__ bool wait_bar(uint64_t *bar, uint32_t parity, uint64_t deadline,
+                                         volatile int *abort_flag, int32_t *status)
+{
+    uint32_t spins = 0;
+    while (!tc::mbar_try_wait(bar, parity)) {
+        if ((++spins & 255u) == 0) {
+            if (*abort_flag) return false;
+            if (tc::globaltimer_ns() > deadline) {
+                *abort_flag = 1;
+                flag(status, HAD_ERR_TIMEOUT);
+                return false;
+            }
+        }
+    }
+    return true;
+}
+
+__device__ __forceinline__ void red_add1(uint32_t saddr)
+{
+    asm volatile("red.shared.add.u32 [%0], %1;" ::"r"(saddr), "r"(1u) : "memory");
+}
+
+__device__ __forceinline__ float ex2(float x)
+{
+    float y;
+    asm("ex2.approx.ftz.f32 %0, %1;" : "=f"(y) : "f"(x));
+    return y;
+}
+
+// Weight of an accumulator value v = 256 s: exp2(c2 (s - m)) evaluated as
+// exp2(k1 * float(1.5*2^23 + v) + k0); the int -> float step is exact and
+// costs one integer add.  The histogram's Z uses the very same expression.
+__device__ __forceinline__ float weight_of(int v, float k1, float k0)
+{
+    return ex2(fmaf(__int_as_float(v + kMagic), k1, k0));
+}
+
+template <int D, bool kDbg>
+__global__ void __launch_bounds__(Cfg<D>::THREADS, 1)
+attention_fwd_kernel(const Params p)
+{
+    using C = Cfg<D>;
+    constexpr int QT = C::QT;
+    extern __shared__ uint8_t smem_raw[];
+    uint8_t *smem = reinterpret_cast<uint8_t *>(
+        (reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~uintptr_t(1023));
+    uint64_t *bar = reinterpret_cast<uint64_t *>(smem + C::OFF_BAR);
+    Bars b;
+    b.q_full = bar;
+    b.k_full = bar + 1;
+    b.k_empty = b.k_full + C::KSTAGES;
+    b.v_full = b.k_empty + C::KSTAGES;
+    b.v_empty = b.v_full + C::VSTAGES;
+    b.grp = b.v_empty + C::VSTAGES;
+    b.drain = b.grp + QT * 9;
+    uint32_t *tmem_holder = reinterpret_cast<uint32_t *>(smem + C::OFF_MISC);
+    volatile int *abort_flag = reinterpret_cast<volatile int *>(smem + C::OFF_MISC + 4);
+
+    const int warp = threadIdx.x >> 5;
+    const int lane = threadIdx.x & 31;
+    const long long head = blockIdx.x / p.ctas_per_head;
+    const int qtile0 = (blockIdx.x % p.ctas_per_head) * QT;
+    const int T = p.ktiles;
+    const uint64_t deadline = tc::globaltimer_ns() + kWaitNs;
+
+    if (threadIdx.x == 0) {
+        tc::mbar_init(b.q_full, 1);
+        for (int s = 0; s < C::KSTAGES; ++s) {
+            tc::mbar_init(b.k_full + s, 1);
+            tc::mbar_init(b.k_empty + s, 1);
+        }
+        for (int s = 0; s < C::VSTAGES; ++s) {
+            tc::mbar_init(b.v_full + s, 1);
+            tc::mbar_init(b.v_empty + s, 1);
+        }
+        for (int g = 0; g < QT; ++g) {
+            for (int s = 0; s < 2; ++s) {
+                tc::mbar_init(b.s_full(g, s), 1);
+                tc::mbar_init(b.s_empty(g, s), kRows);
+                tc::mbar_init(b.p_full(g, s), kRows);
+                tc::mbar_init(b.p_empty(g, s), 1);
+            }
+            tc::mbar_init(b.o_full(g), 1);
+        }
+        tc::mbar_init(b.drain, 1);
+        *abort_flag = 0;
+        tc::fence_mbar_init();
+    }
+    if (warp == 0) tc::tmem_alloc(tmem_holder, C::TMEM_COLS);
+    tc::fence_before_sync();
+    __syncthreads();
+    tc::fence_after_sync();
+    const uint32_t tmem = *tmem_holder;
+
+    if (warp == 0) {
+        // ------------------------------------------------------------ producer
+        if (lane == 0) {
+            const int8_t *qsrc = p.qop + (head * p.qtiles + qtile0) * (long long)C::QBYTES;
+            const int8_t *ksrc = p.kop + head * (long long)T * C::KBYTES;
+            const uint8_t *vsrc = reinterpret_cast<const uint8_t *>(p.vop) +
+                                  head * (long long)T * C::VBYTES;
+            tc::mbar_expect_tx(b.q_full, QT * C::QBYTES);
+            tc::bulk_g2s(smem + C::OFF_Q, qsrc, QT * C::QBYTES, b.q_full);
+            int issued_k = 0, issued_v = 0;
+            bool ok = true;
+            for (int u = 0; u < 2 * T && ok; ++u) {
+                const int j = u < T ? u : u - T;
+                const int ks = u % C::KSTAGES;
+                ok = wait_bar(b.k_empty + ks, ((u / C::KSTAGES) & 1) ^ 1, deadline, abort_flag,
+                              p.status);
+                if (!ok) break;
+                tc::mbar_expect_tx(b.k_full + ks, C::KBYTES);
+                tc::bulk_g2s(smem + C::OFF_K + ks * C::KBYTES, ksrc + (long long)j * C::KBYTES,
+                             C::KBYTES, b.k_full + ks);
+                issued_k = u + 1;
+                if (u >= T) {
+                    const int vs = j % C::VSTAGES;
+                    ok = wait_bar(b.v_empty + vs, ((j / C::VSTAGES) & 1) ^ 1, deadline,
+                                  abort_flag, p.status);
+                    if (!ok) break;
+                    tc::mbar_expect_tx(b.v_full + vs, C::VBYTES);
+                    tc::bulk_g2s(smem + C::OFF_V + vs * C::VBYTES,
+                                 vsrc + (long long)j * C::VBYTES, C::VBYTES, b.v_full + vs);
+                    issued_v = j + 1;
+                }
+            }
+            if (!ok) {
+                // let every copy already in flight land before the CTA exits
+                const uint64_t drain_deadline = tc::globaltimer_ns() + kWaitNs / 4;
+                volatile int never = 0;
+                wait_bar(b.q_full, 0, drain_deadline, &never, p.status);
+                for (int u = (issued_k > C::KSTAGES ? issued_k - C::KSTAGES : 0); u < issued_k; ++u)
+                    wait_bar(b.k_full + u % C::KSTAGES, (u / C::KSTAGES) & 1, drain_deadline,
+                             &never, p.status);
+                for (int j = (issued_v > C::VSTAGES ? issued_v - C::VSTAGES : 0); j < issued_v; ++j)
+                    wait_bar(b.v_full + j % C::VSTAGES, (j / C::VSTAGES) & 1, drain_deadline,
+                             &never, p.status);
+            }
+        }
+    } else if (warp == 1) {
+        // ------------------------------------------------------------ MMA issuer
+        if (lane == 0) {
+            const uint32_t q_addr = tc::smem_u32(smem + C::OFF_Q);
+            const uint32_t k_addr = tc::smem_u32(smem + C::OFF_K);
+            const uint32_t v_addr = tc::smem_u32(smem + C::OFF_V);
+            bool ok = wait_bar(b.q_full, 0, deadline, abort_flag, p.status);
+            tc::fence_after_sync();
+            auto pv = [&](int j) -> bool {
+                const int vs = j % C::VSTAGES;
+                if (!wait_bar(b.v_full + vs, (j / C::VSTAGES) & 1, deadline, abort_flag, p.status))
+                    return false;
+                const int pb = j & 1;
+                for (int g = 0; g < QT; ++g) {
+                    if (!wait_bar(b.p_full(g, pb), (j >> 1) & 1, deadline, abort_flag, p.status))
+                        return false;
+                    tc::fence_after_sync();
+                    const uint32_t gcol = g * C::GROUP_COLS;
+#pragma unroll
+                    for (int kk = 0; kk < kKeys / 16; ++kk) {
+                        const uint64_t bdesc =
+                            tc::smem_desc(v_addr + vs * C::VBYTES + kk * 256, 128, 8 * 128);
+                        tc::mma_f16_ts(tmem + gcol + C::O_COL,
+                                       tmem + gcol + C::P_COL + pb * 32 + kk * 8, bdesc,
+                                       C::IDESC_PV, (j > 0 || kk > 0) ? 1u : 0u);
+                    }
+                    tc::mma_commit(b.p_empty(g, pb));
+                }
+                tc::mma_commit(b.v_empty + vs);
+                return true;
+            };
+            for (int u = 0; u < 2 * T && ok; ++u) {
+                const int ks = u % C::KSTAGES;
+                ok = wait_bar(b.k_full + ks, (u / C::KSTAGES) & 1, deadline, abort_flag, p.status);
+                if (!ok) break;
+                const int sb = u & 1;
+                for (int g = 0; g < QT && ok; ++g) {
+                    ok = wait_bar(b.s_empty(g, sb), ((u >> 1) & 1) ^ 1, deadline, abort_flag,
+                                  p.status);
+                    if (!ok) break;
+                    tc::fence_after_sync();
+                    const uint32_t scol = g * C::GROUP_COLS + C::S_COL + sb * 64;
+#pragma unroll
+                    for (int kk = 0; kk < D / 32; ++kk) {
+                        const uint64_t adesc =
+                            tc::smem_desc(q_addr + g * C::QBYTES + kk * 256, 128, D * 8);
+                        const uint64_t bdesc =
+                            tc::smem_desc(k_addr + ks * C::KBYTES + kk * 256, 128, D * 8);
+                        tc::mma_i8_ss(tmem + scol, adesc, bdesc, C::IDESC_QK, kk > 0 ? 1u : 0u);
+                    }
+                    tc::mma_commit(b.s_full(g, sb));
+                }
+                if (!ok) break;
+                tc::mma_commit(b.k_empty + ks);
+                if (u >= T + 1) ok = pv(u - T - 1);
+            }
+            if (ok) ok = pv(T - 1);
+            if (ok)
+                for (int g = 0; g < QT; ++g) tc::mma_commit(b.o_full(g));
+            // drain: wait until every MMA this thread issued has completed
+            tc::mma_commit(b.drain);
+            volatile int never = 0;
+            wait_bar(b.drain, 0, tc::globaltimer_ns() + kWaitNs / 4, &never, p.status);
+        }
+    } else {
+        // ------------------------------------------------------------ epilogue
+        const int g = (warp - 2) >> 2;                // query tile of this warp
+        const int quarter = warp & 3;                 // TMEM lanes 32*quarter ...
+        const int r = quarter * 32 + lane;            // row within the tile
+        const int row = (qtile0 + g) * kRows + r;     // query index within the head
+        const bool active = row < p.n;
+        const uint32_t lane_base = tmem + ((uint32_t)(quarter * 32) << 16) + g * C::GROUP_COLS;
+        uint32_t *hist = reinterpret_cast<uint32_t *>(smem + C::OFF_HIST + g * C::HIST_BYTES);
+        uint32_t *hcol = hist + r;                    // hist[bin][r] at hcol[bin * kRows]
+        for (int bin = 0; bin < C::BINS; ++bin) hcol[bin * kRows] = 0;
+        // bin of accumulator value v = 256 s is (D - s)/2, at byte offset
+        // bin * 512 = 256 D - v from this row's bin 0
+        const uint32_t hbase = tc::smem_u32(hcol) + 256u * D;
+        bool ok = true;
+
+        // pass 1: histogram of the logits of this row
+        for (int j = 0; j < T && ok; ++j) {
+            const int sb = j & 1;
+            ok = __all_sync(kFullMask, wait_bar(b.s_full(g, sb), (j >> 1) & 1, deadline,
+                                                abort_flag, p.status));
+            if (!ok) break;
+            tc::fence_after_sync();
+            uint32_t s0[32], s1[32];
+            const uint32_t scol = C::S_COL + sb * 64;
+            tc::tmem_ld32(lane_base + scol, s0);
+            tc::tmem_ld32(lane_base + scol + 32, s1);
+            tc::tmem_wait_ld();
+            tc::fence_before_sync();
+            tc::mbar_arrive(b.s_empty(g, sb));
+            const int valid = min(kKeys, p.n - j * kKeys);
+            if (valid == kKeys) {
+#pragma unroll
+                for (int c = 0; c < 32; ++c) red_add1(hbase - s0[c]);
+#pragma unroll
+                for (int c = 0; c < 32; ++c) red_add1(hbase - s1[c]);
+            } else {
+#pragma unroll
+                for (int c = 0; c < 32; ++c)
+                    if (c < valid) red_add1(hbase - s0[c]);
+#pragma unroll
+                for (int c = 0; c < 32; ++c)
+                    if (32 + c < valid) red_add1(hbase - s1[c]);
+            }
+        }
+
+        // threshold level t (as a Hamming distance), quota q, max, Z
+        int t = C::BINS - 1, hmin = C::BINS - 1;
+        int quota = 0;
+        {
+            int below = 0;
+            bool found = false, seen = false;
+            for (int bin = 0; bin < C::BINS; ++bin) {
+                const int c = (int)hcol[bin * kRows];
+                if (!seen && c) { hmin = bin; seen = true; }
+                if (!found) {
+                    if (below + c >= p.N) { t = bin; quota = p.N - below; found = true; }
+                    else below += c;
+                }
+            }
+        }
+        const int vt = 256 * (D - 2 * t);             // accumulator value of the threshold
+        const int vm = 256 * (D - 2 * hmin);          // ... of the row maximum
+        const float k1 = p.c2 * (1.0f / 256.0f);
+        const float k0 = -fmaf((float)vm, k1, 0.0f) - 12582912.0f * k1;
+        float Z = 0.0f;
+        for (int bin = hmin; bin < t; ++bin)
+            Z += (float)hcol[bin * kRows] * weight_of(256 * (D - 2 * bin), k1, k0);
+        Z += (float)quota * weight_of(vt, k1, k0);
+        int rem = quota;                              // ties still to keep
+        int kept = 0;
+        const long long obase = ((head * p.n) + row) * (long long)p.N;
+
+        // pass 2: P = kept weights (fp16) -> TMEM; the MMA warp does O += P V
+        for (int j = 0; j < T && ok; ++j) {
+            const int u = T + j;
+            const int sb = u & 1;
+            ok = __all_sync(kFullMask, wait_bar(b.s_full(g, sb), (u >> 1) & 1, deadline,
+                                                abort_flag, p.status));
+            if (!ok) break;
+            tc::fence_after_sync();
+            uint32_t s[64];
+            const uint32_t scol = C::S_COL + sb * 64;
+            tc::tmem_ld32(lane_base + scol, *reinterpret_cast<uint32_t(*)[32]>(s));
+            tc::tmem_ld32(lane_base + scol + 32, *reinterpret_cast<uint32_t(*)[32]>(s + 32));
+            tc::tmem_wait_ld();
+            tc::fence_before_sync();
+            tc::mbar_arrive(b.s_empty(g, sb));
+            const int pb = j & 1;
+            ok = __all_sync(kFullMask, wait_bar(b.p_empty(g, pb), ((j >> 1) & 1) ^ 1, deadline,
+                                                abort_flag, p.status));
+            if (!ok) break;
+            const int valid = min(kKeys, p.n - j * kKeys);
+            uint32_t packed[32];
+#pragma unroll
+            for (int c = 0; c < 64; c += 2) {
+                float w2[2];
+#pragma unroll
+                for (int e = 0; e < 2; ++e) {
+                    const int v = (int)s[c + e];
+                    const bool in = (c + e) < valid;
+                    const bool tie = in && (v == vt);
+                    const bool keep = in && ((v > vt) || (tie && rem > 0));
+                    rem -= tie ? 1 : 0;
+                    const float w = weight_of(v, k1, k0);
+                    w2[e] = keep ? w : 0.0f;
+                    if (kDbg) {
+                        if (keep && active) {
+                            if (p.dbg_idx) p.dbg_idx[obase + kept] = j * kKeys + c + e;
+                            if (p.dbg_logits) p.dbg_logits[obase + kept] = (int16_t)(v / 256);
+                            ++kept;
+                        }
+                    }
+                }
+                __half2 h = __floats2half2_rn(w2[0], w2[1]);
+                packed[c >> 1] = *reinterpret_cast<uint32_t *>(&h);
+            }
+            tc::tmem_st32(lane_base + C::P_COL + pb * 32, packed);
+            tc::tmem_wait_st();
+            tc::fence_before_sync();
+            tc::mbar_arrive(b.p_full(g, pb));
+        }
+
+        // output: O / Z * 2^e_h
+        if (ok) ok = __all_sync(kFullMask, wait_bar(b.o_full(g), 0, deadline, abort_flag, p.status));
+        if (ok) {
+            tc::fence_after_sync();
+            const float scale = ldexpf(1.0f, p.vexp[head]) / Z;
+            float *orow = p.out + ((head * p.n) + row) * (long long)D;
+#pragma unroll
+            for (int c0 = 0; c0 < D; c0 += 32) {
+                uint32_t o[32];
+                tc::tmem_ld32(lane_base + C::O_COL + c0, o);
+                tc::tmem_wait_ld();
+                if (active) {
+#pragma unroll
+                    for (int c = 0; c < 32; c += 4) {
+                        float4 v = make_float4(__uint_as_float(o[c]) * scale,
+                                               __uint_as_float(o[c + 1]) * scale,
+                                               __uint_as_float(o[c + 2]) * scale,
+                                               __uint_as_float(o[c + 3]) * scale);
+                        *reinterpret_cast<float4 *>(orow + c0 + c) = v;
+                    }
+                }
+            }
+        }
+    }
+
+    tc::fence_before_sync();
+    __syncthreads();
+    if (warp == 0) {
+        tc::fence_after_sync();
+        tc::tmem_dealloc(tmem, C::TMEM_COLS);
+    }
+}
+
+}  // namespace fused
+}  // namespace had

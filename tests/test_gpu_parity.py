@@ -191,7 +191,8 @@ def test_golden_handworked(had):
         want = np.zeros(case["d"])
         for col, ex in exp[key]["out_nonzero"].items():
             want[int(col)] = _golden.closed_form(ex)
-        assert np.allclose(out[0, 0, r].cpu().numpy(), want, rtol=1e-5, atol=1e-6)
+        # P enters the value product as fp16: within the output tolerance
+        assert_close(out[0, 0, r].cpu().numpy(), want, f"golden {key}")
 
 
 def test_sign_edge_values_on_device(had):
