@@ -173,6 +173,12 @@ def max_over_ranks(value, world, device):
     return float(t.item())
 
 
+def aggregate(tokens_per_rank, ms_local, world, device):
+    """Whole-job throughput: every rank's tokens over the slowest rank's time."""
+    ms = max_over_ranks(ms_local, world, device)
+    return tokens_per_rank * world / (ms * 1e-3), ms
+
+
 def barrier(world):
     if world > 1:
         import torch.distributed as dist
@@ -284,11 +290,8 @@ def run_had(args, world, rank, local):
     torch.cuda.synchronize()
     barrier(world)
     clock_info = clocks.stop()
-    ms = sum(s.elapsed_time(e) for s, e in zip(starts, ends)) / args.steps
-    ms = max_over_ranks(ms, world, dev)
-
-    tokens_per_rank = cfg.tokens
-    value = tokens_per_rank * world / (ms * 1e-3)
+    ms_local = sum(s.elapsed_time(e) for s, e in zip(starts, ends)) / args.steps
+    value, ms = aggregate(cfg.tokens, ms_local, world, dev)
 
     # per-kernel view: the same work through the unfused entry points, so
     # each kernel of the step can be bracketed by its own events
