@@ -137,6 +137,40 @@ HAD_API had_status_t had_attention_fwd(const void *Q, const void *K, const void 
                                int32_t *dev_status, cudaStream_t stream);
 
 /*
+ * had_attention_fwd for callers that cannot allocate device memory.
+ *
+ * The paper has no counterpart to this entry point; it exists for callers
+ * that cannot call cudaMalloc (code running under another runtime's
+ * allocator, plugins handed only their input and output buffers, processes
+ * whose device memory is reserved up front).  It computes exactly what
+ * had_attention_fwd computes, with the same kernels, but takes its
+ * workspace from a fixed device array inside the library instead of a
+ * caller buffer, and allocates nothing.
+ *   - Limit: had_workspace_bytes(HAD_OP_ATTENTION_FWD, ...) must not exceed
+ *     had_noalloc_scratch_bytes() (80 MiB, enough for B=4 H=16 n=4096
+ *     d=64); larger sizes return HAD_ERR_WORKSPACE before any launch.
+ *   - The array is part of the loaded module: every GPU that loads the
+ *     library holds it until the process exits.
+ *   - The first call on each device looks up the array's device address
+ *     (cudaGetSymbolAddress, with that device current) and caches it; make
+ *     that first call before any stream capture.
+ *   - Every call shares the one array per device and leaves its contents
+ *     behind; the call re-initialises everything it reads.  Calls whose
+ *     kernels overlap on the GPU (different streams, or host threads
+ *     without ordering) race on the array and give undefined results.
+ * Arguments are those of had_attention_fwd without the debug outputs and
+ * the workspace.
+ */
+HAD_API had_status_t had_attention_fwd_noalloc(const void *Q, const void *K, const void *V,
+                                               had_dtype_t dt, const float *sigma_q,
+                                               const float *sigma_k, int B, int H, int n,
+                                               int d, int N, float tau, float *out,
+                                               int32_t *dev_status, cudaStream_t stream);
+
+/* Size in bytes of the fixed array had_attention_fwd_noalloc works in. */
+HAD_API size_t had_noalloc_scratch_bytes(void);
+
+/*
  * Workspace bytes an operation needs for these sizes (0 if none), or
  * (size_t)-1 for unsupported or invalid sizes.
  */

@@ -3,6 +3,7 @@
 // kernels included below; this file only validates and enqueues.
 #include <climits>
 #include <cstdint>
+#include <mutex>
 #include <cuda_runtime.h>
 
 #include "had.h"
@@ -212,6 +213,37 @@ had_status_t launch_fused(const void *Q, const void *K, const void *V, const flo
                                                 dbg_lg, ws, w, status, st);
 }
 
+// Fixed scratch of had_attention_fwd_noalloc.  Some callers cannot call
+// cudaMalloc at all (code running inside another runtime's allocator, a
+// plugin that is handed only input and output buffers, or a process whose
+// device memory is fully reserved up front), so this entry point takes its
+// workspace from a statically sized device array instead.  The array is part
+// of the module: every GPU that loads the library holds it until the process
+// exits.
+constexpr size_t kNoAllocScratchBytes = size_t(80) << 20;   // 80 MiB
+static __device__ __align__(256) unsigned char g_noalloc_scratch[kNoAllocScratchBytes];
+
+// In host code `g_noalloc_scratch` is only a stand-in symbol, never a device
+// address; the real address is looked up once per device, with that device
+// current, and cached here.
+constexpr int kMaxDevices = 64;
+void *g_noalloc_ptr[kMaxDevices] = {};
+std::mutex g_noalloc_mutex;
+
+had_status_t noalloc_scratch(void **ptr)
+{
+    int dev = 0;
+    if (cudaGetDevice(&dev) != cudaSuccess || dev < 0 || dev >= kMaxDevices) return HAD_ERR_CUDA;
+    std::lock_guard<std::mutex> lock(g_noalloc_mutex);
+    if (!g_noalloc_ptr[dev]) {
+        void *p = nullptr;
+        if (cudaGetSymbolAddress(&p, g_noalloc_scratch) != cudaSuccess || !p) return HAD_ERR_CUDA;
+        g_noalloc_ptr[dev] = p;
+    }
+    *ptr = g_noalloc_ptr[dev];
+    return HAD_OK;
+}
+
 }  // namespace
 
 extern "C" {
@@ -283,6 +315,34 @@ had_status_t had_attention_fwd(const void *Q, const void *K, const void *V, had_
     return launch_fused<float>(Q, K, V, sigma_q, sigma_k, B, H, n, d, N, tau, out, dbg_idx,
                                dbg_logits, base, w, dev_status, stream);
 }
+
+had_status_t had_attention_fwd_noalloc(const void *Q, const void *K, const void *V,
+                                       had_dtype_t dt, const float *sigma_q,
+                                       const float *sigma_k, int B, int H, int n, int d, int N,
+                                       float tau, float *out, int32_t *dev_status,
+                                       cudaStream_t stream)
+{
+    had_status_t s = check_topn(B, H, n, d, N);
+    if (s != HAD_OK) return s;
+    if (dt != HAD_BF16 && dt != HAD_F32) return HAD_ERR_INVALID_ARG;
+    if (!Q || !K || !V || !sigma_q || !sigma_k || !out) return HAD_ERR_INVALID_ARG;
+    if (!aligned16(Q) || !aligned16(K) || !aligned16(V) || !aligned16(out))
+        return HAD_ERR_INVALID_ARG;
+    if (!(tau == tau) || tau > 3.0e38f || tau < -3.0e38f) return HAD_ERR_INVALID_ARG;
+    const FwdWorkspace w = fwd_layout(B, H, n, d, N);
+    if (w.total > kNoAllocScratchBytes) return HAD_ERR_WORKSPACE;
+    if ((long long)B * H * w.qtiles > INT_MAX) return HAD_ERR_UNSUPPORTED;
+    void *scratch = nullptr;
+    if ((s = noalloc_scratch(&scratch)) != HAD_OK) return s;
+    char *base = static_cast<char *>(scratch);
+    if (dt == HAD_BF16)
+        return launch_fused<__nv_bfloat16>(Q, K, V, sigma_q, sigma_k, B, H, n, d, N, tau, out,
+                                           nullptr, nullptr, base, w, dev_status, stream);
+    return launch_fused<float>(Q, K, V, sigma_q, sigma_k, B, H, n, d, N, tau, out, nullptr,
+                               nullptr, base, w, dev_status, stream);
+}
+
+size_t had_noalloc_scratch_bytes(void) { return kNoAllocScratchBytes; }
 
 size_t had_workspace_bytes(int op, int B, int H, int n, int d, int N)
 {

@@ -52,6 +52,8 @@ def _load():
         "had_sparse_softmax_av": [vp, vp, vp, i32, i32, i32, i32, i32, i32, f32, vp, vp, vp, vp],
         "had_attention_fwd": [vp, vp, vp, i32, vp, vp, i32, i32, i32, i32, i32, f32, vp, vp, vp,
                               vp, sz, vp, vp],
+        "had_attention_fwd_noalloc": [vp, vp, vp, i32, vp, vp, i32, i32, i32, i32, i32, f32, vp,
+                                      vp, vp],
     }
     for name, args in sig.items():
         fn = getattr(lib, name)
@@ -61,6 +63,8 @@ def _load():
     lib.had_workspace_bytes.restype = ctypes.c_size_t
     lib.had_launch_count.argtypes = [i32] * 6
     lib.had_launch_count.restype = ctypes.c_int
+    lib.had_noalloc_scratch_bytes.argtypes = []
+    lib.had_noalloc_scratch_bytes.restype = ctypes.c_size_t
     lib.had_status_string.argtypes = [ctypes.c_int]
     lib.had_status_string.restype = ctypes.c_char_p
     return lib
@@ -216,6 +220,34 @@ def had_attention_fwd(Q, K, V, sigma_q, sigma_k, N, tau, out=None, dbg_idx=None,
                                 _ptr(dev_status), _stream(stream))
     _check(st, "had_attention_fwd")
     return out
+
+
+def had_attention_fwd_noalloc(Q, K, V, sigma_q, sigma_k, N, tau, out, dev_status=None,
+                              stream=None):
+    """had_attention_fwd for callers that cannot allocate device memory.
+
+    The library works in a fixed device array of had_noalloc_scratch_bytes()
+    bytes instead of a workspace, so nothing is allocated here either: the
+    caller passes every tensor, `out` included.  Sizes whose workspace
+    exceeds the array raise HadError(HAD_ERR_WORKSPACE).  Calls that overlap
+    on the GPU share the array and race.
+    """
+    _dev(Q, "Q")
+    B, H, n, d = _shape4(Q, "Q")
+    _dev(K, "K", Q.dtype, (B, H, n, d))
+    _dev(V, "V", Q.dtype, (B, H, n, d))
+    _dev(sigma_q, "sigma_q", torch.float32, (H,))
+    _dev(sigma_k, "sigma_k", torch.float32, (H,))
+    _dev(out, "out", torch.float32, (B, H, n, d))
+    st = _lib.had_attention_fwd_noalloc(_ptr(Q), _ptr(K), _ptr(V), _dtype_code(Q), _ptr(sigma_q),
+                                        _ptr(sigma_k), B, H, n, d, N, ctypes.c_float(tau),
+                                        _ptr(out), _ptr(dev_status), _stream(stream))
+    _check(st, "had_attention_fwd_noalloc")
+    return out
+
+
+def had_noalloc_scratch_bytes() -> int:
+    return int(_lib.had_noalloc_scratch_bytes())
 
 
 def workspace(B, H, n, d, N, device="cuda"):
