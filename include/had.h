@@ -125,6 +125,7 @@ HAD_API had_status_t had_sparse_softmax_av(const int32_t *idx, const int16_t *lo
  *   out       [B,H,n,d] float out
  *   dbg_idx, dbg_logits  [B,H,n,N] optional outputs of the kept set (may be
  *             NULL; when given they hold exactly what had_hamming_topn would)
+ *   tau       softmax temperature, finite and >= 0 (else HAD_ERR_INVALID_ARG)
  *   ws        workspace of had_workspace_bytes(HAD_OP_ATTENTION_FWD, ...)
  * The n x n logit matrix never goes to memory.
  */

@@ -124,7 +124,7 @@ had_status_t launch_av(const int32_t *idx, const int16_t *lg, const void *V, had
 // Workspace of the fused forward: tensor-core operand tiles of Q, K and V^T
 // and the per-head V scale.
 struct FwdWorkspace {
-    size_t qop, kop, vop, vmax, vexp, total;
+    size_t qop, kop, vop, qbits, kbits, vmax, vexp, miss_rows, total;
     int qtiles, ktiles;
 };
 
@@ -140,9 +140,12 @@ FwdWorkspace fwd_layout(int B, int H, int n, int d, int N)
     w.qop = 0;
     w.kop = w.qop + round_up(bh * w.qtiles * had::fused::kRows * d);
     w.vop = w.kop + round_up(bh * w.ktiles * had::fused::kKeys * d);
-    w.vmax = w.vop + round_up(bh * w.ktiles * had::fused::kKeys * d * 2);
-    w.vexp = w.vmax + round_up(bh * 4);
-    w.total = w.vexp + round_up(bh * 4);
+    w.qbits = w.vop + round_up(bh * w.ktiles * had::fused::kKeys * d * 2);
+    w.kbits = w.qbits + round_up(bh * n * (d / 8));
+    w.vmax = w.kbits + round_up(bh * n * (d / 8));
+    w.vexp = w.vmax + round_up((bh + 1) * 4);         // vmax[BH] then the miss counter
+    w.miss_rows = w.vexp + round_up(bh * 4);
+    w.total = w.miss_rows + round_up(bh * (size_t)w.qtiles * had::fused::kRows * 4);
     return w;
 }
 
@@ -157,18 +160,27 @@ had_status_t launch_fused_typed(const T *Q, const T *K, const T *V, const float 
     auto *qop = reinterpret_cast<int8_t *>(ws + w.qop);
     auto *kop = reinterpret_cast<int8_t *>(ws + w.kop);
     auto *vop = reinterpret_cast<__half *>(ws + w.vop);
+    auto *qbits = reinterpret_cast<uint32_t *>(ws + w.qbits);
+    auto *kbits = reinterpret_cast<uint32_t *>(ws + w.kbits);
     auto *vmax = reinterpret_cast<unsigned int *>(ws + w.vmax);
+    auto *miss_count = reinterpret_cast<int *>(ws + w.vmax) + bh;
     auto *vexp = reinterpret_cast<int *>(ws + w.vexp);
-    if (cudaMemsetAsync(vmax, 0, bh * 4, st) != cudaSuccess) return HAD_ERR_CUDA;
+    auto *miss_rows = reinterpret_cast<int *>(ws + w.miss_rows);
+    if (cudaMemsetAsync(vmax, 0, (bh + 1) * 4, st) != cudaSuccess) return HAD_ERR_CUDA;
     const long long qchunks = bh * w.qtiles * had::fused::kRows * (D / 16);
     const long long kchunks = bh * w.ktiles * had::fused::kKeys * (D / 16);
+    // Q as +/-4 and K as +/-1: the i8 MMA accumulates 4 s
     had::prep::sign_operand_kernel<T><<<grid_for(qchunks, 256), 256, 0, st>>>(
-        Q, sq, H, n, D, had::fused::kRows, w.qtiles, qchunks, qop, status);
+        Q, sq, H, n, D, had::fused::kRows, w.qtiles, qchunks, 0x04u, 0xFCu, qop,
+        reinterpret_cast<uint16_t *>(qbits), status);
     had::prep::sign_operand_kernel<T><<<grid_for(kchunks, 256), 256, 0, st>>>(
-        K, sk, H, n, D, had::fused::kKeys, w.ktiles, kchunks, kop, status);
-    const long long vgroups = bh * n * D / 8;
-    had::prep::vmax_kernel<T><<<grid_for(vgroups, 256), 256, 0, st>>>(
-        V, (long long)n * D / 8, vgroups, vmax);
+        K, sk, H, n, D, had::fused::kKeys, w.ktiles, kchunks, 0x01u, 0xFFu, kop,
+        reinterpret_cast<uint16_t *>(kbits), status);
+    const long long vgroups_per_head = (long long)n * D / 8;
+    const int chunks = (int)((vgroups_per_head + 4095) / 4096);   // 32 KiB of bf16 per CTA
+    if (bh * chunks > INT_MAX) return HAD_ERR_UNSUPPORTED;
+    had::prep::vmax_kernel<T><<<(unsigned)(bh * chunks), 256, 0, st>>>(V, vgroups_per_head,
+                                                                      chunks, vmax);
     had::prep::v_operand_kernel<T, D><<<(unsigned)(bh * w.ktiles), 256, 0, st>>>(
         V, n, vmax, vop, vexp);
     had_status_t s = launched();
@@ -188,6 +200,9 @@ had_status_t launch_fused_typed(const T *Q, const T *K, const T *V, const float 
     p.dbg_idx = dbg_idx;
     p.dbg_logits = dbg_lg;
     p.status = status;
+    p.miss_count = miss_count;
+    p.miss_rows = miss_rows;
+    p.sample_tiles = w.ktiles / 16 > 4 ? w.ktiles / 16 : 4;
     p.n = n;
     p.N = N;
     p.qtiles = w.qtiles;
@@ -196,6 +211,8 @@ had_status_t launch_fused_typed(const T *Q, const T *K, const T *V, const float 
     p.c2 = tau * 1.4426950408889634f;
     const long long blocks = bh * p.ctas_per_head;
     kernel<<<(unsigned)blocks, C::THREADS, C::SMEM_BYTES, st>>>(p);
+    had::fused::fixup_rows_kernel<T, D><<<148 * 2, 256, 0, st>>>(
+        qbits, kbits, V, n, N, tau, miss_count, miss_rows, out, dbg_idx, dbg_lg);
     return launched();
 }
 
@@ -304,7 +321,7 @@ had_status_t had_attention_fwd(const void *Q, const void *K, const void *V, had_
     if (!aligned16(Q) || !aligned16(K) || !aligned16(V) || !aligned16(out) ||
         (dbg_idx && !aligned16(dbg_idx)) || (dbg_logits && !aligned16(dbg_logits)))
         return HAD_ERR_INVALID_ARG;
-    if (!(tau == tau) || tau > 3.0e38f || tau < -3.0e38f) return HAD_ERR_INVALID_ARG;
+    if (!(tau >= 0.0f) || tau > 3.0e38f) return HAD_ERR_INVALID_ARG;
     const FwdWorkspace w = fwd_layout(B, H, n, d, N);
     if (!ws || ws_bytes < w.total || !aligned16(ws)) return HAD_ERR_WORKSPACE;
     if ((long long)B * H * w.qtiles > INT_MAX) return HAD_ERR_UNSUPPORTED;
@@ -328,7 +345,7 @@ had_status_t had_attention_fwd_noalloc(const void *Q, const void *K, const void 
     if (!Q || !K || !V || !sigma_q || !sigma_k || !out) return HAD_ERR_INVALID_ARG;
     if (!aligned16(Q) || !aligned16(K) || !aligned16(V) || !aligned16(out))
         return HAD_ERR_INVALID_ARG;
-    if (!(tau == tau) || tau > 3.0e38f || tau < -3.0e38f) return HAD_ERR_INVALID_ARG;
+    if (!(tau >= 0.0f) || tau > 3.0e38f) return HAD_ERR_INVALID_ARG;
     const FwdWorkspace w = fwd_layout(B, H, n, d, N);
     if (w.total > kNoAllocScratchBytes) return HAD_ERR_WORKSPACE;
     if ((long long)B * H * w.qtiles > INT_MAX) return HAD_ERR_UNSUPPORTED;
@@ -369,7 +386,7 @@ int had_launch_count(int op, int B, int H, int n, int d, int N)
     case HAD_OP_SPARSE_SOFTMAX_AV:
         return check_topn(B, H, n, d, N) == HAD_OK ? 1 : -1;
     case HAD_OP_ATTENTION_FWD:
-        return check_topn(B, H, n, d, N) == HAD_OK ? 5 : -1;
+        return check_topn(B, H, n, d, N) == HAD_OK ? 6 : -1;
     default:
         return -1;
     }

@@ -5,18 +5,21 @@
 //
 // A CTA owns QT tiles of 128 query rows of one head (TMEM lane i = row i of
 // a tile) and streams the head's keys in tiles of 64, twice:
-//   pass 1  S = Q K^T on the tensor core (+/-16 int8 operands, so the s32
-//           accumulator holds 256*s); each epilogue thread reads its row of
-//           S and counts the logits in a per-row histogram of d+1 levels in
-//           shared memory (one shared-memory reduction per logit, addressed
-//           straight from the accumulator value).  From the histogram: the
-//           threshold level, the number q of keys kept at it, the row
-//           maximum m and the softmax normaliser Z, all exact.
-//   pass 2  S again; the thread turns its row into P = exp(tau (s - m)) for
-//           logits above the threshold and for the first q logits at it
+//   pass 1  S = Q K^T on the tensor core (+/-4 x +/-1 int8 operands, so the
+//           s32 accumulator holds 4 s); each epilogue thread reads its row.
+//           The first key tiles are counted exactly into a per-row histogram
+//           of the d+1 logit levels (shared memory); it places a window of
+//           three levels around the row's threshold, and the remaining tiles
+//           only update four 8-bit cumulative counters packed in one
+//           register (one shifted add per logit).  That yields the exact
+//           threshold level t and the number q of keys kept at it whenever t
+//           falls inside the window; rows where it does not are listed and
+//           recomputed exactly by fixup_rows_kernel.
+//   pass 2  S again; the thread turns its row into P = exp(tau (s - ref))
+//           for logits above the threshold and for the first q logits at it
 //           (ascending key index: the lower index wins the tie), 0 elsewhere,
-//           packs P to fp16 pairs in TMEM, and the tensor core accumulates
-//           O += P V (fp16 operands, f32 accumulate) in TMEM.
+//           sums them into Z, packs P to fp16 pairs in TMEM, and the tensor
+//           core accumulates O += P V (fp16 operands, f32 accumulate).
 // The n x n logits never leave the SM.
 //
 // Warp roles: warp 0 bulk-copies Q once and K (twice) / V (once) tiles into
@@ -27,8 +30,10 @@
 // and MMAs drain, frees its TMEM and returns.
 #pragma once
 #include <cuda_fp16.h>
+#include <type_traits>
 
 #include "had_common.cuh"
+#include "had_av.cuh"
 #include "had_prep.cuh"
 #include "had_tc.cuh"
 
@@ -37,7 +42,6 @@ namespace fused {
 
 constexpr int kRows = 128;
 constexpr int kKeys = 64;
-constexpr int kOperandScale = 16;                   // +/-16 int8: accumulator = 256 s
 constexpr uint64_t kWaitNs = 2000000000ull;         // 2 s: far beyond any real wait
 constexpr int kMagic = 0x4B400000;                  // bits of 1.5 * 2^23
 
@@ -49,7 +53,7 @@ struct Cfg {
     static constexpr int KBYTES = kKeys * D;              // int8 K tile
     static constexpr int VBYTES = D * kKeys * 2;          // fp16 V^T tile
     static constexpr int KSTAGES = 4;
-    static constexpr int VSTAGES = D == 64 ? 3 : 2;
+    static constexpr int VSTAGES = 3;
     static constexpr int BINS = D + 1;
     static constexpr int HIST_BYTES = BINS * kRows * 4;   // per query tile
     static constexpr uint32_t TMEM_COLS = 512;
@@ -81,6 +85,9 @@ struct Params {
     int32_t *dbg_idx;         // [BH][n][N] or null
     int16_t *dbg_logits;      // [BH][n][N] or null
     int32_t *status;
+    int *miss_count;          // rows whose threshold fell outside the window
+    int *miss_rows;           // their flat row ids (head * n + row)
+    int sample_tiles;         // key tiles counted exactly before the window
     int n, N;
     int qtiles;               // query tiles per head in qop (a multiple of QT)
     int ktiles;
@@ -131,12 +138,23 @@ __device__ __forceinline__ float ex2(float x)
     return y;
 }
 
-// Weight of an accumulator value v = 256 s: exp2(c2 (s - m)) evaluated as
-// exp2(k1 * float(1.5*2^23 + v) + k0); the int -> float step is exact and
-// costs one integer add.  The histogram's Z uses the very same expression.
+// Weight of an accumulator value v (a multiple of the logit):
+// exp2(k1 * (v - ref)) evaluated as exp2(k1 * float(1.5*2^23 + v) + k0) with
+// k0 = -k1 * (ref + 1.5*2^23); the int -> float step is exact and costs one
+// integer add.
 __device__ __forceinline__ float weight_of(int v, float k1, float k0)
 {
     return ex2(fmaf(__int_as_float(v + kMagic), k1, k0));
+}
+
+// Increment of the four cumulative 8-bit window counters for a logit whose
+// counter index is amount / 8 (amount <= 0: every counter; >= 32: none).
+// shl.b32 clamps shift amounts above 32, which gives the "none" case.
+__device__ __forceinline__ uint32_t window_inc(int amount)
+{
+    uint32_t r;
+    asm("shl.b32 %0, %1, %2;" : "=r"(r) : "r"(0x01010101u), "r"((uint32_t)max(amount, 0)));
+    return r;
 }
 
 template <int D, bool kDbg>
@@ -272,15 +290,15 @@ attention_fwd_kernel(const Params p)
                 tc::mma_commit(b.v_empty + vs);
                 return true;
             };
-            for (int u = 0; u < 2 * T && ok; ++u) {
+            auto qk = [&](int u) -> bool {
                 const int ks = u % C::KSTAGES;
-                ok = wait_bar(b.k_full + ks, (u / C::KSTAGES) & 1, deadline, abort_flag, p.status);
-                if (!ok) break;
+                if (!wait_bar(b.k_full + ks, (u / C::KSTAGES) & 1, deadline, abort_flag, p.status))
+                    return false;
                 const int sb = u & 1;
-                for (int g = 0; g < QT && ok; ++g) {
-                    ok = wait_bar(b.s_empty(g, sb), ((u >> 1) & 1) ^ 1, deadline, abort_flag,
-                                  p.status);
-                    if (!ok) break;
+                for (int g = 0; g < QT; ++g) {
+                    if (!wait_bar(b.s_empty(g, sb), ((u >> 1) & 1) ^ 1, deadline, abort_flag,
+                                  p.status))
+                        return false;
                     tc::fence_after_sync();
                     const uint32_t scol = g * C::GROUP_COLS + C::S_COL + sb * 64;
 #pragma unroll
@@ -293,11 +311,24 @@ attention_fwd_kernel(const Params p)
                     }
                     tc::mma_commit(b.s_full(g, sb));
                 }
-                if (!ok) break;
                 tc::mma_commit(b.k_empty + ks);
-                if (u >= T + 1) ok = pv(u - T - 1);
+                return true;
+            };
+            // The epilogue consumes S tiles in pairs, so MMAs go in pairs too:
+            // the QK^T of pair k is issued as soon as the epilogue has loaded
+            // pair k-1, before the P V of pair k-1, which waits for its P.
+            for (int pass = 0; pass < 2 && ok; ++pass) {
+                for (int j = 0; j < T && ok; j += 2) {
+                    const int cnt = min(2, T - j);
+                    for (int k = 0; k < cnt && ok; ++k) ok = qk(pass * T + j + k);
+                    if (pass == 1 && j >= 2)
+                        for (int k = 0; k < 2 && ok; ++k) ok = pv(j - 2 + k);
+                }
             }
-            if (ok) ok = pv(T - 1);
+            if (ok) {
+                const int last = (T - 1) & ~1;            // first tile of the last pair
+                for (int i = last; i < T && ok; ++i) ok = pv(i);
+            }
             if (ok)
                 for (int g = 0; g < QT; ++g) tc::mma_commit(b.o_full(g));
             // drain: wait until every MMA this thread issued has completed
@@ -316,105 +347,173 @@ attention_fwd_kernel(const Params p)
         uint32_t *hist = reinterpret_cast<uint32_t *>(smem + C::OFF_HIST + g * C::HIST_BYTES);
         uint32_t *hcol = hist + r;                    // hist[bin][r] at hcol[bin * kRows]
         for (int bin = 0; bin < C::BINS; ++bin) hcol[bin * kRows] = 0;
-        // bin of accumulator value v = 256 s is (D - s)/2, at byte offset
-        // bin * 512 = 256 D - v from this row's bin 0
+        // The accumulator holds v = 4 s.  The level of a logit is its Hamming
+        // distance (D - s)/2; its histogram bin sits (D - s) * 256 bytes =
+        // 256 D - 64 v past this row's bin 0.
         const uint32_t hbase = tc::smem_u32(hcol) + 256u * D;
+        const int A = min(T, p.sample_tiles);         // tiles counted exactly
         bool ok = true;
+        using I0 = std::integral_constant<int, 0>;
+        using I64 = std::integral_constant<int, 64>;
+        using BT = std::integral_constant<bool, true>;
+        using BF = std::integral_constant<bool, false>;
 
-        // pass 1: histogram of the logits of this row
-        for (int j = 0; j < T && ok; ++j) {
-            const int sb = j & 1;
-            ok = __all_sync(kFullMask, wait_bar(b.s_full(g, sb), (j >> 1) & 1, deadline,
-                                                abort_flag, p.status));
-            if (!ok) break;
+        // S tiles travel in pairs: both accumulators are waited for, loaded
+        // with one tcgen05.wait::ld and released together, so the load
+        // latency and the MMA round trip are paid once per two tiles.
+        uint32_t s[128];
+        auto load_tiles = [&](int u, int cnt) -> bool {
+            for (int k = 0; k < cnt; ++k) {
+                const int uk = u + k;
+                if (!__all_sync(kFullMask, wait_bar(b.s_full(g, uk & 1), (uk >> 1) & 1,
+                                                    deadline, abort_flag, p.status)))
+                    return false;
+            }
             tc::fence_after_sync();
-            uint32_t s0[32], s1[32];
-            const uint32_t scol = C::S_COL + sb * 64;
-            tc::tmem_ld32(lane_base + scol, s0);
-            tc::tmem_ld32(lane_base + scol + 32, s1);
+            tc::tmem_ld32(lane_base + C::S_COL + (u & 1) * 64, *reinterpret_cast<uint32_t(*)[32]>(s));
+            tc::tmem_ld32(lane_base + C::S_COL + (u & 1) * 64 + 32,
+                          *reinterpret_cast<uint32_t(*)[32]>(s + 32));
+            if (cnt > 1) {
+                tc::tmem_ld32(lane_base + C::S_COL + ((u + 1) & 1) * 64,
+                              *reinterpret_cast<uint32_t(*)[32]>(s + 64));
+                tc::tmem_ld32(lane_base + C::S_COL + ((u + 1) & 1) * 64 + 32,
+                              *reinterpret_cast<uint32_t(*)[32]>(s + 96));
+            }
             tc::tmem_wait_ld();
             tc::fence_before_sync();
-            tc::mbar_arrive(b.s_empty(g, sb));
-            const int valid = min(kKeys, p.n - j * kKeys);
-            if (valid == kKeys) {
-#pragma unroll
-                for (int c = 0; c < 32; ++c) red_add1(hbase - s0[c]);
-#pragma unroll
-                for (int c = 0; c < 32; ++c) red_add1(hbase - s1[c]);
-            } else {
-#pragma unroll
-                for (int c = 0; c < 32; ++c)
-                    if (c < valid) red_add1(hbase - s0[c]);
-#pragma unroll
-                for (int c = 0; c < 32; ++c)
-                    if (32 + c < valid) red_add1(hbase - s1[c]);
-            }
-        }
+            for (int k = 0; k < cnt; ++k) tc::mbar_arrive(b.s_empty(g, (u + k) & 1));
+            return true;
+        };
 
-        // threshold level t (as a Hamming distance), quota q, max, Z
-        int t = C::BINS - 1, hmin = C::BINS - 1;
-        int quota = 0;
-        {
-            int below = 0;
-            bool found = false, seen = false;
+        // pass 1a: exact histogram of the first A key tiles
+        auto hist_tile = [&](auto off, auto full, int valid) {
+            constexpr int O = decltype(off)::value;
+#pragma unroll
+            for (int c = 0; c < 64; ++c)
+                if (decltype(full)::value || c < valid) red_add1(hbase - (s[O + c] << 6));
+        };
+        // pass 1b: four cumulative 8-bit window counters in one register
+        uint32_t acc = 0;
+        int tot0 = 0, tot1 = 0, tot2 = 0, tot3 = 0;
+        int cshift = 0, L0 = 0, hmin = C::BINS - 1;
+        auto flush = [&]() {
+            tot0 += (int)(acc & 0xFFu);
+            tot1 += (int)((acc >> 8) & 0xFFu);
+            tot2 += (int)((acc >> 16) & 0xFFu);
+            tot3 += (int)(acc >> 24);
+            acc = 0;
+        };
+        auto window_tile = [&](auto off, auto full, int valid) {
+            constexpr int O = decltype(off)::value;
+#pragma unroll
+            for (int c = 0; c < 64; ++c)
+                if (decltype(full)::value || c < valid) acc += window_inc(cshift - (int)s[O + c]);
+        };
+        // Window from the sample: est = the level of the sample's
+        // (N * sampled / n)-th best key.  Levels L0 = est - 1 .. est + 1 are
+        // resolved exactly; the rest of the row updates four cumulative
+        // counters f_k = #{level <= L0 - 1 + k}, k = 0..3.
+        auto place_window = [&]() {
+            const int sampled = min(p.n, A * kKeys);
+            const int ns = max(1, (int)(((long long)p.N * sampled + p.n / 2) / p.n));
+            int cum = 0, est = C::BINS - 1;
+            bool seen = false, found = false;
             for (int bin = 0; bin < C::BINS; ++bin) {
                 const int c = (int)hcol[bin * kRows];
                 if (!seen && c) { hmin = bin; seen = true; }
-                if (!found) {
-                    if (below + c >= p.N) { t = bin; quota = p.N - below; found = true; }
-                    else below += c;
-                }
+                cum += c;
+                if (!found && cum >= ns) { est = bin; found = true; }
+            }
+            L0 = est - 1;
+            cshift = 4 * D - 8 * L0 + 8;              // 8 * (level - L0 + 1) = cshift - v
+        };
+        auto pass1_tile = [&](int j, auto off) {
+            const int valid = min(kKeys, p.n - j * kKeys);
+            if (j < A) {
+                if (valid == kKeys) hist_tile(off, BT{}, valid);
+                else hist_tile(off, BF{}, valid);
+                if (j == A - 1) place_window();
+            } else {
+                if (valid == kKeys) window_tile(off, BT{}, valid);
+                else window_tile(off, BF{}, valid);
+                if ((j - A) % 3 == 2) flush();        // fields stay below 3 * 64 < 256
+            }
+        };
+        for (int j = 0; j < T && ok; j += 2) {
+            const int cnt = min(2, T - j);
+            ok = load_tiles(j, cnt);
+            if (!ok) break;
+            pass1_tile(j, I0{});
+            if (cnt > 1) pass1_tile(j + 1, I64{});
+        }
+        flush();
+
+        // threshold level t and the number q of keys kept at it
+        int t = -1, quota = 0;
+        bool miss = false;
+        if (A >= T) {
+            int below = 0;
+            for (int bin = 0; bin < C::BINS; ++bin) {
+                const int c = (int)hcol[bin * kRows];
+                if (below + c >= p.N) { t = bin; quota = p.N - below; break; }
+                below += c;
+            }
+        } else {
+            int f0 = tot0, f1 = tot1, f2 = tot2, f3 = tot3;
+            for (int bin = 0; bin < C::BINS; ++bin) {
+                const int c = (int)hcol[bin * kRows];
+                if (bin <= L0 - 1) f0 += c;
+                if (bin <= L0) f1 += c;
+                if (bin <= L0 + 1) f2 += c;
+                if (bin <= L0 + 2) f3 += c;
+            }
+            if (f0 < p.N && f3 >= p.N) {
+                if (f1 >= p.N) { t = L0; quota = p.N - f0; }
+                else if (f2 >= p.N) { t = L0 + 1; quota = p.N - f1; }
+                else { t = L0 + 2; quota = p.N - f2; }
+            } else {
+                miss = true;
             }
         }
-        const int vt = 256 * (D - 2 * t);             // accumulator value of the threshold
-        const int vm = 256 * (D - 2 * hmin);          // ... of the row maximum
-        const float k1 = p.c2 * (1.0f / 256.0f);
-        const float k0 = -fmaf((float)vm, k1, 0.0f) - 12582912.0f * k1;
-        float Z = 0.0f;
-        for (int bin = hmin; bin < t; ++bin)
-            Z += (float)hcol[bin * kRows] * weight_of(256 * (D - 2 * bin), k1, k0);
-        Z += (float)quota * weight_of(vt, k1, k0);
+        if (miss && active) {
+            const int slot = atomicAdd(p.miss_count, 1);
+            p.miss_rows[slot] = (int)(head * p.n + row);
+        }
+        // missed rows keep nothing here; the fix-up kernel rewrites them
+        const int vt = miss ? 4 * (D + 2) : 4 * (D - 2 * t);
+        if (miss) quota = 0;
+        // softmax reference: the sample's best logit, raised if needed so that
+        // no weight can exceed the fp16 range (s <= D)
+        const float c2q = p.c2 * 0.25f;               // exponent per unit of v
+        const int headroom = c2q > 1.0e-6f ? (int)fminf(floorf(15.99f / c2q), 1.0e6f) : 1000000;
+        const int ref = max(4 * (D - 2 * hmin), 4 * D - headroom);
+        const float k0 = -fmaf((float)ref, c2q, 0.0f) - 12582912.0f * c2q;
         int rem = quota;                              // ties still to keep
         int kept = 0;
+        float Z = 0.0f;
         const long long obase = ((head * p.n) + row) * (long long)p.N;
 
         // pass 2: P = kept weights (fp16) -> TMEM; the MMA warp does O += P V
-        for (int j = 0; j < T && ok; ++j) {
-            const int u = T + j;
-            const int sb = u & 1;
-            ok = __all_sync(kFullMask, wait_bar(b.s_full(g, sb), (u >> 1) & 1, deadline,
-                                                abort_flag, p.status));
-            if (!ok) break;
-            tc::fence_after_sync();
-            uint32_t s[64];
-            const uint32_t scol = C::S_COL + sb * 64;
-            tc::tmem_ld32(lane_base + scol, *reinterpret_cast<uint32_t(*)[32]>(s));
-            tc::tmem_ld32(lane_base + scol + 32, *reinterpret_cast<uint32_t(*)[32]>(s + 32));
-            tc::tmem_wait_ld();
-            tc::fence_before_sync();
-            tc::mbar_arrive(b.s_empty(g, sb));
-            const int pb = j & 1;
-            ok = __all_sync(kFullMask, wait_bar(b.p_empty(g, pb), ((j >> 1) & 1) ^ 1, deadline,
-                                                abort_flag, p.status));
-            if (!ok) break;
-            const int valid = min(kKeys, p.n - j * kKeys);
+        auto pass2_tile = [&](int j, auto off, auto full, int valid) {
+            constexpr int O = decltype(off)::value;
             uint32_t packed[32];
 #pragma unroll
             for (int c = 0; c < 64; c += 2) {
                 float w2[2];
 #pragma unroll
                 for (int e = 0; e < 2; ++e) {
-                    const int v = (int)s[c + e];
-                    const bool in = (c + e) < valid;
+                    const int v = (int)s[O + c + e];
+                    const bool in = decltype(full)::value || (c + e) < valid;
                     const bool tie = in && (v == vt);
                     const bool keep = in && ((v > vt) || (tie && rem > 0));
                     rem -= tie ? 1 : 0;
-                    const float w = weight_of(v, k1, k0);
-                    w2[e] = keep ? w : 0.0f;
+                    const float w = keep ? weight_of(v, c2q, k0) : 0.0f;
+                    Z += w;
+                    w2[e] = w;
                     if (kDbg) {
                         if (keep && active) {
                             if (p.dbg_idx) p.dbg_idx[obase + kept] = j * kKeys + c + e;
-                            if (p.dbg_logits) p.dbg_logits[obase + kept] = (int16_t)(v / 256);
+                            if (p.dbg_logits) p.dbg_logits[obase + kept] = (int16_t)(v / 4);
                             ++kept;
                         }
                     }
@@ -422,11 +521,22 @@ attention_fwd_kernel(const Params p)
                 __half2 h = __floats2half2_rn(w2[0], w2[1]);
                 packed[c >> 1] = *reinterpret_cast<uint32_t *>(&h);
             }
-            tc::tmem_st32(lane_base + C::P_COL + pb * 32, packed);
+            tc::tmem_st32(lane_base + C::P_COL + (j & 1) * 32, packed);
+        };
+        for (int j = 0; j < T && ok; ++j) {
+            ok = load_tiles(T + j, 1);
+            if (!ok) break;
+            ok = __all_sync(kFullMask, wait_bar(b.p_empty(g, j & 1), ((j >> 1) & 1) ^ 1, deadline,
+                                                abort_flag, p.status));
+            if (!ok) break;
+            const int valid = min(kKeys, p.n - j * kKeys);
+            if (valid == kKeys) pass2_tile(j, I0{}, BT{}, valid);
+            else pass2_tile(j, I0{}, BF{}, valid);
             tc::tmem_wait_st();
             tc::fence_before_sync();
-            tc::mbar_arrive(b.p_full(g, pb));
+            tc::mbar_arrive(b.p_full(g, j & 1));
         }
+        if (!(Z > 0.0f)) Z = 1.0f;                    // missed or inactive rows only
 
         // output: O / Z * 2^e_h
         if (ok) ok = __all_sync(kFullMask, wait_bar(b.o_full(g), 0, deadline, abort_flag, p.status));
@@ -458,6 +568,111 @@ attention_fwd_kernel(const Params p)
     if (warp == 0) {
         tc::fence_after_sync();
         tc::tmem_dealloc(tmem, C::TMEM_COLS);
+    }
+}
+
+// Exact recomputation of the rows the fused kernel listed: one warp per row,
+// Hamming distances from the packed bits, histogram -> threshold and quota,
+// then the kept keys in ascending index order (ballot prefix counts decide
+// the ties), exp(tau (s - m)) weights in fp32 and the gathered V rows.
+template <typename T, int D>
+__global__ void __launch_bounds__(256)
+fixup_rows_kernel(const uint32_t *__restrict__ qbits, const uint32_t *__restrict__ kbits,
+                  const T *__restrict__ V, int n, int N, float tau,
+                  const int *__restrict__ miss_count, const int *__restrict__ miss_rows,
+                  float *__restrict__ out, int32_t *dbg_idx, int16_t *dbg_logits)
+{
+    constexpr int DW = D / 32, BINS = D + 1, PER = D / 32;
+    __shared__ int hist[8][BINS];
+    const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
+    const int count = *miss_count;
+    for (int m = blockIdx.x * 8 + warp; m < count; m += gridDim.x * 8) {
+        const int r = miss_rows[m];
+        const long long head = r / n;
+        uint32_t q[DW];
+#pragma unroll
+        for (int w = 0; w < DW; ++w) q[w] = qbits[(long long)r * DW + w];
+        const uint32_t *kh = kbits + head * n * DW;
+        for (int b = lane; b < BINS; b += 32) hist[warp][b] = 0;
+        __syncwarp();
+#pragma unroll 4
+        for (int j = lane; j < n; j += 32) {
+            int h = 0;
+#pragma unroll
+            for (int w = 0; w < DW; ++w) h += __popc(q[w] ^ kh[(long long)j * DW + w]);
+            atomicAdd(&hist[warp][h], 1);
+        }
+        __syncwarp();
+        int t = BINS - 1, quota = 0, hmin = BINS - 1, below = 0;
+        bool found = false, seen = false;
+        for (int b = 0; b < BINS; ++b) {
+            const int c = hist[warp][b];
+            if (!seen && c) { hmin = b; seen = true; }
+            if (!found) {
+                if (below + c >= N) { t = b; quota = N - below; found = true; }
+                else below += c;
+            }
+        }
+        __syncwarp();
+        const int smax = D - 2 * hmin;
+        float acc[PER];
+#pragma unroll
+        for (int e = 0; e < PER; ++e) acc[e] = 0.0f;
+        float z = 0.0f;
+        int ties_before = 0, kept_before = 0;
+        const unsigned below_me = (1u << lane) - 1u;
+        const T *vh = V + head * n * (long long)D;
+        for (int j0 = 0; j0 < n; j0 += 32) {
+            const int j = j0 + lane;
+            int h = BINS;
+            if (j < n) {
+                h = 0;
+#pragma unroll
+                for (int w = 0; w < DW; ++w) h += __popc(q[w] ^ kh[(long long)j * DW + w]);
+            }
+            const bool tie = (h == t);
+            const unsigned tmask = __ballot_sync(kFullMask, tie);
+            const int rank = ties_before + __popc(tmask & below_me);
+            const bool keep = (j < n) && (h < t || (tie && rank < quota));
+            ties_before += __popc(tmask);
+            const unsigned kmask = __ballot_sync(kFullMask, keep);
+            const int s = D - 2 * h;
+            const float w = keep ? expf(tau * (float)(s - smax)) : 0.0f;
+            if (keep && (dbg_idx || dbg_logits)) {
+                const long long pos = (long long)r * N + kept_before + __popc(kmask & below_me);
+                if (dbg_idx) dbg_idx[pos] = j;
+                if (dbg_logits) dbg_logits[pos] = (int16_t)s;
+            }
+            kept_before += __popc(kmask);
+            // gather the kept V rows four at a time so their loads overlap
+            unsigned mm = kmask;
+            while (mm) {
+                int jj[4];
+                float ww[4];
+#pragma unroll
+                for (int u = 0; u < 4; ++u) {
+                    const bool has = mm != 0u;        // warp-uniform
+                    const int src = has ? __ffs(mm) - 1 : 0;
+                    if (has) mm &= mm - 1u;
+                    jj[u] = __shfl_sync(kFullMask, j, src);
+                    ww[u] = __shfl_sync(kFullMask, w, src);
+                    if (!has) { jj[u] = j0; ww[u] = 0.0f; }
+                }
+                float v[4][PER];
+#pragma unroll
+                for (int u = 0; u < 4; ++u)
+                    VRow<T, PER>::load(vh + (long long)jj[u] * D + lane * PER, v[u]);
+#pragma unroll
+                for (int u = 0; u < 4; ++u) {
+#pragma unroll
+                    for (int e = 0; e < PER; ++e) acc[e] = fmaf(ww[u], v[u][e], acc[e]);
+                    z += ww[u];
+                }
+            }
+        }
+        float *orow = out + (long long)r * D + lane * PER;
+#pragma unroll
+        for (int e = 0; e < PER; ++e) orow[e] = acc[e] / z;
     }
 }
 

@@ -7,11 +7,13 @@
 // 128 bytes apart, row groups (8 rows) (K bytes / 16) * 128 bytes apart.
 // Tiles are stored contiguously so the kernel moves each with one bulk copy.
 //
-//   Qop [BH][qtiles] tiles of 128 rows x d int8 (+16 / -16, 0 padding;
+//   Qop [BH][qtiles] tiles of 128 rows x d int8 (+4 / -4, 0 padding;
 //                    qtiles >= ceil(n/128), the extra tiles all padding)
-//   Kop [BH][ceil(n/64)] tiles of 64 keys x d int8 (+16 / -16, 0 padding)
-// The +/-16 scale makes the s32 accumulator hold 256 * s, which the fused
-// kernel uses directly as a byte offset into its per-row histogram.
+//   Kop [BH][ceil(n/64)] tiles of 64 keys x d int8 (+1 / -1, 0 padding)
+//   Qbits, Kbits [BH][n][d/32] the same signs bit-packed (1 = -1)
+// The +/-4 x +/-1 scaling makes the s32 accumulator hold 4 * s, which the
+// fused kernel turns into histogram addresses and counter shifts with one
+// integer add.
 //   Vop [BH][ceil(n/64)]  tiles of V^T: d rows x 64 keys fp16, scaled by
 //                         2^-e_h so the head's largest |v| lies in
 //                         [2^14, 2^15) (bf16 -> fp16 then loses no bits for
@@ -39,10 +41,13 @@ __device__ __forceinline__ uint32_t core_offset(uint32_t row, uint32_t kbyte, ui
 
 // One thread per 16 consecutive elements of a row -> 16 int8 signs.
 // Works for Q (tile 128) and K (tile 64): `tile_rows` selects the tiling.
+// The packed copy is written as 16-bit halves: chunk kc of a row is bits
+// 16*(kc%2) .. 16*(kc%2)+15 of word kc/2.
 template <typename T>
 __global__ void __launch_bounds__(256)
 sign_operand_kernel(const T *__restrict__ x, const float *__restrict__ sigma, int H, int n,
-                    int d, int tile_rows, int tiles, long long chunks, int8_t *__restrict__ op,
+                    int d, int tile_rows, int tiles, long long chunks, uint32_t pos,
+                    uint32_t neg, int8_t *__restrict__ op, uint16_t *__restrict__ bits,
                     int32_t *status)
 {
     const int cpr = d >> 4;                                  // chunks per row
@@ -64,15 +69,20 @@ sign_operand_kernel(const T *__restrict__ x, const float *__restrict__ sigma, in
             Load8<T>::run(src, lo);
             Load8<T>::run(src + 8, hi);
             uint32_t w[4];
+            uint32_t packed = 0;
 #pragma unroll
             for (int q = 0; q < 4; ++q) {
                 uint32_t word = 0;
 #pragma unroll
-                for (int b = 0; b < 4; ++b)
-                    word |= (negative_bit(v[4 * q + b], rule) ? 0xF0u : 0x10u) << (8 * b);
+                for (int b = 0; b < 4; ++b) {
+                    const uint32_t nb = negative_bit(v[4 * q + b], rule);
+                    word |= (nb ? neg : pos) << (8 * b);
+                    packed |= nb << (4 * q + b);
+                }
                 w[q] = word;
             }
             out = make_uint4(w[0], w[1], w[2], w[3]);
+            bits[(head * n + r) * (long long)cpr + kc] = (uint16_t)packed;
         }
         const int t = r / tile_rows;
         const uint32_t rr = (uint32_t)(r % tile_rows);
@@ -82,40 +92,34 @@ sign_operand_kernel(const T *__restrict__ x, const float *__restrict__ sigma, in
 }
 
 // Largest |v| of each head, as ordered float bits (non-negative floats
-// compare like unsigned integers).  vmax must be zeroed beforehand.
+// compare like unsigned integers; NaN counts as infinity).  Each CTA reduces
+// one contiguous chunk of one head and issues a single atomicMax.  vmax must
+// be zeroed beforehand.
 template <typename T>
 __global__ void __launch_bounds__(256)
-vmax_kernel(const T *__restrict__ v, long long groups_per_head, long long groups,
+vmax_kernel(const T *__restrict__ v, long long groups_per_head, int chunks_per_head,
             unsigned int *__restrict__ vmax)
 {
-    for (long long g0 = blockIdx.x * (long long)blockDim.x; g0 < groups;
-         g0 += (long long)gridDim.x * blockDim.x) {
-        const long long g = g0 + threadIdx.x;
-        const bool valid = g < groups;
-        const long long head = valid ? g / groups_per_head : -1;
-        float m = 0.0f;
-        if (valid) {
-            float e[8];
-            Load8<T>::run(v + g * 8, e);
-            bool nan = false;
+    __shared__ float wmax[8];
+    const long long head = blockIdx.x / chunks_per_head;
+    const int chunk = blockIdx.x % chunks_per_head;
+    const long long per = (groups_per_head + chunks_per_head - 1) / chunks_per_head;
+    const long long g_beg = head * groups_per_head + chunk * per;
+    const long long g_end = head * groups_per_head + min(groups_per_head, (chunk + 1) * per);
+    float m = 0.0f;
+    for (long long g = g_beg + threadIdx.x; g < g_end; g += blockDim.x) {
+        float e[8];
+        Load8<T>::run(v + g * 8, e);
 #pragma unroll
-            for (int k = 0; k < 8; ++k) {
-                m = fmaxf(m, fabsf(e[k]));
-                nan |= isnan(e[k]);
-            }
-            if (nan) m = __int_as_float(0x7f800000);         // NaN: treat like inf
-        }
-        // lane 0 is valid whenever any lane is; reduce per warp when the
-        // warp lies in one head, otherwise one atomic per lane
-        const long long h0 = __shfl_sync(kFullMask, head, 0);
-        const bool same = __all_sync(kFullMask, head == h0 || head < 0);
-        if (same && h0 >= 0) {
+        for (int k = 0; k < 8; ++k) m = isnan(e[k]) ? __int_as_float(0x7f800000) : fmaxf(m, fabsf(e[k]));
+    }
 #pragma unroll
-            for (int o = 16; o > 0; o >>= 1) m = fmaxf(m, __shfl_xor_sync(kFullMask, m, o));
-            if ((threadIdx.x & 31) == 0) atomicMax(vmax + h0, __float_as_uint(m));
-        } else if (valid) {
-            atomicMax(vmax + head, __float_as_uint(m));
-        }
+    for (int o = 16; o > 0; o >>= 1) m = fmaxf(m, __shfl_xor_sync(kFullMask, m, o));
+    if ((threadIdx.x & 31) == 0) wmax[threadIdx.x >> 5] = m;
+    __syncthreads();
+    if (threadIdx.x == 0) {
+        for (int w = 1; w < (int)(blockDim.x >> 5); ++w) m = fmaxf(m, wmax[w]);
+        atomicMax(vmax + head, __float_as_uint(m));
     }
 }
 
