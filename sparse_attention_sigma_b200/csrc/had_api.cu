@@ -211,7 +211,7 @@ had_status_t launch_fused_typed(const T *Q, const T *K, const T *V, const float 
     p.c2 = tau * 1.4426950408889634f;
     const long long blocks = bh * p.ctas_per_head;
     kernel<<<(unsigned)blocks, C::THREADS, C::SMEM_BYTES, st>>>(p);
-    had::fused::fixup_rows_kernel<T, D><<<148 * 2, 256, 0, st>>>(
+    had::fused::fixup_rows_kernel<T, D><<<148 * 4, 256, 0, st>>>(
         qbits, kbits, V, n, N, tau, miss_count, miss_rows, out, dbg_idx, dbg_lg);
     return launched();
 }

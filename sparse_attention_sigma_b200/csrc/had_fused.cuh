@@ -571,10 +571,14 @@ attention_fwd_kernel(const Params p)
     }
 }
 
-// Exact recomputation of the rows the fused kernel listed: one warp per row,
-// Hamming distances from the packed bits, histogram -> threshold and quota,
-// then the kept keys in ascending index order (ballot prefix counts decide
-// the ties), exp(tau (s - m)) weights in fp32 and the gathered V rows.
+// Exact recomputation of the rows the fused kernel listed.  One CTA of
+// eight warps per row: Hamming distances from the packed bits, a shared
+// histogram -> threshold level and quota, then each warp takes one
+// contiguous range of keys.  Per-warp counts of ties and of keys above the
+// threshold, prefix-summed across warps, give every warp its share of the
+// quota (ties go to the lower key index) and its output positions; the warp
+// gathers its kept V rows with exp(tau (s - m)) weights in fp32 and the
+// partial sums meet in shared memory.
 template <typename T, int D>
 __global__ void __launch_bounds__(256)
 fixup_rows_kernel(const uint32_t *__restrict__ qbits, const uint32_t *__restrict__ kbits,
@@ -582,66 +586,89 @@ fixup_rows_kernel(const uint32_t *__restrict__ qbits, const uint32_t *__restrict
                   const int *__restrict__ miss_count, const int *__restrict__ miss_rows,
                   float *__restrict__ out, int32_t *dbg_idx, int16_t *dbg_logits)
 {
-    constexpr int DW = D / 32, BINS = D + 1, PER = D / 32;
-    __shared__ int hist[8][BINS];
+    constexpr int DW = D / 32, BINS = D + 1, PER = D / 32, NW = 8;
+    __shared__ int hist[BINS];
+    __shared__ int wties[NW], wabove[NW];
+    __shared__ float opart[NW][D];
+    __shared__ float zpart[NW];
+    __shared__ int sh_t, sh_quota, sh_hmin;
     const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
+    const unsigned below_me = (1u << lane) - 1u;
     const int count = *miss_count;
-    for (int m = blockIdx.x * 8 + warp; m < count; m += gridDim.x * 8) {
+    // each warp's key range: a multiple of 32 keys
+    const int span = ((n + NW - 1) / NW + 31) / 32 * 32;
+    const int jb = min(n, warp * span), je = min(n, jb + span);
+    for (int m = blockIdx.x; m < count; m += gridDim.x) {
         const int r = miss_rows[m];
         const long long head = r / n;
         uint32_t q[DW];
 #pragma unroll
         for (int w = 0; w < DW; ++w) q[w] = qbits[(long long)r * DW + w];
         const uint32_t *kh = kbits + head * n * DW;
-        for (int b = lane; b < BINS; b += 32) hist[warp][b] = 0;
-        __syncwarp();
-#pragma unroll 4
-        for (int j = lane; j < n; j += 32) {
+        auto ham = [&](int j) {
             int h = 0;
 #pragma unroll
             for (int w = 0; w < DW; ++w) h += __popc(q[w] ^ kh[(long long)j * DW + w]);
-            atomicAdd(&hist[warp][h], 1);
-        }
-        __syncwarp();
-        int t = BINS - 1, quota = 0, hmin = BINS - 1, below = 0;
-        bool found = false, seen = false;
-        for (int b = 0; b < BINS; ++b) {
-            const int c = hist[warp][b];
-            if (!seen && c) { hmin = b; seen = true; }
-            if (!found) {
-                if (below + c >= N) { t = b; quota = N - below; found = true; }
-                else below += c;
+            return h;
+        };
+        for (int b = threadIdx.x; b < BINS; b += blockDim.x) hist[b] = 0;
+        __syncthreads();
+        for (int j = threadIdx.x; j < n; j += blockDim.x) atomicAdd(&hist[ham(j)], 1);
+        __syncthreads();
+        if (threadIdx.x == 0) {
+            int t = BINS - 1, quota = 0, hmin = BINS - 1, below = 0;
+            bool found = false, seen = false;
+            for (int b = 0; b < BINS; ++b) {
+                const int c = hist[b];
+                if (!seen && c) { hmin = b; seen = true; }
+                if (!found) {
+                    if (below + c >= N) { t = b; quota = N - below; found = true; }
+                    else below += c;
+                }
             }
+            sh_t = t; sh_quota = quota; sh_hmin = hmin;
         }
-        __syncwarp();
-        const int smax = D - 2 * hmin;
+        __syncthreads();
+        const int t = sh_t, quota = sh_quota, smax = D - 2 * sh_hmin;
+        // counts of this warp's range
+        int nt = 0, na = 0;
+        for (int j = jb + lane; j < je; j += 32) {
+            const int h = ham(j);
+            nt += (h == t);
+            na += (h < t);
+        }
+#pragma unroll
+        for (int o = 16; o > 0; o >>= 1) {
+            nt += __shfl_xor_sync(kFullMask, nt, o);
+            na += __shfl_xor_sync(kFullMask, na, o);
+        }
+        if (lane == 0) { wties[warp] = nt; wabove[warp] = na; }
+        __syncthreads();
+        int ties_before = 0, kept_before = 0;
+        for (int w = 0; w < warp; ++w) {
+            kept_before += wabove[w] + min(max(quota - ties_before, 0), wties[w]);
+            ties_before += wties[w];
+        }
         float acc[PER];
 #pragma unroll
         for (int e = 0; e < PER; ++e) acc[e] = 0.0f;
         float z = 0.0f;
-        int ties_before = 0, kept_before = 0;
-        const unsigned below_me = (1u << lane) - 1u;
         const T *vh = V + head * n * (long long)D;
-        for (int j0 = 0; j0 < n; j0 += 32) {
+        for (int j0 = jb; j0 < je; j0 += 32) {
             const int j = j0 + lane;
-            int h = BINS;
-            if (j < n) {
-                h = 0;
-#pragma unroll
-                for (int w = 0; w < DW; ++w) h += __popc(q[w] ^ kh[(long long)j * DW + w]);
-            }
+            const int h = j < je ? ham(j) : BINS;
             const bool tie = (h == t);
             const unsigned tmask = __ballot_sync(kFullMask, tie);
             const int rank = ties_before + __popc(tmask & below_me);
-            const bool keep = (j < n) && (h < t || (tie && rank < quota));
+            const bool keep = (h < t) || (tie && rank < quota);
             ties_before += __popc(tmask);
             const unsigned kmask = __ballot_sync(kFullMask, keep);
-            const int s = D - 2 * h;
-            const float w = keep ? expf(tau * (float)(s - smax)) : 0.0f;
+            const int sv = D - 2 * h;
+            const float w = keep ? expf(tau * (float)(sv - smax)) : 0.0f;
             if (keep && (dbg_idx || dbg_logits)) {
                 const long long pos = (long long)r * N + kept_before + __popc(kmask & below_me);
                 if (dbg_idx) dbg_idx[pos] = j;
-                if (dbg_logits) dbg_logits[pos] = (int16_t)s;
+                if (dbg_logits) dbg_logits[pos] = (int16_t)sv;
             }
             kept_before += __popc(kmask);
             // gather the kept V rows four at a time so their loads overlap
@@ -670,9 +697,20 @@ fixup_rows_kernel(const uint32_t *__restrict__ qbits, const uint32_t *__restrict
                 }
             }
         }
-        float *orow = out + (long long)r * D + lane * PER;
 #pragma unroll
-        for (int e = 0; e < PER; ++e) orow[e] = acc[e] / z;
+        for (int e = 0; e < PER; ++e) opart[warp][lane * PER + e] = acc[e];
+        if (lane == 0) zpart[warp] = z;
+        __syncthreads();
+        float zt = 0.0f;
+#pragma unroll
+        for (int w = 0; w < NW; ++w) zt += zpart[w];
+        for (int c = threadIdx.x; c < D; c += blockDim.x) {
+            float o = 0.0f;
+#pragma unroll
+            for (int w = 0; w < NW; ++w) o += opart[w][c];
+            out[(long long)r * D + c] = o / zt;
+        }
+        __syncthreads();
     }
 }
 
