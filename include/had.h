@@ -148,8 +148,8 @@ HAD_API had_status_t had_attention_fwd(const void *Q, const void *K, const void 
  * workspace from a fixed device array inside the library instead of a
  * caller buffer, and allocates nothing.
  *   - Limit: had_workspace_bytes(HAD_OP_ATTENTION_FWD, ...) must not exceed
- *     had_noalloc_scratch_bytes() (80 MiB, enough for B=4 H=16 n=4096
- *     d=64); larger sizes return HAD_ERR_WORKSPACE before any launch.
+ *     had_noalloc_scratch_bytes() (96 MiB, enough for B=4 H=16 n=4096
+ *     d=64 N=512); larger sizes return HAD_ERR_WORKSPACE before any launch.
  *   - The array is part of the loaded module: every GPU that loads the
  *     library holds it until the process exits.
  *   - The first call on each device looks up the array's device address

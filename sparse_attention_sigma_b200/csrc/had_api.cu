@@ -124,7 +124,7 @@ had_status_t launch_av(const int32_t *idx, const int16_t *lg, const void *V, had
 // Workspace of the fused forward: tensor-core operand tiles of Q, K and V^T
 // and the per-head V scale.
 struct FwdWorkspace {
-    size_t qop, kop, vop, qbits, kbits, vmax, vexp, miss_rows, total;
+    size_t qop, qop2, kop, vop, qbits, kbits, vmax, vexp, miss_rows, total;
     int qtiles, ktiles;
 };
 
@@ -138,7 +138,8 @@ FwdWorkspace fwd_layout(int B, int H, int n, int d, int N)
     w.qtiles = (w.qtiles + qt - 1) / qt * qt;
     w.ktiles = (n + had::fused::kKeys - 1) / had::fused::kKeys;
     w.qop = 0;
-    w.kop = w.qop + round_up(bh * w.qtiles * had::fused::kRows * d);
+    w.qop2 = w.qop + round_up(bh * w.qtiles * had::fused::kRows * d);
+    w.kop = w.qop2 + round_up(bh * w.qtiles * had::fused::kRows * d);
     w.vop = w.kop + round_up(bh * w.ktiles * had::fused::kKeys * d);
     w.qbits = w.vop + round_up(bh * w.ktiles * had::fused::kKeys * d * 2);
     w.kbits = w.qbits + round_up(bh * n * (d / 8));
@@ -158,6 +159,7 @@ had_status_t launch_fused_typed(const T *Q, const T *K, const T *V, const float 
     using C = had::fused::Cfg<D>;
     const long long bh = (long long)B * H;
     auto *qop = reinterpret_cast<int8_t *>(ws + w.qop);
+    auto *qop2 = reinterpret_cast<int8_t *>(ws + w.qop2);
     auto *kop = reinterpret_cast<int8_t *>(ws + w.kop);
     auto *vop = reinterpret_cast<__half *>(ws + w.vop);
     auto *qbits = reinterpret_cast<uint32_t *>(ws + w.qbits);
@@ -169,13 +171,13 @@ had_status_t launch_fused_typed(const T *Q, const T *K, const T *V, const float 
     if (cudaMemsetAsync(vmax, 0, (bh + 1) * 4, st) != cudaSuccess) return HAD_ERR_CUDA;
     const long long qchunks = bh * w.qtiles * had::fused::kRows * (D / 16);
     const long long kchunks = bh * w.ktiles * had::fused::kKeys * (D / 16);
-    // Q as +/-4 and K as +/-1: the i8 MMA accumulates 4 s
+    // Q as +/-1 and +/-64, K as +/-4: the i8 MMA accumulates 4 s or 256 s
     had::prep::sign_operand_kernel<T><<<grid_for(qchunks, 256), 256, 0, st>>>(
-        Q, sq, H, n, D, had::fused::kRows, w.qtiles, qchunks, 0x04u, 0xFCu, qop,
-        reinterpret_cast<uint16_t *>(qbits), status);
+        Q, sq, H, n, D, had::fused::kRows, w.qtiles, qchunks, 0x01u, 0xFFu, qop, 0x40u, 0xC0u,
+        qop2, reinterpret_cast<uint16_t *>(qbits), status);
     had::prep::sign_operand_kernel<T><<<grid_for(kchunks, 256), 256, 0, st>>>(
-        K, sk, H, n, D, had::fused::kKeys, w.ktiles, kchunks, 0x01u, 0xFFu, kop,
-        reinterpret_cast<uint16_t *>(kbits), status);
+        K, sk, H, n, D, had::fused::kKeys, w.ktiles, kchunks, 0x04u, 0xFCu, kop, 0u, 0u,
+        nullptr, reinterpret_cast<uint16_t *>(kbits), status);
     const long long vgroups_per_head = (long long)n * D / 8;
     const int chunks = (int)((vgroups_per_head + 4095) / 4096);   // 32 KiB of bf16 per CTA
     if (bh * chunks > INT_MAX) return HAD_ERR_UNSUPPORTED;
@@ -193,6 +195,7 @@ had_status_t launch_fused_typed(const T *Q, const T *K, const T *V, const float 
         return HAD_ERR_CUDA;
     had::fused::Params p;
     p.qop = qop;
+    p.qop2 = qop2;
     p.kop = kop;
     p.vop = vop;
     p.vexp = vexp;
@@ -237,7 +240,7 @@ had_status_t launch_fused(const void *Q, const void *K, const void *V, const flo
 // workspace from a statically sized device array instead.  The array is part
 // of the module: every GPU that loads the library holds it until the process
 // exits.
-constexpr size_t kNoAllocScratchBytes = size_t(80) << 20;   // 80 MiB
+constexpr size_t kNoAllocScratchBytes = size_t(96) << 20;   // 96 MiB
 static __device__ __align__(256) unsigned char g_noalloc_scratch[kNoAllocScratchBytes];
 
 // In host code `g_noalloc_scratch` is only a stand-in symbol, never a device

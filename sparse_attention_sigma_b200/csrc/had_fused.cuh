@@ -64,12 +64,13 @@ struct Cfg {
     static_assert(QT * GROUP_COLS <= TMEM_COLS || QT == 1, "TMEM budget");
     static_assert(O_COL + D <= (QT == 1 ? TMEM_COLS : GROUP_COLS), "TMEM budget");
     // shared memory layout (offsets from a 1024-aligned base)
-    static constexpr int OFF_Q = 0;
-    static constexpr int OFF_K = OFF_Q + QT * QBYTES;
+    static constexpr int OFF_Q = 0;                       // Q as +/-1 (pass 1)
+    static constexpr int OFF_Q2 = OFF_Q + QT * QBYTES;     // Q as +/-64 (pass 2)
+    static constexpr int OFF_K = OFF_Q2 + QT * QBYTES;
     static constexpr int OFF_V = OFF_K + KSTAGES * KBYTES;
     static constexpr int OFF_HIST = OFF_V + VSTAGES * VBYTES;
     static constexpr int OFF_BAR = OFF_HIST + QT * HIST_BYTES;
-    static constexpr int NBARS = 1 + 2 * KSTAGES + 2 * VSTAGES + QT * 9 + 1;
+    static constexpr int NBARS = 1 + 2 * KSTAGES + 2 * VSTAGES + 9 + 1;
     static constexpr int OFF_MISC = OFF_BAR + NBARS * 8;
     static constexpr int SMEM_BYTES = OFF_MISC + 16 + 1024;   // + alignment slack
     static constexpr uint32_t IDESC_QK = tc::idesc(2, 1, 1, kRows, kKeys);   // s32 <- s8 x s8
@@ -77,8 +78,9 @@ struct Cfg {
 };
 
 struct Params {
-    const int8_t *qop;        // [BH][qtiles] 128 x D int8 tiles (+/-16)
-    const int8_t *kop;        // [BH][ktiles] 64 x D int8 tiles (+/-16)
+    const int8_t *qop;        // [BH][qtiles] 128 x D int8 tiles (+/-1)
+    const int8_t *qop2;       // [BH][qtiles] 128 x D int8 tiles (+/-64)
+    const int8_t *kop;        // [BH][ktiles] 64 x D int8 tiles (+/-4)
     const __half *vop;        // [BH][ktiles] D x 64 fp16 tiles (V^T, scaled)
     const int *vexp;          // [BH] power of two of the V scale
     float *out;               // [BH][n][D]
@@ -99,13 +101,14 @@ struct Bars {
     uint64_t *q_full;
     uint64_t *k_full, *k_empty;     // [KSTAGES]
     uint64_t *v_full, *v_empty;     // [VSTAGES]
-    uint64_t *grp;                  // [QT][9]: s_full[2] s_empty[2] p_full[2] p_empty[2] o_full
+    // shared by all query tiles of the CTA:
+    uint64_t *grp;                  // s_full[2] s_empty[2] p_full[2] p_empty[2] o_full
     uint64_t *drain;
-    __device__ uint64_t *s_full(int g, int b) const { return grp + g * 9 + b; }
-    __device__ uint64_t *s_empty(int g, int b) const { return grp + g * 9 + 2 + b; }
-    __device__ uint64_t *p_full(int g, int b) const { return grp + g * 9 + 4 + b; }
-    __device__ uint64_t *p_empty(int g, int b) const { return grp + g * 9 + 6 + b; }
-    __device__ uint64_t *o_full(int g) const { return grp + g * 9 + 8; }
+    __device__ uint64_t *s_full(int b) const { return grp + b; }
+    __device__ uint64_t *s_empty(int b) const { return grp + 2 + b; }
+    __device__ uint64_t *p_full(int b) const { return grp + 4 + b; }
+    __device__ uint64_t *p_empty(int b) const { return grp + 6 + b; }
+    __device__ uint64_t *o_full() const { return grp + 8; }
 };
 
 // Bounded wait: false if the deadline passed or another role aborted.
@@ -129,6 +132,13 @@ __device__ __forceinline__ bool wait_bar(uint64_t *bar, uint32_t parity, uint64_
 __device__ __forceinline__ void red_add1(uint32_t saddr)
 {
     asm volatile("red.shared.add.u32 [%0], %1;" ::"r"(saddr), "r"(1u) : "memory");
+}
+
+__device__ __forceinline__ float lds_f32(uint32_t saddr)
+{
+    float v;
+    asm volatile("ld.shared.f32 %0, [%1];" : "=f"(v) : "r"(saddr) : "memory");
+    return v;
 }
 
 __device__ __forceinline__ float ex2(float x)
@@ -174,7 +184,7 @@ attention_fwd_kernel(const Params p)
     b.v_full = b.k_empty + C::KSTAGES;
     b.v_empty = b.v_full + C::VSTAGES;
     b.grp = b.v_empty + C::VSTAGES;
-    b.drain = b.grp + QT * 9;
+    b.drain = b.grp + 9;
     uint32_t *tmem_holder = reinterpret_cast<uint32_t *>(smem + C::OFF_MISC);
     volatile int *abort_flag = reinterpret_cast<volatile int *>(smem + C::OFF_MISC + 4);
 
@@ -195,15 +205,13 @@ attention_fwd_kernel(const Params p)
             tc::mbar_init(b.v_full + s, 1);
             tc::mbar_init(b.v_empty + s, 1);
         }
-        for (int g = 0; g < QT; ++g) {
-            for (int s = 0; s < 2; ++s) {
-                tc::mbar_init(b.s_full(g, s), 1);
-                tc::mbar_init(b.s_empty(g, s), kRows);
-                tc::mbar_init(b.p_full(g, s), kRows);
-                tc::mbar_init(b.p_empty(g, s), 1);
-            }
-            tc::mbar_init(b.o_full(g), 1);
+        for (int s = 0; s < 2; ++s) {
+            tc::mbar_init(b.s_full(s), 1);
+            tc::mbar_init(b.s_empty(s), 4 * QT);        // one arrive per epilogue warp
+            tc::mbar_init(b.p_full(s), 4 * QT);
+            tc::mbar_init(b.p_empty(s), 1);
         }
+        tc::mbar_init(b.o_full(), 1);
         tc::mbar_init(b.drain, 1);
         *abort_flag = 0;
         tc::fence_mbar_init();
@@ -221,8 +229,10 @@ attention_fwd_kernel(const Params p)
             const int8_t *ksrc = p.kop + head * (long long)T * C::KBYTES;
             const uint8_t *vsrc = reinterpret_cast<const uint8_t *>(p.vop) +
                                   head * (long long)T * C::VBYTES;
-            tc::mbar_expect_tx(b.q_full, QT * C::QBYTES);
+            const int8_t *qsrc2 = p.qop2 + (head * p.qtiles + qtile0) * (long long)C::QBYTES;
+            tc::mbar_expect_tx(b.q_full, 2 * QT * C::QBYTES);
             tc::bulk_g2s(smem + C::OFF_Q, qsrc, QT * C::QBYTES, b.q_full);
+            tc::bulk_g2s(smem + C::OFF_Q2, qsrc2, QT * C::QBYTES, b.q_full);
             int issued_k = 0, issued_v = 0;
             bool ok = true;
             for (int u = 0; u < 2 * T && ok; ++u) {
@@ -262,55 +272,56 @@ attention_fwd_kernel(const Params p)
     } else if (warp == 1) {
         // ------------------------------------------------------------ MMA issuer
         if (lane == 0) {
-            const uint32_t q_addr = tc::smem_u32(smem + C::OFF_Q);
-            const uint32_t k_addr = tc::smem_u32(smem + C::OFF_K);
-            const uint32_t v_addr = tc::smem_u32(smem + C::OFF_V);
+            // Descriptors are computed once; a tile or K step moves only the
+            // start-address field (bits 0-13, in 16-byte units).
+            // the two query tiles sit QBYTES apart in both Q buffers
+            const uint64_t dq1 = tc::smem_desc(tc::smem_u32(smem + C::OFF_Q), 128, D * 8);
+            const uint64_t dq2 = tc::smem_desc(tc::smem_u32(smem + C::OFF_Q2), 128, D * 8);
+            const uint64_t dk = tc::smem_desc(tc::smem_u32(smem + C::OFF_K), 128, D * 8);
+            const uint64_t dv = tc::smem_desc(tc::smem_u32(smem + C::OFF_V), 128, 8 * 128);
             bool ok = wait_bar(b.q_full, 0, deadline, abort_flag, p.status);
             tc::fence_after_sync();
             auto pv = [&](int j) -> bool {
                 const int vs = j % C::VSTAGES;
-                if (!wait_bar(b.v_full + vs, (j / C::VSTAGES) & 1, deadline, abort_flag, p.status))
-                    return false;
                 const int pb = j & 1;
+                if (!wait_bar(b.v_full + vs, (j / C::VSTAGES) & 1, deadline, abort_flag, p.status) ||
+                    !wait_bar(b.p_full(pb), (j >> 1) & 1, deadline, abort_flag, p.status))
+                    return false;
+                tc::fence_after_sync();
+                const uint64_t dvs = dv + (uint64_t)((vs * C::VBYTES) >> 4);
+#pragma unroll
                 for (int g = 0; g < QT; ++g) {
-                    if (!wait_bar(b.p_full(g, pb), (j >> 1) & 1, deadline, abort_flag, p.status))
-                        return false;
-                    tc::fence_after_sync();
                     const uint32_t gcol = g * C::GROUP_COLS;
 #pragma unroll
-                    for (int kk = 0; kk < kKeys / 16; ++kk) {
-                        const uint64_t bdesc =
-                            tc::smem_desc(v_addr + vs * C::VBYTES + kk * 256, 128, 8 * 128);
+                    for (int kk = 0; kk < kKeys / 16; ++kk)
                         tc::mma_f16_ts(tmem + gcol + C::O_COL,
-                                       tmem + gcol + C::P_COL + pb * 32 + kk * 8, bdesc,
-                                       C::IDESC_PV, (j > 0 || kk > 0) ? 1u : 0u);
-                    }
-                    tc::mma_commit(b.p_empty(g, pb));
+                                       tmem + gcol + C::P_COL + pb * 32 + kk * 8,
+                                       dvs + (uint64_t)(kk * 16), C::IDESC_PV,
+                                       (j > 0 || kk > 0) ? 1u : 0u);
                 }
+                tc::mma_commit(b.p_empty(pb));
                 tc::mma_commit(b.v_empty + vs);
                 return true;
             };
             auto qk = [&](int u) -> bool {
                 const int ks = u % C::KSTAGES;
-                if (!wait_bar(b.k_full + ks, (u / C::KSTAGES) & 1, deadline, abort_flag, p.status))
-                    return false;
                 const int sb = u & 1;
+                if (!wait_bar(b.k_full + ks, (u / C::KSTAGES) & 1, deadline, abort_flag, p.status) ||
+                    !wait_bar(b.s_empty(sb), ((u >> 1) & 1) ^ 1, deadline, abort_flag, p.status))
+                    return false;
+                tc::fence_after_sync();
+                const uint64_t dks = dk + (uint64_t)((ks * C::KBYTES) >> 4);
+                const uint64_t dqp = u < T ? dq1 : dq2;
+#pragma unroll
                 for (int g = 0; g < QT; ++g) {
-                    if (!wait_bar(b.s_empty(g, sb), ((u >> 1) & 1) ^ 1, deadline, abort_flag,
-                                  p.status))
-                        return false;
-                    tc::fence_after_sync();
                     const uint32_t scol = g * C::GROUP_COLS + C::S_COL + sb * 64;
 #pragma unroll
-                    for (int kk = 0; kk < D / 32; ++kk) {
-                        const uint64_t adesc =
-                            tc::smem_desc(q_addr + g * C::QBYTES + kk * 256, 128, D * 8);
-                        const uint64_t bdesc =
-                            tc::smem_desc(k_addr + ks * C::KBYTES + kk * 256, 128, D * 8);
-                        tc::mma_i8_ss(tmem + scol, adesc, bdesc, C::IDESC_QK, kk > 0 ? 1u : 0u);
-                    }
-                    tc::mma_commit(b.s_full(g, sb));
+                    for (int kk = 0; kk < D / 32; ++kk)
+                        tc::mma_i8_ss(tmem + scol,
+                                      dqp + (uint64_t)((g * C::QBYTES) >> 4) + (uint64_t)(kk * 16),
+                                      dks + (uint64_t)(kk * 16), C::IDESC_QK, kk > 0 ? 1u : 0u);
                 }
+                tc::mma_commit(b.s_full(sb));
                 tc::mma_commit(b.k_empty + ks);
                 return true;
             };
@@ -329,8 +340,7 @@ attention_fwd_kernel(const Params p)
                 const int last = (T - 1) & ~1;            // first tile of the last pair
                 for (int i = last; i < T && ok; ++i) ok = pv(i);
             }
-            if (ok)
-                for (int g = 0; g < QT; ++g) tc::mma_commit(b.o_full(g));
+            if (ok) tc::mma_commit(b.o_full());
             // drain: wait until every MMA this thread issued has completed
             tc::mma_commit(b.drain);
             volatile int never = 0;
@@ -365,7 +375,7 @@ attention_fwd_kernel(const Params p)
         auto load_tiles = [&](int u, int cnt) -> bool {
             for (int k = 0; k < cnt; ++k) {
                 const int uk = u + k;
-                if (!__all_sync(kFullMask, wait_bar(b.s_full(g, uk & 1), (uk >> 1) & 1,
+                if (!__all_sync(kFullMask, wait_bar(b.s_full(uk & 1), (uk >> 1) & 1,
                                                     deadline, abort_flag, p.status)))
                     return false;
             }
@@ -381,7 +391,9 @@ attention_fwd_kernel(const Params p)
             }
             tc::tmem_wait_ld();
             tc::fence_before_sync();
-            for (int k = 0; k < cnt; ++k) tc::mbar_arrive(b.s_empty(g, (u + k) & 1));
+            __syncwarp();
+            if (lane == 0)
+                for (int k = 0; k < cnt; ++k) tc::mbar_arrive(b.s_empty((u + k) & 1));
             return true;
         };
 
@@ -393,21 +405,26 @@ attention_fwd_kernel(const Params p)
                 if (decltype(full)::value || c < valid) red_add1(hbase - (s[O + c] << 6));
         };
         // pass 1b: four cumulative 8-bit window counters in one register
-        uint32_t acc = 0;
+        // four independent counter registers keep the adds off one chain
+        uint32_t acc[4] = {0u, 0u, 0u, 0u};
         int tot0 = 0, tot1 = 0, tot2 = 0, tot3 = 0;
         int cshift = 0, L0 = 0, hmin = C::BINS - 1;
         auto flush = [&]() {
-            tot0 += (int)(acc & 0xFFu);
-            tot1 += (int)((acc >> 8) & 0xFFu);
-            tot2 += (int)((acc >> 16) & 0xFFu);
-            tot3 += (int)(acc >> 24);
-            acc = 0;
+#pragma unroll
+            for (int a = 0; a < 4; ++a) {
+                tot0 += (int)(acc[a] & 0xFFu);
+                tot1 += (int)((acc[a] >> 8) & 0xFFu);
+                tot2 += (int)((acc[a] >> 16) & 0xFFu);
+                tot3 += (int)(acc[a] >> 24);
+                acc[a] = 0u;
+            }
         };
         auto window_tile = [&](auto off, auto full, int valid) {
             constexpr int O = decltype(off)::value;
 #pragma unroll
             for (int c = 0; c < 64; ++c)
-                if (decltype(full)::value || c < valid) acc += window_inc(cshift - (int)s[O + c]);
+                if (decltype(full)::value || c < valid)
+                    acc[c & 3] += window_inc(cshift - (int)s[O + c]);
         };
         // Window from the sample: est = the level of the sample's
         // (N * sampled / n)-th best key.  Levels L0 = est - 1 .. est + 1 are
@@ -480,17 +497,24 @@ attention_fwd_kernel(const Params p)
             p.miss_rows[slot] = (int)(head * p.n + row);
         }
         // missed rows keep nothing here; the fix-up kernel rewrites them
-        const int vt = miss ? 4 * (D + 2) : 4 * (D - 2 * t);
-        if (miss) quota = 0;
-        // softmax reference: the sample's best logit, raised if needed so that
-        // no weight can exceed the fp16 range (s <= D)
-        const float c2q = p.c2 * 0.25f;               // exponent per unit of v
-        const int headroom = c2q > 1.0e-6f ? (int)fminf(floorf(15.99f / c2q), 1.0e6f) : 1000000;
-        const int ref = max(4 * (D - 2 * hmin), 4 * D - headroom);
-        const float k0 = -fmaf((float)ref, c2q, 0.0f) - 12582912.0f * c2q;
+        if (miss) { t = -1; quota = 0; }
+        // Softmax reference: the sample's best logit, raised if needed so that
+        // no weight can exceed the fp16 range (s <= D).  The histogram column
+        // becomes the row's weight table: level l holds exp2(c2 (s_l - ref))
+        // for l <= t and 0 beyond the threshold, so pass 2 reads a logit's
+        // weight with one shared load at the same address its histogram bin
+        // had.
+        {
+            const int headroom = p.c2 > 1.0e-6f ? (int)fminf(floorf(15.99f / p.c2), 1.0e6f) : 1000000;
+            const int ref = max(D - 2 * hmin, D - headroom);
+            for (int bin = 0; bin < C::BINS; ++bin)
+                hcol[bin * kRows] =
+                    bin <= t ? __float_as_uint(ex2(p.c2 * (float)(D - 2 * bin - ref))) : 0u;
+        }
+        const uint32_t vt = 256u * (uint32_t)(D - 2 * t);   // accumulator value of the threshold
         int rem = quota;                              // ties still to keep
         int kept = 0;
-        float Z = 0.0f;
+        float zacc[4] = {0.0f, 0.0f, 0.0f, 0.0f};
         const long long obase = ((head * p.n) + row) * (long long)p.N;
 
         // pass 2: P = kept weights (fp16) -> TMEM; the MMA warp does O += P V
@@ -502,18 +526,19 @@ attention_fwd_kernel(const Params p)
                 float w2[2];
 #pragma unroll
                 for (int e = 0; e < 2; ++e) {
-                    const int v = (int)s[O + c + e];
+                    const uint32_t v = s[O + c + e];          // 256 s
                     const bool in = decltype(full)::value || (c + e) < valid;
-                    const bool tie = in && (v == vt);
-                    const bool keep = in && ((v > vt) || (tie && rem > 0));
+                    float w = lds_f32(hbase - v);            // 0 below the threshold
+                    const bool tie = (v == vt);
+                    const bool drop = !in || (tie && rem <= 0);
                     rem -= tie ? 1 : 0;
-                    const float w = keep ? weight_of(v, c2q, k0) : 0.0f;
-                    Z += w;
+                    w = drop ? 0.0f : w;
+                    zacc[e + (c & 2)] += w;
                     w2[e] = w;
                     if (kDbg) {
-                        if (keep && active) {
+                        if (active && !drop && ((int)v > (int)vt || tie)) {
                             if (p.dbg_idx) p.dbg_idx[obase + kept] = j * kKeys + c + e;
-                            if (p.dbg_logits) p.dbg_logits[obase + kept] = (int16_t)(v / 4);
+                            if (p.dbg_logits) p.dbg_logits[obase + kept] = (int16_t)((int)v / 256);
                             ++kept;
                         }
                     }
@@ -526,7 +551,7 @@ attention_fwd_kernel(const Params p)
         for (int j = 0; j < T && ok; ++j) {
             ok = load_tiles(T + j, 1);
             if (!ok) break;
-            ok = __all_sync(kFullMask, wait_bar(b.p_empty(g, j & 1), ((j >> 1) & 1) ^ 1, deadline,
+            ok = __all_sync(kFullMask, wait_bar(b.p_empty(j & 1), ((j >> 1) & 1) ^ 1, deadline,
                                                 abort_flag, p.status));
             if (!ok) break;
             const int valid = min(kKeys, p.n - j * kKeys);
@@ -534,12 +559,14 @@ attention_fwd_kernel(const Params p)
             else pass2_tile(j, I0{}, BF{}, valid);
             tc::tmem_wait_st();
             tc::fence_before_sync();
-            tc::mbar_arrive(b.p_full(g, j & 1));
+            __syncwarp();
+            if (lane == 0) tc::mbar_arrive(b.p_full(j & 1));
         }
+        float Z = (zacc[0] + zacc[1]) + (zacc[2] + zacc[3]);
         if (!(Z > 0.0f)) Z = 1.0f;                    // missed or inactive rows only
 
         // output: O / Z * 2^e_h
-        if (ok) ok = __all_sync(kFullMask, wait_bar(b.o_full(g), 0, deadline, abort_flag, p.status));
+        if (ok) ok = __all_sync(kFullMask, wait_bar(b.o_full(), 0, deadline, abort_flag, p.status));
         if (ok) {
             tc::fence_after_sync();
             const float scale = ldexpf(1.0f, p.vexp[head]) / Z;

@@ -7,13 +7,15 @@
 // 128 bytes apart, row groups (8 rows) (K bytes / 16) * 128 bytes apart.
 // Tiles are stored contiguously so the kernel moves each with one bulk copy.
 //
-//   Qop [BH][qtiles] tiles of 128 rows x d int8 (+4 / -4, 0 padding;
-//                    qtiles >= ceil(n/128), the extra tiles all padding)
-//   Kop [BH][ceil(n/64)] tiles of 64 keys x d int8 (+1 / -1, 0 padding)
+//   Qop1, Qop2 [BH][qtiles] tiles of 128 rows x d int8: the signs as +/-1
+//                    and as +/-64 (0 padding; qtiles >= ceil(n/128), the
+//                    extra tiles all padding)
+//   Kop [BH][ceil(n/64)] tiles of 64 keys x d int8 (+4 / -4, 0 padding)
 //   Qbits, Kbits [BH][n][d/32] the same signs bit-packed (1 = -1)
-// The +/-4 x +/-1 scaling makes the s32 accumulator hold 4 * s, which the
-// fused kernel turns into histogram addresses and counter shifts with one
-// integer add.
+// With K as +/-4 the s32 accumulator holds 4 s against Qop1 (the counter
+// shifts of the fused kernel's first pass are one integer add away) and
+// 256 s against Qop2 (the byte offset of the logit's level in its per-row
+// tables, again one integer add away).
 //   Vop [BH][ceil(n/64)]  tiles of V^T: d rows x 64 keys fp16, scaled by
 //                         2^-e_h so the head's largest |v| lies in
 //                         [2^14, 2^15) (bf16 -> fp16 then loses no bits for
@@ -43,12 +45,13 @@ __device__ __forceinline__ uint32_t core_offset(uint32_t row, uint32_t kbyte, ui
 // Works for Q (tile 128) and K (tile 64): `tile_rows` selects the tiling.
 // The packed copy is written as 16-bit halves: chunk kc of a row is bits
 // 16*(kc%2) .. 16*(kc%2)+15 of word kc/2.
+// `op2` (may be null) receives a second copy with the codes pos2 / neg2.
 template <typename T>
 __global__ void __launch_bounds__(256)
 sign_operand_kernel(const T *__restrict__ x, const float *__restrict__ sigma, int H, int n,
                     int d, int tile_rows, int tiles, long long chunks, uint32_t pos,
-                    uint32_t neg, int8_t *__restrict__ op, uint16_t *__restrict__ bits,
-                    int32_t *status)
+                    uint32_t neg, int8_t *__restrict__ op, uint32_t pos2, uint32_t neg2,
+                    int8_t *__restrict__ op2, uint16_t *__restrict__ bits, int32_t *status)
 {
     const int cpr = d >> 4;                                  // chunks per row
     const long long padded_rows = (long long)tiles * tile_rows;
@@ -58,7 +61,7 @@ sign_operand_kernel(const T *__restrict__ x, const float *__restrict__ sigma, in
         const int kc = (int)(c % cpr);
         const long long head = prow / padded_rows;
         const int r = (int)(prow % padded_rows);             // row within the head
-        uint4 out = make_uint4(0, 0, 0, 0);
+        uint4 out = make_uint4(0, 0, 0, 0), out2 = make_uint4(0, 0, 0, 0);
         if (r < n) {
             const SignRule rule = sign_rule(__ldg(sigma + (head % H)));
             if (rule.bad) flag(status, HAD_ERR_BAD_SIGMA);
@@ -68,26 +71,33 @@ sign_operand_kernel(const T *__restrict__ x, const float *__restrict__ sigma, in
             float (&hi)[8] = *reinterpret_cast<float(*)[8]>(v + 8);
             Load8<T>::run(src, lo);
             Load8<T>::run(src + 8, hi);
-            uint32_t w[4];
+            uint32_t w[4], w2[4];
             uint32_t packed = 0;
 #pragma unroll
             for (int q = 0; q < 4; ++q) {
-                uint32_t word = 0;
+                uint32_t word = 0, word2 = 0;
 #pragma unroll
                 for (int b = 0; b < 4; ++b) {
                     const uint32_t nb = negative_bit(v[4 * q + b], rule);
                     word |= (nb ? neg : pos) << (8 * b);
+                    word2 |= (nb ? neg2 : pos2) << (8 * b);
                     packed |= nb << (4 * q + b);
                 }
                 w[q] = word;
+                w2[q] = word2;
             }
             out = make_uint4(w[0], w[1], w[2], w[3]);
+            out2 = make_uint4(w2[0], w2[1], w2[2], w2[3]);
             bits[(head * n + r) * (long long)cpr + kc] = (uint16_t)packed;
         }
         const int t = r / tile_rows;
         const uint32_t rr = (uint32_t)(r % tile_rows);
         int8_t *tile = op + ((head * tiles + t) * (long long)tile_rows * d);
         *reinterpret_cast<uint4 *>(tile + core_offset(rr, kc * 16, d)) = out;
+        if (op2) {
+            int8_t *tile2 = op2 + ((head * tiles + t) * (long long)tile_rows * d);
+            *reinterpret_cast<uint4 *>(tile2 + core_offset(rr, kc * 16, d)) = out2;
+        }
     }
 }
 
