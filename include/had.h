@@ -72,7 +72,9 @@ typedef enum {
     HAD_OP_BINARIZE_PACK = 0,     /* had_binarize_pack */
     HAD_OP_HAMMING_TOPN = 1,      /* had_hamming_topn */
     HAD_OP_ATTENTION_FWD = 2,     /* had_attention_fwd */
-    HAD_OP_SPARSE_SOFTMAX_AV = 3  /* had_sparse_softmax_av */
+    HAD_OP_SPARSE_SOFTMAX_AV = 3, /* had_sparse_softmax_av */
+    HAD_OP_ATTENTION_PREPARE = 4, /* had_attention_prepare */
+    HAD_OP_ATTENTION_CORE = 5     /* had_attention_core */
 } had_op_t;
 
 /*
@@ -136,6 +138,26 @@ HAD_API had_status_t had_attention_fwd(const void *Q, const void *K, const void 
                                float *out, int32_t *dbg_idx, int16_t *dbg_logits,
                                void *ws, size_t ws_bytes,
                                int32_t *dev_status, cudaStream_t stream);
+
+/*
+ * had_attention_fwd in two stages sharing one workspace (same size as
+ * had_attention_fwd's): had_attention_prepare standardizes and signs Q and K
+ * into tensor-core operand tiles and packed bits and converts V, and
+ * had_attention_core runs the fused kernel (and the exact recomputation of
+ * any row whose threshold fell outside its sampled window) on them.  The
+ * two in order on one stream compute exactly what had_attention_fwd does;
+ * core reads only the workspace and V.  Arguments as had_attention_fwd.
+ */
+HAD_API had_status_t had_attention_prepare(const void *Q, const void *K, const void *V,
+                                           had_dtype_t dt, const float *sigma_q,
+                                           const float *sigma_k, int B, int H, int n, int d,
+                                           int N, void *ws, size_t ws_bytes,
+                                           int32_t *dev_status, cudaStream_t stream);
+
+HAD_API had_status_t had_attention_core(const void *V, had_dtype_t dt, int B, int H, int n,
+                                        int d, int N, float tau, float *out, int32_t *dbg_idx,
+                                        int16_t *dbg_logits, void *ws, size_t ws_bytes,
+                                        int32_t *dev_status, cudaStream_t stream);
 
 /*
  * had_attention_fwd for callers that cannot allocate device memory.

@@ -150,13 +150,13 @@ FwdWorkspace fwd_layout(int B, int H, int n, int d, int N)
     return w;
 }
 
+// Operand preparation: Q/K signs as tensor-core tiles and packed bits,
+// V^T in fp16 with its per-head scale.
 template <typename T, int D>
-had_status_t launch_fused_typed(const T *Q, const T *K, const T *V, const float *sq,
-                                const float *sk, int B, int H, int n, int N, float tau,
-                                float *out, int32_t *dbg_idx, int16_t *dbg_lg, char *ws,
-                                const FwdWorkspace &w, int32_t *status, cudaStream_t st)
+had_status_t prep_typed(const T *Q, const T *K, const T *V, const float *sq, const float *sk,
+                        int B, int H, int n, char *ws, const FwdWorkspace &w, int32_t *status,
+                        cudaStream_t st)
 {
-    using C = had::fused::Cfg<D>;
     const long long bh = (long long)B * H;
     auto *qop = reinterpret_cast<int8_t *>(ws + w.qop);
     auto *qop2 = reinterpret_cast<int8_t *>(ws + w.qop2);
@@ -165,9 +165,8 @@ had_status_t launch_fused_typed(const T *Q, const T *K, const T *V, const float 
     auto *qbits = reinterpret_cast<uint32_t *>(ws + w.qbits);
     auto *kbits = reinterpret_cast<uint32_t *>(ws + w.kbits);
     auto *vmax = reinterpret_cast<unsigned int *>(ws + w.vmax);
-    auto *miss_count = reinterpret_cast<int *>(ws + w.vmax) + bh;
     auto *vexp = reinterpret_cast<int *>(ws + w.vexp);
-    auto *miss_rows = reinterpret_cast<int *>(ws + w.miss_rows);
+    // vmax[BH] and the miss counter that follows it start at zero
     if (cudaMemsetAsync(vmax, 0, (bh + 1) * 4, st) != cudaSuccess) return HAD_ERR_CUDA;
     const long long qchunks = bh * w.qtiles * had::fused::kRows * (D / 16);
     const long long kchunks = bh * w.ktiles * had::fused::kKeys * (D / 16);
@@ -185,26 +184,39 @@ had_status_t launch_fused_typed(const T *Q, const T *K, const T *V, const float 
                                                                       chunks, vmax);
     had::prep::v_operand_kernel<T, D><<<(unsigned)(bh * w.ktiles), 256, 0, st>>>(
         V, n, vmax, vop, vexp);
-    had_status_t s = launched();
-    if (s != HAD_OK) return s;
+    return launched();
+}
+
+// The fused kernel on prepared operands, then the exact fix-up of the rows
+// whose threshold fell outside the sampled window.
+template <typename T, int D>
+had_status_t core_typed(const T *V, int B, int H, int n, int N, float tau, float *out,
+                        int32_t *dbg_idx, int16_t *dbg_lg, char *ws, const FwdWorkspace &w,
+                        int32_t *status, cudaStream_t st)
+{
+    using C = had::fused::Cfg<D>;
+    const long long bh = (long long)B * H;
     const bool dbg = dbg_idx != nullptr || dbg_lg != nullptr;
     auto kernel = dbg ? had::fused::attention_fwd_kernel<D, true>
                       : had::fused::attention_fwd_kernel<D, false>;
     if (cudaFuncSetAttribute(kernel, cudaFuncAttributeMaxDynamicSharedMemorySize,
                              C::SMEM_BYTES) != cudaSuccess)
         return HAD_ERR_CUDA;
+    auto *qbits = reinterpret_cast<uint32_t *>(ws + w.qbits);
+    auto *kbits = reinterpret_cast<uint32_t *>(ws + w.kbits);
+    auto *miss_count = reinterpret_cast<int *>(ws + w.vmax) + bh;
     had::fused::Params p;
-    p.qop = qop;
-    p.qop2 = qop2;
-    p.kop = kop;
-    p.vop = vop;
-    p.vexp = vexp;
+    p.qop = reinterpret_cast<int8_t *>(ws + w.qop);
+    p.qop2 = reinterpret_cast<int8_t *>(ws + w.qop2);
+    p.kop = reinterpret_cast<int8_t *>(ws + w.kop);
+    p.vop = reinterpret_cast<__half *>(ws + w.vop);
+    p.vexp = reinterpret_cast<int *>(ws + w.vexp);
     p.out = out;
     p.dbg_idx = dbg_idx;
     p.dbg_logits = dbg_lg;
     p.status = status;
     p.miss_count = miss_count;
-    p.miss_rows = miss_rows;
+    p.miss_rows = reinterpret_cast<int *>(ws + w.miss_rows);
     p.sample_tiles = w.ktiles / 16 > 4 ? w.ktiles / 16 : 4;
     p.n = n;
     p.N = N;
@@ -215,8 +227,19 @@ had_status_t launch_fused_typed(const T *Q, const T *K, const T *V, const float 
     const long long blocks = bh * p.ctas_per_head;
     kernel<<<(unsigned)blocks, C::THREADS, C::SMEM_BYTES, st>>>(p);
     had::fused::fixup_rows_kernel<T, D><<<148 * 4, 256, 0, st>>>(
-        qbits, kbits, V, n, N, tau, miss_count, miss_rows, out, dbg_idx, dbg_lg);
+        qbits, kbits, V, n, N, tau, miss_count, p.miss_rows, out, dbg_idx, dbg_lg);
     return launched();
+}
+
+template <typename T, int D>
+had_status_t launch_fused_typed(const T *Q, const T *K, const T *V, const float *sq,
+                                const float *sk, int B, int H, int n, int N, float tau,
+                                float *out, int32_t *dbg_idx, int16_t *dbg_lg, char *ws,
+                                const FwdWorkspace &w, int32_t *status, cudaStream_t st)
+{
+    had_status_t s = prep_typed<T, D>(Q, K, V, sq, sk, B, H, n, ws, w, status, st);
+    if (s != HAD_OK) return s;
+    return core_typed<T, D>(V, B, H, n, N, tau, out, dbg_idx, dbg_lg, ws, w, status, st);
 }
 
 template <typename T>
@@ -336,6 +359,66 @@ had_status_t had_attention_fwd(const void *Q, const void *K, const void *V, had_
                                dbg_logits, base, w, dev_status, stream);
 }
 
+had_status_t had_attention_prepare(const void *Q, const void *K, const void *V, had_dtype_t dt,
+                                   const float *sigma_q, const float *sigma_k, int B, int H,
+                                   int n, int d, int N, void *ws, size_t ws_bytes,
+                                   int32_t *dev_status, cudaStream_t stream)
+{
+    had_status_t s = check_topn(B, H, n, d, N);
+    if (s != HAD_OK) return s;
+    if (dt != HAD_BF16 && dt != HAD_F32) return HAD_ERR_INVALID_ARG;
+    if (!Q || !K || !V || !sigma_q || !sigma_k) return HAD_ERR_INVALID_ARG;
+    if (!aligned16(Q) || !aligned16(K) || !aligned16(V)) return HAD_ERR_INVALID_ARG;
+    const FwdWorkspace w = fwd_layout(B, H, n, d, N);
+    if (!ws || ws_bytes < w.total || !aligned16(ws)) return HAD_ERR_WORKSPACE;
+    if ((long long)B * H * w.qtiles > INT_MAX) return HAD_ERR_UNSUPPORTED;
+    char *base = static_cast<char *>(ws);
+    if (dt == HAD_BF16) {
+        const auto *q = static_cast<const __nv_bfloat16 *>(Q), *k = static_cast<const __nv_bfloat16 *>(K),
+                   *v = static_cast<const __nv_bfloat16 *>(V);
+        return d == 64 ? prep_typed<__nv_bfloat16, 64>(q, k, v, sigma_q, sigma_k, B, H, n, base, w,
+                                                       dev_status, stream)
+                       : prep_typed<__nv_bfloat16, 128>(q, k, v, sigma_q, sigma_k, B, H, n, base,
+                                                        w, dev_status, stream);
+    }
+    const auto *q = static_cast<const float *>(Q), *k = static_cast<const float *>(K),
+               *v = static_cast<const float *>(V);
+    return d == 64 ? prep_typed<float, 64>(q, k, v, sigma_q, sigma_k, B, H, n, base, w,
+                                           dev_status, stream)
+                   : prep_typed<float, 128>(q, k, v, sigma_q, sigma_k, B, H, n, base, w,
+                                            dev_status, stream);
+}
+
+had_status_t had_attention_core(const void *V, had_dtype_t dt, int B, int H, int n, int d, int N,
+                                float tau, float *out, int32_t *dbg_idx, int16_t *dbg_logits,
+                                void *ws, size_t ws_bytes, int32_t *dev_status,
+                                cudaStream_t stream)
+{
+    had_status_t s = check_topn(B, H, n, d, N);
+    if (s != HAD_OK) return s;
+    if (dt != HAD_BF16 && dt != HAD_F32) return HAD_ERR_INVALID_ARG;
+    if (!V || !out || !aligned16(V) || !aligned16(out) || (dbg_idx && !aligned16(dbg_idx)) ||
+        (dbg_logits && !aligned16(dbg_logits)))
+        return HAD_ERR_INVALID_ARG;
+    if (!(tau >= 0.0f) || tau > 3.0e38f) return HAD_ERR_INVALID_ARG;
+    const FwdWorkspace w = fwd_layout(B, H, n, d, N);
+    if (!ws || ws_bytes < w.total || !aligned16(ws)) return HAD_ERR_WORKSPACE;
+    if ((long long)B * H * w.qtiles > INT_MAX) return HAD_ERR_UNSUPPORTED;
+    char *base = static_cast<char *>(ws);
+    if (dt == HAD_BF16) {
+        const auto *v = static_cast<const __nv_bfloat16 *>(V);
+        return d == 64 ? core_typed<__nv_bfloat16, 64>(v, B, H, n, N, tau, out, dbg_idx, dbg_logits,
+                                                       base, w, dev_status, stream)
+                       : core_typed<__nv_bfloat16, 128>(v, B, H, n, N, tau, out, dbg_idx,
+                                                        dbg_logits, base, w, dev_status, stream);
+    }
+    const auto *v = static_cast<const float *>(V);
+    return d == 64 ? core_typed<float, 64>(v, B, H, n, N, tau, out, dbg_idx, dbg_logits, base, w,
+                                           dev_status, stream)
+                   : core_typed<float, 128>(v, B, H, n, N, tau, out, dbg_idx, dbg_logits, base, w,
+                                            dev_status, stream);
+}
+
 had_status_t had_attention_fwd_noalloc(const void *Q, const void *K, const void *V,
                                        had_dtype_t dt, const float *sigma_q,
                                        const float *sigma_k, int B, int H, int n, int d, int N,
@@ -373,6 +456,8 @@ size_t had_workspace_bytes(int op, int B, int H, int n, int d, int N)
     case HAD_OP_SPARSE_SOFTMAX_AV:
         return check_topn(B, H, n, d, N) == HAD_OK ? 0 : (size_t)-1;
     case HAD_OP_ATTENTION_FWD:
+    case HAD_OP_ATTENTION_PREPARE:
+    case HAD_OP_ATTENTION_CORE:
         if (check_topn(B, H, n, d, N) != HAD_OK) return (size_t)-1;
         return fwd_layout(B, H, n, d, N).total;
     default:
@@ -390,6 +475,10 @@ int had_launch_count(int op, int B, int H, int n, int d, int N)
         return check_topn(B, H, n, d, N) == HAD_OK ? 1 : -1;
     case HAD_OP_ATTENTION_FWD:
         return check_topn(B, H, n, d, N) == HAD_OK ? 6 : -1;
+    case HAD_OP_ATTENTION_PREPARE:
+        return check_topn(B, H, n, d, N) == HAD_OK ? 4 : -1;
+    case HAD_OP_ATTENTION_CORE:
+        return check_topn(B, H, n, d, N) == HAD_OK ? 2 : -1;
     default:
         return -1;
     }

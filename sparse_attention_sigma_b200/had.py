@@ -31,6 +31,8 @@ HAD_OP_BINARIZE_PACK = 0
 HAD_OP_HAMMING_TOPN = 1
 HAD_OP_ATTENTION_FWD = 2
 HAD_OP_SPARSE_SOFTMAX_AV = 3
+HAD_OP_ATTENTION_PREPARE = 4
+HAD_OP_ATTENTION_CORE = 5
 
 
 class HadError(RuntimeError):
@@ -54,6 +56,8 @@ def _load():
                               vp, sz, vp, vp],
         "had_attention_fwd_noalloc": [vp, vp, vp, i32, vp, vp, i32, i32, i32, i32, i32, f32, vp,
                                       vp, vp],
+        "had_attention_prepare": [vp, vp, vp, i32, vp, vp, i32, i32, i32, i32, i32, vp, sz, vp, vp],
+        "had_attention_core": [vp, i32, i32, i32, i32, i32, i32, f32, vp, vp, vp, vp, sz, vp, vp],
     }
     for name, args in sig.items():
         fn = getattr(lib, name)
@@ -219,6 +223,42 @@ def had_attention_fwd(Q, K, V, sigma_q, sigma_k, N, tau, out=None, dbg_idx=None,
                                 _ptr(dbg_idx), _ptr(dbg_logits), _ptr(ws), ws.numel(),
                                 _ptr(dev_status), _stream(stream))
     _check(st, "had_attention_fwd")
+    return out
+
+
+def had_attention_prepare(Q, K, V, sigma_q, sigma_k, N, ws, dev_status=None, stream=None):
+    """First stage of had_attention_fwd: operand tiles and packed bits into ws."""
+    _dev(Q, "Q")
+    B, H, n, d = _shape4(Q, "Q")
+    _dev(K, "K", Q.dtype, (B, H, n, d))
+    _dev(V, "V", Q.dtype, (B, H, n, d))
+    _dev(sigma_q, "sigma_q", torch.float32, (H,))
+    _dev(sigma_k, "sigma_k", torch.float32, (H,))
+    _dev(ws, "ws", torch.uint8)
+    st = _lib.had_attention_prepare(_ptr(Q), _ptr(K), _ptr(V), _dtype_code(Q), _ptr(sigma_q),
+                                    _ptr(sigma_k), B, H, n, d, N, _ptr(ws), ws.numel(),
+                                    _ptr(dev_status), _stream(stream))
+    _check(st, "had_attention_prepare")
+    return ws
+
+
+def had_attention_core(V, N, tau, ws, out=None, dbg_idx=None, dbg_logits=None, dev_status=None,
+                       stream=None):
+    """Second stage of had_attention_fwd: the fused kernel on the prepared ws."""
+    _dev(V, "V")
+    B, H, n, d = _shape4(V, "V")
+    _dev(ws, "ws", torch.uint8)
+    if out is None:
+        out = torch.empty((B, H, n, d), dtype=torch.float32, device=V.device)
+    _dev(out, "out", torch.float32, (B, H, n, d))
+    if dbg_idx is not None:
+        _dev(dbg_idx, "dbg_idx", torch.int32, (B, H, n, N))
+    if dbg_logits is not None:
+        _dev(dbg_logits, "dbg_logits", torch.int16, (B, H, n, N))
+    st = _lib.had_attention_core(_ptr(V), _dtype_code(V), B, H, n, d, N, ctypes.c_float(tau),
+                                 _ptr(out), _ptr(dbg_idx), _ptr(dbg_logits), _ptr(ws),
+                                 ws.numel(), _ptr(dev_status), _stream(stream))
+    _check(st, "had_attention_core")
     return out
 
 

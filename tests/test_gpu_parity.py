@@ -244,3 +244,32 @@ def test_out_of_range_index_flagged(had):
     had.had_sparse_softmax_av(idx, lg, c.gv, c.tau, dev_status=status)
     torch.cuda.synchronize()
     assert status.item() & (1 << had.HAD_ERR_INVALID_ARG)
+
+
+def test_prepare_then_core_equals_fwd(had):
+    c = random_case(2, 3, 700, 64, 90, 15)
+    ref = had.had_attention_fwd(c.gq, c.gk, c.gv, c.gsq, c.gsk, c.N, c.tau)
+    ws = had.workspace(c.B, c.H, c.n, c.d, c.N)
+    had.had_attention_prepare(c.gq, c.gk, c.gv, c.gsq, c.gsk, c.N, ws)
+    out = had.had_attention_core(c.gv, c.N, c.tau, ws)
+    torch.cuda.synchronize()
+    assert torch.equal(out, ref)
+
+
+def test_tau_zero_is_uniform_over_kept(had):
+    c = random_case(1, 2, 300, 64, 40, 16, tau=0.0)
+    idx = torch.empty((1, 2, 300, 40), dtype=torch.int32, device="cuda")
+    out = had.had_attention_fwd(c.gq, c.gk, c.gv, c.gsq, c.gsk, c.N, 0.0, dbg_idx=idx)
+    torch.cuda.synchronize()
+    v = c.v.double()
+    ii = idx.long().cpu()
+    mean = torch.stack([torch.stack([v[0, h, ii[0, h, i]].mean(0) for i in range(300)])
+                        for h in range(2)])[None]
+    assert_close(out.cpu().numpy(), mean.numpy(), "tau = 0")
+
+
+def test_negative_tau_rejected(had):
+    c = random_case(1, 1, 64, 64, 8, 17)
+    with pytest.raises(had.HadError) as e:
+        had.had_attention_fwd(c.gq, c.gk, c.gv, c.gsq, c.gsk, c.N, -0.1)
+    assert e.value.status == had.HAD_ERR_INVALID_ARG
