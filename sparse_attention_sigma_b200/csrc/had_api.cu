@@ -124,8 +124,8 @@ had_status_t launch_av(const int32_t *idx, const int16_t *lg, const void *V, had
 // Workspace of the fused forward: tensor-core operand tiles of Q, K and V^T
 // and the per-head V scale.
 struct FwdWorkspace {
-    size_t qop, qop2, kop, vop, qbits, kbits, vmax, vexp, miss_rows, total;
-    int qtiles, ktiles;
+    size_t qop, qop2, kop, vop, qbits, kbits, vpart, miss, vexp, miss_rows, total;
+    int qtiles, ktiles, vchunks;
 };
 
 FwdWorkspace fwd_layout(int B, int H, int n, int d, int N)
@@ -137,53 +137,43 @@ FwdWorkspace fwd_layout(int B, int H, int n, int d, int N)
     w.qtiles = (n + had::fused::kRows - 1) / had::fused::kRows;
     w.qtiles = (w.qtiles + qt - 1) / qt * qt;
     w.ktiles = (n + had::fused::kKeys - 1) / had::fused::kKeys;
+    // V chunks of 8192 elements for the per-head maximum
+    w.vchunks = (int)(((size_t)n * d + 8191) / 8192);
     w.qop = 0;
     w.qop2 = w.qop + round_up(bh * w.qtiles * had::fused::kRows * d);
     w.kop = w.qop2 + round_up(bh * w.qtiles * had::fused::kRows * d);
     w.vop = w.kop + round_up(bh * w.ktiles * had::fused::kKeys * d);
     w.qbits = w.vop + round_up(bh * w.ktiles * had::fused::kKeys * d * 2);
     w.kbits = w.qbits + round_up(bh * n * (d / 8));
-    w.vmax = w.kbits + round_up(bh * n * (d / 8));
-    w.vexp = w.vmax + round_up((bh + 1) * 4);         // vmax[BH] then the miss counter
+    w.vpart = w.kbits + round_up(bh * n * (d / 8));
+    w.miss = w.vpart + round_up(bh * w.vchunks * 4);
+    w.vexp = w.miss + round_up(4);
     w.miss_rows = w.vexp + round_up(bh * 4);
     w.total = w.miss_rows + round_up(bh * (size_t)w.qtiles * had::fused::kRows * 4);
     return w;
 }
 
-// Operand preparation: Q/K signs as tensor-core tiles and packed bits,
-// V^T in fp16 with its per-head scale.
+// Operand preparation: Q/K signs as tensor-core tiles and packed bits and
+// the V chunk maxima in one launch, then V^T in fp16 with its per-head scale.
 template <typename T, int D>
 had_status_t prep_typed(const T *Q, const T *K, const T *V, const float *sq, const float *sk,
                         int B, int H, int n, char *ws, const FwdWorkspace &w, int32_t *status,
                         cudaStream_t st)
 {
     const long long bh = (long long)B * H;
-    auto *qop = reinterpret_cast<int8_t *>(ws + w.qop);
-    auto *qop2 = reinterpret_cast<int8_t *>(ws + w.qop2);
-    auto *kop = reinterpret_cast<int8_t *>(ws + w.kop);
-    auto *vop = reinterpret_cast<__half *>(ws + w.vop);
-    auto *qbits = reinterpret_cast<uint32_t *>(ws + w.qbits);
-    auto *kbits = reinterpret_cast<uint32_t *>(ws + w.kbits);
-    auto *vmax = reinterpret_cast<unsigned int *>(ws + w.vmax);
-    auto *vexp = reinterpret_cast<int *>(ws + w.vexp);
-    // vmax[BH] and the miss counter that follows it start at zero
-    if (cudaMemsetAsync(vmax, 0, (bh + 1) * 4, st) != cudaSuccess) return HAD_ERR_CUDA;
-    const long long qchunks = bh * w.qtiles * had::fused::kRows * (D / 16);
-    const long long kchunks = bh * w.ktiles * had::fused::kKeys * (D / 16);
+    const long long blocks = bh * (w.qtiles + w.ktiles + w.vchunks);
+    if (blocks > INT_MAX || bh * w.ktiles > INT_MAX) return HAD_ERR_UNSUPPORTED;
+    auto *vpart = reinterpret_cast<float *>(ws + w.vpart);
     // Q as +/-1 and +/-64, K as +/-4: the i8 MMA accumulates 4 s or 256 s
-    had::prep::sign_operand_kernel<T><<<grid_for(qchunks, 256), 256, 0, st>>>(
-        Q, sq, H, n, D, had::fused::kRows, w.qtiles, qchunks, 0x01u, 0xFFu, qop, 0x40u, 0xC0u,
-        qop2, reinterpret_cast<uint16_t *>(qbits), status);
-    had::prep::sign_operand_kernel<T><<<grid_for(kchunks, 256), 256, 0, st>>>(
-        K, sk, H, n, D, had::fused::kKeys, w.ktiles, kchunks, 0x04u, 0xFCu, kop, 0u, 0u,
-        nullptr, reinterpret_cast<uint16_t *>(kbits), status);
-    const long long vgroups_per_head = (long long)n * D / 8;
-    const int chunks = (int)((vgroups_per_head + 4095) / 4096);   // 32 KiB of bf16 per CTA
-    if (bh * chunks > INT_MAX) return HAD_ERR_UNSUPPORTED;
-    had::prep::vmax_kernel<T><<<(unsigned)(bh * chunks), 256, 0, st>>>(V, vgroups_per_head,
-                                                                      chunks, vmax);
+    had::prep::operands_kernel<T, D><<<(unsigned)blocks, 256, 0, st>>>(
+        Q, K, V, sq, sk, H, n, (int)bh, w.qtiles, w.ktiles, w.vchunks,
+        reinterpret_cast<int8_t *>(ws + w.qop), reinterpret_cast<int8_t *>(ws + w.qop2),
+        reinterpret_cast<int8_t *>(ws + w.kop), reinterpret_cast<uint16_t *>(ws + w.qbits),
+        reinterpret_cast<uint16_t *>(ws + w.kbits), vpart, reinterpret_cast<int *>(ws + w.miss),
+        status);
     had::prep::v_operand_kernel<T, D><<<(unsigned)(bh * w.ktiles), 256, 0, st>>>(
-        V, n, vmax, vop, vexp);
+        V, n, vpart, w.vchunks, reinterpret_cast<__half *>(ws + w.vop),
+        reinterpret_cast<int *>(ws + w.vexp));
     return launched();
 }
 
@@ -204,7 +194,7 @@ had_status_t core_typed(const T *V, int B, int H, int n, int N, float tau, float
         return HAD_ERR_CUDA;
     auto *qbits = reinterpret_cast<uint32_t *>(ws + w.qbits);
     auto *kbits = reinterpret_cast<uint32_t *>(ws + w.kbits);
-    auto *miss_count = reinterpret_cast<int *>(ws + w.vmax) + bh;
+    auto *miss_count = reinterpret_cast<int *>(ws + w.miss);
     had::fused::Params p;
     p.qop = reinterpret_cast<int8_t *>(ws + w.qop);
     p.qop2 = reinterpret_cast<int8_t *>(ws + w.qop2);
@@ -474,9 +464,9 @@ int had_launch_count(int op, int B, int H, int n, int d, int N)
     case HAD_OP_SPARSE_SOFTMAX_AV:
         return check_topn(B, H, n, d, N) == HAD_OK ? 1 : -1;
     case HAD_OP_ATTENTION_FWD:
-        return check_topn(B, H, n, d, N) == HAD_OK ? 6 : -1;
-    case HAD_OP_ATTENTION_PREPARE:
         return check_topn(B, H, n, d, N) == HAD_OK ? 4 : -1;
+    case HAD_OP_ATTENTION_PREPARE:
+        return check_topn(B, H, n, d, N) == HAD_OK ? 2 : -1;
     case HAD_OP_ATTENTION_CORE:
         return check_topn(B, H, n, d, N) == HAD_OK ? 2 : -1;
     default:

@@ -14,12 +14,18 @@
 //           register (one shifted add per logit).  That yields the exact
 //           threshold level t and the number q of keys kept at it whenever t
 //           falls inside the window; rows where it does not are listed and
-//           recomputed exactly by fixup_rows_kernel.
-//   pass 2  S again; the thread turns its row into P = exp(tau (s - ref))
-//           for logits above the threshold and for the first q logits at it
-//           (ascending key index: the lower index wins the tie), 0 elsewhere,
-//           sums them into Z, packs P to fp16 pairs in TMEM, and the tensor
-//           core accumulates O += P V (fp16 operands, f32 accumulate).
+//           recomputed exactly by fixup_rows_kernel.  Each tile's counter
+//           word is also kept in TMEM, so the row knows in which tile its
+//           tie quota runs out.
+//   pass 2  S again (Q now +/-64: the accumulator holds 256 s, a byte
+//           offset into the row's weight table); the thread turns its row
+//           into P = exp(tau (s - ref)) for logits above the threshold and
+//           for the first q logits at it (ascending key index: the lower
+//           index wins the tie), 0 elsewhere, sums them into Z, packs P to
+//           fp16 pairs in TMEM, and the tensor core accumulates O += P V
+//           (fp16 operands, f32 accumulate).  Only the sampled tiles and the
+//           tile where some row's quota runs out count ties key by key; in
+//           every other tile one table load gives a key's weight.
 // The n x n logits never leave the SM.
 //
 // Warp roles: warp 0 bulk-copies Q once and K (twice) / V (once) tiles into
@@ -61,6 +67,10 @@ struct Cfg {
     static constexpr uint32_t S_COL = 0;                  // + 64 * buffer: s32, 64 keys
     static constexpr uint32_t P_COL = 128;                // + 32 * buffer: fp16 pairs
     static constexpr uint32_t O_COL = 192;                // f32, D columns
+    // pass 1 only: one word of window counts per key tile, in the P and O
+    // columns (unused until pass 2)
+    static constexpr uint32_t STASH_COL = P_COL;
+    static constexpr int STASH_CAP = (QT == 1 ? O_COL + D : GROUP_COLS) - P_COL;
     static_assert(QT * GROUP_COLS <= TMEM_COLS || QT == 1, "TMEM budget");
     static_assert(O_COL + D <= (QT == 1 ? TMEM_COLS : GROUP_COLS), "TMEM budget");
     // shared memory layout (offsets from a 1024-aligned base)
@@ -274,7 +284,7 @@ attention_fwd_kernel(const Params p)
         if (lane == 0) {
             // Descriptors are computed once; a tile or K step moves only the
             // start-address field (bits 0-13, in 16-byte units).
-            // the two query tiles sit QBYTES apart in both Q buffers
+            // the query tiles sit QBYTES apart in both Q buffers
             const uint64_t dq1 = tc::smem_desc(tc::smem_u32(smem + C::OFF_Q), 128, D * 8);
             const uint64_t dq2 = tc::smem_desc(tc::smem_u32(smem + C::OFF_Q2), 128, D * 8);
             const uint64_t dk = tc::smem_desc(tc::smem_u32(smem + C::OFF_K), 128, D * 8);
@@ -325,20 +335,14 @@ attention_fwd_kernel(const Params p)
                 tc::mma_commit(b.k_empty + ks);
                 return true;
             };
-            // The epilogue consumes S tiles in pairs, so MMAs go in pairs too:
-            // the QK^T of pair k is issued as soon as the epilogue has loaded
-            // pair k-1, before the P V of pair k-1, which waits for its P.
-            for (int pass = 0; pass < 2 && ok; ++pass) {
-                for (int j = 0; j < T && ok; j += 2) {
-                    const int cnt = min(2, T - j);
-                    for (int k = 0; k < cnt && ok; ++k) ok = qk(pass * T + j + k);
-                    if (pass == 1 && j >= 2)
-                        for (int k = 0; k < 2 && ok; ++k) ok = pv(j - 2 + k);
-                }
-            }
-            if (ok) {
-                const int last = (T - 1) & ~1;            // first tile of the last pair
-                for (int i = last; i < T && ok; ++i) ok = pv(i);
+            // The epilogue frees an S buffer half-way through its tile and
+            // hands over P at the end of it, so in pass 2 the QK^T of tile
+            // j + 2 goes before the P V of tile j.
+            for (int u = 0; u < T && ok; ++u) ok = qk(u);
+            for (int u = T; u < T + min(T, 2) && ok; ++u) ok = qk(u);
+            for (int j = 0; j < T && ok; ++j) {
+                if (j + 2 < T) ok = qk(T + j + 2);
+                if (ok) ok = pv(j);
             }
             if (ok) tc::mma_commit(b.o_full());
             // drain: wait until every MMA this thread issued has completed
@@ -362,69 +366,59 @@ attention_fwd_kernel(const Params p)
         // 256 D - 64 v past this row's bin 0.
         const uint32_t hbase = tc::smem_u32(hcol) + 256u * D;
         const int A = min(T, p.sample_tiles);         // tiles counted exactly
+        // Pass 1 keeps one word of window counts per key tile in the TMEM
+        // columns that P and O only use in pass 2; from it each row learns
+        // the one tile where its tie quota runs out, and every other tile of
+        // pass 2 needs no per-key tie bookkeeping.
+        const bool stash_ok = !kDbg && T - A <= C::STASH_CAP;
+        const int fast_from = stash_ok ? A : T;
         bool ok = true;
-        using I0 = std::integral_constant<int, 0>;
-        using I64 = std::integral_constant<int, 64>;
         using BT = std::integral_constant<bool, true>;
         using BF = std::integral_constant<bool, false>;
 
-        // S tiles travel in pairs: both accumulators are waited for, loaded
-        // with one tcgen05.wait::ld and released together, so the load
-        // latency and the MMA round trip are paid once per two tiles.
-        uint32_t s[128];
-        auto load_tiles = [&](int u, int cnt) -> bool {
-            for (int k = 0; k < cnt; ++k) {
-                const int uk = u + k;
-                if (!__all_sync(kFullMask, wait_bar(b.s_full(uk & 1), (uk >> 1) & 1,
-                                                    deadline, abort_flag, p.status)))
-                    return false;
-            }
+        // Each S tile is read in two halves of 32 columns; the load of the
+        // next half is in flight while the current one is processed.
+        uint32_t sa[32], sb[32];
+        auto ld_half = [&](int u, int h, uint32_t (&rr)[32]) {
+            tc::tmem_ld32(lane_base + C::S_COL + (u & 1) * 64 + h * 32, rr);
+        };
+        auto wait_s = [&](int u) -> bool {
+            const bool w = __all_sync(kFullMask, wait_bar(b.s_full(u & 1), (u >> 1) & 1, deadline,
+                                                          abort_flag, p.status));
             tc::fence_after_sync();
-            tc::tmem_ld32(lane_base + C::S_COL + (u & 1) * 64, *reinterpret_cast<uint32_t(*)[32]>(s));
-            tc::tmem_ld32(lane_base + C::S_COL + (u & 1) * 64 + 32,
-                          *reinterpret_cast<uint32_t(*)[32]>(s + 32));
-            if (cnt > 1) {
-                tc::tmem_ld32(lane_base + C::S_COL + ((u + 1) & 1) * 64,
-                              *reinterpret_cast<uint32_t(*)[32]>(s + 64));
-                tc::tmem_ld32(lane_base + C::S_COL + ((u + 1) & 1) * 64 + 32,
-                              *reinterpret_cast<uint32_t(*)[32]>(s + 96));
-            }
-            tc::tmem_wait_ld();
+            return w;
+        };
+        auto release_s = [&](int u) {
             tc::fence_before_sync();
             __syncwarp();
-            if (lane == 0)
-                for (int k = 0; k < cnt; ++k) tc::mbar_arrive(b.s_empty((u + k) & 1));
-            return true;
+            if (lane == 0) tc::mbar_arrive(b.s_empty(u & 1));
         };
+        auto half_valid = [&](int j, int h) { return min(32, p.n - j * kKeys - h * 32); };
 
         // pass 1a: exact histogram of the first A key tiles
-        auto hist_tile = [&](auto off, auto full, int valid) {
-            constexpr int O = decltype(off)::value;
+        auto hist_half = [&](const uint32_t (&rr)[32], auto full, int valid) {
 #pragma unroll
-            for (int c = 0; c < 64; ++c)
-                if (decltype(full)::value || c < valid) red_add1(hbase - (s[O + c] << 6));
+            for (int c = 0; c < 32; ++c)
+                if (decltype(full)::value || c < valid) red_add1(hbase - (rr[c] << 6));
         };
-        // pass 1b: four cumulative 8-bit window counters in one register
+        // pass 1b: four cumulative 8-bit window counters in one register;
         // four independent counter registers keep the adds off one chain
         uint32_t acc[4] = {0u, 0u, 0u, 0u};
+        uint32_t run = 0u;                            // sum of up to three tile words
         int tot0 = 0, tot1 = 0, tot2 = 0, tot3 = 0;
         int cshift = 0, L0 = 0, hmin = C::BINS - 1;
         auto flush = [&]() {
-#pragma unroll
-            for (int a = 0; a < 4; ++a) {
-                tot0 += (int)(acc[a] & 0xFFu);
-                tot1 += (int)((acc[a] >> 8) & 0xFFu);
-                tot2 += (int)((acc[a] >> 16) & 0xFFu);
-                tot3 += (int)(acc[a] >> 24);
-                acc[a] = 0u;
-            }
+            tot0 += (int)(run & 0xFFu);
+            tot1 += (int)((run >> 8) & 0xFFu);
+            tot2 += (int)((run >> 16) & 0xFFu);
+            tot3 += (int)(run >> 24);
+            run = 0u;
         };
-        auto window_tile = [&](auto off, auto full, int valid) {
-            constexpr int O = decltype(off)::value;
+        auto window_half = [&](const uint32_t (&rr)[32], auto full, int valid) {
 #pragma unroll
-            for (int c = 0; c < 64; ++c)
+            for (int c = 0; c < 32; ++c)
                 if (decltype(full)::value || c < valid)
-                    acc[c & 3] += window_inc(cshift - (int)s[O + c]);
+                    acc[c & 3] += window_inc(cshift - (int)rr[c]);
         };
         // Window from the sample: est = the level of the sample's
         // (N * sampled / n)-th best key.  Levels L0 = est - 1 .. est + 1 are
@@ -444,24 +438,44 @@ attention_fwd_kernel(const Params p)
             L0 = est - 1;
             cshift = 4 * D - 8 * L0 + 8;              // 8 * (level - L0 + 1) = cshift - v
         };
-        auto pass1_tile = [&](int j, auto off) {
-            const int valid = min(kKeys, p.n - j * kKeys);
+        auto pass1_half = [&](int j, int h, const uint32_t (&rr)[32]) {
+            const int valid = half_valid(j, h);
             if (j < A) {
-                if (valid == kKeys) hist_tile(off, BT{}, valid);
-                else hist_tile(off, BF{}, valid);
-                if (j == A - 1) place_window();
+                if (valid >= 32) hist_half(rr, BT{}, 32);
+                else hist_half(rr, BF{}, valid);
             } else {
-                if (valid == kKeys) window_tile(off, BT{}, valid);
-                else window_tile(off, BF{}, valid);
-                if ((j - A) % 3 == 2) flush();        // fields stay below 3 * 64 < 256
+                if (valid >= 32) window_half(rr, BT{}, 32);
+                else window_half(rr, BF{}, valid);
             }
         };
-        for (int j = 0; j < T && ok; j += 2) {
-            const int cnt = min(2, T - j);
-            ok = load_tiles(j, cnt);
-            if (!ok) break;
-            pass1_tile(j, I0{});
-            if (cnt > 1) pass1_tile(j + 1, I64{});
+        auto pass1_end_tile = [&](int j) {
+            if (j == A - 1) place_window();
+            if (j >= A) {
+                const uint32_t w = (acc[0] + acc[1]) + (acc[2] + acc[3]);   // fields <= 64
+                acc[0] = acc[1] = acc[2] = acc[3] = 0u;
+                run += w;
+                if ((j - A) % 3 == 2) flush();        // fields stay below 3 * 64 < 256
+                if (stash_ok) tc::tmem_st1(lane_base + C::STASH_COL + (j - A), w);
+            }
+        };
+        ok = wait_s(0);
+        if (ok) {
+            ld_half(0, 0, sa);
+            tc::tmem_wait_ld(sa);
+        }
+        for (int j = 0; j < T && ok; ++j) {
+            ld_half(j, 1, sb);
+            pass1_half(j, 0, sa);
+            tc::tmem_wait_ld(sb);
+            release_s(j);
+            const bool more = j + 1 < T;
+            if (more) {
+                ok = wait_s(j + 1);
+                if (ok) ld_half(j + 1, 0, sa);
+            }
+            pass1_half(j, 1, sb);
+            pass1_end_tile(j);
+            if (more && ok) tc::tmem_wait_ld(sa);
         }
         flush();
 
@@ -492,12 +506,47 @@ attention_fwd_kernel(const Params p)
                 miss = true;
             }
         }
+        // Where the tie quota runs out.  The sampled tiles hold the first
+        // hist[t] keys at level t; past them, tile words give each tile's
+        // count at t.  Ties are kept in full before tile jstar, kstar of them
+        // (the lowest indices) inside it, and none after it: from tile
+        // zero_at on the weight table maps level t to 0.
+        int zero_at = T, jstar = -1, kstar = 0;
+        if (stash_ok && ok && A < T) {
+            tc::tmem_wait_st();
+            const bool want = t >= 0 && !miss;
+            const int ts = t - L0 + 1;                // 1..3: field of level t in a tile word
+            const int rem0 = want ? quota - (int)hcol[t * kRows] : 0;
+            bool found = !want || rem0 <= 0;
+            if (want && rem0 <= 0) zero_at = A;
+            int cum = 0;
+            for (int c0 = 0; c0 < T - A; c0 += 32) {
+                uint32_t w[32];
+                tc::tmem_ld32(lane_base + C::STASH_COL + c0, w);
+                tc::tmem_wait_ld(w);
+#pragma unroll
+                for (int i = 0; i < 32; ++i) {
+                    const int jj = c0 + i;
+                    if (!found && jj < T - A) {
+                        const int cnt = (int)((w[i] >> (8 * ts)) & 0xFFu) -
+                                        (int)((w[i] >> (8 * ts - 8)) & 0xFFu);
+                        if (cum + cnt >= rem0) {
+                            found = true;
+                            zero_at = A + jj + 1;
+                            if (rem0 - cum < cnt) { jstar = A + jj; kstar = rem0 - cum; }
+                        }
+                        cum += cnt;
+                    }
+                }
+            }
+            if (!found) miss = true;                  // counts disagree: recompute the row
+        }
         if (miss && active) {
             const int slot = atomicAdd(p.miss_count, 1);
             p.miss_rows[slot] = (int)(head * p.n + row);
         }
         // missed rows keep nothing here; the fix-up kernel rewrites them
-        if (miss) { t = -1; quota = 0; }
+        if (miss) { t = -1; quota = 0; zero_at = T; jstar = -1; }
         // Softmax reference: the sample's best logit, raised if needed so that
         // no weight can exceed the fp16 range (s <= D).  The histogram column
         // becomes the row's weight table: level l holds exp2(c2 (s_l - ref))
@@ -512,55 +561,99 @@ attention_fwd_kernel(const Params p)
                     bin <= t ? __float_as_uint(ex2(p.c2 * (float)(D - 2 * bin - ref))) : 0u;
         }
         const uint32_t vt = 256u * (uint32_t)(D - 2 * t);   // accumulator value of the threshold
-        int rem = quota;                              // ties still to keep
+        int rem = quota;                              // ties still to keep (slow tiles before fast_from)
         int kept = 0;
         float zacc[4] = {0.0f, 0.0f, 0.0f, 0.0f};
         const long long obase = ((head * p.n) + row) * (long long)p.N;
+        constexpr int kAll = 1 << 30;
 
         // pass 2: P = kept weights (fp16) -> TMEM; the MMA warp does O += P V
-        auto pass2_tile = [&](int j, auto off, auto full, int valid) {
-            constexpr int O = decltype(off)::value;
-            uint32_t packed[32];
+        // Fast half: the table alone decides (0 beyond the threshold).
+        auto fast_half = [&](const uint32_t (&rr)[32], uint32_t (&pk)[16]) {
 #pragma unroll
-            for (int c = 0; c < 64; c += 2) {
+            for (int c = 0; c < 32; c += 2) {
+                const float w0 = lds_f32(hbase - rr[c]);
+                const float w1 = lds_f32(hbase - rr[c + 1]);
+                zacc[c & 2] += w0;
+                zacc[(c & 2) + 1] += w1;
+                __half2 h2 = __floats2half2_rn(w0, w1);
+                pk[c >> 1] = *reinterpret_cast<uint32_t *>(&h2);
+            }
+        };
+        // Slow half: ties at the threshold are kept while rl > 0, in
+        // ascending key order; keys past n weigh nothing.
+        auto slow_half = [&](int key0, const uint32_t (&rr)[32], uint32_t (&pk)[16], int &rl,
+                             auto full, int valid) {
+#pragma unroll
+            for (int c = 0; c < 32; c += 2) {
                 float w2[2];
 #pragma unroll
                 for (int e = 0; e < 2; ++e) {
-                    const uint32_t v = s[O + c + e];          // 256 s
+                    const uint32_t v = rr[c + e];            // 256 s
                     const bool in = decltype(full)::value || (c + e) < valid;
                     float w = lds_f32(hbase - v);            // 0 below the threshold
                     const bool tie = (v == vt);
-                    const bool drop = !in || (tie && rem <= 0);
-                    rem -= tie ? 1 : 0;
+                    const bool drop = !in || (tie && rl <= 0);
+                    rl -= tie ? 1 : 0;
                     w = drop ? 0.0f : w;
                     zacc[e + (c & 2)] += w;
                     w2[e] = w;
                     if (kDbg) {
                         if (active && !drop && ((int)v > (int)vt || tie)) {
-                            if (p.dbg_idx) p.dbg_idx[obase + kept] = j * kKeys + c + e;
+                            if (p.dbg_idx) p.dbg_idx[obase + kept] = key0 + c + e;
                             if (p.dbg_logits) p.dbg_logits[obase + kept] = (int16_t)((int)v / 256);
                             ++kept;
                         }
                     }
                 }
-                __half2 h = __floats2half2_rn(w2[0], w2[1]);
-                packed[c >> 1] = *reinterpret_cast<uint32_t *>(&h);
+                __half2 h2 = __floats2half2_rn(w2[0], w2[1]);
+                pk[c >> 1] = *reinterpret_cast<uint32_t *>(&h2);
             }
-            tc::tmem_st32(lane_base + C::P_COL + (j & 1) * 32, packed);
         };
+        auto pass2_half = [&](int j, int h, bool slow, const uint32_t (&rr)[32],
+                              uint32_t (&pk)[16], int &rl) {
+            if (!slow) {
+                fast_half(rr, pk);
+            } else {
+                const int valid = half_valid(j, h);
+                if (valid >= 32) slow_half(j * kKeys + h * 32, rr, pk, rl, BT{}, 32);
+                else slow_half(j * kKeys + h * 32, rr, pk, rl, BF{}, valid);
+            }
+        };
+        if (ok) ok = wait_s(T);
+        if (ok) {
+            ld_half(T, 0, sa);
+            tc::tmem_wait_ld(sa);
+        }
         for (int j = 0; j < T && ok; ++j) {
-            ok = load_tiles(T + j, 1);
-            if (!ok) break;
+            const int u = T + j;
+            if (j == zero_at) hcol[t * kRows] = 0u;  // ties past the quota weigh nothing now
+            const bool slow = j < fast_from || half_valid(j, 1) < 32 ||
+                              __any_sync(kFullMask, j == jstar);
+            int rl = j < fast_from ? rem : (j == jstar ? kstar : kAll);
+            uint32_t pk[16];
+            ld_half(u, 1, sb);
+            pass2_half(j, 0, slow, sa, pk, rl);
             ok = __all_sync(kFullMask, wait_bar(b.p_empty(j & 1), ((j >> 1) & 1) ^ 1, deadline,
                                                 abort_flag, p.status));
-            if (!ok) break;
-            const int valid = min(kKeys, p.n - j * kKeys);
-            if (valid == kKeys) pass2_tile(j, I0{}, BT{}, valid);
-            else pass2_tile(j, I0{}, BF{}, valid);
-            tc::tmem_wait_st();
+            if (ok) tc::tmem_st16(lane_base + C::P_COL + (j & 1) * 32, pk);
+            tc::tmem_wait_ld(sb);
+            release_s(u);
+            const bool more = j + 1 < T;
+            if (more && ok) {
+                ok = wait_s(u + 1);
+                if (ok) ld_half(u + 1, 0, sa);
+            }
+            pass2_half(j, 1, slow, sb, pk, rl);
+            if (j < fast_from) rem = rl;
+            if (ok) {
+                tc::tmem_st16(lane_base + C::P_COL + (j & 1) * 32 + 16, pk);
+                tc::tmem_wait_st();
+            }
             tc::fence_before_sync();
             __syncwarp();
-            if (lane == 0) tc::mbar_arrive(b.p_full(j & 1));
+            if (ok && lane == 0) tc::mbar_arrive(b.p_full(j & 1));
+            if (more && ok) tc::tmem_wait_ld(sa);
         }
         float Z = (zacc[0] + zacc[1]) + (zacc[2] + zacc[3]);
         if (!(Z > 0.0f)) Z = 1.0f;                    // missed or inactive rows only
@@ -575,7 +668,7 @@ attention_fwd_kernel(const Params p)
             for (int c0 = 0; c0 < D; c0 += 32) {
                 uint32_t o[32];
                 tc::tmem_ld32(lane_base + C::O_COL + c0, o);
-                tc::tmem_wait_ld();
+                tc::tmem_wait_ld(o);
                 if (active) {
 #pragma unroll
                     for (int c = 0; c < 32; c += 4) {
@@ -599,13 +692,23 @@ attention_fwd_kernel(const Params p)
 }
 
 // Exact recomputation of the rows the fused kernel listed.  One CTA of
-// eight warps per row: Hamming distances from the packed bits, a shared
-// histogram -> threshold level and quota, then each warp takes one
-// contiguous range of keys.  Per-warp counts of ties and of keys above the
-// threshold, prefix-summed across warps, give every warp its share of the
-// quota (ties go to the lower key index) and its output positions; the warp
-// gathers its kept V rows with exp(tau (s - m)) weights in fp32 and the
-// partial sums meet in shared memory.
+// eight warps per row, over the keys in segments of kFixSeg:
+//   1. the Hamming distance of every key to the row (packed bits, loads of
+//      several keys in flight per thread) into a shared byte array, and
+//      their histogram -> threshold level t and quota q;
+//   2. per segment, each warp takes one contiguous range of it; per-warp
+//      counts of ties and of keys above the threshold, prefix-summed across
+//      warps (and carried across segments), give every warp its share of
+//      the quota (ties go to the lower key index) and its output positions;
+//   3. the warp lists its kept keys with their weights exp(tau (s - m)) in
+//      shared memory and gathers their V rows eight at a time (lane l owns
+//      D/32 columns, so each row is one coalesced read), accumulating fp32;
+//      the partial sums meet in shared memory.
+// For n <= kFixSeg the distances of step 1 are kept for step 2; longer rows
+// recompute each segment's distances.
+constexpr int kFixSeg = 16384;
+constexpr int kFixList = 256;                     // kept keys a warp lists per round
+
 template <typename T, int D>
 __global__ void __launch_bounds__(256)
 fixup_rows_kernel(const uint32_t *__restrict__ qbits, const uint32_t *__restrict__ kbits,
@@ -614,17 +717,17 @@ fixup_rows_kernel(const uint32_t *__restrict__ qbits, const uint32_t *__restrict
                   float *__restrict__ out, int32_t *dbg_idx, int16_t *dbg_logits)
 {
     constexpr int DW = D / 32, BINS = D + 1, PER = D / 32, NW = 8;
+    __shared__ uint8_t dist[kFixSeg];
     __shared__ int hist[BINS];
     __shared__ int wties[NW], wabove[NW];
+    __shared__ int lidx[NW][kFixList];
+    __shared__ float lw[NW][kFixList];
     __shared__ float opart[NW][D];
     __shared__ float zpart[NW];
     __shared__ int sh_t, sh_quota, sh_hmin;
     const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
     const unsigned below_me = (1u << lane) - 1u;
     const int count = *miss_count;
-    // each warp's key range: a multiple of 32 keys
-    const int span = ((n + NW - 1) / NW + 31) / 32 * 32;
-    const int jb = min(n, warp * span), je = min(n, jb + span);
     for (int m = blockIdx.x; m < count; m += gridDim.x) {
         const int r = miss_rows[m];
         const long long head = r / n;
@@ -632,16 +735,36 @@ fixup_rows_kernel(const uint32_t *__restrict__ qbits, const uint32_t *__restrict
 #pragma unroll
         for (int w = 0; w < DW; ++w) q[w] = qbits[(long long)r * DW + w];
         const uint32_t *kh = kbits + head * n * DW;
-        auto ham = [&](int j) {
-            int h = 0;
+        // distances of keys [s0, s1) into dist[j - s0], four keys in flight per thread
+        auto fill = [&](int s0, int s1) {
+            for (int j0 = s0 + threadIdx.x; j0 < s1; j0 += 4 * blockDim.x) {
+                uint32_t kw[4][DW];
 #pragma unroll
-            for (int w = 0; w < DW; ++w) h += __popc(q[w] ^ kh[(long long)j * DW + w]);
-            return h;
+                for (int u = 0; u < 4; ++u) {
+                    const int j = j0 + u * blockDim.x;
+#pragma unroll
+                    for (int w = 0; w < DW; ++w)
+                        kw[u][w] = j < s1 ? __ldg(kh + (long long)j * DW + w) : 0u;
+                }
+#pragma unroll
+                for (int u = 0; u < 4; ++u) {
+                    const int j = j0 + u * blockDim.x;
+                    int h = 0;
+#pragma unroll
+                    for (int w = 0; w < DW; ++w) h += __popc(q[w] ^ kw[u][w]);
+                    if (j < s1) dist[j - s0] = (uint8_t)h;
+                }
+            }
         };
         for (int b = threadIdx.x; b < BINS; b += blockDim.x) hist[b] = 0;
         __syncthreads();
-        for (int j = threadIdx.x; j < n; j += blockDim.x) atomicAdd(&hist[ham(j)], 1);
-        __syncthreads();
+        for (int s0 = 0; s0 < n; s0 += kFixSeg) {
+            const int s1 = min(n, s0 + kFixSeg);
+            fill(s0, s1);
+            __syncthreads();
+            for (int j = threadIdx.x; j < s1 - s0; j += blockDim.x) atomicAdd(&hist[dist[j]], 1);
+            __syncthreads();
+        }
         if (threadIdx.x == 0) {
             int t = BINS - 1, quota = 0, hmin = BINS - 1, below = 0;
             bool found = false, seen = false;
@@ -657,72 +780,96 @@ fixup_rows_kernel(const uint32_t *__restrict__ qbits, const uint32_t *__restrict
         }
         __syncthreads();
         const int t = sh_t, quota = sh_quota, smax = D - 2 * sh_hmin;
-        // counts of this warp's range
-        int nt = 0, na = 0;
-        for (int j = jb + lane; j < je; j += 32) {
-            const int h = ham(j);
-            nt += (h == t);
-            na += (h < t);
-        }
-#pragma unroll
-        for (int o = 16; o > 0; o >>= 1) {
-            nt += __shfl_xor_sync(kFullMask, nt, o);
-            na += __shfl_xor_sync(kFullMask, na, o);
-        }
-        if (lane == 0) { wties[warp] = nt; wabove[warp] = na; }
-        __syncthreads();
-        int ties_before = 0, kept_before = 0;
-        for (int w = 0; w < warp; ++w) {
-            kept_before += wabove[w] + min(max(quota - ties_before, 0), wties[w]);
-            ties_before += wties[w];
-        }
+        int ties_all = 0, kept_all = 0;           // over earlier segments (block-uniform)
         float acc[PER];
 #pragma unroll
         for (int e = 0; e < PER; ++e) acc[e] = 0.0f;
         float z = 0.0f;
         const T *vh = V + head * n * (long long)D;
-        for (int j0 = jb; j0 < je; j0 += 32) {
-            const int j = j0 + lane;
-            const int h = j < je ? ham(j) : BINS;
-            const bool tie = (h == t);
-            const unsigned tmask = __ballot_sync(kFullMask, tie);
-            const int rank = ties_before + __popc(tmask & below_me);
-            const bool keep = (h < t) || (tie && rank < quota);
-            ties_before += __popc(tmask);
-            const unsigned kmask = __ballot_sync(kFullMask, keep);
-            const int sv = D - 2 * h;
-            const float w = keep ? expf(tau * (float)(sv - smax)) : 0.0f;
-            if (keep && (dbg_idx || dbg_logits)) {
-                const long long pos = (long long)r * N + kept_before + __popc(kmask & below_me);
-                if (dbg_idx) dbg_idx[pos] = j;
-                if (dbg_logits) dbg_logits[pos] = (int16_t)sv;
+        for (int s0 = 0; s0 < n; s0 += kFixSeg) {
+            const int s1 = min(n, s0 + kFixSeg);
+            if (n > kFixSeg) {
+                __syncthreads();
+                fill(s0, s1);
+                __syncthreads();
             }
-            kept_before += __popc(kmask);
-            // gather the kept V rows four at a time so their loads overlap
-            unsigned mm = kmask;
-            while (mm) {
-                int jj[4];
-                float ww[4];
-#pragma unroll
-                for (int u = 0; u < 4; ++u) {
-                    const bool has = mm != 0u;        // warp-uniform
-                    const int src = has ? __ffs(mm) - 1 : 0;
-                    if (has) mm &= mm - 1u;
-                    jj[u] = __shfl_sync(kFullMask, j, src);
-                    ww[u] = __shfl_sync(kFullMask, w, src);
-                    if (!has) { jj[u] = j0; ww[u] = 0.0f; }
-                }
-                float v[4][PER];
-#pragma unroll
-                for (int u = 0; u < 4; ++u)
-                    VRow<T, PER>::load(vh + (long long)jj[u] * D + lane * PER, v[u]);
-#pragma unroll
-                for (int u = 0; u < 4; ++u) {
-#pragma unroll
-                    for (int e = 0; e < PER; ++e) acc[e] = fmaf(ww[u], v[u][e], acc[e]);
-                    z += ww[u];
-                }
+            // this warp's range of the segment: a multiple of 32 keys
+            const int len = s1 - s0;
+            const int span = ((len + NW - 1) / NW + 31) / 32 * 32;
+            const int jb = min(len, warp * span), je = min(len, jb + span);
+            int nt = 0, na = 0;
+            for (int j = jb + lane; j < je; j += 32) {
+                const int h = dist[j];
+                nt += (h == t);
+                na += (h < t);
             }
+#pragma unroll
+            for (int o = 16; o > 0; o >>= 1) {
+                nt += __shfl_xor_sync(kFullMask, nt, o);
+                na += __shfl_xor_sync(kFullMask, na, o);
+            }
+            if (lane == 0) { wties[warp] = nt; wabove[warp] = na; }
+            __syncthreads();
+            int ties_before = ties_all, kept_before = kept_all;
+            {
+                int tb = ties_all, ka = kept_all;
+                for (int w = 0; w < NW; ++w) {
+                    const int take = wabove[w] + min(max(quota - tb, 0), wties[w]);
+                    if (w == warp) { ties_before = tb; kept_before = ka; }
+                    tb += wties[w];
+                    ka += take;
+                }
+                ties_all = tb;
+                kept_all = ka;
+            }
+            for (int base = jb; base < je; base += kFixList) {
+                const int lim = min(je, base + kFixList);
+                int cnt = 0;
+                for (int j0 = base; j0 < lim; j0 += 32) {
+                    const int j = j0 + lane;
+                    const int h = j < lim ? dist[j] : BINS;
+                    const bool tie = (h == t);
+                    const unsigned tmask = __ballot_sync(kFullMask, tie);
+                    const int rank = ties_before + __popc(tmask & below_me);
+                    const bool keep = (h < t) || (tie && rank < quota);
+                    ties_before += __popc(tmask);
+                    const unsigned kmask = __ballot_sync(kFullMask, keep);
+                    if (keep) {
+                        const int sv = D - 2 * h;
+                        const int slot = cnt + __popc(kmask & below_me);
+                        lidx[warp][slot] = s0 + j;
+                        lw[warp][slot] = expf(tau * (float)(sv - smax));
+                        if (dbg_idx || dbg_logits) {
+                            const long long pos = (long long)r * N + kept_before + slot;
+                            if (dbg_idx) dbg_idx[pos] = s0 + j;
+                            if (dbg_logits) dbg_logits[pos] = (int16_t)sv;
+                        }
+                    }
+                    cnt += __popc(kmask);
+                }
+                kept_before += cnt;
+                __syncwarp();
+                // gather the listed V rows, eight loads in flight per lane
+                for (int i0 = 0; i0 < cnt; i0 += 8) {
+                    float v[8][PER];
+                    float ww[8];
+#pragma unroll
+                    for (int u = 0; u < 8; ++u) {
+                        const bool has = i0 + u < cnt;
+                        const int jj = has ? lidx[warp][i0 + u] : 0;
+                        ww[u] = has ? lw[warp][i0 + u] : 0.0f;
+                        VRow<T, PER>::load(vh + (long long)jj * D + lane * PER, v[u]);
+                    }
+#pragma unroll
+                    for (int u = 0; u < 8; ++u) {
+#pragma unroll
+                        for (int e = 0; e < PER; ++e) acc[e] = fmaf(ww[u], v[u][e], acc[e]);
+                        z += ww[u];
+                    }
+                }
+                __syncwarp();
+            }
+            __syncthreads();
         }
 #pragma unroll
         for (int e = 0; e < PER; ++e) opart[warp][lane * PER + e] = acc[e];

@@ -41,87 +41,116 @@ __device__ __forceinline__ uint32_t core_offset(uint32_t row, uint32_t kbyte, ui
     return ((row >> 3) * (kbytes >> 4) + (kbyte >> 4)) * 128u + (row & 7u) * 16u + (kbyte & 15u);
 }
 
-// One thread per 16 consecutive elements of a row -> 16 int8 signs.
-// Works for Q (tile 128) and K (tile 64): `tile_rows` selects the tiling.
-// The packed copy is written as 16-bit halves: chunk kc of a row is bits
-// 16*(kc%2) .. 16*(kc%2)+15 of word kc/2.
-// `op2` (may be null) receives a second copy with the codes pos2 / neg2.
+// Signs of 16 consecutive elements as int8 codes (pos / neg) in four words,
+// and as 16 packed bits (1 = negative).
 template <typename T>
-__global__ void __launch_bounds__(256)
-sign_operand_kernel(const T *__restrict__ x, const float *__restrict__ sigma, int H, int n,
-                    int d, int tile_rows, int tiles, long long chunks, uint32_t pos,
-                    uint32_t neg, int8_t *__restrict__ op, uint32_t pos2, uint32_t neg2,
-                    int8_t *__restrict__ op2, uint16_t *__restrict__ bits, int32_t *status)
+__device__ __forceinline__ uint32_t sign16(const T *src, const SignRule &rule, uint32_t pos,
+                                           uint32_t neg, uint32_t (&w)[4])
 {
-    const int cpr = d >> 4;                                  // chunks per row
-    const long long padded_rows = (long long)tiles * tile_rows;
-    for (long long c = blockIdx.x * (long long)blockDim.x + threadIdx.x; c < chunks;
-         c += (long long)gridDim.x * blockDim.x) {
-        const long long prow = c / cpr;                      // padded row over all heads
-        const int kc = (int)(c % cpr);
-        const long long head = prow / padded_rows;
-        const int r = (int)(prow % padded_rows);             // row within the head
-        uint4 out = make_uint4(0, 0, 0, 0), out2 = make_uint4(0, 0, 0, 0);
-        if (r < n) {
-            const SignRule rule = sign_rule(__ldg(sigma + (head % H)));
-            if (rule.bad) flag(status, HAD_ERR_BAD_SIGMA);
-            const T *src = x + (head * n + r) * (long long)d + kc * 16;
-            float v[16];
-            float (&lo)[8] = *reinterpret_cast<float(*)[8]>(v);
-            float (&hi)[8] = *reinterpret_cast<float(*)[8]>(v + 8);
-            Load8<T>::run(src, lo);
-            Load8<T>::run(src + 8, hi);
-            uint32_t w[4], w2[4];
-            uint32_t packed = 0;
+    float v[16];
+    Load8<T>::run(src, *reinterpret_cast<float(*)[8]>(v));
+    Load8<T>::run(src + 8, *reinterpret_cast<float(*)[8]>(v + 8));
+    uint32_t packed = 0;
 #pragma unroll
-            for (int q = 0; q < 4; ++q) {
-                uint32_t word = 0, word2 = 0;
+    for (int q = 0; q < 4; ++q) {
+        uint32_t word = 0;
 #pragma unroll
-                for (int b = 0; b < 4; ++b) {
-                    const uint32_t nb = negative_bit(v[4 * q + b], rule);
-                    word |= (nb ? neg : pos) << (8 * b);
-                    word2 |= (nb ? neg2 : pos2) << (8 * b);
-                    packed |= nb << (4 * q + b);
-                }
-                w[q] = word;
-                w2[q] = word2;
-            }
-            out = make_uint4(w[0], w[1], w[2], w[3]);
-            out2 = make_uint4(w2[0], w2[1], w2[2], w2[3]);
-            bits[(head * n + r) * (long long)cpr + kc] = (uint16_t)packed;
+        for (int b = 0; b < 4; ++b) {
+            const uint32_t nb = negative_bit(v[4 * q + b], rule);
+            word |= (nb ? neg : pos) << (8 * b);
+            packed |= nb << (4 * q + b);
         }
-        const int t = r / tile_rows;
-        const uint32_t rr = (uint32_t)(r % tile_rows);
-        int8_t *tile = op + ((head * tiles + t) * (long long)tile_rows * d);
-        *reinterpret_cast<uint4 *>(tile + core_offset(rr, kc * 16, d)) = out;
-        if (op2) {
-            int8_t *tile2 = op2 + ((head * tiles + t) * (long long)tile_rows * d);
-            *reinterpret_cast<uint4 *>(tile2 + core_offset(rr, kc * 16, d)) = out2;
-        }
+        w[q] = word;
     }
+    return packed;
 }
 
-// Largest |v| of each head, as ordered float bits (non-negative floats
-// compare like unsigned integers; NaN counts as infinity).  Each CTA reduces
-// one contiguous chunk of one head and issues a single atomicMax.  vmax must
-// be zeroed beforehand.
-template <typename T>
-__global__ void __launch_bounds__(256)
-vmax_kernel(const T *__restrict__ v, long long groups_per_head, int chunks_per_head,
-            unsigned int *__restrict__ vmax)
+// Rewrite of four code words from one code pair to another (a byte-wise map
+// pos -> pos2, everything else -> neg2).
+__device__ __forceinline__ uint4 recode(const uint32_t (&w)[4], uint32_t pos, uint32_t pos2,
+                                        uint32_t neg2)
 {
-    __shared__ float wmax[8];
-    const long long head = blockIdx.x / chunks_per_head;
-    const int chunk = blockIdx.x % chunks_per_head;
-    const long long per = (groups_per_head + chunks_per_head - 1) / chunks_per_head;
-    const long long g_beg = head * groups_per_head + chunk * per;
-    const long long g_end = head * groups_per_head + min(groups_per_head, (chunk + 1) * per);
-    float m = 0.0f;
-    for (long long g = g_beg + threadIdx.x; g < g_end; g += blockDim.x) {
-        float e[8];
-        Load8<T>::run(v + g * 8, e);
+    uint32_t o[4];
 #pragma unroll
-        for (int k = 0; k < 8; ++k) m = isnan(e[k]) ? __int_as_float(0x7f800000) : fmaxf(m, fabsf(e[k]));
+    for (int q = 0; q < 4; ++q) {
+        uint32_t word = 0;
+#pragma unroll
+        for (int b = 0; b < 4; ++b)
+            word |= (((w[q] >> (8 * b)) & 0xFFu) == pos ? pos2 : neg2) << (8 * b);
+        o[q] = word;
+    }
+    return make_uint4(o[0], o[1], o[2], o[3]);
+}
+
+// All operand preparation that needs only the inputs, in one launch.  Block
+// b of the grid takes, in this order:
+//   b <  BH*qtiles            one 128-row Q tile -> Qop1 (+/-1), Qop2 (+/-64), Qbits
+//   b <  BH*(qtiles+ktiles)   one 64-key K tile  -> Kop (+/-4), Kbits
+//   otherwise                 one chunk of V     -> the chunk's largest |v|
+// Rows past n are written as zero padding.  A thread handles 16 consecutive
+// elements of a row; the packed bits are written as 16-bit halves (chunk kc
+// of a row is bits 16*(kc%2) .. of word kc/2).  Block 0 also zeroes the miss
+// counter of the fused kernel.
+template <typename T, int D>
+__global__ void __launch_bounds__(256)
+operands_kernel(const T *__restrict__ Q, const T *__restrict__ K, const T *__restrict__ V,
+                const float *__restrict__ sq, const float *__restrict__ sk, int H, int n,
+                int bh, int qtiles, int ktiles, int vchunks, int8_t *__restrict__ qop,
+                int8_t *__restrict__ qop2, int8_t *__restrict__ kop,
+                uint16_t *__restrict__ qbits, uint16_t *__restrict__ kbits,
+                float *__restrict__ vpart, int *__restrict__ miss_count, int32_t *status)
+{
+    constexpr int CPR = D / 16;                                // 16-element chunks per row
+    const int b = blockIdx.x;
+    if (b == 0 && threadIdx.x == 0) *miss_count = 0;
+    const int nq = bh * qtiles, nk = bh * ktiles;
+    if (b < nq + nk) {
+        const bool isq = b < nq;
+        const int tiles = isq ? qtiles : ktiles;
+        const int bb = isq ? b : b - nq;
+        const int head = bb / tiles;
+        const int t = bb - head * tiles;
+        const int rows = isq ? kQRows : kKeys;
+        const T *x = isq ? Q : K;
+        const SignRule rule = sign_rule(__ldg((isq ? sq : sk) + head % H));
+        if (rule.bad && threadIdx.x == 0) flag(status, HAD_ERR_BAD_SIGMA);
+        int8_t *tile = (isq ? qop : kop) + (size_t)bb * rows * D;
+        int8_t *tile2 = qop2 + (size_t)bb * rows * D;
+        uint16_t *bits = isq ? qbits : kbits;
+        const uint32_t pos = isq ? 0x01u : 0x04u, neg = isq ? 0xFFu : 0xFCu;
+        for (int c = threadIdx.x; c < rows * CPR; c += blockDim.x) {
+            const int r = c / CPR, kc = c % CPR;
+            const int row = t * rows + r;
+            uint32_t w[4] = {0u, 0u, 0u, 0u};
+            if (row < n) {
+                const size_t e = ((size_t)head * n + row) * D + kc * 16;
+                const uint32_t packed = sign16<T>(x + e, rule, pos, neg, w);
+                bits[e / 16] = (uint16_t)packed;
+            }
+            const uint32_t off = core_offset(r, kc * 16, D);
+            *reinterpret_cast<uint4 *>(tile + off) = make_uint4(w[0], w[1], w[2], w[3]);
+            if (isq)
+                *reinterpret_cast<uint4 *>(tile2 + off) =
+                    row < n ? recode(w, 0x01u, 0x40u, 0xC0u) : make_uint4(0u, 0u, 0u, 0u);
+        }
+        return;
+    }
+    // largest |v| of one chunk of one head, as a float (NaN counts as inf)
+    __shared__ float wmax[8];
+    const int bb = b - nq - nk;
+    const int head = bb / vchunks;
+    const int chunk = bb - head * vchunks;
+    const long long groups = (long long)n * D / 8;             // 8-element groups per head
+    const long long per = (groups + vchunks - 1) / vchunks;
+    const long long g0 = chunk * per, g1 = min(groups, g0 + per);
+    const T *vh = V + (size_t)head * n * D;
+    float m = 0.0f;
+    for (long long g = g0 + threadIdx.x; g < g1; g += blockDim.x) {
+        float e[8];
+        Load8<T>::run(vh + g * 8, e);
+#pragma unroll
+        for (int k = 0; k < 8; ++k)
+            m = isnan(e[k]) ? __int_as_float(0x7f800000) : fmaxf(m, fabsf(e[k]));
     }
 #pragma unroll
     for (int o = 16; o > 0; o >>= 1) m = fmaxf(m, __shfl_xor_sync(kFullMask, m, o));
@@ -129,33 +158,42 @@ vmax_kernel(const T *__restrict__ v, long long groups_per_head, int chunks_per_h
     __syncthreads();
     if (threadIdx.x == 0) {
         for (int w = 1; w < (int)(blockDim.x >> 5); ++w) m = fmaxf(m, wmax[w]);
-        atomicMax(vmax + head, __float_as_uint(m));
+        vpart[bb] = m;
     }
 }
 
 // Power-of-two scale exponent of a head from its largest |v|.
-__device__ __forceinline__ int vscale_exp(unsigned int bits)
+__device__ __forceinline__ int vscale_exp(float m)
 {
-    const float m = __uint_as_float(bits);
     if (!(m > 0.0f) || !isfinite(m)) return 0;
     int e;
     frexpf(m, &e);            // m = f * 2^e, f in [0.5, 1)  ->  m < 2^e
     return e - 15;            // m * 2^-(e-15) in [2^14, 2^15)
 }
 
-// One CTA per (head, 64-key tile): transpose the tile through shared memory
-// and write V^T as fp16 core matrices.  Writes e_h for every head (by the
+// One CTA per (head, 64-key tile): the head's largest |v| from the chunk
+// maxima of operands_kernel, then the tile transposed through shared memory
+// and written as V^T fp16 core matrices.  Writes e_h for every head (by the
 // CTA of tile 0).
 template <typename T, int D>
 __global__ void __launch_bounds__(256)
-v_operand_kernel(const T *__restrict__ v, int n, const unsigned int *__restrict__ vmax,
+v_operand_kernel(const T *__restrict__ v, int n, const float *__restrict__ vpart, int vchunks,
                  __half *__restrict__ op, int *__restrict__ vexp)
 {
     __shared__ float tile[kKeys][D + 1];
+    __shared__ float head_max;
     const int tiles = (n + kKeys - 1) / kKeys;
     const long long head = blockIdx.x / tiles;
     const int t = blockIdx.x % tiles;
-    const int e = vscale_exp(vmax[head]);
+    if (threadIdx.x < 32) {
+        float m = 0.0f;
+        for (int c = threadIdx.x; c < vchunks; c += 32) m = fmaxf(m, vpart[head * vchunks + c]);
+#pragma unroll
+        for (int o = 16; o > 0; o >>= 1) m = fmaxf(m, __shfl_xor_sync(kFullMask, m, o));
+        if (threadIdx.x == 0) head_max = m;
+    }
+    __syncthreads();
+    const int e = vscale_exp(head_max);
     const float scale = ldexpf(1.0f, -e);
     if (t == 0 && threadIdx.x == 0) vexp[head] = e;
     // load 64 keys x D values (coalesced, 8 elements per thread-iteration)
