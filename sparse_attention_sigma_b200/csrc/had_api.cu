@@ -147,7 +147,7 @@ FwdWorkspace fwd_layout(int B, int H, int n, int d, int N)
     w.kbits = w.qbits + round_up(bh * n * (d / 8));
     w.vpart = w.kbits + round_up(bh * n * (d / 8));
     w.miss = w.vpart + round_up(bh * w.vchunks * 4);
-    w.vexp = w.miss + round_up(4);
+    w.vexp = w.miss + round_up(8);                      // miss counter, fix-up done counter
     w.miss_rows = w.vexp + round_up(bh * 4);
     w.total = w.miss_rows + round_up(bh * (size_t)w.qtiles * had::fused::kRows * 4);
     return w;
@@ -189,8 +189,11 @@ had_status_t core_typed(const T *V, int B, int H, int n, int N, float tau, float
     const bool dbg = dbg_idx != nullptr || dbg_lg != nullptr;
     auto kernel = dbg ? had::fused::attention_fwd_kernel<D, true>
                       : had::fused::attention_fwd_kernel<D, false>;
+    // the CTA takes most of the unified L1 as shared memory
     if (cudaFuncSetAttribute(kernel, cudaFuncAttributeMaxDynamicSharedMemorySize,
-                             C::SMEM_BYTES) != cudaSuccess)
+                             C::SMEM_BYTES) != cudaSuccess ||
+        cudaFuncSetAttribute(kernel, cudaFuncAttributePreferredSharedMemoryCarveout,
+                             cudaSharedmemCarveoutMaxShared) != cudaSuccess)
         return HAD_ERR_CUDA;
     auto *qbits = reinterpret_cast<uint32_t *>(ws + w.qbits);
     auto *kbits = reinterpret_cast<uint32_t *>(ws + w.kbits);
@@ -207,6 +210,7 @@ had_status_t core_typed(const T *V, int B, int H, int n, int N, float tau, float
     p.status = status;
     p.miss_count = miss_count;
     p.miss_rows = reinterpret_cast<int *>(ws + w.miss_rows);
+    p.miss_cap = (long long)bh * w.qtiles * had::fused::kRows;
     p.sample_tiles = w.ktiles / 16 > 4 ? w.ktiles / 16 : 4;
     p.n = n;
     p.N = N;
@@ -217,7 +221,7 @@ had_status_t core_typed(const T *V, int B, int H, int n, int N, float tau, float
     const long long blocks = bh * p.ctas_per_head;
     kernel<<<(unsigned)blocks, C::THREADS, C::SMEM_BYTES, st>>>(p);
     had::fused::fixup_rows_kernel<T, D><<<148 * 4, 256, 0, st>>>(
-        qbits, kbits, V, n, N, tau, miss_count, p.miss_rows, out, dbg_idx, dbg_lg);
+        qbits, kbits, V, n, N, tau, miss_count, miss_count + 1, p.miss_rows, out, dbg_idx, dbg_lg);
     return launched();
 }
 

@@ -31,9 +31,13 @@
 // Warp roles: warp 0 bulk-copies Q once and K (twice) / V (once) tiles into
 // shared-memory rings; warp 1 issues every MMA from one thread; warps
 // 2 .. 2+4*QT-1 are the epilogue, one query row per thread, four warps per
-// query tile.  The QT tiles share every K and V tile.  Every wait is bounded
-// by a deadline: a CTA that hits it flags HAD_ERR_TIMEOUT, lets its copies
-// and MMAs drain, frees its TMEM and returns.
+// query tile.  The QT tiles share every K and V tile.  Each query tile has
+// three S buffers in TMEM, so the QK^T of a tile is issued about one and a
+// half tiles before the epilogue reads it; in pass 2 the tile's P is written
+// over the first half of its own S, and the P V that reads it frees the
+// buffer for the next QK^T in the MMA thread's (in-order) stream.  Every
+// wait is bounded by a deadline: a CTA that hits it flags HAD_ERR_TIMEOUT,
+// lets its copies and MMAs drain, frees its TMEM and returns.
 #pragma once
 #include <cuda_fp16.h>
 #include <type_traits>
@@ -60,17 +64,19 @@ struct Cfg {
     static constexpr int VBYTES = D * kKeys * 2;          // fp16 V^T tile
     static constexpr int KSTAGES = 4;
     static constexpr int VSTAGES = 3;
+    static constexpr int SBUF = 3;                        // S buffers per query tile
     static constexpr int BINS = D + 1;
     static constexpr int HIST_BYTES = BINS * kRows * 4;   // per query tile
     static constexpr uint32_t TMEM_COLS = 512;
     static constexpr uint32_t GROUP_COLS = 256;           // TMEM columns per query tile
-    static constexpr uint32_t S_COL = 0;                  // + 64 * buffer: s32, 64 keys
-    static constexpr uint32_t P_COL = 128;                // + 32 * buffer: fp16 pairs
-    static constexpr uint32_t O_COL = 192;                // f32, D columns
-    // pass 1 only: one word of window counts per key tile, in the P and O
-    // columns (unused until pass 2)
-    static constexpr uint32_t STASH_COL = P_COL;
-    static constexpr int STASH_CAP = (QT == 1 ? O_COL + D : GROUP_COLS) - P_COL;
+    // S of key tile u in buffer u % SBUF (s32, 64 columns); in pass 2 the
+    // tile's P (fp16 pairs, 32 columns) overwrites the first half of its S.
+    static constexpr uint32_t S_COL = 0;
+    static constexpr uint32_t O_COL = SBUF * 64;          // f32, D columns
+    // pass 1 only: one word of window counts per key tile, in the O columns
+    // (unused until the first P V)
+    static constexpr uint32_t STASH_COL = O_COL;
+    static constexpr int STASH_CAP = D;
     static_assert(QT * GROUP_COLS <= TMEM_COLS || QT == 1, "TMEM budget");
     static_assert(O_COL + D <= (QT == 1 ? TMEM_COLS : GROUP_COLS), "TMEM budget");
     // shared memory layout (offsets from a 1024-aligned base)
@@ -80,7 +86,7 @@ struct Cfg {
     static constexpr int OFF_V = OFF_K + KSTAGES * KBYTES;
     static constexpr int OFF_HIST = OFF_V + VSTAGES * VBYTES;
     static constexpr int OFF_BAR = OFF_HIST + QT * HIST_BYTES;
-    static constexpr int NBARS = 1 + 2 * KSTAGES + 2 * VSTAGES + 9 + 1;
+    static constexpr int NBARS = 1 + 2 * KSTAGES + 2 * VSTAGES + 3 * SBUF + 2;
     static constexpr int OFF_MISC = OFF_BAR + NBARS * 8;
     static constexpr int SMEM_BYTES = OFF_MISC + 16 + 1024;   // + alignment slack
     static constexpr uint32_t IDESC_QK = tc::idesc(2, 1, 1, kRows, kKeys);   // s32 <- s8 x s8
@@ -99,6 +105,7 @@ struct Params {
     int32_t *status;
     int *miss_count;          // rows whose threshold fell outside the window
     int *miss_rows;           // their flat row ids (head * n + row)
+    long long miss_cap;       // entries of miss_rows (every row of the grid)
     int sample_tiles;         // key tiles counted exactly before the window
     int n, N;
     int qtiles;               // query tiles per head in qop (a multiple of QT)
@@ -112,13 +119,12 @@ struct Bars {
     uint64_t *k_full, *k_empty;     // [KSTAGES]
     uint64_t *v_full, *v_empty;     // [VSTAGES]
     // shared by all query tiles of the CTA:
-    uint64_t *grp;                  // s_full[2] s_empty[2] p_full[2] p_empty[2] o_full
-    uint64_t *drain;
+    uint64_t *grp;                  // s_full[SBUF] s_empty[SBUF] p_full[SBUF] o_full drain
     __device__ uint64_t *s_full(int b) const { return grp + b; }
-    __device__ uint64_t *s_empty(int b) const { return grp + 2 + b; }
-    __device__ uint64_t *p_full(int b) const { return grp + 4 + b; }
-    __device__ uint64_t *p_empty(int b) const { return grp + 6 + b; }
-    __device__ uint64_t *o_full() const { return grp + 8; }
+    __device__ uint64_t *s_empty(int b) const { return grp + 3 + b; }
+    __device__ uint64_t *p_full(int b) const { return grp + 6 + b; }
+    __device__ uint64_t *o_full() const { return grp + 9; }
+    __device__ uint64_t *drain() const { return grp + 10; }
 };
 
 // Bounded wait: false if the deadline passed or another role aborted.
@@ -194,7 +200,6 @@ attention_fwd_kernel(const Params p)
     b.v_full = b.k_empty + C::KSTAGES;
     b.v_empty = b.v_full + C::VSTAGES;
     b.grp = b.v_empty + C::VSTAGES;
-    b.drain = b.grp + 9;
     uint32_t *tmem_holder = reinterpret_cast<uint32_t *>(smem + C::OFF_MISC);
     volatile int *abort_flag = reinterpret_cast<volatile int *>(smem + C::OFF_MISC + 4);
 
@@ -215,14 +220,13 @@ attention_fwd_kernel(const Params p)
             tc::mbar_init(b.v_full + s, 1);
             tc::mbar_init(b.v_empty + s, 1);
         }
-        for (int s = 0; s < 2; ++s) {
+        for (int s = 0; s < C::SBUF; ++s) {
             tc::mbar_init(b.s_full(s), 1);
             tc::mbar_init(b.s_empty(s), 4 * QT);        // one arrive per epilogue warp
             tc::mbar_init(b.p_full(s), 4 * QT);
-            tc::mbar_init(b.p_empty(s), 1);
         }
         tc::mbar_init(b.o_full(), 1);
-        tc::mbar_init(b.drain, 1);
+        tc::mbar_init(b.drain(), 1);
         *abort_flag = 0;
         tc::fence_mbar_init();
     }
@@ -291,33 +295,41 @@ attention_fwd_kernel(const Params p)
             const uint64_t dv = tc::smem_desc(tc::smem_u32(smem + C::OFF_V), 128, 8 * 128);
             bool ok = wait_bar(b.q_full, 0, deadline, abort_flag, p.status);
             tc::fence_after_sync();
+            // O += P V for pass-2 key tile j; P sits in the S buffer of tile T + j.
             auto pv = [&](int j) -> bool {
                 const int vs = j % C::VSTAGES;
-                const int pb = j & 1;
                 if (!wait_bar(b.v_full + vs, (j / C::VSTAGES) & 1, deadline, abort_flag, p.status) ||
-                    !wait_bar(b.p_full(pb), (j >> 1) & 1, deadline, abort_flag, p.status))
+                    !wait_bar(b.p_full(j % C::SBUF), (j / C::SBUF) & 1, deadline, abort_flag,
+                              p.status))
                     return false;
                 tc::fence_after_sync();
                 const uint64_t dvs = dv + (uint64_t)((vs * C::VBYTES) >> 4);
+                const uint32_t pcol = C::S_COL + ((T + j) % C::SBUF) * 64;
 #pragma unroll
                 for (int g = 0; g < QT; ++g) {
                     const uint32_t gcol = g * C::GROUP_COLS;
 #pragma unroll
                     for (int kk = 0; kk < kKeys / 16; ++kk)
-                        tc::mma_f16_ts(tmem + gcol + C::O_COL,
-                                       tmem + gcol + C::P_COL + pb * 32 + kk * 8,
+                        tc::mma_f16_ts(tmem + gcol + C::O_COL, tmem + gcol + pcol + kk * 8,
                                        dvs + (uint64_t)(kk * 16), C::IDESC_PV,
                                        (j > 0 || kk > 0) ? 1u : 0u);
                 }
-                tc::mma_commit(b.p_empty(pb));
                 tc::mma_commit(b.v_empty + vs);
                 return true;
             };
+            // S = Q K^T for key tile u of the stream (pass 1: u < T).  Its
+            // buffer u % SBUF last held tile u - SBUF: a pass-1 tile is given
+            // back by the epilogue (s_empty); a pass-2 tile is free once the
+            // P V that read its P is issued, which happens earlier in this
+            // thread's (in-order) stream.
             auto qk = [&](int u) -> bool {
                 const int ks = u % C::KSTAGES;
-                const int sb = u & 1;
-                if (!wait_bar(b.k_full + ks, (u / C::KSTAGES) & 1, deadline, abort_flag, p.status) ||
-                    !wait_bar(b.s_empty(sb), ((u >> 1) & 1) ^ 1, deadline, abort_flag, p.status))
+                const int sb = u % C::SBUF;
+                const int prev = u - C::SBUF;
+                if (!wait_bar(b.k_full + ks, (u / C::KSTAGES) & 1, deadline, abort_flag, p.status))
+                    return false;
+                if (prev >= 0 && prev < T &&
+                    !wait_bar(b.s_empty(sb), (prev / C::SBUF) & 1, deadline, abort_flag, p.status))
                     return false;
                 tc::fence_after_sync();
                 const uint64_t dks = dk + (uint64_t)((ks * C::KBYTES) >> 4);
@@ -335,20 +347,19 @@ attention_fwd_kernel(const Params p)
                 tc::mma_commit(b.k_empty + ks);
                 return true;
             };
-            // The epilogue frees an S buffer half-way through its tile and
-            // hands over P at the end of it, so in pass 2 the QK^T of tile
-            // j + 2 goes before the P V of tile j.
+            // Pass 1, then the first SBUF tiles of pass 2; after that each
+            // P V frees the buffer for the QK^T SBUF tiles ahead.
             for (int u = 0; u < T && ok; ++u) ok = qk(u);
-            for (int u = T; u < T + min(T, 2) && ok; ++u) ok = qk(u);
+            for (int u = T; u < T + min(T, C::SBUF) && ok; ++u) ok = qk(u);
             for (int j = 0; j < T && ok; ++j) {
-                if (j + 2 < T) ok = qk(T + j + 2);
-                if (ok) ok = pv(j);
+                ok = pv(j);
+                if (ok && j + C::SBUF < T) ok = qk(T + j + C::SBUF);
             }
             if (ok) tc::mma_commit(b.o_full());
             // drain: wait until every MMA this thread issued has completed
-            tc::mma_commit(b.drain);
+            tc::mma_commit(b.drain());
             volatile int never = 0;
-            wait_bar(b.drain, 0, tc::globaltimer_ns() + kWaitNs / 4, &never, p.status);
+            wait_bar(b.drain(), 0, tc::globaltimer_ns() + kWaitNs / 4, &never, p.status);
         }
     } else {
         // ------------------------------------------------------------ epilogue
@@ -380,18 +391,18 @@ attention_fwd_kernel(const Params p)
         // next half is in flight while the current one is processed.
         uint32_t sa[32], sb[32];
         auto ld_half = [&](int u, int h, uint32_t (&rr)[32]) {
-            tc::tmem_ld32(lane_base + C::S_COL + (u & 1) * 64 + h * 32, rr);
+            tc::tmem_ld32(lane_base + C::S_COL + (u % C::SBUF) * 64 + h * 32, rr);
         };
         auto wait_s = [&](int u) -> bool {
-            const bool w = __all_sync(kFullMask, wait_bar(b.s_full(u & 1), (u >> 1) & 1, deadline,
-                                                          abort_flag, p.status));
+            const bool w = __all_sync(kFullMask, wait_bar(b.s_full(u % C::SBUF), (u / C::SBUF) & 1,
+                                                          deadline, abort_flag, p.status));
             tc::fence_after_sync();
             return w;
         };
         auto release_s = [&](int u) {
             tc::fence_before_sync();
             __syncwarp();
-            if (lane == 0) tc::mbar_arrive(b.s_empty(u & 1));
+            if (lane == 0) tc::mbar_arrive(b.s_empty(u % C::SBUF));
         };
         auto half_valid = [&](int j, int h) { return min(32, p.n - j * kKeys - h * 32); };
 
@@ -543,7 +554,7 @@ attention_fwd_kernel(const Params p)
         }
         if (miss && active) {
             const int slot = atomicAdd(p.miss_count, 1);
-            p.miss_rows[slot] = (int)(head * p.n + row);
+            if (slot < p.miss_cap) p.miss_rows[slot] = (int)(head * p.n + row);
         }
         // missed rows keep nothing here; the fix-up kernel rewrites them
         if (miss) { t = -1; quota = 0; zero_at = T; jstar = -1; }
@@ -632,27 +643,23 @@ attention_fwd_kernel(const Params p)
                               __any_sync(kFullMask, j == jstar);
             int rl = j < fast_from ? rem : (j == jstar ? kstar : kAll);
             uint32_t pk[16];
+            const uint32_t pcol = lane_base + C::S_COL + (u % C::SBUF) * 64;   // P over S
             ld_half(u, 1, sb);
             pass2_half(j, 0, slow, sa, pk, rl);
-            ok = __all_sync(kFullMask, wait_bar(b.p_empty(j & 1), ((j >> 1) & 1) ^ 1, deadline,
-                                                abort_flag, p.status));
-            if (ok) tc::tmem_st16(lane_base + C::P_COL + (j & 1) * 32, pk);
+            tc::tmem_st16(pcol, pk);                  // S columns 0-15 are already read
             tc::tmem_wait_ld(sb);
-            release_s(u);
             const bool more = j + 1 < T;
-            if (more && ok) {
+            if (more) {
                 ok = wait_s(u + 1);
                 if (ok) ld_half(u + 1, 0, sa);
             }
             pass2_half(j, 1, slow, sb, pk, rl);
             if (j < fast_from) rem = rl;
-            if (ok) {
-                tc::tmem_st16(lane_base + C::P_COL + (j & 1) * 32 + 16, pk);
-                tc::tmem_wait_st();
-            }
+            tc::tmem_st16(pcol + 16, pk);
+            tc::tmem_wait_st();
             tc::fence_before_sync();
             __syncwarp();
-            if (ok && lane == 0) tc::mbar_arrive(b.p_full(j & 1));
+            if (ok && lane == 0) tc::mbar_arrive(b.p_full(j % C::SBUF));
             if (more && ok) tc::tmem_wait_ld(sa);
         }
         float Z = (zacc[0] + zacc[1]) + (zacc[2] + zacc[3]);
@@ -705,7 +712,8 @@ attention_fwd_kernel(const Params p)
 //      D/32 columns, so each row is one coalesced read), accumulating fp32;
 //      the partial sums meet in shared memory.
 // For n <= kFixSeg the distances of step 1 are kept for step 2; longer rows
-// recompute each segment's distances.
+// recompute each segment's distances.  The last CTA to finish zeroes the
+// miss counter (and its own done counter) for the next fused pass.
 constexpr int kFixSeg = 16384;
 constexpr int kFixList = 256;                     // kept keys a warp lists per round
 
@@ -713,7 +721,8 @@ template <typename T, int D>
 __global__ void __launch_bounds__(256)
 fixup_rows_kernel(const uint32_t *__restrict__ qbits, const uint32_t *__restrict__ kbits,
                   const T *__restrict__ V, int n, int N, float tau,
-                  const int *__restrict__ miss_count, const int *__restrict__ miss_rows,
+                  int *__restrict__ miss_count, int *__restrict__ done_count,
+                  const int *__restrict__ miss_rows,
                   float *__restrict__ out, int32_t *dbg_idx, int16_t *dbg_logits)
 {
     constexpr int DW = D / 32, BINS = D + 1, PER = D / 32, NW = 8;
@@ -885,6 +894,14 @@ fixup_rows_kernel(const uint32_t *__restrict__ qbits, const uint32_t *__restrict
             out[(long long)r * D + c] = o / zt;
         }
         __syncthreads();
+    }
+    if (threadIdx.x == 0) {
+        __threadfence();
+        if (atomicAdd(done_count, 1) == (int)gridDim.x - 1) {
+            *miss_count = 0;
+            *done_count = 0;
+            __threadfence();
+        }
     }
 }
 

@@ -90,7 +90,9 @@ __device__ __forceinline__ uint4 recode(const uint32_t (&w)[4], uint32_t pos, ui
 // Rows past n are written as zero padding.  A thread handles 16 consecutive
 // elements of a row; the packed bits are written as 16-bit halves (chunk kc
 // of a row is bits 16*(kc%2) .. of word kc/2).  Block 0 also zeroes the miss
-// counter of the fused kernel.
+// counter of the fused kernel and the done counter of the fix-up kernel
+// (which zeroes both again when it finishes, so the fused stage can run
+// again on the same operands).
 template <typename T, int D>
 __global__ void __launch_bounds__(256)
 operands_kernel(const T *__restrict__ Q, const T *__restrict__ K, const T *__restrict__ V,
@@ -102,7 +104,7 @@ operands_kernel(const T *__restrict__ Q, const T *__restrict__ K, const T *__res
 {
     constexpr int CPR = D / 16;                                // 16-element chunks per row
     const int b = blockIdx.x;
-    if (b == 0 && threadIdx.x == 0) *miss_count = 0;
+    if (b == 0 && threadIdx.x < 2) miss_count[threadIdx.x] = 0;   // miss and fix-up done counters
     const int nq = bh * qtiles, nk = bh * ktiles;
     if (b < nq + nk) {
         const bool isq = b < nq;

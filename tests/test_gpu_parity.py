@@ -254,6 +254,11 @@ def test_prepare_then_core_equals_fwd(had):
     out = had.had_attention_core(c.gv, c.N, c.tau, ws)
     torch.cuda.synchronize()
     assert torch.equal(out, ref)
+    # the core stage may run again on the same prepared operands
+    for _ in range(3):
+        again = had.had_attention_core(c.gv, c.N, c.tau, ws)
+        torch.cuda.synchronize()
+        assert torch.equal(again, ref)
 
 
 def test_tau_zero_is_uniform_over_kept(had):
