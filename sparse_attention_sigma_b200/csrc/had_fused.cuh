@@ -62,8 +62,11 @@ struct Cfg {
     static constexpr int QBYTES = kRows * D;              // int8 Q tile
     static constexpr int KBYTES = kKeys * D;              // int8 K tile
     static constexpr int VBYTES = D * kKeys * 2;          // fp16 V^T tile
-    static constexpr int KSTAGES = 4;
-    static constexpr int VSTAGES = 3;
+    // Deep K and V rings: a bulk copy takes a few microseconds to land.
+    // Stages are released in pairs (one commit per two tiles).
+    static constexpr int KSTAGES = D == 64 ? 8 : 6;
+    static constexpr int VSTAGES = 4;
+    static_assert(KSTAGES % 2 == 0 && VSTAGES % 2 == 0, "stages are released in pairs");
     static constexpr int SBUF = 3;                        // S buffers per query tile
     static constexpr int BINS = D + 1;
     static constexpr int HIST_BYTES = BINS * kRows * 4;   // per query tile
@@ -86,7 +89,7 @@ struct Cfg {
     static constexpr int OFF_V = OFF_K + KSTAGES * KBYTES;
     static constexpr int OFF_HIST = OFF_V + VSTAGES * VBYTES;
     static constexpr int OFF_BAR = OFF_HIST + QT * HIST_BYTES;
-    static constexpr int NBARS = 1 + 2 * KSTAGES + 2 * VSTAGES + 3 * SBUF + 2;
+    static constexpr int NBARS = 1 + KSTAGES + KSTAGES / 2 + VSTAGES + VSTAGES / 2 + 3 * SBUF + 2;
     static constexpr int OFF_MISC = OFF_BAR + NBARS * 8;
     static constexpr int SMEM_BYTES = OFF_MISC + 16 + 1024;   // + alignment slack
     static constexpr uint32_t IDESC_QK = tc::idesc(2, 1, 1, kRows, kKeys);   // s32 <- s8 x s8
@@ -116,8 +119,8 @@ struct Params {
 
 struct Bars {
     uint64_t *q_full;
-    uint64_t *k_full, *k_empty;     // [KSTAGES]
-    uint64_t *v_full, *v_empty;     // [VSTAGES]
+    uint64_t *k_full, *k_empty;     // [KSTAGES], [KSTAGES / 2]: one per pair of stages
+    uint64_t *v_full, *v_empty;     // [VSTAGES], [VSTAGES / 2]
     // shared by all query tiles of the CTA:
     uint64_t *grp;                  // s_full[SBUF] s_empty[SBUF] p_full[SBUF] o_full drain
     __device__ uint64_t *s_full(int b) const { return grp + b; }
@@ -197,9 +200,9 @@ attention_fwd_kernel(const Params p)
     b.q_full = bar;
     b.k_full = bar + 1;
     b.k_empty = b.k_full + C::KSTAGES;
-    b.v_full = b.k_empty + C::KSTAGES;
+    b.v_full = b.k_empty + C::KSTAGES / 2;
     b.v_empty = b.v_full + C::VSTAGES;
-    b.grp = b.v_empty + C::VSTAGES;
+    b.grp = b.v_empty + C::VSTAGES / 2;
     uint32_t *tmem_holder = reinterpret_cast<uint32_t *>(smem + C::OFF_MISC);
     volatile int *abort_flag = reinterpret_cast<volatile int *>(smem + C::OFF_MISC + 4);
 
@@ -212,14 +215,10 @@ attention_fwd_kernel(const Params p)
 
     if (threadIdx.x == 0) {
         tc::mbar_init(b.q_full, 1);
-        for (int s = 0; s < C::KSTAGES; ++s) {
-            tc::mbar_init(b.k_full + s, 1);
-            tc::mbar_init(b.k_empty + s, 1);
-        }
-        for (int s = 0; s < C::VSTAGES; ++s) {
-            tc::mbar_init(b.v_full + s, 1);
-            tc::mbar_init(b.v_empty + s, 1);
-        }
+        for (int s = 0; s < C::KSTAGES; ++s) tc::mbar_init(b.k_full + s, 1);
+        for (int s = 0; s < C::KSTAGES / 2; ++s) tc::mbar_init(b.k_empty + s, 1);
+        for (int s = 0; s < C::VSTAGES; ++s) tc::mbar_init(b.v_full + s, 1);
+        for (int s = 0; s < C::VSTAGES / 2; ++s) tc::mbar_init(b.v_empty + s, 1);
         for (int s = 0; s < C::SBUF; ++s) {
             tc::mbar_init(b.s_full(s), 1);
             tc::mbar_init(b.s_empty(s), 4 * QT);        // one arrive per epilogue warp
@@ -252,18 +251,23 @@ attention_fwd_kernel(const Params p)
             for (int u = 0; u < 2 * T && ok; ++u) {
                 const int j = u < T ? u : u - T;
                 const int ks = u % C::KSTAGES;
-                ok = wait_bar(b.k_empty + ks, ((u / C::KSTAGES) & 1) ^ 1, deadline, abort_flag,
-                              p.status);
-                if (!ok) break;
+                // a pair of stages comes back when both of its tiles' QK^T are done
+                if ((u & 1) == 0) {
+                    ok = wait_bar(b.k_empty + (u / 2) % (C::KSTAGES / 2),
+                                  ((u / C::KSTAGES) & 1) ^ 1, deadline, abort_flag, p.status);
+                    if (!ok) break;
+                }
                 tc::mbar_expect_tx(b.k_full + ks, C::KBYTES);
                 tc::bulk_g2s(smem + C::OFF_K + ks * C::KBYTES, ksrc + (long long)j * C::KBYTES,
                              C::KBYTES, b.k_full + ks);
                 issued_k = u + 1;
                 if (u >= T) {
                     const int vs = j % C::VSTAGES;
-                    ok = wait_bar(b.v_empty + vs, ((j / C::VSTAGES) & 1) ^ 1, deadline,
-                                  abort_flag, p.status);
-                    if (!ok) break;
+                    if ((j & 1) == 0) {
+                        ok = wait_bar(b.v_empty + (j / 2) % (C::VSTAGES / 2),
+                                      ((j / C::VSTAGES) & 1) ^ 1, deadline, abort_flag, p.status);
+                        if (!ok) break;
+                    }
                     tc::mbar_expect_tx(b.v_full + vs, C::VBYTES);
                     tc::bulk_g2s(smem + C::OFF_V + vs * C::VBYTES,
                                  vsrc + (long long)j * C::VBYTES, C::VBYTES, b.v_full + vs);
@@ -314,7 +318,7 @@ attention_fwd_kernel(const Params p)
                                        dvs + (uint64_t)(kk * 16), C::IDESC_PV,
                                        (j > 0 || kk > 0) ? 1u : 0u);
                 }
-                tc::mma_commit(b.v_empty + vs);
+                if (j & 1) tc::mma_commit(b.v_empty + (j / 2) % (C::VSTAGES / 2));
                 return true;
             };
             // S = Q K^T for key tile u of the stream (pass 1: u < T).  Its
@@ -344,7 +348,7 @@ attention_fwd_kernel(const Params p)
                                       dks + (uint64_t)(kk * 16), C::IDESC_QK, kk > 0 ? 1u : 0u);
                 }
                 tc::mma_commit(b.s_full(sb));
-                tc::mma_commit(b.k_empty + ks);
+                if (u & 1) tc::mma_commit(b.k_empty + (u / 2) % (C::KSTAGES / 2));
                 return true;
             };
             // Pass 1, then the first SBUF tiles of pass 2; after that each
