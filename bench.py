@@ -262,10 +262,15 @@ def source_digest():
     return h.hexdigest()
 
 
+def fused_kernel_name(cfg):
+    """The fused kernel had_attention_core runs for this workload (no debug outputs)."""
+    return "attention_fwd_kernel"
+
+
 def stored_traffic(cfg):
     """DRAM bytes per launch of the fused kernel from the committed ncu summary,
     or None when the summary belongs to other sources or another workload."""
-    path = os.path.join(ROOT, "profiles", f"attention_fwd_kernel_{cfg.name}.md")
+    path = os.path.join(ROOT, "profiles", f"{fused_kernel_name(cfg)}_{cfg.name}.md")
     if not os.path.exists(path):
         return None
     fields = {}
@@ -371,7 +376,7 @@ def run_had(args, world, rank, local):
                    "l2": "flushed between steps (256 MiB write outside the timed events)"},
         "roofline": {"bound": "tensor", "achieved": achieved, "peak": peak_eff,
                      "unit": "TFLOP/s", "frac": achieved / peak_eff, "traffic": traffic,
-                     "kernel": "had_attention_core: attention_fwd_kernel + fixup_rows_kernel",
+                     "kernel": f"had_attention_core: {fused_kernel_name(cfg)} + fixup_rows_kernel",
                      "core_ms": core_ms, "whole_call_frac": model["t_roof"] / (ms * 1e-3),
                      "t_roof_us": model["t_roof"] * 1e6, "t_hbm_us": model["t_hbm"] * 1e6,
                      "t_tc_us": model["t_tc"] * 1e6, "t_alu_us": model["t_alu"] * 1e6,

@@ -58,15 +58,22 @@ constexpr int kMagic = 0x4B400000;                  // bits of 1.5 * 2^23
 template <int D>
 struct Cfg {
     static constexpr int QT = D == 64 ? 2 : 1;            // query tiles per CTA
-    static constexpr int THREADS = 32 * (2 + 4 * QT);
+    // warp 0 producer, warp 1 MMA issuer of query tile 0, warps 2 .. 1+4*QT
+    // epilogue, warp 2+4*QT MMA issuer of query tile 1 (QT = 2)
+    static constexpr int THREADS = 32 * (2 + 4 * QT + (QT - 1));
     static constexpr int QBYTES = kRows * D;              // int8 Q tile
     static constexpr int KBYTES = kKeys * D;              // int8 K tile
     static constexpr int VBYTES = D * kKeys * 2;          // fp16 V^T tile
-    // Deep K and V rings: a bulk copy takes a few microseconds to land.
-    // Stages are released in pairs (one commit per two tiles).
-    static constexpr int KSTAGES = D == 64 ? 8 : 6;
-    static constexpr int VSTAGES = 4;
-    static_assert(KSTAGES % 2 == 0 && VSTAGES % 2 == 0, "stages are released in pairs");
+    // K and V move in groups of consecutive tiles, 16 KB per bulk copy: a
+    // cp.async.bulk costs an SM about the same time whatever its size up to
+    // 16 KB, so few large copies keep the operand stream off the critical
+    // path.  Rings of KGROUPS / VGROUPS groups; one commit frees a group.
+    static constexpr int GK = 16384 / KBYTES;             // K tiles per copy
+    static constexpr int GV = 16384 / VBYTES;             // V tiles per copy
+    static constexpr int KGROUPS = 3;
+    static constexpr int VGROUPS = 3;
+    static constexpr int KSTAGES = KGROUPS * GK;          // K tile slots
+    static constexpr int VSTAGES = VGROUPS * GV;          // V tile slots
     static constexpr int SBUF = 3;                        // S buffers per query tile
     static constexpr int BINS = D + 1;
     static constexpr int HIST_BYTES = BINS * kRows * 4;   // per query tile
@@ -89,7 +96,7 @@ struct Cfg {
     static constexpr int OFF_V = OFF_K + KSTAGES * KBYTES;
     static constexpr int OFF_HIST = OFF_V + VSTAGES * VBYTES;
     static constexpr int OFF_BAR = OFF_HIST + QT * HIST_BYTES;
-    static constexpr int NBARS = 1 + KSTAGES + KSTAGES / 2 + VSTAGES + VSTAGES / 2 + 3 * SBUF + 2;
+    static constexpr int NBARS = 1 + 2 * KGROUPS + 2 * VGROUPS + QT * (3 * SBUF + 2);
     static constexpr int OFF_MISC = OFF_BAR + NBARS * 8;
     static constexpr int SMEM_BYTES = OFF_MISC + 16 + 1024;   // + alignment slack
     static constexpr uint32_t IDESC_QK = tc::idesc(2, 1, 1, kRows, kKeys);   // s32 <- s8 x s8
@@ -119,15 +126,16 @@ struct Params {
 
 struct Bars {
     uint64_t *q_full;
-    uint64_t *k_full, *k_empty;     // [KSTAGES], [KSTAGES / 2]: one per pair of stages
-    uint64_t *v_full, *v_empty;     // [VSTAGES], [VSTAGES / 2]
-    // shared by all query tiles of the CTA:
-    uint64_t *grp;                  // s_full[SBUF] s_empty[SBUF] p_full[SBUF] o_full drain
-    __device__ uint64_t *s_full(int b) const { return grp + b; }
-    __device__ uint64_t *s_empty(int b) const { return grp + 3 + b; }
-    __device__ uint64_t *p_full(int b) const { return grp + 6 + b; }
-    __device__ uint64_t *o_full() const { return grp + 9; }
-    __device__ uint64_t *drain() const { return grp + 10; }
+    uint64_t *k_full, *k_empty;     // [KGROUPS]
+    uint64_t *v_full, *v_empty;     // [VGROUPS]
+    // per query tile g (each has its own MMA issuer):
+    // s_full[SBUF] s_empty[SBUF] p_full[SBUF] o_full drain
+    uint64_t *grp;
+    __device__ uint64_t *s_full(int g, int b) const { return grp + 11 * g + b; }
+    __device__ uint64_t *s_empty(int g, int b) const { return grp + 11 * g + 3 + b; }
+    __device__ uint64_t *p_full(int g, int b) const { return grp + 11 * g + 6 + b; }
+    __device__ uint64_t *o_full(int g) const { return grp + 11 * g + 9; }
+    __device__ uint64_t *drain(int g) const { return grp + 11 * g + 10; }
 };
 
 // Bounded wait: false if the deadline passed or another role aborted.
@@ -199,10 +207,10 @@ attention_fwd_kernel(const Params p)
     Bars b;
     b.q_full = bar;
     b.k_full = bar + 1;
-    b.k_empty = b.k_full + C::KSTAGES;
-    b.v_full = b.k_empty + C::KSTAGES / 2;
-    b.v_empty = b.v_full + C::VSTAGES;
-    b.grp = b.v_empty + C::VSTAGES / 2;
+    b.k_empty = b.k_full + C::KGROUPS;
+    b.v_full = b.k_empty + C::KGROUPS;
+    b.v_empty = b.v_full + C::VGROUPS;
+    b.grp = b.v_empty + C::VGROUPS;
     uint32_t *tmem_holder = reinterpret_cast<uint32_t *>(smem + C::OFF_MISC);
     volatile int *abort_flag = reinterpret_cast<volatile int *>(smem + C::OFF_MISC + 4);
 
@@ -215,17 +223,23 @@ attention_fwd_kernel(const Params p)
 
     if (threadIdx.x == 0) {
         tc::mbar_init(b.q_full, 1);
-        for (int s = 0; s < C::KSTAGES; ++s) tc::mbar_init(b.k_full + s, 1);
-        for (int s = 0; s < C::KSTAGES / 2; ++s) tc::mbar_init(b.k_empty + s, 1);
-        for (int s = 0; s < C::VSTAGES; ++s) tc::mbar_init(b.v_full + s, 1);
-        for (int s = 0; s < C::VSTAGES / 2; ++s) tc::mbar_init(b.v_empty + s, 1);
-        for (int s = 0; s < C::SBUF; ++s) {
-            tc::mbar_init(b.s_full(s), 1);
-            tc::mbar_init(b.s_empty(s), 4 * QT);        // one arrive per epilogue warp
-            tc::mbar_init(b.p_full(s), 4 * QT);
+        for (int s = 0; s < C::KGROUPS; ++s) {
+            tc::mbar_init(b.k_full + s, 1);
+            tc::mbar_init(b.k_empty + s, QT);             // one commit per MMA issuer
         }
-        tc::mbar_init(b.o_full(), 1);
-        tc::mbar_init(b.drain(), 1);
+        for (int s = 0; s < C::VGROUPS; ++s) {
+            tc::mbar_init(b.v_full + s, 1);
+            tc::mbar_init(b.v_empty + s, QT);
+        }
+        for (int g = 0; g < QT; ++g) {
+            for (int s = 0; s < C::SBUF; ++s) {
+                tc::mbar_init(b.s_full(g, s), 1);
+                tc::mbar_init(b.s_empty(g, s), 4);      // one arrive per epilogue warp
+                tc::mbar_init(b.p_full(g, s), 4);
+            }
+            tc::mbar_init(b.o_full(g), 1);
+            tc::mbar_init(b.drain(g), 1);
+        }
         *abort_flag = 0;
         tc::fence_mbar_init();
     }
@@ -246,32 +260,40 @@ attention_fwd_kernel(const Params p)
             tc::mbar_expect_tx(b.q_full, 2 * QT * C::QBYTES);
             tc::bulk_g2s(smem + C::OFF_Q, qsrc, QT * C::QBYTES, b.q_full);
             tc::bulk_g2s(smem + C::OFF_Q2, qsrc2, QT * C::QBYTES, b.q_full);
+            // Group G of the K stream holds key tiles GK*q .. of pass G / nkg
+            // (q = G % nkg); V group H holds key tiles GV*H .. (pass 2 only).
+            const int nkg = (T + C::GK - 1) / C::GK;
             int issued_k = 0, issued_v = 0;
             bool ok = true;
-            for (int u = 0; u < 2 * T && ok; ++u) {
-                const int j = u < T ? u : u - T;
-                const int ks = u % C::KSTAGES;
-                // a pair of stages comes back when both of its tiles' QK^T are done
-                if ((u & 1) == 0) {
-                    ok = wait_bar(b.k_empty + (u / 2) % (C::KSTAGES / 2),
-                                  ((u / C::KSTAGES) & 1) ^ 1, deadline, abort_flag, p.status);
-                    if (!ok) break;
-                }
-                tc::mbar_expect_tx(b.k_full + ks, C::KBYTES);
-                tc::bulk_g2s(smem + C::OFF_K + ks * C::KBYTES, ksrc + (long long)j * C::KBYTES,
-                             C::KBYTES, b.k_full + ks);
-                issued_k = u + 1;
-                if (u >= T) {
-                    const int vs = j % C::VSTAGES;
-                    if ((j & 1) == 0) {
-                        ok = wait_bar(b.v_empty + (j / 2) % (C::VSTAGES / 2),
-                                      ((j / C::VSTAGES) & 1) ^ 1, deadline, abort_flag, p.status);
-                        if (!ok) break;
-                    }
-                    tc::mbar_expect_tx(b.v_full + vs, C::VBYTES);
-                    tc::bulk_g2s(smem + C::OFF_V + vs * C::VBYTES,
-                                 vsrc + (long long)j * C::VBYTES, C::VBYTES, b.v_full + vs);
-                    issued_v = j + 1;
+            auto load_v = [&](int H) -> bool {
+                const int vs = H % C::VGROUPS;
+                if (!wait_bar(b.v_empty + vs, ((H / C::VGROUPS) & 1) ^ 1, deadline, abort_flag,
+                              p.status))
+                    return false;
+                const int cnt = min(C::GV, T - H * C::GV);
+                tc::mbar_expect_tx(b.v_full + vs, cnt * C::VBYTES);
+                tc::bulk_g2s(smem + C::OFF_V + vs * C::GV * C::VBYTES,
+                             vsrc + (long long)H * C::GV * C::VBYTES, cnt * C::VBYTES,
+                             b.v_full + vs);
+                issued_v = H + 1;
+                return true;
+            };
+            for (int G = 0; G < 2 * nkg && ok; ++G) {
+                const int pass = G / nkg, q = G % nkg;
+                const int ks = G % C::KGROUPS;
+                ok = wait_bar(b.k_empty + ks, ((G / C::KGROUPS) & 1) ^ 1, deadline, abort_flag,
+                              p.status);
+                if (!ok) break;
+                const int cnt = min(C::GK, T - q * C::GK);
+                tc::mbar_expect_tx(b.k_full + ks, cnt * C::KBYTES);
+                tc::bulk_g2s(smem + C::OFF_K + ks * C::GK * C::KBYTES,
+                             ksrc + (long long)q * C::GK * C::KBYTES, cnt * C::KBYTES,
+                             b.k_full + ks);
+                issued_k = G + 1;
+                // pass 2: the V groups of these key tiles follow their K group
+                if (pass == 1) {
+                    const int hend = (q * C::GK + cnt + C::GV - 1) / C::GV;
+                    for (int H = issued_v; H < hend && ok; ++H) ok = load_v(H);
                 }
             }
             if (!ok) {
@@ -279,76 +301,85 @@ attention_fwd_kernel(const Params p)
                 const uint64_t drain_deadline = tc::globaltimer_ns() + kWaitNs / 4;
                 volatile int never = 0;
                 wait_bar(b.q_full, 0, drain_deadline, &never, p.status);
-                for (int u = (issued_k > C::KSTAGES ? issued_k - C::KSTAGES : 0); u < issued_k; ++u)
-                    wait_bar(b.k_full + u % C::KSTAGES, (u / C::KSTAGES) & 1, drain_deadline,
+                for (int G = (issued_k > C::KGROUPS ? issued_k - C::KGROUPS : 0); G < issued_k; ++G)
+                    wait_bar(b.k_full + G % C::KGROUPS, (G / C::KGROUPS) & 1, drain_deadline,
                              &never, p.status);
-                for (int j = (issued_v > C::VSTAGES ? issued_v - C::VSTAGES : 0); j < issued_v; ++j)
-                    wait_bar(b.v_full + j % C::VSTAGES, (j / C::VSTAGES) & 1, drain_deadline,
+                for (int H = (issued_v > C::VGROUPS ? issued_v - C::VGROUPS : 0); H < issued_v; ++H)
+                    wait_bar(b.v_full + H % C::VGROUPS, (H / C::VGROUPS) & 1, drain_deadline,
                              &never, p.status);
             }
         }
-    } else if (warp == 1) {
-        // ------------------------------------------------------------ MMA issuer
+    } else if (warp == 1 || warp == 2 + 4 * QT) {
+        // ------------------------------------------------------------ MMA issuers
+        // One thread per query tile g issues that tile's MMAs; the two
+        // issuers share only the K and V rings (each commits once per group).
         if (lane == 0) {
+            const int g = warp == 1 ? 0 : 1;
             // Descriptors are computed once; a tile or K step moves only the
             // start-address field (bits 0-13, in 16-byte units).
-            // the query tiles sit QBYTES apart in both Q buffers
-            const uint64_t dq1 = tc::smem_desc(tc::smem_u32(smem + C::OFF_Q), 128, D * 8);
-            const uint64_t dq2 = tc::smem_desc(tc::smem_u32(smem + C::OFF_Q2), 128, D * 8);
+            const uint64_t dq1 =
+                tc::smem_desc(tc::smem_u32(smem + C::OFF_Q + g * C::QBYTES), 128, D * 8);
+            const uint64_t dq2 =
+                tc::smem_desc(tc::smem_u32(smem + C::OFF_Q2 + g * C::QBYTES), 128, D * 8);
             const uint64_t dk = tc::smem_desc(tc::smem_u32(smem + C::OFF_K), 128, D * 8);
             const uint64_t dv = tc::smem_desc(tc::smem_u32(smem + C::OFF_V), 128, 8 * 128);
+            const uint32_t gcol = g * C::GROUP_COLS;
             bool ok = wait_bar(b.q_full, 0, deadline, abort_flag, p.status);
             tc::fence_after_sync();
-            // O += P V for pass-2 key tile j; P sits in the S buffer of tile T + j.
+            const int nkg = (T + C::GK - 1) / C::GK;
+            // O += P V for pass-2 key tile j; P sits in the S buffer of tile
+            // T + j.  The V group's barrier is waited for at its first tile.
             auto pv = [&](int j) -> bool {
-                const int vs = j % C::VSTAGES;
-                if (!wait_bar(b.v_full + vs, (j / C::VSTAGES) & 1, deadline, abort_flag, p.status) ||
-                    !wait_bar(b.p_full(j % C::SBUF), (j / C::SBUF) & 1, deadline, abort_flag,
+                const int H = j / C::GV;
+                const int vg = H % C::VGROUPS;
+                const int vs = vg * C::GV + j % C::GV;        // tile slot in the V ring
+                if ((j % C::GV == 0 &&
+                     !wait_bar(b.v_full + vg, (H / C::VGROUPS) & 1, deadline, abort_flag,
+                               p.status)) ||
+                    !wait_bar(b.p_full(g, j % C::SBUF), (j / C::SBUF) & 1, deadline, abort_flag,
                               p.status))
                     return false;
                 tc::fence_after_sync();
                 const uint64_t dvs = dv + (uint64_t)((vs * C::VBYTES) >> 4);
                 const uint32_t pcol = C::S_COL + ((T + j) % C::SBUF) * 64;
 #pragma unroll
-                for (int g = 0; g < QT; ++g) {
-                    const uint32_t gcol = g * C::GROUP_COLS;
-#pragma unroll
-                    for (int kk = 0; kk < kKeys / 16; ++kk)
-                        tc::mma_f16_ts(tmem + gcol + C::O_COL, tmem + gcol + pcol + kk * 8,
-                                       dvs + (uint64_t)(kk * 16), C::IDESC_PV,
-                                       (j > 0 || kk > 0) ? 1u : 0u);
-                }
-                if (j & 1) tc::mma_commit(b.v_empty + (j / 2) % (C::VSTAGES / 2));
+                for (int kk = 0; kk < kKeys / 16; ++kk)
+                    tc::mma_f16_ts(tmem + gcol + C::O_COL, tmem + gcol + pcol + kk * 8,
+                                   dvs + (uint64_t)(kk * 16), C::IDESC_PV,
+                                   (j > 0 || kk > 0) ? 1u : 0u);
+                if (j % C::GV == C::GV - 1 || j == T - 1) tc::mma_commit(b.v_empty + vg);
                 return true;
             };
             // S = Q K^T for key tile u of the stream (pass 1: u < T).  Its
             // buffer u % SBUF last held tile u - SBUF: a pass-1 tile is given
             // back by the epilogue (s_empty); a pass-2 tile is free once the
             // P V that read its P is issued, which happens earlier in this
-            // thread's (in-order) stream.
+            // thread's (in-order) stream.  The K group's barrier is waited
+            // for at its first tile.
             auto qk = [&](int u) -> bool {
-                const int ks = u % C::KSTAGES;
+                const int jt = u < T ? u : u - T;             // key tile
+                const int G = (u < T ? 0 : nkg) + jt / C::GK;  // its K group
+                const int kg = G % C::KGROUPS;
+                const int ks = kg * C::GK + jt % C::GK;         // tile slot in the K ring
                 const int sb = u % C::SBUF;
                 const int prev = u - C::SBUF;
-                if (!wait_bar(b.k_full + ks, (u / C::KSTAGES) & 1, deadline, abort_flag, p.status))
+                if (jt % C::GK == 0 &&
+                    !wait_bar(b.k_full + kg, (G / C::KGROUPS) & 1, deadline, abort_flag, p.status))
                     return false;
                 if (prev >= 0 && prev < T &&
-                    !wait_bar(b.s_empty(sb), (prev / C::SBUF) & 1, deadline, abort_flag, p.status))
+                    !wait_bar(b.s_empty(g, sb), (prev / C::SBUF) & 1, deadline, abort_flag,
+                              p.status))
                     return false;
                 tc::fence_after_sync();
                 const uint64_t dks = dk + (uint64_t)((ks * C::KBYTES) >> 4);
                 const uint64_t dqp = u < T ? dq1 : dq2;
+                const uint32_t scol = gcol + C::S_COL + sb * 64;
 #pragma unroll
-                for (int g = 0; g < QT; ++g) {
-                    const uint32_t scol = g * C::GROUP_COLS + C::S_COL + sb * 64;
-#pragma unroll
-                    for (int kk = 0; kk < D / 32; ++kk)
-                        tc::mma_i8_ss(tmem + scol,
-                                      dqp + (uint64_t)((g * C::QBYTES) >> 4) + (uint64_t)(kk * 16),
-                                      dks + (uint64_t)(kk * 16), C::IDESC_QK, kk > 0 ? 1u : 0u);
-                }
-                tc::mma_commit(b.s_full(sb));
-                if (u & 1) tc::mma_commit(b.k_empty + (u / 2) % (C::KSTAGES / 2));
+                for (int kk = 0; kk < D / 32; ++kk)
+                    tc::mma_i8_ss(tmem + scol, dqp + (uint64_t)(kk * 16), dks + (uint64_t)(kk * 16),
+                                  C::IDESC_QK, kk > 0 ? 1u : 0u);
+                tc::mma_commit(b.s_full(g, sb));
+                if (jt % C::GK == C::GK - 1 || jt == T - 1) tc::mma_commit(b.k_empty + kg);
                 return true;
             };
             // Pass 1, then the first SBUF tiles of pass 2; after that each
@@ -359,11 +390,11 @@ attention_fwd_kernel(const Params p)
                 ok = pv(j);
                 if (ok && j + C::SBUF < T) ok = qk(T + j + C::SBUF);
             }
-            if (ok) tc::mma_commit(b.o_full());
+            if (ok) tc::mma_commit(b.o_full(g));
             // drain: wait until every MMA this thread issued has completed
-            tc::mma_commit(b.drain());
+            tc::mma_commit(b.drain(g));
             volatile int never = 0;
-            wait_bar(b.drain(), 0, tc::globaltimer_ns() + kWaitNs / 4, &never, p.status);
+            wait_bar(b.drain(g), 0, tc::globaltimer_ns() + kWaitNs / 4, &never, p.status);
         }
     } else {
         // ------------------------------------------------------------ epilogue
@@ -398,15 +429,16 @@ attention_fwd_kernel(const Params p)
             tc::tmem_ld32(lane_base + C::S_COL + (u % C::SBUF) * 64 + h * 32, rr);
         };
         auto wait_s = [&](int u) -> bool {
-            const bool w = __all_sync(kFullMask, wait_bar(b.s_full(u % C::SBUF), (u / C::SBUF) & 1,
-                                                          deadline, abort_flag, p.status));
+            const bool w = __all_sync(kFullMask, wait_bar(b.s_full(g, u % C::SBUF),
+                                                          (u / C::SBUF) & 1, deadline, abort_flag,
+                                                          p.status));
             tc::fence_after_sync();
             return w;
         };
         auto release_s = [&](int u) {
             tc::fence_before_sync();
             __syncwarp();
-            if (lane == 0) tc::mbar_arrive(b.s_empty(u % C::SBUF));
+            if (lane == 0) tc::mbar_arrive(b.s_empty(g, u % C::SBUF));
         };
         auto half_valid = [&](int j, int h) { return min(32, p.n - j * kKeys - h * 32); };
 
@@ -663,14 +695,14 @@ attention_fwd_kernel(const Params p)
             tc::tmem_wait_st();
             tc::fence_before_sync();
             __syncwarp();
-            if (ok && lane == 0) tc::mbar_arrive(b.p_full(j % C::SBUF));
+            if (ok && lane == 0) tc::mbar_arrive(b.p_full(g, j % C::SBUF));
             if (more && ok) tc::tmem_wait_ld(sa);
         }
         float Z = (zacc[0] + zacc[1]) + (zacc[2] + zacc[3]);
         if (!(Z > 0.0f)) Z = 1.0f;                    // missed or inactive rows only
 
         // output: O / Z * 2^e_h
-        if (ok) ok = __all_sync(kFullMask, wait_bar(b.o_full(), 0, deadline, abort_flag, p.status));
+        if (ok) ok = __all_sync(kFullMask, wait_bar(b.o_full(g), 0, deadline, abort_flag, p.status));
         if (ok) {
             tc::fence_after_sync();
             const float scale = ldexpf(1.0f, p.vexp[head]) / Z;
