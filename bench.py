@@ -390,38 +390,73 @@ def run_had(args, world, rank, local):
 
 
 def end_to_end(had, cfg, q, k, v, gsq, gsk, ws, dev, steps, world):
-    """Same call with inputs copied from pinned host memory and O copied back."""
+    """Same call with inputs copied from pinned host memory and O copied back.
+
+    Every step copies its Q, K, V host -> device, runs had_attention_fwd and
+    copies its O device -> host.  Steps are pipelined the way a serving loop
+    would run them: two sets of device buffers, the upload of step i + 1 on
+    one stream, the compute of step i on another and the download of step
+    i - 1 on a third, ordered by events.  The timed region runs from before
+    the first upload to after the last download.
+    """
     hq, hk, hv = q.pin_memory(), k.pin_memory(), v.pin_memory()
-    ho = torch.empty((cfg.B, cfg.H, cfg.n, cfg.d), dtype=torch.float32).pin_memory()
-    gq = torch.empty_like(q, device=dev)
-    gk = torch.empty_like(k, device=dev)
-    gv = torch.empty_like(v, device=dev)
-    out = torch.empty(ho.shape, dtype=torch.float32, device=dev)
-    stream = torch.cuda.current_stream()
+    ho = [torch.empty((cfg.B, cfg.H, cfg.n, cfg.d), dtype=torch.float32).pin_memory()
+          for _ in range(2)]
+    bufs = []
+    for i in range(2):
+        bufs.append({"q": torch.empty_like(q, device=dev), "k": torch.empty_like(k, device=dev),
+                     "v": torch.empty_like(v, device=dev),
+                     "out": torch.empty(ho[0].shape, dtype=torch.float32, device=dev),
+                     "ws": ws if i == 0 else had.workspace(cfg.B, cfg.H, cfg.n, cfg.d, cfg.N,
+                                                         device=dev)})
+    s_up, s_comp, s_down = (torch.cuda.Stream(device=dev) for _ in range(3))
+    ev = lambda: torch.cuda.Event(enable_timing=False)
+    up_done = [ev(), ev()]
+    comp_done = [ev(), ev()]
+    down_done = [ev(), ev()]
+    used = [False, False]
 
-    def step():
-        gq.copy_(hq, non_blocking=True)
-        gk.copy_(hk, non_blocking=True)
-        gv.copy_(hv, non_blocking=True)
-        had.had_attention_fwd(gq, gk, gv, gsq, gsk, cfg.N, cfg.tau, out=out, ws=ws)
-        ho.copy_(out, non_blocking=True)
+    def step(i):
+        b, h = bufs[i % 2], ho[i % 2]
+        with torch.cuda.stream(s_up):
+            if used[i % 2]:
+                s_up.wait_event(comp_done[i % 2])     # the compute of step i - 2 read them
+            b["q"].copy_(hq, non_blocking=True)
+            b["k"].copy_(hk, non_blocking=True)
+            b["v"].copy_(hv, non_blocking=True)
+            up_done[i % 2].record(s_up)
+        with torch.cuda.stream(s_comp):
+            s_comp.wait_event(up_done[i % 2])
+            if used[i % 2]:
+                s_comp.wait_event(down_done[i % 2])   # out of step i - 2 is on the host
+            had.had_attention_fwd(b["q"], b["k"], b["v"], gsq, gsk, cfg.N, cfg.tau,
+                                  out=b["out"], ws=b["ws"], stream=s_comp)
+            comp_done[i % 2].record(s_comp)
+        with torch.cuda.stream(s_down):
+            s_down.wait_event(comp_done[i % 2])
+            h.copy_(b["out"], non_blocking=True)
+            down_done[i % 2].record(s_down)
+        used[i % 2] = True
 
-    for _ in range(2):
-        step()
+    for i in range(2):
+        step(i)
     torch.cuda.synchronize()
     s = torch.cuda.Event(enable_timing=True)
     e = torch.cuda.Event(enable_timing=True)
     barrier(world)
-    s.record(stream)
-    for _ in range(steps):
-        step()
-    e.record(stream)
+    s.record(s_up)
+    for i in range(steps):
+        step(i)
+    for st in (s_up, s_comp):
+        s_down.wait_stream(st)
+    e.record(s_down)
     torch.cuda.synchronize()
     ms = max_over_ranks(s.elapsed_time(e) / steps, world, dev)
     h2d = (q.numel() + k.numel() + v.numel()) * q.element_size()
     return {"value": cfg.tokens * world / (ms * 1e-3), "unit": "tokens/s",
-            "h2d_bytes_per_step": h2d, "d2h_bytes_per_step": ho.numel() * 4,
-            "ms_per_step": ms}
+            "h2d_bytes_per_step": h2d, "d2h_bytes_per_step": ho[0].numel() * 4,
+            "ms_per_step": ms,
+            "pipelining": "two buffer sets; upload, compute and download on three streams"}
 
 
 def main():

@@ -42,7 +42,10 @@ __device__ __forceinline__ uint32_t core_offset(uint32_t row, uint32_t kbyte, ui
 }
 
 // Signs of 16 consecutive elements as int8 codes (pos / neg) in four words,
-// and as 16 packed bits (1 = negative).
+// and as 16 packed bits (1 = negative).  With a normal sigma an element at
+// or below -sigma * 2^-100 is surely negative after the division and one at
+// or above zero surely not; only elements strictly between (never seen in
+// practice, but possible) take the exact division, all 16 then together.
 template <typename T>
 __device__ __forceinline__ uint32_t sign16(const T *src, const SignRule &rule, uint32_t pos,
                                            uint32_t neg, uint32_t (&w)[4])
@@ -51,16 +54,24 @@ __device__ __forceinline__ uint32_t sign16(const T *src, const SignRule &rule, u
     Load8<T>::run(src, *reinterpret_cast<float(*)[8]>(v));
     Load8<T>::run(src + 8, *reinterpret_cast<float(*)[8]>(v + 8));
     uint32_t packed = 0;
+    bool unsure = !rule.fast;
+#pragma unroll
+    for (int i = 0; i < 16; ++i) {
+        packed |= (uint32_t)(v[i] <= -rule.thr) << i;
+        unsure |= (v[i] < 0.0f) && (v[i] > -rule.thr);
+    }
+    if (unsure) {
+        packed = 0;
+#pragma unroll
+        for (int i = 0; i < 16; ++i) packed |= negative_bit(v[i], rule) << i;
+    }
+    // byte b of word q is pos, or neg where bit 4q+b is set
+    const uint32_t flip = (pos ^ neg) & 0xFFu;
 #pragma unroll
     for (int q = 0; q < 4; ++q) {
-        uint32_t word = 0;
-#pragma unroll
-        for (int b = 0; b < 4; ++b) {
-            const uint32_t nb = negative_bit(v[4 * q + b], rule);
-            word |= (nb ? neg : pos) << (8 * b);
-            packed |= nb << (4 * q + b);
-        }
-        w[q] = word;
+        const uint32_t x = (packed >> (4 * q)) & 0xFu;
+        const uint32_t spread = (x & 1u) | ((x & 2u) << 7) | ((x & 4u) << 14) | ((x & 8u) << 21);
+        w[q] = (pos * 0x01010101u) ^ (spread * flip);
     }
     return packed;
 }

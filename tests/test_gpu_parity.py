@@ -278,3 +278,26 @@ def test_negative_tau_rejected(had):
     with pytest.raises(had.HadError) as e:
         had.had_attention_fwd(c.gq, c.gk, c.gv, c.gsq, c.gsk, c.N, -0.1)
     assert e.value.status == had.HAD_ERR_INVALID_ARG
+
+
+def test_window_misses_take_the_exact_fixup(had):
+    """Every row misses its sampled window: the first key tiles (the sample)
+    hold keys far from all queries, so the sample places the window well
+    above the true threshold level; the fix-up kernel recomputes each row."""
+    B, H, n, d, N = 1, 2, 1024, 64, 64
+    g = torch.Generator().manual_seed(77)
+    c = torch.randn(1, H, 1, d, generator=g)
+    q = (c + 0.3 * torch.randn(B, H, n, d, generator=g)).to(torch.bfloat16)
+    k = torch.randn(B, H, n, d, generator=g)
+    k[:, :, :256] = -c + 0.3 * torch.randn(B, H, 256, d, generator=g)
+    k = k.to(torch.bfloat16)
+    v = torch.randn(B, H, n, d, generator=g).to(torch.bfloat16)
+    case = Case(q, k, v, synth.per_head_sigma(q), synth.per_head_sigma(k), N, 1 / math.sqrt(d))
+    rows = all_rows(case)
+    # on the host: the window the sample places misses the threshold level
+    s = oracle.logits_rows(case.sq, case.sk, rows)
+    lev = (d - s) // 2
+    t = np.sort(lev, axis=1)[:, N - 1]
+    est = np.sort(lev[:, :256], axis=1)[:, max(1, round(N * 256 / n)) - 1]
+    assert np.mean(np.abs(t - est) > 1) > 0.9
+    _check_fused(had, case, rows)
