@@ -48,6 +48,10 @@ def _load():
             lp, lp, lp, c_int, c_long, c_long, c_long, c_long, c_long,
             ctypes.c_float, lp, c_long, lp, lp, lp, lp, c_int]
         lib.had_oracle_attention_rows.restype = c_int
+        lib.had_oracle_topn_mass_rows.argtypes = [
+            lp, lp, c_long, c_long, c_long, c_long, ctypes.c_double, lp, c_int, lp,
+            c_long, lp, c_int]
+        lib.had_oracle_topn_mass_rows.restype = c_int
         lib.had_oracle_max_threads.argtypes = []
         lib.had_oracle_max_threads.restype = c_int
         _lib = lib
@@ -137,6 +141,28 @@ def attention_rows(sq, sk, v, tau, N, rows, threads=0):
     if rc != 0:
         raise ValueError("oracle rejected the arguments (N must be in [1, n])")
     return idx, lg, p, out
+
+
+def topn_mass_rows(sq, sk, tau, p, rows, threads=0):
+    """Top-N mass retention for the given flat query rows.
+
+    Returns nmin [R, len(p)] int32: for each row and threshold p_k in (0, 1],
+    the smallest N whose N largest weights of the full softmax over all keys
+    (temperature tau, in fp64) hold at least p_k of the row's total.
+    """
+    sq = np.ascontiguousarray(sq, dtype=np.int8)
+    sk = np.ascontiguousarray(sk, dtype=np.int8)
+    B, H, n, d = sq.shape
+    assert sk.shape == sq.shape
+    rows = _rows_array(rows, B * H * n)
+    pv = np.ascontiguousarray(p, dtype=np.float64).reshape(-1)
+    out = np.empty((rows.size, pv.size), dtype=np.int32)
+    rc = _load().had_oracle_topn_mass_rows(
+        _ptr(sq), _ptr(sk), B, H, n, d, float(tau), _ptr(pv), int(pv.size), _ptr(rows),
+        rows.size, _ptr(out), int(threads))
+    if rc != 0:
+        raise ValueError("oracle rejected the arguments (each p must be in (0, 1])")
+    return out
 
 
 def attention(sq, sk, v, tau, N, threads=0):

@@ -240,6 +240,92 @@ int had_oracle_attention_rows(const int8_t *sq, const int8_t *sk,
 }
 
 /* Number of OpenMP threads a parallel region would use (1 without OpenMP). */
+/* Larger weight first. */
+static int by_weight_desc(const void *a, const void *b)
+{
+    double x = *(const double *)a, y = *(const double *)b;
+    return (x < y) - (x > y);
+}
+
+/*
+ * Top-N mass retention: the pages' premise that a small N keeps most of the
+ * softmax mass of a row (pith.science review, the "concrete test" and the
+ * free-parameter notes on N).  For each listed row and each threshold p_k
+ * in (0, 1]: the smallest N such that the N largest weights of the full
+ * softmax over all n keys (temperature tau, binarized logits) hold at least
+ * p_k of the row's total.  Plain definition in fp64: weights
+ * exp(tau (s_j - max s)), sorted in descending order, summed one by one;
+ * the total Z is the same running sum at N = n, and N is the first count
+ * whose running sum reaches p_k * Z.  Returns 0, or -1 on bad arguments or
+ * an allocation failure.
+ */
+int had_oracle_topn_mass_rows(const int8_t *sq, const int8_t *sk, long B,
+                              long H, long n, long d, double tau,
+                              const double *p, int np, const int64_t *rows,
+                              long nrows, int32_t *nmin_out, int nthreads)
+{
+    (void)B;
+    (void)H;
+    if (n < 1 || d < 1 || np < 1)
+        return -1;
+    for (int k = 0; k < np; ++k)
+        if (!(p[k] > 0.0) || p[k] > 1.0)
+            return -1;
+    int failed = 0;
+#ifdef _OPENMP
+    if (nthreads > 0)
+        omp_set_num_threads(nthreads);
+#pragma omp parallel
+#endif
+    {
+        int32_t *s = (int32_t *)malloc(sizeof(int32_t) * (size_t)n);
+        double *w = (double *)malloc(sizeof(double) * (size_t)n);
+        double *cum = (double *)malloc(sizeof(double) * (size_t)n);
+#ifdef _OPENMP
+#pragma omp for schedule(dynamic, 4)
+#endif
+        for (long t = 0; t < nrows; ++t) {
+            if (!s || !w || !cum) {
+#ifdef _OPENMP
+#pragma omp atomic write
+#endif
+                failed = 1;
+                continue;
+            }
+            long r = (long)rows[t];
+            long head = r / n;
+            row_logits(sq + r * d, sk + head * n * d, n, d, s);
+            int32_t m = s[0];
+            for (long j = 1; j < n; ++j)
+                if (s[j] > m)
+                    m = s[j];
+            for (long j = 0; j < n; ++j)
+                w[j] = exp(tau * (double)(s[j] - m));
+            qsort(w, (size_t)n, sizeof(double), by_weight_desc);
+            double acc = 0.0;
+            for (long j = 0; j < n; ++j) {
+                acc += w[j];
+                cum[j] = acc;
+            }
+            const double Z = cum[n - 1];
+            for (int k = 0; k < np; ++k) {
+                const double target = p[k] * Z;
+                long N = n;
+                for (long j = 0; j < n; ++j)
+                    if (cum[j] >= target) {
+                        N = j + 1;
+                        break;
+                    }
+                nmin_out[t * np + k] = (int32_t)N;
+            }
+        }
+        free(s);
+        free(w);
+        free(cum);
+    }
+    return failed ? -1 : 0;
+}
+
 int had_oracle_max_threads(void)
 {
 #ifdef _OPENMP

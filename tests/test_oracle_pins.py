@@ -332,3 +332,65 @@ def test_oracle_rejects_bad_N(N):
     sq, sk, v = _binarized((1, 1, 50, 64), seed=90)
     with pytest.raises(ValueError):
         oracle.attention(sq, sk, v, 0.125, N)
+
+
+# ------------------------------------------------------ top-N mass retention
+# The smallest N whose N largest softmax weights (full softmax over all keys)
+# reach a fraction p of the row's total; pinned by closed forms and by an
+# independent numpy brute force.
+
+
+def test_mass_all_keys_equal_is_ceil_p_n():
+    # equal logits: every weight is 1, so N = ceil(p n)
+    sq, sk, _ = _binarized((1, 1, 40, 64), seed=100)
+    sk[...] = sk[:, :, :1]
+    p = [0.1, 0.25, 0.5, 0.9, 1.0]
+    got = oracle.topn_mass_rows(sq, sk, 0.125, p, np.arange(40))
+    assert (got == np.array([math.ceil(x * 40) for x in p])[None, :]).all()
+
+
+def test_mass_two_levels_closed_form():
+    # k1 keys equal to the query (logit d) and the rest its negation (-d):
+    # weights 1 and e = exp(-2 tau d); Z = k1 + (n - k1) e
+    n, d, k1, tau = 64, 64, 5, 0.03
+    rng = np.random.default_rng(3)
+    q = np.where(rng.random(d) < 0.5, -1, 1).astype(np.int8)
+    sq = np.broadcast_to(q, (1, 1, n, d)).copy()
+    sk = np.broadcast_to(-q, (1, 1, n, d)).copy()
+    sk[0, 0, 7:7 + k1] = q
+    e = math.exp(-2 * tau * d)
+    Z = k1 + (n - k1) * e
+    p = [0.2, k1 / Z - 1e-9, 0.9, 0.99]
+    got = oracle.topn_mass_rows(sq, sk, tau, p, [0])[0]
+    for pk, g in zip(p, got):
+        t = pk * Z
+        want = math.ceil(t - 1e-12) if t <= k1 else k1 + math.ceil((t - k1) / e - 1e-9)
+        assert g == want, (pk, g, want)
+
+
+def test_mass_matches_numpy_brute_force():
+    sq, sk, _ = _binarized((1, 2, 300, 64), seed=110)
+    p = np.array([0.5, 0.9, 0.95, 0.99])
+    tau = 0.125
+    got = oracle.topn_mass_rows(sq, sk, tau, p, np.arange(600))
+    s = np.einsum("hik,hjk->hij", sq[0].astype(np.float64), sk[0].astype(np.float64))
+    w = np.exp(tau * (s - s.max(axis=-1, keepdims=True))).reshape(600, 300)
+    cum = np.cumsum(-np.sort(-w, axis=1), axis=1)
+    want = np.stack([np.argmax(cum >= pk * cum[:, -1:], axis=1) + 1 for pk in p], axis=1)
+    # equal up to fp64 rounding at an exact boundary (none is expected here)
+    assert np.array_equal(got, want)
+
+
+def test_mass_monotone_in_p_and_bounded():
+    sq, sk, _ = _binarized((1, 1, 200, 64), seed=120)
+    p = np.linspace(0.05, 1.0, 20)
+    got = oracle.topn_mass_rows(sq, sk, 0.125, p, np.arange(200))
+    assert (np.diff(got, axis=1) >= 0).all()
+    assert (got >= 1).all() and (got <= 200).all()
+
+
+@pytest.mark.parametrize("p", [0.0, -0.5, 1.5])
+def test_mass_rejects_bad_p(p):
+    sq, sk, _ = _binarized((1, 1, 10, 64), seed=130)
+    with pytest.raises(ValueError):
+        oracle.topn_mass_rows(sq, sk, 0.125, [p], [0])
