@@ -48,6 +48,8 @@ def parse():
                     help="target CPU time of the oracle baseline sample")
     ap.add_argument("--no-e2e", action="store_true")
     ap.add_argument("--no-cpu-baseline", action="store_true")
+    ap.add_argument("--mode", choices=["attention", "mass"], default="attention",
+                    help="mass: time the top-N mass-retention diagnostic instead")
     return ap.parse_args()
 
 
@@ -459,12 +461,62 @@ def end_to_end(had, cfg, q, k, v, gsq, gsk, ws, dev, steps, world):
             "pipelining": "two buffer sets; upload, compute and download on three streams"}
 
 
+def run_mass(args, world, rank, local):
+    """The top-N mass-retention diagnostic (had_topn_mass) on the workload's
+    binarized Q and K: rows per second, against the popcount roofline of its
+    histogram pass (d/32 popcounts per (query, key) pair at 16 per clock per
+    SM)."""
+    from sparse_attention_sigma_b200 import had
+    cfg = synth.CONFIGS[args.config]
+    dev = torch.device("cuda", local)
+    torch.cuda.set_device(dev)
+    q, k, _, sgq, sgk = synth.make_inputs(cfg)
+    qb = had.had_binarize_pack(q.to(dev), sgq.to(dev))
+    kb = had.had_binarize_pack(k.to(dev), sgk.to(dev))
+    p = [0.9, 0.95, 0.99]
+    nmin = torch.empty((cfg.B, cfg.H, cfg.n, len(p)), dtype=torch.int32, device=dev)
+    step = lambda: had.had_topn_mass(qb, kb, cfg.d, cfg.tau, p, nmin=nmin)
+    for _ in range(max(3, args.warmup)):
+        step()
+    torch.cuda.synchronize()
+    s = torch.cuda.Event(enable_timing=True)
+    e = torch.cuda.Event(enable_timing=True)
+    barrier(world)
+    s.record()
+    for _ in range(args.steps):
+        step()
+    e.record()
+    torch.cuda.synchronize()
+    ms = max_over_ranks(s.elapsed_time(e) / args.steps, world, dev)
+    rows = cfg.B * cfg.H * cfg.n * world
+    popc = cfg.B * cfg.H * cfg.n * cfg.n * (cfg.d // 32) * world
+    peak = SM_COUNT * 16 * 1.965e9 * world
+    med = nmin.reshape(-1, len(p)).float().median(dim=0).values.tolist()
+    if rank == 0:
+        print(json.dumps({
+            "metric": "top-N mass-retention diagnostic rows/sec", "value": rows / (ms * 1e-3),
+            "unit": "rows/s", "n_gpus": world, "steps": args.steps, "warmup": args.warmup,
+            "ms_per_step": ms, "higher_is_better": True, "scaling": "weak", "dtype": "u32/f64",
+            "data": "synthetic", "impl": "had_topn_mass",
+            "config": {"workload": cfg.describe(),
+                       "p": p},
+            "median_nmin": dict(zip([str(x) for x in p], med)),
+            "roofline": {"bound": "alu", "achieved": popc / (ms * 1e-3) / 1e12,
+                         "peak": peak / 1e12, "unit": "Tpopc/s",
+                         "frac": popc / (ms * 1e-3) / peak,
+                         "note": "popcount pipe, 16/clk/SM at 1.965 GHz"},
+            "gpu_launches": args.steps,
+        }), flush=True)
+
+
 def main():
     args = parse()
     world, rank, local = dist_setup(args)
     try:
         if args.impl == "reference":
             run_reference(args, world, rank)
+        elif args.mode == "mass":
+            run_mass(args, world, rank, local)
         else:
             run_had(args, world, rank, local)
     finally:

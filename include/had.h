@@ -74,7 +74,8 @@ typedef enum {
     HAD_OP_ATTENTION_FWD = 2,     /* had_attention_fwd */
     HAD_OP_SPARSE_SOFTMAX_AV = 3, /* had_sparse_softmax_av */
     HAD_OP_ATTENTION_PREPARE = 4, /* had_attention_prepare */
-    HAD_OP_ATTENTION_CORE = 5     /* had_attention_core */
+    HAD_OP_ATTENTION_CORE = 5,    /* had_attention_core */
+    HAD_OP_TOPN_MASS = 6          /* had_topn_mass */
 } had_op_t;
 
 /*
@@ -158,6 +159,26 @@ HAD_API had_status_t had_attention_core(const void *V, had_dtype_t dt, int B, in
                                         int d, int N, float tau, float *out, int32_t *dbg_idx,
                                         int16_t *dbg_logits, void *ws, size_t ws_bytes,
                                         int32_t *dev_status, cudaStream_t stream);
+
+/*
+ * Top-N mass retention diagnostic ("Hamming Attention Distillation",
+ * pith.science review: the concrete test of the premise that a small N keeps
+ * most of the softmax mass, and the free-parameter notes on N).  For every
+ * query row and every threshold p[k]: the smallest N such that the N
+ * largest weights of the full softmax over all n keys (temperature tau,
+ * binarized logits s = d - 2 Hamming) hold at least p[k] of the row's total.
+ * Computed from the row's histogram of logit levels, in fp64.
+ *   qbits, kbits  [B,H,n,d/32] uint32 (device), as had_binarize_pack writes
+ *   tau           >= 0
+ *   p             np thresholds in (0, 1] (HOST memory, read during the call)
+ *   np            1 .. 8
+ *   nmin          [B,H,n,np] int32 out (device)
+ * No workspace.  Invalid arguments return HAD_ERR_INVALID_ARG before any
+ * launch; d outside {64, 128} returns HAD_ERR_UNSUPPORTED.
+ */
+HAD_API had_status_t had_topn_mass(const uint32_t *qbits, const uint32_t *kbits, int B, int H,
+                                   int n, int d, float tau, const double *p, int np,
+                                   int32_t *nmin, int32_t *dev_status, cudaStream_t stream);
 
 /*
  * had_attention_fwd for callers that cannot allocate device memory.

@@ -13,6 +13,7 @@
 #include "had_av.cuh"
 #include "had_prep.cuh"
 #include "had_fused.cuh"
+#include "had_mass.cuh"
 
 namespace {
 
@@ -281,6 +282,21 @@ had_status_t noalloc_scratch(void **ptr)
     return HAD_OK;
 }
 
+template <int DW>
+had_status_t launch_mass_dw(const uint32_t *qb, const uint32_t *kb, int B, int H, int n,
+                            float tau, const had::MassP &ps, int32_t *nmin, cudaStream_t st)
+{
+    constexpr int smem = had::mass_smem_bytes<DW>();
+    if (cudaFuncSetAttribute(had::topn_mass_kernel<DW>,
+                             cudaFuncAttributeMaxDynamicSharedMemorySize, smem) != cudaSuccess)
+        return HAD_ERR_CUDA;
+    const long long blocks = (long long)((n + had::kTopnRows - 1) / had::kTopnRows) * B * H;
+    if (blocks > INT_MAX) return HAD_ERR_UNSUPPORTED;
+    had::topn_mass_kernel<DW><<<(unsigned)blocks, had::kTopnRows, smem, st>>>(
+        qb, kb, n, (double)tau, ps, nmin);
+    return launched();
+}
+
 }  // namespace
 
 extern "C" {
@@ -441,6 +457,26 @@ had_status_t had_attention_fwd_noalloc(const void *Q, const void *K, const void 
 
 size_t had_noalloc_scratch_bytes(void) { return kNoAllocScratchBytes; }
 
+had_status_t had_topn_mass(const uint32_t *qbits, const uint32_t *kbits, int B, int H, int n,
+                           int d, float tau, const double *p, int np, int32_t *nmin,
+                           int32_t *dev_status, cudaStream_t stream)
+{
+    (void)dev_status;
+    had_status_t s = check_shape(B, H, n, d);
+    if (s != HAD_OK) return s;
+    if (!qbits || !kbits || !nmin || !p) return HAD_ERR_INVALID_ARG;
+    if (!aligned16(qbits) || !aligned16(kbits) || !aligned16(nmin)) return HAD_ERR_INVALID_ARG;
+    if (np < 1 || np > had::kMassMaxP || !(tau >= 0.0f) || !isfinite(tau)) return HAD_ERR_INVALID_ARG;
+    had::MassP ps{};
+    ps.np = np;
+    for (int k = 0; k < np; ++k) {
+        if (!(p[k] > 0.0) || p[k] > 1.0) return HAD_ERR_INVALID_ARG;
+        ps.p[k] = p[k];
+    }
+    return d == 64 ? launch_mass_dw<2>(qbits, kbits, B, H, n, tau, ps, nmin, stream)
+                   : launch_mass_dw<4>(qbits, kbits, B, H, n, tau, ps, nmin, stream);
+}
+
 size_t had_workspace_bytes(int op, int B, int H, int n, int d, int N)
 {
     switch (op) {
@@ -454,6 +490,8 @@ size_t had_workspace_bytes(int op, int B, int H, int n, int d, int N)
     case HAD_OP_ATTENTION_CORE:
         if (check_topn(B, H, n, d, N) != HAD_OK) return (size_t)-1;
         return fwd_layout(B, H, n, d, N).total;
+    case HAD_OP_TOPN_MASS:
+        return check_shape(B, H, n, d) == HAD_OK ? 0 : (size_t)-1;
     default:
         return (size_t)-1;
     }
@@ -473,6 +511,8 @@ int had_launch_count(int op, int B, int H, int n, int d, int N)
         return check_topn(B, H, n, d, N) == HAD_OK ? 2 : -1;
     case HAD_OP_ATTENTION_CORE:
         return check_topn(B, H, n, d, N) == HAD_OK ? 2 : -1;
+    case HAD_OP_TOPN_MASS:
+        return check_shape(B, H, n, d) == HAD_OK ? 1 : -1;
     default:
         return -1;
     }

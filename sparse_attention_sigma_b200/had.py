@@ -33,6 +33,7 @@ HAD_OP_ATTENTION_FWD = 2
 HAD_OP_SPARSE_SOFTMAX_AV = 3
 HAD_OP_ATTENTION_PREPARE = 4
 HAD_OP_ATTENTION_CORE = 5
+HAD_OP_TOPN_MASS = 6
 
 
 class HadError(RuntimeError):
@@ -58,6 +59,7 @@ def _load():
                                       vp, vp],
         "had_attention_prepare": [vp, vp, vp, i32, vp, vp, i32, i32, i32, i32, i32, vp, sz, vp, vp],
         "had_attention_core": [vp, i32, i32, i32, i32, i32, i32, f32, vp, vp, vp, vp, sz, vp, vp],
+        "had_topn_mass": [vp, vp, i32, i32, i32, i32, f32, vp, i32, vp, vp, vp],
     }
     for name, args in sig.items():
         fn = getattr(lib, name)
@@ -171,6 +173,25 @@ def had_hamming_topn(qbits, kbits, d, N, idx=None, logits=None, ws=None, dev_sta
                                _stream(stream))
     _check(st, "had_hamming_topn")
     return idx, logits
+
+
+def had_topn_mass(qbits, kbits, d, tau, p, nmin=None, dev_status=None, stream=None):
+    """Top-N mass retention: nmin [B,H,n,len(p)] int32, the smallest N whose N
+    largest softmax weights (over all keys) hold at least p[k] of a row's mass."""
+    _dev(qbits, "qbits", torch.int32)
+    B, H, n, w = _shape4(qbits, "qbits")
+    if w * 32 != d:
+        raise ValueError("qbits last dimension must be d/32")
+    _dev(kbits, "kbits", torch.int32, (B, H, n, w))
+    pv = (ctypes.c_double * len(p))(*[float(x) for x in p])
+    if nmin is None:
+        nmin = torch.empty((B, H, n, len(p)), dtype=torch.int32, device=qbits.device)
+    _dev(nmin, "nmin", torch.int32, (B, H, n, len(p)))
+    st = _lib.had_topn_mass(_ptr(qbits), _ptr(kbits), B, H, n, d, ctypes.c_float(tau),
+                            ctypes.cast(pv, ctypes.c_void_p), len(p), _ptr(nmin),
+                            _ptr(dev_status), _stream(stream))
+    _check(st, "had_topn_mass")
+    return nmin
 
 
 def had_sparse_softmax_av(idx, logits, V, tau, out=None, p=None, want_p=False, dev_status=None,

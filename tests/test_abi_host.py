@@ -83,3 +83,25 @@ def test_argument_errors_return_before_any_cuda_call(lib):
     # misaligned pointer
     assert f(vp(4097), fake, fake, 0, fake, fake, 1, 1, 8, 64, 2, 0.1, fake, None, None,
              fake, 1 << 20, None, None) == 1
+
+
+def test_topn_mass_argument_errors_return_before_any_cuda_call(lib):
+    f = lib.had_topn_mass
+    vp, i = ctypes.c_void_p, ctypes.c_int
+    f.argtypes = [vp, vp, i, i, i, i, ctypes.c_float, vp, i, vp, vp, vp]
+    f.restype = ctypes.c_int
+    fake = vp(4096)        # never dereferenced: the checks fail first
+    good = (ctypes.c_double * 3)(0.5, 0.9, 1.0)
+    bad = (ctypes.c_double * 1)(1.5)
+    p = lambda a: ctypes.cast(a, vp)
+    assert f(fake, fake, 1, 1, 8, 96, 0.1, p(good), 3, fake, None, None) == 2    # d
+    assert f(fake, fake, 1, 1, 8, 64, 0.1, p(good), 0, fake, None, None) == 1    # np = 0
+    assert f(fake, fake, 1, 1, 8, 64, 0.1, p(good), 9, fake, None, None) == 1    # np > 8
+    assert f(fake, fake, 1, 1, 8, 64, 0.1, p(bad), 1, fake, None, None) == 1     # p > 1
+    assert f(fake, fake, 1, 1, 8, 64, -0.1, p(good), 3, fake, None, None) == 1   # tau < 0
+    assert f(fake, fake, 1, 1, 8, 64, 0.1, None, 3, fake, None, None) == 1       # no p
+    lib.had_workspace_bytes.restype = ctypes.c_size_t
+    lib.had_workspace_bytes.argtypes = [ctypes.c_int] * 6
+    lib.had_launch_count.argtypes = [ctypes.c_int] * 6
+    assert lib.had_workspace_bytes(6, 1, 1, 8, 64, 0) == 0
+    assert lib.had_launch_count(6, 1, 1, 8, 64, 0) == 1

@@ -301,3 +301,39 @@ def test_window_misses_take_the_exact_fixup(had):
     est = np.sort(lev[:, :256], axis=1)[:, max(1, round(N * 256 / n)) - 1]
     assert np.mean(np.abs(t - est) > 1) > 0.9
     _check_fused(had, case, rows)
+
+
+def _mass_check(had, c, p, rows):
+    """Kernel vs oracle, exact except where the fp64 sums put p Z within
+    rounding of a boundary (then the two may differ by one key)."""
+    qb = had.had_binarize_pack(c.gq, c.gsq)
+    kb = had.had_binarize_pack(c.gk, c.gsk)
+    got = had.had_topn_mass(qb, kb, c.d, c.tau, p).reshape(-1, len(p)).cpu().numpy()[rows]
+    tau32 = float(np.float32(c.tau))           # the C ABI takes tau as fp32
+    want = oracle.topn_mass_rows(c.sq, c.sk, tau32, p, rows)
+    diff = np.argwhere(got != want)
+    if len(diff):
+        s = oracle.logits_rows(c.sq, c.sk, rows).astype(np.float64)
+        w = np.exp(tau32 * (s - s.max(axis=1, keepdims=True)))
+        cum = np.cumsum(-np.sort(-w, axis=1), axis=1)
+        for r, k in diff:
+            assert abs(int(got[r, k]) - int(want[r, k])) == 1
+            lo = min(got[r, k], want[r, k]) - 1
+            tgt = p[k] * cum[r, -1]
+            assert abs(cum[r, lo] - tgt) <= 1e-12 * cum[r, -1], (r, k)
+    return got
+
+
+@pytest.mark.parametrize("B,H,n,d,seed", [(1, 2, 300, 64, 11), (2, 1, 257, 128, 12),
+                                          (1, 1, 1, 64, 13)])
+def test_topn_mass_small_all_rows(had, B, H, n, d, seed):
+    c = random_case(B, H, n, d, max(1, n // 8), seed)
+    p = [0.5, 0.9, 0.95, 0.99, 1.0]
+    got = _mass_check(had, c, p, all_rows(c))
+    assert (np.diff(got, axis=1) >= 0).all()
+
+
+def test_topn_mass_long_workload_sampled(had):
+    c = config_case("long")
+    rows = synth.sample_rows(synth.CONFIGS["long"], 256, seed=21)
+    _mass_check(had, c, [0.9, 0.95, 0.99], rows)
