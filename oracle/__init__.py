@@ -48,6 +48,10 @@ def _load():
             lp, lp, lp, c_int, c_long, c_long, c_long, c_long, c_long,
             ctypes.c_float, lp, c_long, lp, lp, lp, lp, c_int]
         lib.had_oracle_attention_rows.restype = c_int
+        lib.had_oracle_attention_causal_rows.argtypes = [
+            lp, lp, lp, c_int, c_long, c_long, c_long, c_long, c_long,
+            ctypes.c_float, lp, c_long, lp, lp, lp, lp, c_int]
+        lib.had_oracle_attention_causal_rows.restype = c_int
         lib.had_oracle_topn_mass_rows.argtypes = [
             lp, lp, c_long, c_long, c_long, c_long, ctypes.c_double, lp, c_int, lp,
             c_long, lp, c_int]
@@ -135,6 +139,30 @@ def attention_rows(sq, sk, v, tau, N, rows, threads=0):
     p = np.empty((R, N), dtype=np.float64)
     out = np.empty((R, d), dtype=np.float32)
     rc = _load().had_oracle_attention_rows(
+        _ptr(sq), _ptr(sk), _ptr(v), _is_bf16(v), B, H, n, d, int(N),
+        ctypes.c_float(float(tau)), _ptr(rows), R, _ptr(idx), _ptr(lg), _ptr(p),
+        _ptr(out), int(threads))
+    if rc != 0:
+        raise ValueError("oracle rejected the arguments (N must be in [1, n])")
+    return idx, lg, p, out
+
+
+def attention_causal_rows(sq, sk, v, tau, N, rows, threads=0):
+    """Causal top-N attention for the given flat query rows: query i of a head
+    sees keys 0..i and keeps min(N, i+1) of them.  Same outputs as
+    attention_rows; empty slots hold idx -1, logit 0, p 0."""
+    sq = np.ascontiguousarray(sq, dtype=np.int8)
+    sk = np.ascontiguousarray(sk, dtype=np.int8)
+    v = np.ascontiguousarray(v)
+    B, H, n, d = sq.shape
+    assert sk.shape == sq.shape and v.shape == sq.shape
+    rows = _rows_array(rows, B * H * n)
+    R = rows.size
+    idx = np.empty((R, N), dtype=np.int32)
+    lg = np.empty((R, N), dtype=np.int16)
+    p = np.empty((R, N), dtype=np.float64)
+    out = np.empty((R, d), dtype=np.float32)
+    rc = _load().had_oracle_attention_causal_rows(
         _ptr(sq), _ptr(sk), _ptr(v), _is_bf16(v), B, H, n, d, int(N),
         ctypes.c_float(float(tau)), _ptr(rows), R, _ptr(idx), _ptr(lg), _ptr(p),
         _ptr(out), int(threads))

@@ -240,6 +240,93 @@ int had_oracle_attention_rows(const int8_t *sq, const int8_t *sk,
 }
 
 /* Number of OpenMP threads a parallel region would use (1 without OpenMP). */
+/*
+ * Causal variant (the review's note that decoder LLMs are the target of the
+ * long-context claims; the pages print no causal rule, so this is the plain
+ * reading): query i of a head sees keys 0 .. i only and keeps the
+ * N_i = min(N, i + 1) largest visible logits, ties to the lower index, in
+ * ascending key order; softmax over the kept logits and the value product
+ * as in the non-causal case.  Slots N_i .. N-1 of a row are empty: idx -1,
+ * logit 0, p 0.
+ */
+int had_oracle_attention_causal_rows(const int8_t *sq, const int8_t *sk,
+                                     const void *v, int v_is_bf16, long B,
+                                     long H, long n, long d, long N,
+                                     float tau, const int64_t *rows,
+                                     long nrows, int32_t *idx_out,
+                                     int16_t *s_out, double *p_out,
+                                     float *o_out, int nthreads)
+{
+    (void)B;
+    (void)H;
+    if (N < 1 || N > n || d < 1 || n < 1)
+        return -1;
+    int failed = 0;
+#ifdef _OPENMP
+    if (nthreads > 0)
+        omp_set_num_threads(nthreads);
+#pragma omp parallel
+#endif
+    {
+        int32_t *s = (int32_t *)malloc(sizeof(int32_t) * (size_t)n);
+        keyed_t *order = (keyed_t *)malloc(sizeof(keyed_t) * (size_t)n);
+        double *e = (double *)malloc(sizeof(double) * (size_t)N);
+#ifdef _OPENMP
+#pragma omp for schedule(dynamic, 4)
+#endif
+        for (long t = 0; t < nrows; ++t) {
+            if (!s || !order || !e) {
+#ifdef _OPENMP
+#pragma omp atomic write
+#endif
+                failed = 1;
+                continue;
+            }
+            long r = (long)rows[t];
+            long head = r / n;
+            long i = r % n;                  /* position of the query */
+            long vis = i + 1;                /* keys 0 .. i are visible */
+            long Ni = N < vis ? N : vis;
+            row_logits(sq + r * d, sk + head * n * d, vis, d, s);
+            for (long j = 0; j < vis; ++j) {
+                order[j].s = s[j];
+                order[j].j = (int32_t)j;
+            }
+            qsort(order, (size_t)vis, sizeof(keyed_t), by_logit_then_index);
+            qsort(order, (size_t)Ni, sizeof(keyed_t), by_index);
+            int32_t m = order[0].s;
+            for (long k = 1; k < Ni; ++k)
+                if (order[k].s > m)
+                    m = order[k].s;
+            double Z = 0.0;
+            for (long k = 0; k < Ni; ++k) {
+                e[k] = exp((double)tau * (double)(order[k].s - m));
+                Z += e[k];
+            }
+            for (long k = 0; k < N; ++k) {
+                const int kept = k < Ni;
+                idx_out[t * N + k] = kept ? order[k].j : -1;
+                s_out[t * N + k] = kept ? (int16_t)order[k].s : 0;
+                if (p_out)
+                    p_out[t * N + k] = kept ? e[k] / Z : 0.0;
+            }
+            const long vbase = head * n * d;
+            for (long c = 0; c < d; ++c) {
+                double acc = 0.0;
+                for (long k = 0; k < Ni; ++k)
+                    acc += (e[k] / Z) *
+                           (double)load_elem(v, v_is_bf16,
+                                             vbase + (long)order[k].j * d + c);
+                o_out[t * d + c] = (float)acc;
+            }
+        }
+        free(s);
+        free(order);
+        free(e);
+    }
+    return failed ? -1 : 0;
+}
+
 /* Larger weight first. */
 static int by_weight_desc(const void *a, const void *b)
 {

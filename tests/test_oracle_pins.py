@@ -394,3 +394,46 @@ def test_mass_rejects_bad_p(p):
     sq, sk, _ = _binarized((1, 1, 10, 64), seed=130)
     with pytest.raises(ValueError):
         oracle.topn_mass_rows(sq, sk, 0.125, [p], [0])
+
+
+# --------------------------------------------------------------- causal variant
+# Query i sees keys 0..i and keeps min(N, i+1) of them; empty slots hold
+# idx -1, logit 0, p 0.
+
+
+def test_causal_last_row_is_the_full_row():
+    sq, sk, v = _binarized((1, 2, 60, 64), seed=140)
+    rows = np.array([59, 119])                    # last position of each head
+    a = oracle.attention_causal_rows(sq, sk, v, 0.125, 12, rows)
+    b = oracle.attention_rows(sq, sk, v, 0.125, 12, rows)
+    for x, y in zip(a, b):
+        assert np.array_equal(x, y)
+
+
+def test_causal_row_is_the_truncated_problem():
+    # row i equals the non-causal answer on keys 0..i with N_i = min(N, i+1)
+    sq, sk, v = _binarized((1, 1, 50, 64), seed=150)
+    N = 9
+    for i in (0, 3, 8, 9, 20, 49):
+        idx, lg, p, out = oracle.attention_causal_rows(sq, sk, v, 0.125, N, [i])
+        Ni = min(N, i + 1)
+        sub = oracle.attention_rows(sq[:, :, :i + 1], sk[:, :, :i + 1], v[:, :, :i + 1],
+                                    0.125, Ni, [i])
+        assert np.array_equal(idx[0, :Ni], sub[0][0]) and (idx[0, Ni:] == -1).all()
+        assert np.array_equal(lg[0, :Ni], sub[1][0]) and (lg[0, Ni:] == 0).all()
+        assert np.array_equal(p[0, :Ni], sub[2][0]) and (p[0, Ni:] == 0).all()
+        assert np.array_equal(out[0], sub[3][0])
+
+
+def test_causal_dense_rows_match_masked_softmax():
+    # with N = n every row keeps all visible keys: a dense masked softmax
+    sq, sk, v = _binarized((1, 1, 40, 64), seed=160)
+    tau = 0.2
+    idx, lg, p, out = oracle.attention_causal_rows(sq, sk, v, tau, 40, np.arange(40))
+    s = torch.tensor(sq[0, 0], dtype=torch.float64) @ torch.tensor(sk[0, 0], dtype=torch.float64).T
+    mask = torch.tril(torch.ones(40, 40, dtype=torch.bool))
+    w = torch.softmax((tau * s).masked_fill(~mask, float("-inf")), dim=-1)
+    ref = (w @ torch.tensor(v[0, 0], dtype=torch.float64)).numpy()
+    assert np.allclose(out, ref, rtol=1e-6, atol=1e-6)
+    assert np.allclose(p.sum(axis=1), 1.0, atol=1e-12)
+    assert (idx[0] == [0] + [-1] * 39).all() and out[0].tolist() == v[0, 0, 0].tolist()
