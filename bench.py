@@ -48,7 +48,7 @@ def parse():
                     help="target CPU time of the oracle baseline sample")
     ap.add_argument("--no-e2e", action="store_true")
     ap.add_argument("--no-cpu-baseline", action="store_true")
-    ap.add_argument("--mode", choices=["attention", "mass"], default="attention",
+    ap.add_argument("--mode", choices=["attention", "mass", "causal"], default="attention",
                     help="mass: time the top-N mass-retention diagnostic instead")
     return ap.parse_args()
 
@@ -509,6 +509,83 @@ def run_mass(args, world, rank, local):
         }), flush=True)
 
 
+def run_causal(args, world, rank, local):
+    """The causal forward (had_attention_causal_fwd) on the workload: tokens per
+    second, issued as its three stages so that each has its own events.  The
+    dominant kernel is the causal top-N selection, bound by the popcount pipe:
+    d/32 popcounts per visible (query, key) pair, n (n + 1) / 2 pairs a head."""
+    from sparse_attention_sigma_b200 import had
+    cfg = synth.CONFIGS[args.config]
+    dev = torch.device("cuda", local)
+    torch.cuda.set_device(dev)
+    stream = torch.cuda.current_stream()
+    q, k, v, sgq, sgk = synth.make_inputs(cfg)
+    gq, gk, gv = q.to(dev), k.to(dev), v.to(dev)
+    gsq, gsk = sgq.to(dev), sgk.to(dev)
+    shape = (cfg.B, cfg.H, cfg.n)
+    qb = torch.empty(shape + (cfg.d // 32,), dtype=torch.int32, device=dev)
+    kb = torch.empty_like(qb)
+    idx = torch.empty(shape + (cfg.N,), dtype=torch.int32, device=dev)
+    lg = torch.empty(shape + (cfg.N,), dtype=torch.int16, device=dev)
+    out = torch.empty(shape + (cfg.d,), dtype=torch.float32, device=dev)
+    flush = torch.empty(L2_FLUSH_BYTES // 4, dtype=torch.float32, device=dev)
+
+    def stages():
+        had.had_binarize_pack(gq, gsq, bits=qb)
+        had.had_binarize_pack(gk, gsk, bits=kb)
+        yield
+        had.had_hamming_topn_causal(qb, kb, cfg.d, cfg.N, idx=idx, logits=lg)
+        yield
+        had.had_sparse_softmax_av(idx, lg, gv, cfg.tau, out=out)
+        yield
+
+    for _ in range(max(3, args.warmup)):
+        for _ in stages():
+            pass
+    # the one-call entry point computes the same thing
+    ref = had.had_attention_causal_fwd(gq, gk, gv, gsq, gsk, cfg.N, cfg.tau)
+    torch.cuda.synchronize()
+    if not torch.equal(ref, out):
+        raise RuntimeError("had_attention_causal_fwd differs from its three stages")
+    clocks = ClockSampler(local)
+    clocks.start()
+    ev = [[torch.cuda.Event(enable_timing=True) for _ in range(4)] for _ in range(args.steps)]
+    barrier(world)
+    torch.cuda.synchronize()
+    for i in range(args.steps):
+        flush.fill_(float(i))
+        ev[i][0].record(stream)
+        for j, _ in enumerate(stages()):
+            ev[i][j + 1].record(stream)
+    torch.cuda.synchronize()
+    barrier(world)
+    clock_info = clocks.stop()
+    stage_ms = [sum(e[j].elapsed_time(e[j + 1]) for e in ev) / args.steps for j in range(3)]
+    value, ms = aggregate(cfg.tokens, sum(stage_ms), world, dev)
+    topn_ms = max_over_ranks(stage_ms[1], world, dev)
+    popc = cfg.B * cfg.H * cfg.n * (cfg.n + 1) // 2 * (cfg.d // 32)
+    peak = SM_COUNT * 16 * 1.965e9
+    if rank != 0:
+        return
+    print(json.dumps({
+        "metric": "HAD causal attention tokens/sec", "value": value, "unit": "tokens/s",
+        "n_gpus": world, "steps": args.steps, "warmup": max(3, args.warmup), "ms_per_step": ms,
+        "higher_is_better": True, "scaling": "weak", "vs_baseline": None, "dtype": "bf16",
+        "data": "synthetic", "impl": "had_attention_causal_fwd",
+        "config": {"workload": cfg.describe(), "causal": True,
+                   "l2": "flushed between steps (256 MiB write outside the timed events)"},
+        "stage_ms": {"binarize_pack": stage_ms[0], "hamming_topn_causal": stage_ms[1],
+                     "sparse_softmax_av": stage_ms[2]},
+        "roofline": {"bound": "alu", "achieved": popc / (topn_ms * 1e-3) / 1e12,
+                     "peak": peak / 1e12, "unit": "Tpopc/s", "frac": popc / (topn_ms * 1e-3) / peak,
+                     "kernel": "topn_simt_kernel (causal)",
+                     "note": "popcount pipe, 16/clk/SM at 1.965 GHz; one popcount per 32 bits "
+                             "of each visible (query, key) pair"},
+        "gpu_launches": 4 * args.steps,
+        "clocks": clock_info,
+    }), flush=True)
+
+
 def main():
     args = parse()
     world, rank, local = dist_setup(args)
@@ -517,6 +594,8 @@ def main():
             run_reference(args, world, rank)
         elif args.mode == "mass":
             run_mass(args, world, rank, local)
+        elif args.mode == "causal":
+            run_causal(args, world, rank, local)
         else:
             run_had(args, world, rank, local)
     finally:

@@ -75,7 +75,8 @@ typedef enum {
     HAD_OP_SPARSE_SOFTMAX_AV = 3, /* had_sparse_softmax_av */
     HAD_OP_ATTENTION_PREPARE = 4, /* had_attention_prepare */
     HAD_OP_ATTENTION_CORE = 5,    /* had_attention_core */
-    HAD_OP_TOPN_MASS = 6          /* had_topn_mass */
+    HAD_OP_TOPN_MASS = 6,         /* had_topn_mass */
+    HAD_OP_ATTENTION_CAUSAL = 7   /* had_attention_causal_fwd */
 } had_op_t;
 
 /*
@@ -112,8 +113,10 @@ HAD_API had_status_t had_hamming_topn(const uint32_t *qbits, const uint32_t *kbi
  *   tau    softmax temperature (1/sqrt(d) in the reference workloads)
  *   out    [B,H,n,d] float out
  *   p      [B,H,n,N] float out, or NULL: the probabilities, same order as idx
- * Every idx entry must lie in [0, n); entries outside it are skipped and
- * flag HAD_ERR_INVALID_ARG in *dev_status.
+ * An idx entry of -1 is an empty slot (as had_hamming_topn_causal writes
+ * them): it gets probability 0 and no error; a row of empty slots gets zeros.
+ * Every other idx entry must lie in [0, n); entries outside it are skipped
+ * and flag HAD_ERR_INVALID_ARG in *dev_status.
  */
 HAD_API had_status_t had_sparse_softmax_av(const int32_t *idx, const int16_t *logits,
                                    const void *V, had_dtype_t dt,
@@ -159,6 +162,33 @@ HAD_API had_status_t had_attention_core(const void *V, had_dtype_t dt, int B, in
                                         int d, int N, float tau, float *out, int32_t *dbg_idx,
                                         int16_t *dbg_logits, void *ws, size_t ws_bytes,
                                         int32_t *dev_status, cudaStream_t stream);
+
+/*
+ * Causal variant.  The pages print no causal rule; this is the plain reading
+ * for decoder use: query i of a head sees keys 0 .. i only and keeps the
+ * N_i = min(N, i + 1) largest visible logits (ties to the lower index), in
+ * ascending key order.  Slots N_i .. N-1 of a row hold idx -1 and logit 0;
+ * had_sparse_softmax_av treats idx -1 as an empty slot (no weight, no
+ * error), so the two compose.  Arguments as had_hamming_topn (no workspace).
+ */
+HAD_API had_status_t had_hamming_topn_causal(const uint32_t *qbits, const uint32_t *kbits,
+                                             int B, int H, int n, int d, int N, int32_t *idx,
+                                             int16_t *logits, int32_t *dev_status,
+                                             cudaStream_t stream);
+
+/*
+ * Causal forward in one call: had_binarize_pack of Q and K, then
+ * had_hamming_topn_causal, then had_sparse_softmax_av, inside a caller
+ * workspace of had_workspace_bytes(HAD_OP_ATTENTION_CAUSAL, ...) bytes
+ * (packed bits and the kept set: about B*H*n*(d/4 + 6 N) bytes).  Arguments
+ * otherwise as had_attention_fwd (no debug outputs).
+ */
+HAD_API had_status_t had_attention_causal_fwd(const void *Q, const void *K, const void *V,
+                                              had_dtype_t dt, const float *sigma_q,
+                                              const float *sigma_k, int B, int H, int n, int d,
+                                              int N, float tau, float *out, void *ws,
+                                              size_t ws_bytes, int32_t *dev_status,
+                                              cudaStream_t stream);
 
 /*
  * Top-N mass retention diagnostic ("Hamming Attention Distillation",

@@ -71,26 +71,47 @@ had_status_t launch_pack(const void *x, had_dtype_t dt, const float *sigma, int 
     return launched();
 }
 
-template <int DW>
+template <int DW, bool kCausal>
 had_status_t launch_topn_dw(const uint32_t *qb, const uint32_t *kb, int B, int H, int n,
                             int N, int32_t *idx, int16_t *lg, cudaStream_t st)
 {
     constexpr int smem = had::topn_smem_bytes<DW>();
     // Set on every call: the attribute belongs to the current device.
-    if (cudaFuncSetAttribute(had::topn_simt_kernel<DW>,
+    if (cudaFuncSetAttribute(had::topn_simt_kernel<DW, kCausal>,
                              cudaFuncAttributeMaxDynamicSharedMemorySize, smem) != cudaSuccess)
         return HAD_ERR_CUDA;
     const long long blocks = (long long)((n + had::kTopnRows - 1) / had::kTopnRows) * B * H;
     if (blocks > INT_MAX) return HAD_ERR_UNSUPPORTED;
-    had::topn_simt_kernel<DW><<<(unsigned)blocks, had::kTopnRows, smem, st>>>(qb, kb, n, N, idx, lg);
+    had::topn_simt_kernel<DW, kCausal><<<(unsigned)blocks, had::kTopnRows, smem, st>>>(
+        qb, kb, n, N, idx, lg);
     return launched();
 }
 
 had_status_t launch_topn(const uint32_t *qb, const uint32_t *kb, int B, int H, int n, int d,
-                         int N, int32_t *idx, int16_t *lg, cudaStream_t st)
+                         int N, int32_t *idx, int16_t *lg, bool causal, cudaStream_t st)
 {
-    return d == 64 ? launch_topn_dw<2>(qb, kb, B, H, n, N, idx, lg, st)
-                   : launch_topn_dw<4>(qb, kb, B, H, n, N, idx, lg, st);
+    if (causal)
+        return d == 64 ? launch_topn_dw<2, true>(qb, kb, B, H, n, N, idx, lg, st)
+                       : launch_topn_dw<4, true>(qb, kb, B, H, n, N, idx, lg, st);
+    return d == 64 ? launch_topn_dw<2, false>(qb, kb, B, H, n, N, idx, lg, st)
+                   : launch_topn_dw<4, false>(qb, kb, B, H, n, N, idx, lg, st);
+}
+
+// Workspace of the causal forward: packed Q and K bits, then the kept set.
+struct CausalWorkspace {
+    size_t qbits, kbits, idx, logits, total;
+};
+
+CausalWorkspace causal_layout(int B, int H, int n, int d, int N)
+{
+    const size_t rows = (size_t)B * H * n;
+    CausalWorkspace w;
+    w.qbits = 0;
+    w.kbits = w.qbits + round_up(rows * (d / 8));
+    w.idx = w.kbits + round_up(rows * (d / 8));
+    w.logits = w.idx + round_up(rows * (size_t)N * 4);
+    w.total = w.logits + round_up(rows * (size_t)N * 2);
+    return w;
 }
 
 had_status_t launch_av(const int32_t *idx, const int16_t *lg, const void *V, had_dtype_t dt,
@@ -325,7 +346,47 @@ had_status_t had_hamming_topn(const uint32_t *qbits, const uint32_t *kbits, int 
     if (!aligned16(qbits) || !aligned16(kbits) || !aligned16(idx) ||
         (logits && !aligned16(logits)))
         return HAD_ERR_INVALID_ARG;
-    return launch_topn(qbits, kbits, B, H, n, d, N, idx, logits, stream);
+    return launch_topn(qbits, kbits, B, H, n, d, N, idx, logits, false, stream);
+}
+
+had_status_t had_hamming_topn_causal(const uint32_t *qbits, const uint32_t *kbits, int B, int H,
+                                     int n, int d, int N, int32_t *idx, int16_t *logits,
+                                     int32_t *dev_status, cudaStream_t stream)
+{
+    (void)dev_status;
+    had_status_t s = check_topn(B, H, n, d, N);
+    if (s != HAD_OK) return s;
+    if (!qbits || !kbits || !idx) return HAD_ERR_INVALID_ARG;
+    if (!aligned16(qbits) || !aligned16(kbits) || !aligned16(idx) ||
+        (logits && !aligned16(logits)))
+        return HAD_ERR_INVALID_ARG;
+    return launch_topn(qbits, kbits, B, H, n, d, N, idx, logits, true, stream);
+}
+
+had_status_t had_attention_causal_fwd(const void *Q, const void *K, const void *V,
+                                      had_dtype_t dt, const float *sigma_q, const float *sigma_k,
+                                      int B, int H, int n, int d, int N, float tau, float *out,
+                                      void *ws, size_t ws_bytes, int32_t *dev_status,
+                                      cudaStream_t stream)
+{
+    had_status_t s = check_topn(B, H, n, d, N);
+    if (s != HAD_OK) return s;
+    if (dt != HAD_BF16 && dt != HAD_F32) return HAD_ERR_INVALID_ARG;
+    if (!Q || !K || !V || !sigma_q || !sigma_k || !out || !ws) return HAD_ERR_INVALID_ARG;
+    if (!aligned16(Q) || !aligned16(K) || !aligned16(V) || !aligned16(out) || !aligned16(ws))
+        return HAD_ERR_INVALID_ARG;
+    if (!(tau == tau) || tau > 3.0e38f || tau < -3.0e38f) return HAD_ERR_INVALID_ARG;
+    const CausalWorkspace w = causal_layout(B, H, n, d, N);
+    if (ws_bytes < w.total) return HAD_ERR_WORKSPACE;
+    char *base = static_cast<char *>(ws);
+    auto *qb = reinterpret_cast<uint32_t *>(base + w.qbits);
+    auto *kb = reinterpret_cast<uint32_t *>(base + w.kbits);
+    auto *idx = reinterpret_cast<int32_t *>(base + w.idx);
+    auto *lg = reinterpret_cast<int16_t *>(base + w.logits);
+    if ((s = launch_pack(Q, dt, sigma_q, B, H, n, d, qb, dev_status, stream)) != HAD_OK) return s;
+    if ((s = launch_pack(K, dt, sigma_k, B, H, n, d, kb, dev_status, stream)) != HAD_OK) return s;
+    if ((s = launch_topn(qb, kb, B, H, n, d, N, idx, lg, true, stream)) != HAD_OK) return s;
+    return launch_av(idx, lg, V, dt, B, H, n, d, N, tau, out, nullptr, dev_status, stream);
 }
 
 had_status_t had_sparse_softmax_av(const int32_t *idx, const int16_t *logits, const void *V,
@@ -492,6 +553,9 @@ size_t had_workspace_bytes(int op, int B, int H, int n, int d, int N)
         return fwd_layout(B, H, n, d, N).total;
     case HAD_OP_TOPN_MASS:
         return check_shape(B, H, n, d) == HAD_OK ? 0 : (size_t)-1;
+    case HAD_OP_ATTENTION_CAUSAL:
+        return check_topn(B, H, n, d, N) == HAD_OK ? causal_layout(B, H, n, d, N).total
+                                                   : (size_t)-1;
     default:
         return (size_t)-1;
     }
@@ -513,6 +577,8 @@ int had_launch_count(int op, int B, int H, int n, int d, int N)
         return check_topn(B, H, n, d, N) == HAD_OK ? 2 : -1;
     case HAD_OP_TOPN_MASS:
         return check_shape(B, H, n, d) == HAD_OK ? 1 : -1;
+    case HAD_OP_ATTENTION_CAUSAL:
+        return check_topn(B, H, n, d, N) == HAD_OK ? 4 : -1;
     default:
         return -1;
     }

@@ -65,8 +65,11 @@ sparse_softmax_av_kernel(const int32_t *__restrict__ idx, const int16_t *__restr
     const int16_t *lr = logits + row * N;
     const T *vh = V + head * n * (long long)D;
 
+    // an index of -1 marks an empty slot (rows of the causal form that see
+    // fewer than N keys): it weighs nothing and takes no part in the max
     int m = -2147483647;
-    for (int k = lane; k < N; k += 32) m = max(m, (int)lr[k]);
+    for (int k = lane; k < N; k += 32)
+        if (ir[k] != -1) m = max(m, (int)lr[k]);
 #pragma unroll
     for (int o = 16; o > 0; o >>= 1) m = max(m, __shfl_xor_sync(kFullMask, m, o));
 
@@ -80,13 +83,21 @@ sparse_softmax_av_kernel(const int32_t *__restrict__ idx, const int16_t *__restr
         float w = 0.0f;
         if (k < N) {
             j = ir[k];
-            w = expf(tau * (float)((int)lr[k] - m));
-            if (j < 0 || j >= n) { flag(status, HAD_ERR_INVALID_ARG); j = 0; w = 0.0f; }
+            if (j == -1) {
+                w = 0.0f;
+            } else if (j < 0 || j >= n) {
+                flag(status, HAD_ERR_INVALID_ARG);
+                j = 0;
+                w = 0.0f;
+            } else {
+                w = expf(tau * (float)((int)lr[k] - m));
+            }
         }
         z += w;
         const int cnt = min(32, N - k0);
         for (int t = 0; t < cnt; ++t) {
             const int jt = __shfl_sync(kFullMask, j, t);
+            if (jt == -1) continue;   // empty slot; the same t on every lane
             const float wt = __shfl_sync(kFullMask, w, t);
             float v[PER];
             VRow<T, PER>::load(vh + (long long)jt * D + lane * PER, v);
@@ -96,7 +107,9 @@ sparse_softmax_av_kernel(const int32_t *__restrict__ idx, const int16_t *__restr
     }
 #pragma unroll
     for (int o = 16; o > 0; o >>= 1) z += __shfl_xor_sync(kFullMask, z, o);
-    const float inv = 1.0f / z;
+    // z >= 1 whenever the row keeps a key (its largest logit weighs 1); a
+    // row of empty slots only gets zeros
+    const float inv = z > 0.0f ? 1.0f / z : 0.0f;
     float *orow = out + row * D + lane * PER;
 #pragma unroll
     for (int e = 0; e < PER; ++e) orow[e] = acc[e] * inv;

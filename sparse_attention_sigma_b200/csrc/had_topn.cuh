@@ -16,6 +16,10 @@
 //           were kept (ascending key index, so the lower index wins).
 // Output per row: the N kept key indices in ascending order, and their
 // logits s = d - 2h.
+//
+// Causal form (kCausal): query i of a head sees keys 0 .. i only and keeps
+// N_i = min(N, i + 1) of them; slots N_i .. N-1 hold idx -1 and logit 0.  A
+// CTA streams keys only up to its last row.
 #pragma once
 #include "had_common.cuh"
 
@@ -30,7 +34,7 @@ constexpr int topn_smem_bytes()
     return ((DW * 32 + 1) * kTopnRows + kTopnKeyChunk * DW) * 4;
 }
 
-template <int DW>
+template <int DW, bool kCausal = false>
 __global__ void __launch_bounds__(kTopnRows)
 topn_simt_kernel(const uint32_t *__restrict__ qbits, const uint32_t *__restrict__ kbits,
                  int n, int N, int32_t *__restrict__ idx, int16_t *__restrict__ logits)
@@ -44,8 +48,13 @@ topn_simt_kernel(const uint32_t *__restrict__ qbits, const uint32_t *__restrict_
     const int tid = threadIdx.x;
     const int tiles = (n + kTopnRows - 1) / kTopnRows;
     const long long head = blockIdx.x / tiles;
-    const int row = (int)(blockIdx.x % tiles) * kTopnRows + tid;
+    const int row0 = (int)(blockIdx.x % tiles) * kTopnRows;
+    const int row = row0 + tid;
     const bool active = row < n;
+    // keys this CTA streams, and the keys this row sees
+    const int n_cta = kCausal ? min(n, row0 + kTopnRows) : n;
+    const int n_row = kCausal ? row + 1 : n;
+    const int N_row = min(N, n_row);
 
     uint32_t q[DW];
 #pragma unroll
@@ -53,13 +62,14 @@ topn_simt_kernel(const uint32_t *__restrict__ qbits, const uint32_t *__restrict_
     for (int b = 0; b < BINS; ++b) hist[b * kTopnRows + tid] = 0;
 
     const uint32_t *kh = kbits + head * n * DW;
-    for (int j0 = 0; j0 < n; j0 += kTopnKeyChunk) {
-        const int cnt = min(kTopnKeyChunk, n - j0);
+    for (int j0 = 0; j0 < n_cta; j0 += kTopnKeyChunk) {
+        const int cnt = min(kTopnKeyChunk, n_cta - j0);
         __syncthreads();
         for (int t = tid; t < cnt * DW; t += kTopnRows) kch[t] = __ldg(kh + (long long)j0 * DW + t);
         __syncthreads();
         if (active) {
-            for (int jj = 0; jj < cnt; ++jj) {
+            const int lim = min(cnt, n_row - j0);
+            for (int jj = 0; jj < lim; ++jj) {
                 int h = 0;
 #pragma unroll
                 for (int w = 0; w < DW; ++w) h += __popc(q[w] ^ kch[jj * DW + w]);
@@ -74,7 +84,7 @@ topn_simt_kernel(const uint32_t *__restrict__ qbits, const uint32_t *__restrict_
         uint32_t below = 0;
         for (int b = 0; b < BINS; ++b) {
             const uint32_t c = hist[b * kTopnRows + tid];
-            if (below + c >= (uint32_t)N) { t = b; quota = (uint32_t)N - below; break; }
+            if (below + c >= (uint32_t)N_row) { t = b; quota = (uint32_t)N_row - below; break; }
             below += c;
         }
     }
@@ -82,13 +92,14 @@ topn_simt_kernel(const uint32_t *__restrict__ qbits, const uint32_t *__restrict_
     const long long obase = (head * n + row) * (long long)N;
     int out = 0;
     uint32_t ties = 0;
-    for (int j0 = 0; j0 < n; j0 += kTopnKeyChunk) {
-        const int cnt = min(kTopnKeyChunk, n - j0);
+    for (int j0 = 0; j0 < n_cta; j0 += kTopnKeyChunk) {
+        const int cnt = min(kTopnKeyChunk, n_cta - j0);
         __syncthreads();
         for (int tt = tid; tt < cnt * DW; tt += kTopnRows) kch[tt] = __ldg(kh + (long long)j0 * DW + tt);
         __syncthreads();
         if (active) {
-            for (int jj = 0; jj < cnt; ++jj) {
+            const int lim = min(cnt, n_row - j0);
+            for (int jj = 0; jj < lim; ++jj) {
                 int h = 0;
 #pragma unroll
                 for (int w = 0; w < DW; ++w) h += __popc(q[w] ^ kch[jj * DW + w]);
@@ -103,6 +114,11 @@ topn_simt_kernel(const uint32_t *__restrict__ qbits, const uint32_t *__restrict_
             }
         }
     }
+    if (kCausal && active)
+        for (int k = out; k < N; ++k) {
+            idx[obase + k] = -1;
+            if (logits) logits[obase + k] = 0;
+        }
 }
 
 }  // namespace had

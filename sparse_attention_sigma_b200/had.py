@@ -34,6 +34,7 @@ HAD_OP_SPARSE_SOFTMAX_AV = 3
 HAD_OP_ATTENTION_PREPARE = 4
 HAD_OP_ATTENTION_CORE = 5
 HAD_OP_TOPN_MASS = 6
+HAD_OP_ATTENTION_CAUSAL = 7
 
 
 class HadError(RuntimeError):
@@ -60,6 +61,9 @@ def _load():
         "had_attention_prepare": [vp, vp, vp, i32, vp, vp, i32, i32, i32, i32, i32, vp, sz, vp, vp],
         "had_attention_core": [vp, i32, i32, i32, i32, i32, i32, f32, vp, vp, vp, vp, sz, vp, vp],
         "had_topn_mass": [vp, vp, i32, i32, i32, i32, f32, vp, i32, vp, vp, vp],
+        "had_hamming_topn_causal": [vp, vp, i32, i32, i32, i32, i32, vp, vp, vp, vp],
+        "had_attention_causal_fwd": [vp, vp, vp, i32, vp, vp, i32, i32, i32, i32, i32, f32, vp,
+                                     vp, sz, vp, vp],
     }
     for name, args in sig.items():
         fn = getattr(lib, name)
@@ -173,6 +177,54 @@ def had_hamming_topn(qbits, kbits, d, N, idx=None, logits=None, ws=None, dev_sta
                                _stream(stream))
     _check(st, "had_hamming_topn")
     return idx, logits
+
+
+def had_hamming_topn_causal(qbits, kbits, d, N, idx=None, logits=None, dev_status=None,
+                            stream=None, want_logits=True):
+    """Causal top-N: query i keeps the min(N, i+1) best of keys 0..i, slots past
+    that hold idx -1 / logit 0; returns (idx [B,H,n,N] int32, logits int16 or None)."""
+    _dev(qbits, "qbits", torch.int32)
+    B, H, n, w = _shape4(qbits, "qbits")
+    if w * 32 != d:
+        raise ValueError("qbits last dimension must be d/32")
+    _dev(kbits, "kbits", torch.int32, (B, H, n, w))
+    if idx is None:
+        idx = torch.empty((B, H, n, N), dtype=torch.int32, device=qbits.device)
+    _dev(idx, "idx", torch.int32, (B, H, n, N))
+    if logits is None and want_logits:
+        logits = torch.empty((B, H, n, N), dtype=torch.int16, device=qbits.device)
+    if logits is not None:
+        _dev(logits, "logits", torch.int16, (B, H, n, N))
+    st = _lib.had_hamming_topn_causal(_ptr(qbits), _ptr(kbits), B, H, n, d, N, _ptr(idx),
+                                      _ptr(logits), _ptr(dev_status), _stream(stream))
+    _check(st, "had_hamming_topn_causal")
+    return idx, logits
+
+
+def had_attention_causal_fwd(Q, K, V, sigma_q, sigma_k, N, tau, out=None, ws=None,
+                             dev_status=None, stream=None):
+    """Causal binarized top-N attention forward; returns out [B,H,n,d] float32."""
+    _dev(Q, "Q")
+    B, H, n, d = _shape4(Q, "Q")
+    _dev(K, "K", Q.dtype, (B, H, n, d))
+    _dev(V, "V", Q.dtype, (B, H, n, d))
+    _dev(sigma_q, "sigma_q", torch.float32, (H,))
+    _dev(sigma_k, "sigma_k", torch.float32, (H,))
+    if out is None:
+        out = torch.empty((B, H, n, d), dtype=torch.float32, device=Q.device)
+    _dev(out, "out", torch.float32, (B, H, n, d))
+    need = had_workspace_bytes(HAD_OP_ATTENTION_CAUSAL, B, H, n, d, N)
+    if need < 0:
+        raise HadError(HAD_ERR_UNSUPPORTED if d not in (64, 128) else HAD_ERR_INVALID_ARG,
+                       "had_attention_causal_fwd")
+    if ws is None:
+        ws = torch.empty(need, dtype=torch.uint8, device=Q.device)
+    st = _lib.had_attention_causal_fwd(_ptr(Q), _ptr(K), _ptr(V), _dtype_code(Q), _ptr(sigma_q),
+                                       _ptr(sigma_k), B, H, n, d, N, ctypes.c_float(tau),
+                                       _ptr(out), _ptr(ws), ws.numel(), _ptr(dev_status),
+                                       _stream(stream))
+    _check(st, "had_attention_causal_fwd")
+    return out
 
 
 def had_topn_mass(qbits, kbits, d, tau, p, nmin=None, dev_status=None, stream=None):

@@ -105,3 +105,34 @@ def test_topn_mass_argument_errors_return_before_any_cuda_call(lib):
     lib.had_launch_count.argtypes = [ctypes.c_int] * 6
     assert lib.had_workspace_bytes(6, 1, 1, 8, 64, 0) == 0
     assert lib.had_launch_count(6, 1, 1, 8, 64, 0) == 1
+
+
+def test_causal_argument_errors_return_before_any_cuda_call(lib):
+    f = lib.had_attention_causal_fwd
+    vp, i, sz = ctypes.c_void_p, ctypes.c_int, ctypes.c_size_t
+    f.argtypes = [vp, vp, vp, i, vp, vp, i, i, i, i, i, ctypes.c_float, vp, vp, sz, vp, vp]
+    f.restype = ctypes.c_int
+    fake = vp(4096)        # never dereferenced: the checks fail first
+    assert f(fake, fake, fake, 0, fake, fake, 1, 1, 8, 96, 2, 0.1, fake, fake, 1 << 20,
+             None, None) == 2                                                    # d
+    assert f(fake, fake, fake, 0, fake, fake, 1, 1, 8, 64, 9, 0.1, fake, fake, 1 << 20,
+             None, None) == 1                                                    # N > n
+    assert f(fake, fake, fake, 0, fake, fake, 1, 1, 8, 64, 2, 0.1, fake, None, 1 << 20,
+             None, None) == 1                                                    # no workspace
+    assert f(fake, fake, fake, 0, fake, fake, 1, 1, 8, 64, 2, 0.1, fake, fake, 16,
+             None, None) == 3                                                    # too small
+    assert f(fake, fake, fake, 0, fake, fake, 1, 1, 8, 64, 2, float("nan"), fake, fake,
+             1 << 20, None, None) == 1                                           # tau NaN
+    g = lib.had_hamming_topn_causal
+    g.argtypes = [vp, vp, i, i, i, i, i, vp, vp, vp, vp]
+    g.restype = ctypes.c_int
+    assert g(fake, fake, 1, 1, 8, 64, 0, fake, fake, None, None) == 1            # N = 0
+    assert g(fake, None, 1, 1, 8, 64, 2, fake, fake, None, None) == 1            # no kbits
+    assert g(fake, fake, 1, 1, 8, 64, 2, vp(4100), fake, None, None) == 1        # misaligned
+    lib.had_workspace_bytes.restype = ctypes.c_size_t
+    lib.had_workspace_bytes.argtypes = [ctypes.c_int] * 6
+    lib.had_launch_count.argtypes = [ctypes.c_int] * 6
+    # packed Q and K bits (8 B per row at d = 64) plus idx and logits (6 B per slot)
+    assert lib.had_workspace_bytes(7, 1, 1, 128, 64, 16) >= 128 * (8 + 8 + 6 * 16)
+    assert lib.had_workspace_bytes(7, 1, 1, 128, 64, 129) == ctypes.c_size_t(-1).value
+    assert lib.had_launch_count(7, 1, 1, 128, 64, 16) == 4

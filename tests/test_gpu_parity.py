@@ -337,3 +337,59 @@ def test_topn_mass_long_workload_sampled(had):
     c = config_case("long")
     rows = synth.sample_rows(synth.CONFIGS["long"], 256, seed=21)
     _mass_check(had, c, [0.9, 0.95, 0.99], rows)
+
+
+def _check_causal(had, c, rows):
+    """Causal top-N and softmax-V against the oracle: kept indices and logits
+    (empty slots included) bit-exact, probabilities and output within the
+    tolerance; the one-call forward equals the three-call composition."""
+    qb, kb = _check_bits(had, c)
+    idx, lg = had.had_hamming_topn_causal(qb, kb, c.d, c.N)
+    out, p = had.had_sparse_softmax_av(idx, lg, c.gv, c.tau, want_p=True)
+    status = torch.zeros(1, dtype=torch.int32, device="cuda")
+    out1 = had.had_attention_causal_fwd(c.gq, c.gk, c.gv, c.gsq, c.gsk, c.N, c.tau,
+                                        dev_status=status)
+    torch.cuda.synchronize()
+    assert status.item() == 0
+    assert torch.equal(out, out1)
+    o_idx, o_lg, o_p, o_out = oracle.attention_causal_rows(c.sq, c.sk, c.v_or, c.tau, c.N, rows)
+    flat = lambda t: t.reshape(-1, t.shape[-1]).cpu().numpy()[rows]
+    assert np.array_equal(flat(idx), o_idx)
+    assert np.array_equal(flat(lg), o_lg)
+    assert_close(flat(p), o_p, "causal p")
+    assert_close(flat(out), o_out, "causal out")
+
+
+@pytest.mark.parametrize("B,H,n,d,N,seed", [(1, 2, 300, 64, 40, 31), (2, 1, 257, 128, 33, 32),
+                                            (1, 1, 1, 64, 1, 33), (1, 2, 130, 64, 130, 34),
+                                            (1, 3, 200, 64, 1, 35)])
+def test_causal_small_all_rows(had, B, H, n, d, N, seed):
+    c = random_case(B, H, n, d, N, seed)
+    _check_causal(had, c, all_rows(c))
+
+
+def test_causal_long_workload_sampled(had):
+    c = config_case("long")
+    cfg = synth.CONFIGS["long"]
+    # the diagonal region (rows that see fewer than N keys, and the first
+    # CTA boundaries) in two heads, plus a seeded sample of the rest
+    early = np.array([0, 1, 2, 127, 128, 129, 255, 510, 511, 512, 513, 4095])
+    heads = np.array([0, cfg.B * cfg.H - 1])
+    rows = np.unique(np.concatenate([(heads[:, None] * cfg.n + early[None, :]).ravel(),
+                                     synth.sample_rows(cfg, 128, seed=41)]))
+    _check_causal(had, c, rows)
+
+
+def test_empty_slots_give_zeros_without_error(had):
+    c = random_case(1, 1, 64, 64, 8, 36)
+    idx = torch.full((1, 1, 64, 8), -1, dtype=torch.int32, device="cuda")
+    idx[0, 0, 1::2, 3] = 5          # odd rows keep one key
+    lg = torch.zeros((1, 1, 64, 8), dtype=torch.int16, device="cuda")
+    status = torch.zeros(1, dtype=torch.int32, device="cuda")
+    out, p = had.had_sparse_softmax_av(idx, lg, c.gv, c.tau, want_p=True, dev_status=status)
+    torch.cuda.synchronize()
+    assert status.item() == 0
+    assert torch.count_nonzero(out[0, 0, 0::2]) == 0 and torch.count_nonzero(p[0, 0, 0::2]) == 0
+    v5 = c.gv[0, 0, 5].float()
+    assert torch.equal(out[0, 0, 1::2], v5.expand(32, -1))
+    assert torch.all(p[0, 0, 1::2, 3] == 1) and p[0, 0, 1::2].sum() == 32
