@@ -18,7 +18,11 @@ LSB-first bit order, the identity dot = d - 2*popcount(xor), logits against a
 float64 matrix product of the signs, top-N against independent sorts and a
 histogram-threshold selection, the N = n case against a dense library
 softmax, closed forms (all keys equal, N = 1), and a hand-worked example
-under ``tests/golden/``.  No function is left unpinned.
+under ``tests/golden/``.  The soft (tanh) codes of the training stages are
+pinned by tanh closed forms (tanh(ln 2) = 3/5, tanh(ln 3) = 4/5, ...), their
+limits (signs at large c, the scaled dot product at small c), oddness, a
+numpy sort with exact ties, and a dense library softmax at N = n.  No
+function is left unpinned.
 """
 import ctypes
 import os
@@ -56,6 +60,16 @@ def _load():
             lp, lp, c_long, c_long, c_long, c_long, ctypes.c_double, lp, c_int, lp,
             c_long, lp, c_int]
         lib.had_oracle_topn_mass_rows.restype = c_int
+        lib.had_oracle_soft_binarize.argtypes = [lp, c_int, lp, ctypes.c_float, c_long,
+                                                 c_long, c_long, c_long, lp]
+        lib.had_oracle_soft_binarize.restype = None
+        lib.had_oracle_soft_logits_rows.argtypes = [lp, lp, c_long, c_long, c_long,
+                                                    c_long, lp, c_long, lp, c_int]
+        lib.had_oracle_soft_logits_rows.restype = None
+        lib.had_oracle_soft_attention_rows.argtypes = [
+            lp, lp, lp, c_int, c_long, c_long, c_long, c_long, c_long,
+            ctypes.c_float, lp, c_long, lp, lp, lp, lp, c_int]
+        lib.had_oracle_soft_attention_rows.restype = c_int
         lib.had_oracle_max_threads.argtypes = []
         lib.had_oracle_max_threads.restype = c_int
         _lib = lib
@@ -203,3 +217,54 @@ def attention(sq, sk, v, tau, N, threads=0):
 
 def lib_path() -> str:
     return os.path.abspath(_build.LIB)
+
+
+def soft_binarize(x, sigma, c):
+    """Soft codes tanh(c * x / sigma[h]) (fp32) for x of shape [B,H,n,d]:
+    the forward pass of the tanh training stages."""
+    x = np.ascontiguousarray(x)
+    sigma = np.ascontiguousarray(sigma, dtype=np.float32)
+    B, H, n, d = x.shape
+    assert sigma.shape == (H,)
+    out = np.empty((B, H, n, d), dtype=np.float32)
+    _load().had_oracle_soft_binarize(_ptr(x), _is_bf16(x), _ptr(sigma), ctypes.c_float(c),
+                                     B, H, n, d, _ptr(out))
+    return out
+
+
+def soft_logits_rows(tq, tk, rows, threads=0):
+    """fp64 logits [len(rows), n] of the soft codes for the given flat query rows."""
+    tq = np.ascontiguousarray(tq, dtype=np.float32)
+    tk = np.ascontiguousarray(tk, dtype=np.float32)
+    B, H, n, d = tq.shape
+    assert tk.shape == tq.shape
+    rows = _rows_array(rows, B * H * n)
+    out = np.empty((rows.size, n), dtype=np.float64)
+    _load().had_oracle_soft_logits_rows(_ptr(tq), _ptr(tk), B, H, n, d, _ptr(rows), rows.size,
+                                        _ptr(out), int(threads))
+    return out
+
+
+def soft_attention_rows(tq, tk, v, tau, N, rows, threads=0):
+    """Top-N attention on the soft codes for the given flat query rows.
+
+    Returns (idx [R, N] int32 ascending, logits [R, N] float64,
+    p [R, N] float64, out [R, d] float32)."""
+    tq = np.ascontiguousarray(tq, dtype=np.float32)
+    tk = np.ascontiguousarray(tk, dtype=np.float32)
+    v = np.ascontiguousarray(v)
+    B, H, n, d = tq.shape
+    assert tk.shape == tq.shape and v.shape == tq.shape
+    rows = _rows_array(rows, B * H * n)
+    R = rows.size
+    idx = np.empty((R, N), dtype=np.int32)
+    lg = np.empty((R, N), dtype=np.float64)
+    p = np.empty((R, N), dtype=np.float64)
+    out = np.empty((R, d), dtype=np.float32)
+    rc = _load().had_oracle_soft_attention_rows(
+        _ptr(tq), _ptr(tk), _ptr(v), _is_bf16(v), B, H, n, d, int(N),
+        ctypes.c_float(float(tau)), _ptr(rows), R, _ptr(idx), _ptr(lg), _ptr(p),
+        _ptr(out), int(threads))
+    if rc != 0:
+        raise ValueError("oracle rejected the arguments (N must be in [1, n])")
+    return idx, lg, p, out

@@ -413,6 +413,164 @@ int had_oracle_topn_mass_rows(const int8_t *sq, const int8_t *sk, long B,
     return failed ? -1 : 0;
 }
 
+/*
+ * Soft binarization, the forward pass of training stages 1-2 (pith.science
+ * review of arXiv 2502.01770: the annealing schedule starts from a scaled
+ * tanh whose scale c moves it toward the sign function, Eq. 13, before the
+ * straight-through stage).  Reading taken: the code of an element is
+ * t = tanh(c * z) with z = x / sigma[h] as in step 1 (fp32 division), the
+ * product c * z rounded to fp32, tanh evaluated in fp64 and rounded to fp32.
+ * The codes are fp32 numbers in (-1, 1), approaching +/-1 as c grows.
+ */
+void had_oracle_soft_binarize(const void *x, int x_is_bf16, const float *sigma,
+                              float c, long B, long H, long n, long d,
+                              float *t_out)
+{
+    for (long b = 0; b < B; ++b)
+        for (long h = 0; h < H; ++h) {
+            float sg = sigma[h];
+            long base = (b * H + h) * n * d;
+            for (long e = 0; e < n * d; ++e) {
+                float z = load_elem(x, x_is_bf16, base + e) / sg;
+                float u = c * z;
+                t_out[base + e] = (float)tanh((double)u);
+            }
+        }
+}
+
+/* Soft logits of one query row: the dot product of the fp32 codes, in fp64. */
+static void row_soft_logits(const float *tq_row, const float *tk_head, long n,
+                            long d, double *s)
+{
+    for (long j = 0; j < n; ++j) {
+        double acc = 0.0;
+        const float *kr = tk_head + j * d;
+        for (long k = 0; k < d; ++k)
+            acc += (double)tq_row[k] * (double)kr[k];
+        s[j] = acc;
+    }
+}
+
+/* Soft logits [nrows, n] (fp64) of a list of flat query rows. */
+void had_oracle_soft_logits_rows(const float *tq, const float *tk, long B,
+                                 long H, long n, long d, const int64_t *rows,
+                                 long nrows, double *s_out, int nthreads)
+{
+    (void)B;
+    (void)H;
+#ifdef _OPENMP
+    if (nthreads > 0)
+        omp_set_num_threads(nthreads);
+#pragma omp parallel for schedule(dynamic, 4)
+#endif
+    for (long t = 0; t < nrows; ++t) {
+        long r = (long)rows[t];
+        long head = r / n;
+        row_soft_logits(tq + r * d, tk + head * n * d, n, d, s_out + t * n);
+    }
+}
+
+typedef struct {
+    double s;
+    int32_t j;
+} keyed_soft_t;
+
+/* Larger logit first; equal logits: lower key index first. */
+static int by_soft_logit_then_index(const void *a, const void *b)
+{
+    const keyed_soft_t *x = (const keyed_soft_t *)a, *y = (const keyed_soft_t *)b;
+    if (x->s != y->s)
+        return (x->s > y->s) ? -1 : 1;
+    return (x->j < y->j) ? -1 : (x->j > y->j);
+}
+
+static int by_soft_index(const void *a, const void *b)
+{
+    const keyed_soft_t *x = (const keyed_soft_t *)a, *y = (const keyed_soft_t *)b;
+    return (x->j < y->j) ? -1 : (x->j > y->j);
+}
+
+/*
+ * Soft attention rows: the logits of the soft codes (fp64 dot products),
+ * then Eqs. 6-7 exactly as for the binarized codes: the N largest logits
+ * (ties to the lower key index) in ascending key order, softmax over them
+ * with temperature tau and the value product, both in fp64.  s_out holds
+ * the kept logits in fp64.  Returns 0, or -1 on a bad argument or an
+ * allocation failure.
+ */
+int had_oracle_soft_attention_rows(const float *tq, const float *tk,
+                                   const void *v, int v_is_bf16, long B,
+                                   long H, long n, long d, long N, float tau,
+                                   const int64_t *rows, long nrows,
+                                   int32_t *idx_out, double *s_out,
+                                   double *p_out, float *o_out, int nthreads)
+{
+    (void)B;
+    (void)H;
+    if (N < 1 || N > n || d < 1 || n < 1)
+        return -1;
+    int failed = 0;
+#ifdef _OPENMP
+    if (nthreads > 0)
+        omp_set_num_threads(nthreads);
+#pragma omp parallel
+#endif
+    {
+        double *s = (double *)malloc(sizeof(double) * (size_t)n);
+        keyed_soft_t *order = (keyed_soft_t *)malloc(sizeof(keyed_soft_t) * (size_t)n);
+        double *e = (double *)malloc(sizeof(double) * (size_t)N);
+#ifdef _OPENMP
+#pragma omp for schedule(dynamic, 4)
+#endif
+        for (long t = 0; t < nrows; ++t) {
+            if (!s || !order || !e) {
+#ifdef _OPENMP
+#pragma omp atomic write
+#endif
+                failed = 1;
+                continue;
+            }
+            long r = (long)rows[t];
+            long head = r / n;
+            row_soft_logits(tq + r * d, tk + head * n * d, n, d, s);
+            for (long j = 0; j < n; ++j) {
+                order[j].s = s[j];
+                order[j].j = (int32_t)j;
+            }
+            qsort(order, (size_t)n, sizeof(keyed_soft_t), by_soft_logit_then_index);
+            qsort(order, (size_t)N, sizeof(keyed_soft_t), by_soft_index);
+            double m = order[0].s;
+            for (long k = 1; k < N; ++k)
+                if (order[k].s > m)
+                    m = order[k].s;
+            double Z = 0.0;
+            for (long k = 0; k < N; ++k) {
+                e[k] = exp((double)tau * (order[k].s - m));
+                Z += e[k];
+            }
+            for (long k = 0; k < N; ++k) {
+                idx_out[t * N + k] = order[k].j;
+                s_out[t * N + k] = order[k].s;
+                if (p_out)
+                    p_out[t * N + k] = e[k] / Z;
+            }
+            const long vbase = head * n * d;
+            for (long c = 0; c < d; ++c) {
+                double acc = 0.0;
+                for (long k = 0; k < N; ++k)
+                    acc += (e[k] / Z) *
+                           (double)load_elem(v, v_is_bf16,
+                                             vbase + (long)order[k].j * d + c);
+                o_out[t * d + c] = (float)acc;
+            }
+        }
+        free(s);
+        free(order);
+        free(e);
+    }
+    return failed ? -1 : 0;
+}
+
 int had_oracle_max_threads(void)
 {
 #ifdef _OPENMP

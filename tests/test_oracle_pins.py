@@ -437,3 +437,108 @@ def test_causal_dense_rows_match_masked_softmax():
     assert np.allclose(out, ref, rtol=1e-6, atol=1e-6)
     assert np.allclose(p.sum(axis=1), 1.0, atol=1e-12)
     assert (idx[0] == [0] + [-1] * 39).all() and out[0].tolist() == v[0, 0, 0].tolist()
+
+
+# ------------------------------------------------- soft (tanh) codes, stages 1-2
+
+
+def _soft_codes(shape, c, seed, min_abs=0.0, dup_keys=0):
+    g = np.random.default_rng(seed)
+    q = g.standard_normal(shape).astype(np.float32)
+    k = g.standard_normal(shape).astype(np.float32)
+    if min_abs:
+        q = np.where(np.abs(q) < min_abs, np.float32(min_abs) * np.sign(q + 1e-30), q)
+        k = np.where(np.abs(k) < min_abs, np.float32(min_abs) * np.sign(k + 1e-30), k)
+    if dup_keys:
+        k[:, :, dup_keys:2 * dup_keys] = k[:, :, :dup_keys]   # exact logit ties
+    v = g.standard_normal(shape).astype(np.float32)
+    sg = np.ones(shape[1], np.float32)
+    return q, k, v, sg, oracle.soft_binarize(q, sg, c), oracle.soft_binarize(k, sg, c)
+
+
+@pytest.mark.parametrize("x,sigma,c,want", [
+    (0.0, 1.0, 1.0, 0.0),
+    (math.log(2.0), 1.0, 1.0, 0.6),              # tanh(ln 2) = 3/5
+    (0.5 * math.log(3.0), 1.0, 1.0, 0.5),        # tanh(ln sqrt 3) = 1/2
+    (math.log(3.0), 1.0, 1.0, 0.8),              # tanh(ln 3) = 4/5
+    (-math.log(3.0), 1.0, 1.0, -0.8),            # odd
+    (0.3, 0.6, 2.0, math.tanh(1.0)),             # c * x / sigma = 1
+    (1e-20, 1.0, 1.0, 1e-20),                    # tanh(u) = u below fp32 resolution
+    (20.0, 1.0, 1.0, 1.0),                       # saturates to exactly +1 in fp32
+    (-3.0, 1.0, 100.0, -1.0),
+])
+def test_soft_code_closed_forms(x, sigma, c, want):
+    t = oracle.soft_binarize(np.full((1, 1, 1, 32), x, np.float32),
+                             np.array([sigma], np.float32), c)
+    # the argument is rounded to fp32 (slope of tanh <= 1) and so is the result
+    assert np.all(np.abs(t.astype(np.float64) - want) <= 1.2e-7 * max(abs(want), 1e-13))
+
+
+def test_soft_codes_bf16_path_matches_widened_fp32():
+    x = torch.randn(1, 2, 8, 64, generator=torch.Generator().manual_seed(5)).to(torch.bfloat16)
+    sg = np.array([0.7, 1.9], np.float32)
+    a = oracle.soft_binarize(synth.to_oracle_array(x), sg, 1.5)
+    b = oracle.soft_binarize(x.float().numpy(), sg, 1.5)
+    assert np.array_equal(a, b)
+
+
+def test_soft_codes_become_signs_at_large_c():
+    q, _, _, sg, tq, _ = _soft_codes((1, 2, 20, 64), 1e4, seed=170, min_abs=0.01)
+    assert np.array_equal(tq, oracle.binarize(q, sg).astype(np.float32))
+
+
+def test_soft_attention_at_large_c_is_the_binarized_path():
+    q, k, v, sg, tq, tk = _soft_codes((1, 2, 70, 64), 1e4, seed=171, min_abs=0.01)
+    sq, sk = oracle.binarize(q, sg), oracle.binarize(k, sg)
+    rows = np.arange(140)
+    a = oracle.soft_attention_rows(tq, tk, v, 0.125, 9, rows)
+    b = oracle.attention_rows(sq, sk, v, 0.125, 9, rows)
+    assert np.array_equal(a[0], b[0])                     # same kept keys, same tie rule
+    assert np.array_equal(a[1], b[1].astype(np.float64))
+    assert np.allclose(a[2], b[2], rtol=0, atol=1e-14)
+    assert np.array_equal(a[3], b[3])
+
+
+def test_soft_logits_at_small_c_are_the_scaled_dot_product():
+    # tanh(u) = u (1 - u^2/3 + ...): s / c^2 -> z_q . z_k as c -> 0
+    q, k, _, sg, tq, tk = _soft_codes((1, 1, 30, 64), 1e-3, seed=172)
+    s = oracle.soft_logits_rows(tq, tk, np.arange(30)) / 1e-6
+    ref = q[0, 0].astype(np.float64) @ k[0, 0].astype(np.float64).T
+    assert np.allclose(s, ref, rtol=1e-4, atol=1e-4)
+    assert not np.allclose(s, ref.T, rtol=1e-2, atol=1e-2)     # orientation: row = query
+
+
+def test_soft_logits_are_odd_in_the_keys():
+    _, _, _, _, tq, tk = _soft_codes((1, 1, 16, 64), 0.8, seed=173)
+    a = oracle.soft_logits_rows(tq, tk, np.arange(16))
+    b = oracle.soft_logits_rows(tq, -tk, np.arange(16))
+    assert np.array_equal(a, -b)
+    assert np.all(np.abs(a) < 64)
+
+
+def test_soft_topn_against_numpy_sort_with_exact_ties():
+    _, _, v, _, tq, tk = _soft_codes((1, 2, 90, 64), 0.9, seed=174, dup_keys=30)
+    rows = np.arange(180)
+    N = 17
+    idx, lg, p, _ = oracle.soft_attention_rows(tq, tk, v, 0.125, N, rows)
+    s = oracle.soft_logits_rows(tq, tk, rows)
+    for t in range(180):
+        order = np.lexsort((np.arange(90), -s[t]))[:N]         # logit desc, index asc
+        want = np.sort(order)
+        assert np.array_equal(idx[t], want)
+        assert np.array_equal(lg[t], s[t, want])
+    # duplicated keys (j and j + 30) tie exactly; the lower index is kept first
+    assert np.array_equal(s[:, :30], s[:, 30:60])
+    assert np.allclose(p.sum(axis=1), 1.0, atol=1e-12)
+
+
+def test_soft_N_equals_n_is_dense_softmax():
+    _, _, v, _, tq, tk = _soft_codes((1, 1, 40, 64), 1.3, seed=175)
+    tau = float(np.float32(0.3))                 # the oracle takes tau as fp32
+    idx, lg, p, out = oracle.soft_attention_rows(tq, tk, v, tau, 40, np.arange(40))
+    s = torch.tensor(oracle.soft_logits_rows(tq, tk, np.arange(40)))
+    w = torch.softmax(tau * s, dim=-1)
+    ref = (w @ torch.tensor(v[0, 0], dtype=torch.float64)).numpy()
+    assert (idx == np.arange(40)).all()
+    assert np.allclose(p, w.numpy(), rtol=1e-12, atol=1e-15)
+    assert np.allclose(out, ref, rtol=1e-6, atol=1e-6)
