@@ -48,7 +48,7 @@ def parse():
                     help="target CPU time of the oracle baseline sample")
     ap.add_argument("--no-e2e", action="store_true")
     ap.add_argument("--no-cpu-baseline", action="store_true")
-    ap.add_argument("--mode", choices=["attention", "mass", "causal"], default="attention",
+    ap.add_argument("--mode", choices=["attention", "mass", "causal", "soft"], default="attention",
                     help="mass: time the top-N mass-retention diagnostic instead")
     return ap.parse_args()
 
@@ -586,6 +586,88 @@ def run_causal(args, world, rank, local):
     }), flush=True)
 
 
+def run_soft(args, world, rank, local):
+    """The soft-code forward (had_soft_attention_fwd, tanh training stages) on
+    the workload with c = 1: tokens per second, issued as its three stages.
+    The top-N stage is dominated by the fp32 logit kernel (2 d flops per
+    (query, key) pair on the CUDA cores); its roofline is the FMA pipe."""
+    from sparse_attention_sigma_b200 import had
+    cfg = synth.CONFIGS[args.config]
+    dev = torch.device("cuda", local)
+    torch.cuda.set_device(dev)
+    stream = torch.cuda.current_stream()
+    c = 1.0
+    q, k, v, sgq, sgk = synth.make_inputs(cfg)
+    gq, gk, gv = q.to(dev), k.to(dev), v.to(dev)
+    gsq, gsk = sgq.to(dev), sgk.to(dev)
+    shape = (cfg.B, cfg.H, cfg.n)
+    tq = torch.empty(shape + (cfg.d,), dtype=torch.float32, device=dev)
+    tk = torch.empty_like(tq)
+    idx = torch.empty(shape + (cfg.N,), dtype=torch.int32, device=dev)
+    lg = torch.empty(shape + (cfg.N,), dtype=torch.float32, device=dev)
+    out = torch.empty(shape + (cfg.d,), dtype=torch.float32, device=dev)
+    ws = torch.empty(had.had_workspace_bytes(had.HAD_OP_SOFT_TOPN, cfg.B, cfg.H, cfg.n, cfg.d,
+                                             cfg.N), dtype=torch.uint8, device=dev)
+    flush = torch.empty(L2_FLUSH_BYTES // 4, dtype=torch.float32, device=dev)
+    launches = (2 + had.had_launch_count(had.HAD_OP_SOFT_TOPN, cfg.B, cfg.H, cfg.n, cfg.d, cfg.N)
+                + 1)
+
+    def stages():
+        had.had_soft_binarize(gq, gsq, c, t=tq)
+        had.had_soft_binarize(gk, gsk, c, t=tk)
+        yield
+        had.had_soft_topn(tq, tk, cfg.N, idx=idx, logits=lg, ws=ws)
+        yield
+        had.had_soft_softmax_av(idx, lg, gv, cfg.tau, out=out)
+        yield
+
+    for _ in range(max(3, args.warmup)):
+        for _ in stages():
+            pass
+    ref = had.had_soft_attention_fwd(gq, gk, gv, gsq, gsk, c, cfg.N, cfg.tau)
+    torch.cuda.synchronize()
+    if not torch.equal(ref, out):
+        raise RuntimeError("had_soft_attention_fwd differs from its three stages")
+    del ref
+    clocks = ClockSampler(local)
+    clocks.start()
+    ev = [[torch.cuda.Event(enable_timing=True) for _ in range(4)] for _ in range(args.steps)]
+    barrier(world)
+    torch.cuda.synchronize()
+    for i in range(args.steps):
+        flush.fill_(float(i))
+        ev[i][0].record(stream)
+        for j, _ in enumerate(stages()):
+            ev[i][j + 1].record(stream)
+    torch.cuda.synchronize()
+    barrier(world)
+    clock_info = clocks.stop()
+    stage_ms = [sum(e[j].elapsed_time(e[j + 1]) for e in ev) / args.steps for j in range(3)]
+    value, ms = aggregate(cfg.tokens, sum(stage_ms), world, dev)
+    topn_ms = max_over_ranks(stage_ms[1], world, dev)
+    flops = 2.0 * cfg.B * cfg.H * cfg.n * cfg.n * cfg.d
+    peak = SM_COUNT * 128 * 2 * 1.965e9
+    if rank != 0:
+        return
+    print(json.dumps({
+        "metric": "HAD soft-code (tanh) attention tokens/sec", "value": value, "unit": "tokens/s",
+        "n_gpus": world, "steps": args.steps, "warmup": max(3, args.warmup), "ms_per_step": ms,
+        "higher_is_better": True, "scaling": "weak", "vs_baseline": None, "dtype": "f32",
+        "data": "synthetic", "impl": "had_soft_attention_fwd",
+        "config": {"workload": cfg.describe(), "c": c,
+                   "l2": "flushed between steps (256 MiB write outside the timed events)"},
+        "stage_ms": {"soft_binarize": stage_ms[0], "soft_topn": stage_ms[1],
+                     "soft_softmax_av": stage_ms[2]},
+        "roofline": {"bound": "alu", "achieved": flops / (topn_ms * 1e-3) / 1e12,
+                     "peak": peak / 1e12, "unit": "TFLOP/s", "frac": flops / (topn_ms * 1e-3) / peak,
+                     "kernel": "had_soft_topn stage: soft_logits_kernel + soft_select_kernel",
+                     "note": "fp32 FMA pipe, 128 lanes/SM at 1.965 GHz; 2 d flops per "
+                             "(query, key) pair of the logits"},
+        "gpu_launches": launches * args.steps,
+        "clocks": clock_info,
+    }), flush=True)
+
+
 def main():
     args = parse()
     world, rank, local = dist_setup(args)
@@ -596,6 +678,8 @@ def main():
             run_mass(args, world, rank, local)
         elif args.mode == "causal":
             run_causal(args, world, rank, local)
+        elif args.mode == "soft":
+            run_soft(args, world, rank, local)
         else:
             run_had(args, world, rank, local)
     finally:

@@ -76,7 +76,11 @@ typedef enum {
     HAD_OP_ATTENTION_PREPARE = 4, /* had_attention_prepare */
     HAD_OP_ATTENTION_CORE = 5,    /* had_attention_core */
     HAD_OP_TOPN_MASS = 6,         /* had_topn_mass */
-    HAD_OP_ATTENTION_CAUSAL = 7   /* had_attention_causal_fwd */
+    HAD_OP_ATTENTION_CAUSAL = 7,  /* had_attention_causal_fwd */
+    HAD_OP_SOFT_BINARIZE = 8,     /* had_soft_binarize */
+    HAD_OP_SOFT_TOPN = 9,         /* had_soft_topn */
+    HAD_OP_SOFT_SOFTMAX_AV = 10,  /* had_soft_softmax_av */
+    HAD_OP_SOFT_ATTENTION_FWD = 11 /* had_soft_attention_fwd */
 } had_op_t;
 
 /*
@@ -189,6 +193,60 @@ HAD_API had_status_t had_attention_causal_fwd(const void *Q, const void *K, cons
                                               int N, float tau, float *out, void *ws,
                                               size_t ws_bytes, int32_t *dev_status,
                                               cudaStream_t stream);
+
+/*
+ * Soft codes for the tanh training stages ("Hamming Attention
+ * Distillation", pith.science review: the annealing schedule trains first
+ * with a c-scaled tanh, Eq. 13, that approaches the sign as c grows).
+ * t = tanh(c * (x / sigma[h])) in fp32: the division and the product are
+ * IEEE round-to-nearest, tanh is CUDA's tanhf (within 2 ulp).
+ *   x      [B,H,n,d] of dtype dt (device); sigma [H] float (device)
+ *   c      the tanh scale, finite and > 0
+ *   t      [B,H,n,d] float out
+ * A sigma <= 0 or non-finite flags HAD_ERR_BAD_SIGMA in *dev_status.
+ * Non-finite x follow tanhf (+-inf -> +-1, NaN -> NaN); NaN codes are
+ * outside the contract of the calls below.
+ */
+HAD_API had_status_t had_soft_binarize(const void *x, had_dtype_t dt, const float *sigma,
+                                       float c, int B, int H, int n, int d, float *t,
+                                       int32_t *dev_status, cudaStream_t stream);
+
+/*
+ * Top-N of the soft logits s_ij = sum_k tq_ik tk_jk (fp32 FMA in the order
+ * k = 0 .. d-1).  Same selection rule as had_hamming_topn: the N largest
+ * (ties to the lower key index, -0 equal to +0), ascending key order.
+ *   tq, tk   [B,H,n,d] float codes (device)
+ *   idx      [B,H,n,N] int32 out;  logits [B,H,n,N] float out, or NULL
+ *   ws       device scratch of had_workspace_bytes(HAD_OP_SOFT_TOPN, ...)
+ *            bytes: the fp32 logit matrices of a group of heads (up to
+ *            2 GiB); groups run one after another (2 launches each)
+ * n is limited to 32768 (HAD_ERR_UNSUPPORTED beyond).
+ */
+HAD_API had_status_t had_soft_topn(const float *tq, const float *tk, int B, int H, int n, int d,
+                                   int N, int32_t *idx, float *logits, void *ws, size_t ws_bytes,
+                                   int32_t *dev_status, cudaStream_t stream);
+
+/*
+ * had_sparse_softmax_av for fp32 logits (the output of had_soft_topn); same
+ * arguments, empty slots and error behaviour.
+ */
+HAD_API had_status_t had_soft_softmax_av(const int32_t *idx, const float *logits, const void *V,
+                                         had_dtype_t dt, int B, int H, int n, int d, int N,
+                                         float tau, float *out, float *p, int32_t *dev_status,
+                                         cudaStream_t stream);
+
+/*
+ * Soft forward in one call: had_soft_binarize of Q and K with scale c, then
+ * had_soft_topn, then had_soft_softmax_av, inside a caller workspace of
+ * had_workspace_bytes(HAD_OP_SOFT_ATTENTION_FWD, ...) bytes (codes, kept
+ * set and the logit scratch).  Other arguments as had_attention_fwd.
+ */
+HAD_API had_status_t had_soft_attention_fwd(const void *Q, const void *K, const void *V,
+                                            had_dtype_t dt, const float *sigma_q,
+                                            const float *sigma_k, float c, int B, int H, int n,
+                                            int d, int N, float tau, float *out, void *ws,
+                                            size_t ws_bytes, int32_t *dev_status,
+                                            cudaStream_t stream);
 
 /*
  * Top-N mass retention diagnostic ("Hamming Attention Distillation",

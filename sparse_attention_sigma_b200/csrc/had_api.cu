@@ -14,6 +14,7 @@
 #include "had_prep.cuh"
 #include "had_fused.cuh"
 #include "had_mass.cuh"
+#include "had_soft.cuh"
 
 namespace {
 
@@ -114,7 +115,8 @@ CausalWorkspace causal_layout(int B, int H, int n, int d, int N)
     return w;
 }
 
-had_status_t launch_av(const int32_t *idx, const int16_t *lg, const void *V, had_dtype_t dt,
+template <typename L>
+had_status_t launch_av(const int32_t *idx, const L *lg, const void *V, had_dtype_t dt,
                        int B, int H, int n, int d, int N, float tau, float *out, float *p,
                        int32_t *status, cudaStream_t st)
 {
@@ -126,18 +128,18 @@ had_status_t launch_av(const int32_t *idx, const int16_t *lg, const void *V, had
     if (dt == HAD_BF16) {
         const auto *v = static_cast<const __nv_bfloat16 *>(V);
         if (d == 64)
-            had::sparse_softmax_av_kernel<__nv_bfloat16, 64><<<grid, threads, 0, st>>>(
+            had::sparse_softmax_av_kernel<__nv_bfloat16, 64, L><<<grid, threads, 0, st>>>(
                 idx, lg, v, n, N, tau, rows, out, p, status);
         else
-            had::sparse_softmax_av_kernel<__nv_bfloat16, 128><<<grid, threads, 0, st>>>(
+            had::sparse_softmax_av_kernel<__nv_bfloat16, 128, L><<<grid, threads, 0, st>>>(
                 idx, lg, v, n, N, tau, rows, out, p, status);
     } else {
         const auto *v = static_cast<const float *>(V);
         if (d == 64)
-            had::sparse_softmax_av_kernel<float, 64><<<grid, threads, 0, st>>>(
+            had::sparse_softmax_av_kernel<float, 64, L><<<grid, threads, 0, st>>>(
                 idx, lg, v, n, N, tau, rows, out, p, status);
         else
-            had::sparse_softmax_av_kernel<float, 128><<<grid, threads, 0, st>>>(
+            had::sparse_softmax_av_kernel<float, 128, L><<<grid, threads, 0, st>>>(
                 idx, lg, v, n, N, tau, rows, out, p, status);
     }
     return launched();
@@ -317,6 +319,116 @@ had_status_t launch_mass_dw(const uint32_t *qb, const uint32_t *kb, int B, int H
         qb, kb, n, (double)tau, ps, nmin);
     return launched();
 }
+
+// Soft-code path: n is bounded by the select kernel's shared memory (one
+// 4-byte key per column of a row).
+constexpr int kSoftMaxN = 32768;
+constexpr size_t kSoftScratchBytes = size_t(2) << 30;   // logits of one group of heads
+
+had_status_t check_soft(int B, int H, int n, int d, int N)
+{
+    had_status_t s = check_topn(B, H, n, d, N);
+    if (s != HAD_OK) return s;
+    return n > kSoftMaxN ? HAD_ERR_UNSUPPORTED : HAD_OK;
+}
+
+long long soft_ld(int n) { return (n + 3LL) / 4 * 4; }
+
+// Heads whose logit matrices share the scratch at one time.
+long long soft_group(int B, int H, int n)
+{
+    const long long per = (long long)n * soft_ld(n) * 4;
+    long long g = (long long)kSoftScratchBytes / per;
+    const long long bh = (long long)B * H;
+    if (g > bh) g = bh;
+    if (g > 65535) g = 65535;
+    return g < 1 ? 1 : g;
+}
+
+size_t soft_scratch_bytes(int B, int H, int n)
+{
+    return round_up((size_t)soft_group(B, H, n) * n * soft_ld(n) * 4);
+}
+
+int soft_passes(int B, int H, int n)
+{
+    const long long g = soft_group(B, H, n);
+    return (int)(((long long)B * H + g - 1) / g);
+}
+
+had_status_t launch_soft_codes(const void *x, had_dtype_t dt, const float *sigma, float c, int B,
+                               int H, int n, int d, float *t, int32_t *status, cudaStream_t st)
+{
+    const long long groups = (long long)B * H * n * d / 8;
+    const int threads = 256;
+    const int grid = grid_for(groups, threads);
+    if (dt == HAD_BF16)
+        had::soft_codes_kernel<__nv_bfloat16><<<grid, threads, 0, st>>>(
+            static_cast<const __nv_bfloat16 *>(x), sigma, c, H, n, d, groups, t, status);
+    else
+        had::soft_codes_kernel<float><<<grid, threads, 0, st>>>(
+            static_cast<const float *>(x), sigma, c, H, n, d, groups, t, status);
+    return launched();
+}
+
+template <int D>
+had_status_t launch_soft_logits(const float *tq, const float *tk, int n, long long heads,
+                                float *S, cudaStream_t st)
+{
+    constexpr int smem = had::soft_logits_smem_bytes<D>();
+    if (cudaFuncSetAttribute(had::soft_logits_kernel<D>,
+                             cudaFuncAttributeMaxDynamicSharedMemorySize, smem) != cudaSuccess)
+        return HAD_ERR_CUDA;
+    const unsigned tiles = (unsigned)((n + had::kSoftTile - 1) / had::kSoftTile);
+    had::soft_logits_kernel<D><<<dim3(tiles, tiles, (unsigned)heads), 256, smem, st>>>(
+        tq, tk, n, soft_ld(n), S);
+    return launched();
+}
+
+// Soft top-N over all heads, one group of heads at a time through the scratch.
+had_status_t launch_soft_topn(const float *tq, const float *tk, int B, int H, int n, int d,
+                              int N, int32_t *idx, float *lg, float *S, cudaStream_t st)
+{
+    const long long bh = (long long)B * H, g = soft_group(B, H, n);
+    const int smem = (int)had::soft_select_smem_bytes(n);
+    auto *select = d == 64 ? had::soft_select_kernel<64> : had::soft_select_kernel<128>;
+    if (cudaFuncSetAttribute(select,
+                             cudaFuncAttributeMaxDynamicSharedMemorySize, smem) != cudaSuccess)
+        return HAD_ERR_CUDA;
+    for (long long h0 = 0; h0 < bh; h0 += g) {
+        const long long heads = bh - h0 < g ? bh - h0 : g;
+        const long long off = h0 * n * (long long)d;
+        had_status_t s = d == 64 ? launch_soft_logits<64>(tq + off, tk + off, n, heads, S, st)
+                                 : launch_soft_logits<128>(tq + off, tk + off, n, heads, S, st);
+        if (s != HAD_OK) return s;
+        const long long rows = heads * n;
+        if (rows > INT_MAX) return HAD_ERR_UNSUPPORTED;
+        select<<<(unsigned)rows, had::kSelThreads, smem, st>>>(
+            S, soft_ld(n), n, N, h0 * n, idx, lg);
+        if ((s = launched()) != HAD_OK) return s;
+    }
+    return HAD_OK;
+}
+
+// Workspace of the soft forward: codes of Q and K, the kept set, the scratch.
+struct SoftWorkspace {
+    size_t tq, tk, idx, logits, scratch, total;
+};
+
+SoftWorkspace soft_layout(int B, int H, int n, int d, int N)
+{
+    const size_t rows = (size_t)B * H * n;
+    SoftWorkspace w;
+    w.tq = 0;
+    w.tk = w.tq + round_up(rows * d * 4);
+    w.idx = w.tk + round_up(rows * d * 4);
+    w.logits = w.idx + round_up(rows * (size_t)N * 4);
+    w.scratch = w.logits + round_up(rows * (size_t)N * 4);
+    w.total = w.scratch + soft_scratch_bytes(B, H, n);
+    return w;
+}
+
+bool finite_float(float x) { return x == x && x < 3.0e38f && x > -3.0e38f; }
 
 }  // namespace
 
@@ -538,6 +650,77 @@ had_status_t had_topn_mass(const uint32_t *qbits, const uint32_t *kbits, int B, 
                    : launch_mass_dw<4>(qbits, kbits, B, H, n, tau, ps, nmin, stream);
 }
 
+had_status_t had_soft_binarize(const void *x, had_dtype_t dt, const float *sigma, float c, int B,
+                               int H, int n, int d, float *t, int32_t *dev_status,
+                               cudaStream_t stream)
+{
+    had_status_t s = check_shape(B, H, n, d);
+    if (s != HAD_OK) return s;
+    if (dt != HAD_BF16 && dt != HAD_F32) return HAD_ERR_INVALID_ARG;
+    if (!x || !sigma || !t) return HAD_ERR_INVALID_ARG;
+    if (!aligned16(x) || !aligned16(t)) return HAD_ERR_INVALID_ARG;
+    if (!finite_float(c) || !(c > 0.0f)) return HAD_ERR_INVALID_ARG;
+    return launch_soft_codes(x, dt, sigma, c, B, H, n, d, t, dev_status, stream);
+}
+
+had_status_t had_soft_topn(const float *tq, const float *tk, int B, int H, int n, int d, int N,
+                           int32_t *idx, float *logits, void *ws, size_t ws_bytes,
+                           int32_t *dev_status, cudaStream_t stream)
+{
+    (void)dev_status;
+    had_status_t s = check_soft(B, H, n, d, N);
+    if (s != HAD_OK) return s;
+    if (!tq || !tk || !idx || !ws) return HAD_ERR_INVALID_ARG;
+    if (!aligned16(tq) || !aligned16(tk) || !aligned16(idx) || !aligned16(ws) ||
+        (logits && !aligned16(logits)))
+        return HAD_ERR_INVALID_ARG;
+    if (ws_bytes < soft_scratch_bytes(B, H, n)) return HAD_ERR_WORKSPACE;
+    return launch_soft_topn(tq, tk, B, H, n, d, N, idx, logits, static_cast<float *>(ws), stream);
+}
+
+had_status_t had_soft_softmax_av(const int32_t *idx, const float *logits, const void *V,
+                                 had_dtype_t dt, int B, int H, int n, int d, int N, float tau,
+                                 float *out, float *p, int32_t *dev_status, cudaStream_t stream)
+{
+    had_status_t s = check_topn(B, H, n, d, N);
+    if (s != HAD_OK) return s;
+    if (dt != HAD_BF16 && dt != HAD_F32) return HAD_ERR_INVALID_ARG;
+    if (!idx || !logits || !V || !out) return HAD_ERR_INVALID_ARG;
+    if (!aligned16(idx) || !aligned16(logits) || !aligned16(V) || !aligned16(out) ||
+        (p && !aligned16(p)))
+        return HAD_ERR_INVALID_ARG;
+    if (!finite_float(tau)) return HAD_ERR_INVALID_ARG;
+    return launch_av(idx, logits, V, dt, B, H, n, d, N, tau, out, p, dev_status, stream);
+}
+
+had_status_t had_soft_attention_fwd(const void *Q, const void *K, const void *V, had_dtype_t dt,
+                                    const float *sigma_q, const float *sigma_k, float c, int B,
+                                    int H, int n, int d, int N, float tau, float *out, void *ws,
+                                    size_t ws_bytes, int32_t *dev_status, cudaStream_t stream)
+{
+    had_status_t s = check_soft(B, H, n, d, N);
+    if (s != HAD_OK) return s;
+    if (dt != HAD_BF16 && dt != HAD_F32) return HAD_ERR_INVALID_ARG;
+    if (!Q || !K || !V || !sigma_q || !sigma_k || !out || !ws) return HAD_ERR_INVALID_ARG;
+    if (!aligned16(Q) || !aligned16(K) || !aligned16(V) || !aligned16(out) || !aligned16(ws))
+        return HAD_ERR_INVALID_ARG;
+    if (!finite_float(c) || !(c > 0.0f) || !finite_float(tau)) return HAD_ERR_INVALID_ARG;
+    const SoftWorkspace w = soft_layout(B, H, n, d, N);
+    if (ws_bytes < w.total) return HAD_ERR_WORKSPACE;
+    char *base = static_cast<char *>(ws);
+    auto *tq = reinterpret_cast<float *>(base + w.tq);
+    auto *tk = reinterpret_cast<float *>(base + w.tk);
+    auto *idx = reinterpret_cast<int32_t *>(base + w.idx);
+    auto *lg = reinterpret_cast<float *>(base + w.logits);
+    auto *S = reinterpret_cast<float *>(base + w.scratch);
+    if ((s = launch_soft_codes(Q, dt, sigma_q, c, B, H, n, d, tq, dev_status, stream)) != HAD_OK)
+        return s;
+    if ((s = launch_soft_codes(K, dt, sigma_k, c, B, H, n, d, tk, dev_status, stream)) != HAD_OK)
+        return s;
+    if ((s = launch_soft_topn(tq, tk, B, H, n, d, N, idx, lg, S, stream)) != HAD_OK) return s;
+    return launch_av(idx, lg, V, dt, B, H, n, d, N, tau, out, nullptr, dev_status, stream);
+}
+
 size_t had_workspace_bytes(int op, int B, int H, int n, int d, int N)
 {
     switch (op) {
@@ -555,6 +738,15 @@ size_t had_workspace_bytes(int op, int B, int H, int n, int d, int N)
         return check_shape(B, H, n, d) == HAD_OK ? 0 : (size_t)-1;
     case HAD_OP_ATTENTION_CAUSAL:
         return check_topn(B, H, n, d, N) == HAD_OK ? causal_layout(B, H, n, d, N).total
+                                                   : (size_t)-1;
+    case HAD_OP_SOFT_BINARIZE:
+        return check_shape(B, H, n, d) == HAD_OK ? 0 : (size_t)-1;
+    case HAD_OP_SOFT_TOPN:
+        return check_soft(B, H, n, d, N) == HAD_OK ? soft_scratch_bytes(B, H, n) : (size_t)-1;
+    case HAD_OP_SOFT_SOFTMAX_AV:
+        return check_topn(B, H, n, d, N) == HAD_OK ? 0 : (size_t)-1;
+    case HAD_OP_SOFT_ATTENTION_FWD:
+        return check_soft(B, H, n, d, N) == HAD_OK ? soft_layout(B, H, n, d, N).total
                                                    : (size_t)-1;
     default:
         return (size_t)-1;
@@ -579,6 +771,14 @@ int had_launch_count(int op, int B, int H, int n, int d, int N)
         return check_shape(B, H, n, d) == HAD_OK ? 1 : -1;
     case HAD_OP_ATTENTION_CAUSAL:
         return check_topn(B, H, n, d, N) == HAD_OK ? 4 : -1;
+    case HAD_OP_SOFT_BINARIZE:
+        return check_shape(B, H, n, d) == HAD_OK ? 1 : -1;
+    case HAD_OP_SOFT_TOPN:
+        return check_soft(B, H, n, d, N) == HAD_OK ? 2 * soft_passes(B, H, n) : -1;
+    case HAD_OP_SOFT_SOFTMAX_AV:
+        return check_topn(B, H, n, d, N) == HAD_OK ? 1 : -1;
+    case HAD_OP_SOFT_ATTENTION_FWD:
+        return check_soft(B, H, n, d, N) == HAD_OK ? 3 + 2 * soft_passes(B, H, n) : -1;
     default:
         return -1;
     }

@@ -79,6 +79,23 @@ struct VSlice {
     }
 };
 
+// Logits arrive as int16 (binarized codes: integers in [-d, d]) or fp32
+// (soft codes); the row maximum and the differences s - m take their type.
+template <typename L>
+struct LogitT;
+template <>
+struct LogitT<int16_t> {
+    using M = int;
+    __device__ __forceinline__ static M lowest() { return -2147483647; }
+    __device__ __forceinline__ static float diff(int16_t s, M m) { return (float)((int)s - m); }
+};
+template <>
+struct LogitT<float> {
+    using M = float;
+    __device__ __forceinline__ static M lowest() { return -__int_as_float(0x7f800000); }
+    __device__ __forceinline__ static float diff(float s, M m) { return s - m; }
+};
+
 // One warp per query row, split into four 8-lane groups.  Kept entries are
 // taken 32 at a time: lane l reads index and logit l of the chunk and
 // computes its weight exp(tau (s - m)) once; then in 8 rounds each group
@@ -88,9 +105,9 @@ struct VSlice {
 // 32 rows in flight per warp: the gather is bound by L2 bandwidth, not by
 // its latency.  The four groups' partial sums are added with two shuffles at
 // the end, and each group stores a quarter of the row.
-template <typename T, int D>
+template <typename T, int D, typename L = int16_t>
 __global__ void __launch_bounds__(256)
-sparse_softmax_av_kernel(const int32_t *__restrict__ idx, const int16_t *__restrict__ logits,
+sparse_softmax_av_kernel(const int32_t *__restrict__ idx, const L *__restrict__ logits,
                          const T *__restrict__ V, int n, int N, float tau, long long rows,
                          float *__restrict__ out, float *__restrict__ p, int32_t *status)
 {
@@ -105,14 +122,15 @@ sparse_softmax_av_kernel(const int32_t *__restrict__ idx, const int16_t *__restr
     if (row >= rows) return;
     const long long head = row / n;
     const int32_t *ir = idx + row * N;
-    const int16_t *lr = logits + row * N;
+    const L *lr = logits + row * N;
     const T *vh = V + head * n * (long long)D;
+    using LT = LogitT<L>;
 
     // an index of -1 marks an empty slot (rows of the causal form that see
     // fewer than N keys): it weighs nothing and takes no part in the max
-    int m = -2147483647;
+    typename LT::M m = LT::lowest();
     for (int k = lane; k < N; k += 32)
-        if (ir[k] != -1) m = max(m, (int)lr[k]);
+        if (ir[k] != -1) m = max(m, (typename LT::M)lr[k]);
 #pragma unroll
     for (int o = 16; o > 0; o >>= 1) m = max(m, __shfl_xor_sync(kFullMask, m, o));
 
@@ -133,7 +151,7 @@ sparse_softmax_av_kernel(const int32_t *__restrict__ idx, const int16_t *__restr
                 j = -1;
                 w = 0.0f;
             } else {
-                w = expf(tau * (float)((int)lr[k] - m));
+                w = expf(tau * LT::diff(lr[k], m));
             }
         }
         z += w;
@@ -188,7 +206,7 @@ sparse_softmax_av_kernel(const int32_t *__restrict__ idx, const int16_t *__restr
     if (p) {
         for (int k = lane; k < N; k += 32) {
             const int j = ir[k];
-            const float w = (j < 0 || j >= n) ? 0.0f : expf(tau * (float)((int)lr[k] - m));
+            const float w = (j < 0 || j >= n) ? 0.0f : expf(tau * LT::diff(lr[k], m));
             p[row * N + k] = w * inv;
         }
     }

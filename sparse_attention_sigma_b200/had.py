@@ -35,6 +35,10 @@ HAD_OP_ATTENTION_PREPARE = 4
 HAD_OP_ATTENTION_CORE = 5
 HAD_OP_TOPN_MASS = 6
 HAD_OP_ATTENTION_CAUSAL = 7
+HAD_OP_SOFT_BINARIZE = 8
+HAD_OP_SOFT_TOPN = 9
+HAD_OP_SOFT_SOFTMAX_AV = 10
+HAD_OP_SOFT_ATTENTION_FWD = 11
 
 
 class HadError(RuntimeError):
@@ -64,6 +68,11 @@ def _load():
         "had_hamming_topn_causal": [vp, vp, i32, i32, i32, i32, i32, vp, vp, vp, vp],
         "had_attention_causal_fwd": [vp, vp, vp, i32, vp, vp, i32, i32, i32, i32, i32, f32, vp,
                                      vp, sz, vp, vp],
+        "had_soft_binarize": [vp, i32, vp, f32, i32, i32, i32, i32, vp, vp, vp],
+        "had_soft_topn": [vp, vp, i32, i32, i32, i32, i32, vp, vp, vp, sz, vp, vp],
+        "had_soft_softmax_av": [vp, vp, vp, i32, i32, i32, i32, i32, i32, f32, vp, vp, vp, vp],
+        "had_soft_attention_fwd": [vp, vp, vp, i32, vp, vp, f32, i32, i32, i32, i32, i32, f32,
+                                   vp, vp, sz, vp, vp],
     }
     for name, args in sig.items():
         fn = getattr(lib, name)
@@ -224,6 +233,94 @@ def had_attention_causal_fwd(Q, K, V, sigma_q, sigma_k, N, tau, out=None, ws=Non
                                        _ptr(out), _ptr(ws), ws.numel(), _ptr(dev_status),
                                        _stream(stream))
     _check(st, "had_attention_causal_fwd")
+    return out
+
+
+def had_soft_binarize(x, sigma, c, t=None, dev_status=None, stream=None):
+    """Soft codes tanh(c * x / sigma[h]) as float32 [B,H,n,d] (tanh training stages)."""
+    _dev(x, "x")
+    B, H, n, d = _shape4(x, "x")
+    _dev(sigma, "sigma", torch.float32, (H,))
+    if t is None:
+        t = torch.empty((B, H, n, d), dtype=torch.float32, device=x.device)
+    _dev(t, "t", torch.float32, (B, H, n, d))
+    st = _lib.had_soft_binarize(_ptr(x), _dtype_code(x), _ptr(sigma), ctypes.c_float(c), B, H,
+                                n, d, _ptr(t), _ptr(dev_status), _stream(stream))
+    _check(st, "had_soft_binarize")
+    return t
+
+
+def had_soft_topn(tq, tk, N, idx=None, logits=None, ws=None, dev_status=None, stream=None,
+                  want_logits=True):
+    """Top-N of the soft logits tq . tk; returns (idx int32, logits float32 or None)."""
+    _dev(tq, "tq", torch.float32)
+    B, H, n, d = _shape4(tq, "tq")
+    _dev(tk, "tk", torch.float32, (B, H, n, d))
+    if idx is None:
+        idx = torch.empty((B, H, n, N), dtype=torch.int32, device=tq.device)
+    _dev(idx, "idx", torch.int32, (B, H, n, N))
+    if logits is None and want_logits:
+        logits = torch.empty((B, H, n, N), dtype=torch.float32, device=tq.device)
+    if logits is not None:
+        _dev(logits, "logits", torch.float32, (B, H, n, N))
+    need = had_workspace_bytes(HAD_OP_SOFT_TOPN, B, H, n, d, N)
+    if need < 0:
+        raise HadError(HAD_ERR_UNSUPPORTED if d not in (64, 128) else HAD_ERR_INVALID_ARG,
+                       "had_soft_topn")
+    if ws is None:
+        ws = torch.empty(need, dtype=torch.uint8, device=tq.device)
+    st = _lib.had_soft_topn(_ptr(tq), _ptr(tk), B, H, n, d, N, _ptr(idx), _ptr(logits),
+                            _ptr(ws), ws.numel(), _ptr(dev_status), _stream(stream))
+    _check(st, "had_soft_topn")
+    return idx, logits
+
+
+def had_soft_softmax_av(idx, logits, V, tau, out=None, p=None, want_p=False, dev_status=None,
+                        stream=None):
+    """Softmax over kept fp32 logits and sparse product with V; returns (out, p or None)."""
+    _dev(V, "V")
+    B, H, n, d = _shape4(V, "V")
+    _dev(idx, "idx", torch.int32)
+    N = int(idx.shape[-1])
+    _dev(idx, "idx", torch.int32, (B, H, n, N))
+    _dev(logits, "logits", torch.float32, (B, H, n, N))
+    if out is None:
+        out = torch.empty((B, H, n, d), dtype=torch.float32, device=V.device)
+    _dev(out, "out", torch.float32, (B, H, n, d))
+    if p is None and want_p:
+        p = torch.empty((B, H, n, N), dtype=torch.float32, device=V.device)
+    if p is not None:
+        _dev(p, "p", torch.float32, (B, H, n, N))
+    st = _lib.had_soft_softmax_av(_ptr(idx), _ptr(logits), _ptr(V), _dtype_code(V), B, H, n, d,
+                                  N, ctypes.c_float(tau), _ptr(out), _ptr(p), _ptr(dev_status),
+                                  _stream(stream))
+    _check(st, "had_soft_softmax_av")
+    return out, p
+
+
+def had_soft_attention_fwd(Q, K, V, sigma_q, sigma_k, c, N, tau, out=None, ws=None,
+                           dev_status=None, stream=None):
+    """Top-N attention on the soft codes tanh(c x / sigma); returns out [B,H,n,d] float32."""
+    _dev(Q, "Q")
+    B, H, n, d = _shape4(Q, "Q")
+    _dev(K, "K", Q.dtype, (B, H, n, d))
+    _dev(V, "V", Q.dtype, (B, H, n, d))
+    _dev(sigma_q, "sigma_q", torch.float32, (H,))
+    _dev(sigma_k, "sigma_k", torch.float32, (H,))
+    if out is None:
+        out = torch.empty((B, H, n, d), dtype=torch.float32, device=Q.device)
+    _dev(out, "out", torch.float32, (B, H, n, d))
+    need = had_workspace_bytes(HAD_OP_SOFT_ATTENTION_FWD, B, H, n, d, N)
+    if need < 0:
+        raise HadError(HAD_ERR_UNSUPPORTED if d not in (64, 128) else HAD_ERR_INVALID_ARG,
+                       "had_soft_attention_fwd")
+    if ws is None:
+        ws = torch.empty(need, dtype=torch.uint8, device=Q.device)
+    st = _lib.had_soft_attention_fwd(_ptr(Q), _ptr(K), _ptr(V), _dtype_code(Q), _ptr(sigma_q),
+                                     _ptr(sigma_k), ctypes.c_float(c), B, H, n, d, N,
+                                     ctypes.c_float(tau), _ptr(out), _ptr(ws), ws.numel(),
+                                     _ptr(dev_status), _stream(stream))
+    _check(st, "had_soft_attention_fwd")
     return out
 
 

@@ -136,3 +136,39 @@ def test_causal_argument_errors_return_before_any_cuda_call(lib):
     assert lib.had_workspace_bytes(7, 1, 1, 128, 64, 16) >= 128 * (8 + 8 + 6 * 16)
     assert lib.had_workspace_bytes(7, 1, 1, 128, 64, 129) == ctypes.c_size_t(-1).value
     assert lib.had_launch_count(7, 1, 1, 128, 64, 16) == 4
+
+
+def test_soft_argument_errors_return_before_any_cuda_call(lib):
+    vp, i, sz, f = ctypes.c_void_p, ctypes.c_int, ctypes.c_size_t, ctypes.c_float
+    fake = vp(4096)        # never dereferenced: the checks fail first
+    b = lib.had_soft_binarize
+    b.argtypes = [vp, i, vp, f, i, i, i, i, vp, vp, vp]
+    b.restype = ctypes.c_int
+    assert b(fake, 0, fake, 1.0, 1, 1, 8, 96, fake, None, None) == 2            # d
+    assert b(fake, 0, fake, 0.0, 1, 1, 8, 64, fake, None, None) == 1            # c = 0
+    assert b(fake, 0, fake, float("inf"), 1, 1, 8, 64, fake, None, None) == 1   # c = inf
+    assert b(fake, 0, fake, 1.0, 1, 1, 8, 64, vp(4100), None, None) == 1        # misaligned
+    t = lib.had_soft_topn
+    t.argtypes = [vp, vp, i, i, i, i, i, vp, vp, vp, sz, vp, vp]
+    t.restype = ctypes.c_int
+    assert t(fake, fake, 1, 1, 8, 64, 9, fake, fake, fake, 1 << 30, None, None) == 1   # N > n
+    assert t(fake, fake, 1, 1, 40000, 64, 9, fake, fake, fake, 1 << 40, None, None) == 2
+    assert t(fake, fake, 1, 1, 8, 64, 2, fake, fake, fake, 16, None, None) == 3        # ws
+    a = lib.had_soft_attention_fwd
+    a.argtypes = [vp, vp, vp, i, vp, vp, f, i, i, i, i, i, f, vp, vp, sz, vp, vp]
+    a.restype = ctypes.c_int
+    assert a(fake, fake, fake, 0, fake, fake, -1.0, 1, 1, 8, 64, 2, 0.1, fake, fake, 1 << 30,
+             None, None) == 1                                                    # c < 0
+    assert a(fake, fake, fake, 0, fake, fake, 1.0, 1, 1, 8, 64, 2, 0.1, fake, fake, 64,
+             None, None) == 3                                                    # ws
+    lib.had_workspace_bytes.restype = ctypes.c_size_t
+    lib.had_workspace_bytes.argtypes = [ctypes.c_int] * 6
+    lib.had_launch_count.argtypes = [ctypes.c_int] * 6
+    # long workload: 64 heads of 64 MiB logits, 32 heads per 2 GiB group -> 2 groups
+    assert lib.had_workspace_bytes(9, 4, 16, 4096, 64, 512) == 2 << 30
+    assert lib.had_launch_count(9, 4, 16, 4096, 64, 512) == 4
+    assert lib.had_launch_count(11, 4, 16, 4096, 64, 512) == 7
+    assert lib.had_launch_count(8, 4, 16, 4096, 64, 512) == 1
+    # ragged n: rows padded to a multiple of 4 floats
+    assert lib.had_workspace_bytes(9, 1, 1, 130, 64, 5) >= 130 * 132 * 4
+    assert lib.had_workspace_bytes(11, 1, 1, 130, 64, 5) >= 130 * (2 * 64 * 4 + 8 * 5) + 130 * 132 * 4

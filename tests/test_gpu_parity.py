@@ -393,3 +393,147 @@ def test_empty_slots_give_zeros_without_error(had):
     v5 = c.gv[0, 0, 5].float()
     assert torch.equal(out[0, 0, 1::2], v5.expand(32, -1))
     assert torch.all(p[0, 0, 1::2, 3] == 1) and p[0, 0, 1::2].sum() == 32
+
+
+# ------------------------------------------------------ soft (tanh) codes
+
+
+def _soft_inputs(B, H, n, d, seed, dtype=torch.bfloat16, dup=0, min_abs=0.0):
+    g = torch.Generator().manual_seed(seed)
+    q = torch.randn(B, H, n, d, generator=g)
+    k = torch.randn(B, H, n, d, generator=g)
+    v = torch.randn(B, H, n, d, generator=g)
+    if min_abs:                    # move small entries out to +-min_abs
+        away = lambda x: torch.where(x.abs() < min_abs,
+                                     torch.where(x >= 0, min_abs, -min_abs), x)
+        q, k = away(q), away(k)
+    if dup:
+        k[:, :, dup:2 * dup] = k[:, :, :dup]
+    q, k, v = q.to(dtype), k.to(dtype), v.to(dtype)
+    return q, k, v, synth.per_head_sigma(q), synth.per_head_sigma(k)
+
+
+def _ulps(got, want):
+    got = np.asarray(got, np.float32)
+    want = np.asarray(want, np.float32)
+    return np.abs(got.astype(np.float64) - want) / np.spacing(np.maximum(np.abs(want), 1e-30))
+
+
+def _soft_error_bound(o_tq, o_tk, rows, n, d):
+    """Bound on |GPU logit - oracle logit| per (row, key): codes within 2 ulp
+    (tanhf) and fp32 accumulation of d products, from sum_k |tq_k| |tk_k|."""
+    tq = np.abs(o_tq.reshape(-1, d)).astype(np.float64)
+    tk = np.abs(o_tk.reshape(-1, n, d)).astype(np.float64)
+    A = np.stack([tq[r] @ tk[r // n].T for r in rows])
+    return (2.0 ** -20 + d * 2.0 ** -23) * A + 1e-30
+
+
+def _check_soft(had, q, k, v, sgq, sgk, c, N, tau, rows, min_unique=0.8):
+    B, H, n, d = q.shape
+    gq, gk, gv = q.cuda(), k.cuda(), v.cuda()
+    gsq, gsk = sgq.cuda(), sgk.cuda()
+    status = torch.zeros(1, dtype=torch.int32, device="cuda")
+    tq = had.had_soft_binarize(gq, gsq, c, dev_status=status)
+    tk = had.had_soft_binarize(gk, gsk, c, dev_status=status)
+    idx, lg = had.had_soft_topn(tq, tk, N)
+    out, p = had.had_soft_softmax_av(idx, lg, gv, tau, want_p=True, dev_status=status)
+    out1 = had.had_soft_attention_fwd(gq, gk, gv, gsq, gsk, c, N, tau, dev_status=status)
+    torch.cuda.synchronize()
+    assert status.item() == 0
+    assert torch.equal(out, out1)
+
+    o_tq = oracle.soft_binarize(synth.to_oracle_array(q), sgq.numpy(), c)
+    o_tk = oracle.soft_binarize(synth.to_oracle_array(k), sgk.numpy(), c)
+    assert _ulps(tq.cpu().numpy(), o_tq).max() <= 2
+    assert _ulps(tk.cpu().numpy(), o_tk).max() <= 2
+
+    o_idx, o_lg, o_p, o_out = oracle.soft_attention_rows(
+        o_tq, o_tk, synth.to_oracle_array(v), tau, N, rows)
+    s_or = oracle.soft_logits_rows(o_tq, o_tk, rows)
+    eps = _soft_error_bound(o_tq, o_tk, rows, n, d)
+    flat = lambda t: t.reshape(-1, t.shape[-1]).cpu().numpy()[rows]
+    g_idx, g_lg, g_p, g_out = flat(idx), flat(lg), flat(p), flat(out)
+    unique = 0
+    for t in range(len(rows)):
+        gi = g_idx[t]
+        assert (np.diff(gi) > 0).all() and gi[0] >= 0 and gi[-1] < n
+        assert (np.abs(g_lg[t].astype(np.float64) - s_or[t, gi]) <= eps[t, gi]).all()
+        kept = np.zeros(n, bool)
+        kept[gi] = True
+        if N < n:
+            # no dropped key can have been seen above a kept one
+            assert (s_or[t, kept] + eps[t, kept]).min() >= (s_or[t, ~kept] - eps[t, ~kept]).max()
+        ok = np.zeros(n, bool)
+        ok[o_idx[t]] = True
+        # The oracle's kept set is fixed beyond rounding when its threshold
+        # value T (with any exact ties at T, which equal codes reproduce
+        # exactly on both sides) is separated from every other value by
+        # more than the error bounds.
+        vals, e = s_or[t], eps[t]
+        T = vals[ok].min()
+        at = vals == T
+        e_T = e[at].max()
+        above = ok & ~at
+        below = ~ok & ~at
+        isolated = ((vals[above] - e[above]).min(initial=np.inf) > T + e_T and
+                    T - e_T > (vals[below] + e[below]).max(initial=-np.inf))
+        if N == n or isolated:
+            unique += 1            # the kept set is fixed beyond rounding: compare all
+            assert np.array_equal(gi, o_idx[t])
+            assert_close(g_out[t], o_out[t], "soft out")
+            assert_close(g_p[t], o_p[t], "soft p")
+    assert unique >= min_unique * len(rows), f"only {unique} of {len(rows)} rows unique"
+    assert np.allclose(g_p.sum(axis=1), 1.0, atol=1e-5)
+
+
+SOFT_SMALL = [
+    # (B, H, n, d, N, seed, c, dtype)
+    (1, 2, 300, 64, 40, 51, 1.0, torch.bfloat16),
+    (2, 1, 257, 128, 33, 52, 2.0, torch.bfloat16),
+    (1, 1, 1, 64, 1, 53, 1.0, torch.bfloat16),
+    (1, 2, 130, 64, 130, 54, 0.5, torch.float32),      # N = n: dense softmax
+    (1, 3, 200, 64, 1, 55, 1.5, torch.float32),        # N = 1
+    (1, 1, 700, 64, 90, 56, 0.2, torch.bfloat16),
+]
+
+
+@pytest.mark.parametrize("B,H,n,d,N,seed,c,dtype", SOFT_SMALL)
+def test_soft_small_all_rows(had, B, H, n, d, N, seed, c, dtype):
+    q, k, v, sgq, sgk = _soft_inputs(B, H, n, d, seed, dtype)
+    _check_soft(had, q, k, v, sgq, sgk, c, N, 1 / math.sqrt(d), np.arange(B * H * n))
+
+
+def test_soft_exact_ties_keep_the_lower_index(had):
+    q, k, v, sgq, sgk = _soft_inputs(1, 2, 160, 64, 57, dup=40)
+    _check_soft(had, q, k, v, sgq, sgk, 1.0, 24, 0.125, np.arange(320))
+    # all keys equal: every logit of a row ties, the first N keys are kept
+    k_all = k[:, :, :1].expand(-1, -1, 160, -1).contiguous()
+    tq = had.had_soft_binarize(q.cuda(), sgq.cuda(), 1.0)
+    tk = had.had_soft_binarize(k_all.cuda(), synth.per_head_sigma(k_all).cuda(), 1.0)
+    idx, _ = had.had_soft_topn(tq, tk, 24)
+    assert (idx.cpu() == torch.arange(24, dtype=torch.int32)).all()
+
+
+def test_soft_at_large_c_is_the_binarized_path(had):
+    # with |x / sigma| >= 0.01 and c = 1e4 every code is exactly +-1, so the
+    # soft path must give the binarized path's kept set, ties included
+    q, k, v, sgq, sgk = _soft_inputs(1, 2, 300, 64, 58, torch.float32, min_abs=0.05)
+    tq = had.had_soft_binarize(q.cuda(), sgq.cuda(), 1e4)
+    tk = had.had_soft_binarize(k.cuda(), sgk.cuda(), 1e4)
+    assert torch.equal(tq.abs(), torch.ones_like(tq))
+    idx, lg = had.had_soft_topn(tq, tk, 37)
+    out, _ = had.had_soft_softmax_av(idx, lg, v.cuda(), 0.125)
+    sq = oracle.binarize(synth.to_oracle_array(q), sgq.numpy())
+    sk = oracle.binarize(synth.to_oracle_array(k), sgk.numpy())
+    o_idx, o_lg, _, o_out = oracle.attention_rows(sq, sk, synth.to_oracle_array(v), 0.125, 37,
+                                                  np.arange(600))
+    assert np.array_equal(idx.reshape(600, 37).cpu().numpy(), o_idx)
+    assert np.array_equal(lg.reshape(600, 37).cpu().numpy(), o_lg.astype(np.float32))
+    assert_close(out.reshape(600, 64).cpu().numpy(), o_out, "soft large-c out")
+
+
+def test_soft_long_workload_sampled(had):
+    cfg = synth.CONFIGS["long"]
+    c = config_case("long")
+    rows = synth.sample_rows(cfg, 192, seed=61)
+    _check_soft(had, c.q, c.k, c.v, c.sgq, c.sgk, 1.0, cfg.N, cfg.tau, rows)
