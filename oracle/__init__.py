@@ -21,7 +21,10 @@ softmax, closed forms (all keys equal, N = 1), and a hand-worked example
 under ``tests/golden/``.  The soft (tanh) codes of the training stages are
 pinned by tanh closed forms (tanh(ln 2) = 3/5, tanh(ln 3) = 4/5, ...), their
 limits (signs at large c, the scaled dot product at small c), oddness, a
-numpy sort with exact ties, and a dense library softmax at N = n.  No
+numpy sort with exact ties, and a dense library softmax at N = n.  The
+straight-through backward is pinned by torch autograd in float64 (the
+surrogate sign, the kept set as a fixed mask), by finite differences of the
+forward in V, and by closed forms (N = 1 and tau = 0 give dQ = dK = 0).  No
 function is left unpinned.
 """
 import ctypes
@@ -70,6 +73,10 @@ def _load():
             lp, lp, lp, c_int, c_long, c_long, c_long, c_long, c_long,
             ctypes.c_float, lp, c_long, lp, lp, lp, lp, c_int]
         lib.had_oracle_soft_attention_rows.restype = c_int
+        lib.had_oracle_attention_bwd.argtypes = [
+            lp, lp, lp, c_int, lp, lp, lp, c_long, c_long, c_long, c_long, c_long,
+            ctypes.c_float, ctypes.c_float, lp, lp, lp, c_int]
+        lib.had_oracle_attention_bwd.restype = c_int
         lib.had_oracle_max_threads.argtypes = []
         lib.had_oracle_max_threads.restype = c_int
         _lib = lib
@@ -268,3 +275,30 @@ def soft_attention_rows(tq, tk, v, tau, N, rows, threads=0):
     if rc != 0:
         raise ValueError("oracle rejected the arguments (N must be in [1, n])")
     return idx, lg, p, out
+
+
+def attention_bwd(q, k, v, sigma_q, sigma_k, dout, tau, N, clip=1.0, threads=0):
+    """Straight-through backward of the binarized top-N forward.
+
+    q, k, v are [B,H,n,d] (float32, or bf16 bit patterns as uint16, all the
+    same); dout is float32 [B,H,n,d].  Returns (dq, dk, dv) as float64
+    [B,H,n,d]: the sign passes the gradient where |x / sigma| <= clip."""
+    q = np.ascontiguousarray(q)
+    k = np.ascontiguousarray(k)
+    v = np.ascontiguousarray(v)
+    dout = np.ascontiguousarray(dout, dtype=np.float32)
+    sigma_q = np.ascontiguousarray(sigma_q, dtype=np.float32)
+    sigma_k = np.ascontiguousarray(sigma_k, dtype=np.float32)
+    B, H, n, d = q.shape
+    assert k.shape == q.shape and v.shape == q.shape and dout.shape == q.shape
+    assert q.dtype == k.dtype == v.dtype
+    dq = np.empty((B, H, n, d), dtype=np.float64)
+    dk = np.empty_like(dq)
+    dv = np.empty_like(dq)
+    rc = _load().had_oracle_attention_bwd(
+        _ptr(q), _ptr(k), _ptr(v), _is_bf16(q), _ptr(sigma_q), _ptr(sigma_k), _ptr(dout),
+        B, H, n, d, int(N), ctypes.c_float(float(tau)), ctypes.c_float(float(clip)),
+        _ptr(dq), _ptr(dk), _ptr(dv), int(threads))
+    if rc != 0:
+        raise ValueError("oracle rejected the arguments (N must be in [1, n])")
+    return dq, dk, dv

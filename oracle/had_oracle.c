@@ -571,6 +571,135 @@ int had_oracle_soft_attention_rows(const float *tq, const float *tk,
     return failed ? -1 : 0;
 }
 
+/*
+ * Backward pass of the binarized forward for the straight-through training
+ * stage (pith.science review of arXiv 2502.01770: after the tanh stages a
+ * straight-through estimator finishes the binarization).  Readings taken:
+ *   - the forward is steps 1-4 above; the top-N mask is a fixed selection
+ *     (no gradient), softmax and value product are differentiated exactly;
+ *   - the sign passes the gradient straight through where |z| <= clip and
+ *     blocks it elsewhere (z = x / sigma in fp32; clip = 1 is the usual
+ *     choice, clip = +inf passes it everywhere); z = x / sigma contributes
+ *     1 / sigma; sigma itself is a data statistic and gets no gradient.
+ * With dO the gradient of the loss with respect to O, per head and query i
+ * over its kept set K_i (p_ij the kept softmax weights):
+ *   dV_j  = sum_{i: j in K_i} p_ij dO_i
+ *   dp_ij = dO_i . V_j,   D_i = sum_j p_ij dp_ij,   ds_ij = tau p_ij (dp_ij - D_i)
+ *   dQb_i = sum_{j in K_i} ds_ij Kb_j,   dKb_j = sum_{i: j in K_i} ds_ij Qb_i
+ *   dQ = dQb * [|zq| <= clip] / sigma_q,  dK likewise.
+ * All in fp64; every head is processed by one thread in a fixed order.
+ * dO is fp32 [B,H,n,d]; dq, dk, dv are fp64 [B,H,n,d].  Returns 0, or -1 on
+ * a bad argument or an allocation failure.
+ */
+int had_oracle_attention_bwd(const void *q, const void *k, const void *v,
+                             int is_bf16, const float *sigma_q,
+                             const float *sigma_k, const float *dout, long B,
+                             long H, long n, long d, long N, float tau,
+                             float clip, double *dq, double *dk, double *dv,
+                             int nthreads)
+{
+    if (N < 1 || N > n || d < 1 || n < 1)
+        return -1;
+    int failed = 0;
+#ifdef _OPENMP
+    if (nthreads > 0)
+        omp_set_num_threads(nthreads);
+#pragma omp parallel
+#endif
+    {
+        int8_t *sq = (int8_t *)malloc((size_t)(n * d));
+        int8_t *sk = (int8_t *)malloc((size_t)(n * d));
+        int32_t *s = (int32_t *)malloc(sizeof(int32_t) * (size_t)n);
+        keyed_t *order = (keyed_t *)malloc(sizeof(keyed_t) * (size_t)n);
+        double *p = (double *)malloc(sizeof(double) * (size_t)N);
+        double *ds = (double *)malloc(sizeof(double) * (size_t)N);
+        double *dqb = (double *)malloc(sizeof(double) * (size_t)(n * d));
+        double *dkb = (double *)malloc(sizeof(double) * (size_t)(n * d));
+#ifdef _OPENMP
+#pragma omp for schedule(dynamic, 1)
+#endif
+        for (long head = 0; head < B * H; ++head) {
+            if (!sq || !sk || !s || !order || !p || !ds || !dqb || !dkb) {
+#ifdef _OPENMP
+#pragma omp atomic write
+#endif
+                failed = 1;
+                continue;
+            }
+            const long h = head % H;
+            const long base = head * n * d;
+            for (long e = 0; e < n * d; ++e) {
+                float zq = load_elem(q, is_bf16, base + e) / sigma_q[h];
+                float zk = load_elem(k, is_bf16, base + e) / sigma_k[h];
+                sq[e] = (zq < 0.0f) ? (int8_t)-1 : (int8_t)1;
+                sk[e] = (zk < 0.0f) ? (int8_t)-1 : (int8_t)1;
+                dqb[e] = 0.0;
+                dkb[e] = 0.0;
+                dv[base + e] = 0.0;
+            }
+            for (long i = 0; i < n; ++i) {
+                /* the forward's kept set and weights */
+                row_logits(sq + i * d, sk, n, d, s);
+                for (long j = 0; j < n; ++j) {
+                    order[j].s = s[j];
+                    order[j].j = (int32_t)j;
+                }
+                qsort(order, (size_t)n, sizeof(keyed_t), by_logit_then_index);
+                qsort(order, (size_t)N, sizeof(keyed_t), by_index);
+                int32_t m = order[0].s;
+                for (long t = 1; t < N; ++t)
+                    if (order[t].s > m)
+                        m = order[t].s;
+                double Z = 0.0;
+                for (long t = 0; t < N; ++t) {
+                    p[t] = exp((double)tau * (double)(order[t].s - m));
+                    Z += p[t];
+                }
+                for (long t = 0; t < N; ++t)
+                    p[t] /= Z;
+                /* dp, D and ds */
+                const float *go = dout + base + i * d;
+                double D = 0.0;
+                for (long t = 0; t < N; ++t) {
+                    const long vj = base + (long)order[t].j * d;
+                    double dp = 0.0;
+                    for (long c = 0; c < d; ++c)
+                        dp += (double)go[c] * (double)load_elem(v, is_bf16, vj + c);
+                    ds[t] = dp;              /* dp for now */
+                    D += p[t] * dp;
+                }
+                for (long t = 0; t < N; ++t)
+                    ds[t] = (double)tau * p[t] * (ds[t] - D);
+                /* scatter to dV, dKb and gather dQb */
+                for (long t = 0; t < N; ++t) {
+                    const long j = order[t].j;
+                    for (long c = 0; c < d; ++c) {
+                        dv[base + j * d + c] += p[t] * (double)go[c];
+                        dkb[j * d + c] += ds[t] * (double)sq[i * d + c];
+                        dqb[i * d + c] += ds[t] * (double)sk[j * d + c];
+                    }
+                }
+            }
+            /* straight-through sign and the 1 / sigma of the standardization */
+            for (long e = 0; e < n * d; ++e) {
+                float zq = load_elem(q, is_bf16, base + e) / sigma_q[h];
+                float zk = load_elem(k, is_bf16, base + e) / sigma_k[h];
+                dq[base + e] = (fabsf(zq) <= clip) ? dqb[e] / (double)sigma_q[h] : 0.0;
+                dk[base + e] = (fabsf(zk) <= clip) ? dkb[e] / (double)sigma_k[h] : 0.0;
+            }
+        }
+        free(sq);
+        free(sk);
+        free(s);
+        free(order);
+        free(p);
+        free(ds);
+        free(dqb);
+        free(dkb);
+    }
+    return failed ? -1 : 0;
+}
+
 int had_oracle_max_threads(void)
 {
 #ifdef _OPENMP

@@ -542,3 +542,105 @@ def test_soft_N_equals_n_is_dense_softmax():
     assert (idx == np.arange(40)).all()
     assert np.allclose(p, w.numpy(), rtol=1e-12, atol=1e-15)
     assert np.allclose(out, ref, rtol=1e-6, atol=1e-6)
+
+
+# ------------------------------------------- straight-through backward
+
+
+def _bwd_case(shape, seed):
+    g = np.random.default_rng(seed)
+    q, k, v, dout = (g.standard_normal(shape).astype(np.float32) for _ in range(4))
+    sq = np.array([0.9, 1.3][:shape[1]], np.float32)
+    sk = np.array([1.1, 0.7][:shape[1]], np.float32)
+    return q, k, v, dout, sq, sk
+
+
+def _autograd_bwd(q, k, v, dout, sgq, sgk, tau, N, clip):
+    """The same gradients by torch autograd in float64: the sign replaced by
+    its straight-through surrogate, the forward oracle's kept set as a
+    fixed mask."""
+    B, H, n, d = q.shape
+    zq = q / sgq[None, :, None, None]                 # fp32, as the sign rule
+    zk = k / sgk[None, :, None, None]
+    idx = oracle.attention_rows(np.where(zq < 0, -1, 1).astype(np.int8),
+                                np.where(zk < 0, -1, 1).astype(np.int8), v, tau, N,
+                                np.arange(B * H * n))[0]
+    kept = torch.zeros(B * H * n, n, dtype=torch.bool)
+    kept[torch.arange(B * H * n)[:, None], torch.tensor(idx, dtype=torch.long)] = True
+    kept = kept.reshape(B, H, n, n)
+
+    def code(x, z, sg):
+        xt = torch.tensor(x, dtype=torch.float64, requires_grad=True)
+        zt = xt / torch.tensor(sg, dtype=torch.float64)[None, :, None, None]
+        m = torch.tensor(np.abs(z) <= clip, dtype=torch.float64)
+        sign = torch.tensor(np.where(z < 0, -1.0, 1.0))
+        return xt, sign + (zt * m - (zt * m).detach())
+
+    xq, bq = code(q, zq, sgq)
+    xk, bk = code(k, zk, sgk)
+    vt = torch.tensor(v, dtype=torch.float64, requires_grad=True)
+    s = (bq @ bk.transpose(-1, -2)).masked_fill(~kept, float("-inf"))
+    o = torch.softmax(tau * s, dim=-1) @ vt
+    (o * torch.tensor(dout, dtype=torch.float64)).sum().backward()
+    return xq.grad.numpy(), xk.grad.numpy(), vt.grad.numpy()
+
+
+@pytest.mark.parametrize("N,clip", [(7, 1.0), (40, 1.0), (5, float("inf")), (12, 0.4)])
+def test_bwd_matches_torch_autograd(N, clip):
+    q, k, v, dout, sgq, sgk = _bwd_case((1, 2, 40, 64), seed=180 + N)
+    tau = float(np.float32(0.3))
+    dq, dk, dv = oracle.attention_bwd(q, k, v, sgq, sgk, dout, tau, N, clip)
+    aq, ak, av = _autograd_bwd(q, k, v, dout, sgq, sgk, tau, N, clip)
+    assert np.allclose(dv, av, rtol=1e-10, atol=1e-12)
+    assert np.allclose(dq, aq, rtol=1e-9, atol=1e-12)
+    assert np.allclose(dk, ak, rtol=1e-9, atol=1e-12)
+    assert np.abs(dq).max() > 1e-3 and np.abs(dk).max() > 1e-3      # not trivially zero
+
+
+def test_bwd_dv_is_the_forward_difference_in_v():
+    # the forward is linear in V: O(V + e E) - O(V) = e P E exactly
+    q, k, v, dout, sgq, sgk = _bwd_case((1, 1, 30, 64), seed=190)
+    sq, sk = oracle.binarize(q, sgq), oracle.binarize(k, sgk)
+    _, _, dv = oracle.attention_bwd(q, k, v, sgq, sgk, dout, 0.25, 6)
+    rows = np.arange(30)
+    base = oracle.attention_rows(sq, sk, v, 0.25, 6, rows)[3].astype(np.float64)
+    for j, c in [(0, 0), (7, 13), (29, 63)]:
+        v2 = v.copy()
+        v2[0, 0, j, c] += np.float32(0.5)
+        o2 = oracle.attention_rows(sq, sk, v2, 0.25, 6, rows)[3].astype(np.float64)
+        fd = ((o2 - base) * dout[0, 0].astype(np.float64)).sum() / 0.5
+        assert abs(fd - dv[0, 0, j, c]) <= 1e-5 * max(1.0, abs(dv[0, 0, j, c]))
+
+
+def test_bwd_closed_forms_N1_and_tau0():
+    q, k, v, dout, sgq, sgk = _bwd_case((1, 2, 24, 64), seed=191)
+    sq, sk = oracle.binarize(q, sgq), oracle.binarize(k, sgk)
+    rows = np.arange(48)
+    # N = 1: p = 1, so ds = 0 and dV_j sums dO of the rows whose one key is j
+    dq, dk, dv = oracle.attention_bwd(q, k, v, sgq, sgk, dout, 0.3, 1)
+    assert not dq.any() and not dk.any()
+    idx = oracle.attention_rows(sq, sk, v, 0.3, 1, rows)[0][:, 0]
+    want = np.zeros_like(dv)
+    for r in rows:
+        want[0, r // 24, idx[r]] += dout[0, r // 24, r % 24]
+    assert np.allclose(dv, want, rtol=0, atol=1e-12)
+    # tau = 0: uniform weights 1/N, again ds = 0
+    dq, dk, dv = oracle.attention_bwd(q, k, v, sgq, sgk, dout, 0.0, 5)
+    assert not dq.any() and not dk.any()
+    idx = oracle.attention_rows(sq, sk, v, 0.0, 5, rows)[0]
+    want = np.zeros_like(dv)
+    for r in rows:
+        for j in idx[r]:
+            want[0, r // 24, j] += dout[0, r // 24, r % 24].astype(np.float64) / 5.0
+    assert np.allclose(dv, want, rtol=0, atol=1e-12)
+
+
+def test_bwd_clip_masks_exactly():
+    q, k, v, dout, sgq, sgk = _bwd_case((1, 2, 30, 64), seed=192)
+    a = oracle.attention_bwd(q, k, v, sgq, sgk, dout, 0.3, 8, clip=float("inf"))
+    b = oracle.attention_bwd(q, k, v, sgq, sgk, dout, 0.3, 8, clip=0.5)
+    zq = q / sgq[None, :, None, None]
+    zk = k / sgk[None, :, None, None]
+    assert np.array_equal(b[0], np.where(np.abs(zq) <= 0.5, a[0], 0.0))
+    assert np.array_equal(b[1], np.where(np.abs(zk) <= 0.5, a[1], 0.0))
+    assert np.array_equal(b[2], a[2])
