@@ -48,7 +48,8 @@ def parse():
                     help="target CPU time of the oracle baseline sample")
     ap.add_argument("--no-e2e", action="store_true")
     ap.add_argument("--no-cpu-baseline", action="store_true")
-    ap.add_argument("--mode", choices=["attention", "mass", "causal", "soft"], default="attention",
+    ap.add_argument("--mode", choices=["attention", "mass", "causal", "soft", "bwd"],
+                    default="attention",
                     help="mass: time the top-N mass-retention diagnostic instead")
     return ap.parse_args()
 
@@ -668,6 +669,90 @@ def run_soft(args, world, rank, local):
     }), flush=True)
 
 
+def run_bwd(args, world, rank, local):
+    """One step of the straight-through training stage on the workload: the
+    fused forward (keeping its kept set) and had_attention_bwd on that set.
+    Tokens per second of the pair; each half has its own events.  The
+    roofline is the backward's algorithmic HBM traffic: Q, K, V read, dO
+    read, dQ, dK, dV written, and the kept set (6 B per kept pair) read."""
+    from sparse_attention_sigma_b200 import had
+    cfg = synth.CONFIGS[args.config]
+    dev = torch.device("cuda", local)
+    torch.cuda.set_device(dev)
+    stream = torch.cuda.current_stream()
+    peaks = measured_peaks()
+    q, k, v, sgq, sgk = synth.make_inputs(cfg)
+    gq, gk, gv = q.to(dev), k.to(dev), v.to(dev)
+    gsq, gsk = sgq.to(dev), sgk.to(dev)
+    shape = (cfg.B, cfg.H, cfg.n)
+    dout = torch.randn(shape + (cfg.d,), generator=torch.Generator().manual_seed(5)).to(dev)
+    out = torch.empty(shape + (cfg.d,), dtype=torch.float32, device=dev)
+    idx = torch.empty(shape + (cfg.N,), dtype=torch.int32, device=dev)
+    lg = torch.empty(shape + (cfg.N,), dtype=torch.int16, device=dev)
+    grads = [torch.empty(shape + (cfg.d,), dtype=torch.float32, device=dev) for _ in range(3)]
+    fws = had.workspace(cfg.B, cfg.H, cfg.n, cfg.d, cfg.N, device=dev)
+    bws = torch.empty(had.had_workspace_bytes(had.HAD_OP_ATTENTION_BWD, cfg.B, cfg.H, cfg.n,
+                                              cfg.d, cfg.N), dtype=torch.uint8, device=dev)
+    flush = torch.empty(L2_FLUSH_BYTES // 4, dtype=torch.float32, device=dev)
+    launches = (had.had_launch_count(had.HAD_OP_ATTENTION_FWD, cfg.B, cfg.H, cfg.n, cfg.d, cfg.N)
+                + had.had_launch_count(had.HAD_OP_ATTENTION_BWD, cfg.B, cfg.H, cfg.n, cfg.d,
+                                       cfg.N) - 1)      # the kept set is given: no recompute
+
+    def fwd():
+        had.had_attention_fwd(gq, gk, gv, gsq, gsk, cfg.N, cfg.tau, out=out, dbg_idx=idx,
+                              dbg_logits=lg, ws=fws)
+
+    def bwd():
+        had.had_attention_bwd(gq, gk, gv, gsq, gsk, dout, cfg.N, cfg.tau, 1.0, idx=idx,
+                              logits=lg, dq=grads[0], dk=grads[1], dv=grads[2], ws=bws)
+
+    for _ in range(max(3, args.warmup)):
+        fwd()
+        bwd()
+    torch.cuda.synchronize()
+    clocks = ClockSampler(local)
+    clocks.start()
+    ev = [[torch.cuda.Event(enable_timing=True) for _ in range(3)] for _ in range(args.steps)]
+    barrier(world)
+    torch.cuda.synchronize()
+    for i in range(args.steps):
+        flush.fill_(float(i))
+        ev[i][0].record(stream)
+        fwd()
+        ev[i][1].record(stream)
+        bwd()
+        ev[i][2].record(stream)
+    torch.cuda.synchronize()
+    barrier(world)
+    clock_info = clocks.stop()
+    fwd_ms = sum(e[0].elapsed_time(e[1]) for e in ev) / args.steps
+    bwd_local = sum(e[1].elapsed_time(e[2]) for e in ev) / args.steps
+    value, ms = aggregate(cfg.tokens, fwd_ms + bwd_local, world, dev)
+    bwd_ms = max_over_ranks(bwd_local, world, dev)
+    elt = 2 if cfg.dtype == "bf16" else 4
+    elems = cfg.B * cfg.H * cfg.n * cfg.d
+    nbytes = elems * (3 * elt + 4 + 12) + cfg.B * cfg.H * cfg.n * cfg.N * 6
+    peak = peaks["hbm_gbs"]
+    if rank != 0:
+        return
+    print(json.dumps({
+        "metric": "HAD straight-through training step (forward + backward) tokens/sec",
+        "value": value, "unit": "tokens/s", "n_gpus": world, "steps": args.steps,
+        "warmup": max(3, args.warmup), "ms_per_step": ms, "higher_is_better": True,
+        "scaling": "weak", "vs_baseline": None, "dtype": cfg.dtype, "data": "synthetic",
+        "impl": "had_attention_fwd + had_attention_bwd",
+        "config": {"workload": cfg.describe(), "clip": 1.0,
+                   "l2": "flushed between steps (256 MiB write outside the timed events)"},
+        "stage_ms": {"forward": fwd_ms, "backward": bwd_ms},
+        "roofline": {"bound": "hbm", "achieved": nbytes / (bwd_ms * 1e-3) / 1e9, "peak": peak,
+                     "unit": "GB/s", "frac": nbytes / (bwd_ms * 1e-3) / 1e9 / peak,
+                     "kernel": "had_attention_bwd (7 launches)", "peaks": peaks["source"],
+                     "note": "algorithmic bytes: Q,K,V,dO read, dQ,dK,dV written, kept set read"},
+        "gpu_launches": launches * args.steps,
+        "clocks": clock_info,
+    }), flush=True)
+
+
 def main():
     args = parse()
     world, rank, local = dist_setup(args)
@@ -680,6 +765,8 @@ def main():
             run_causal(args, world, rank, local)
         elif args.mode == "soft":
             run_soft(args, world, rank, local)
+        elif args.mode == "bwd":
+            run_bwd(args, world, rank, local)
         else:
             run_had(args, world, rank, local)
     finally:

@@ -80,7 +80,8 @@ typedef enum {
     HAD_OP_SOFT_BINARIZE = 8,     /* had_soft_binarize */
     HAD_OP_SOFT_TOPN = 9,         /* had_soft_topn */
     HAD_OP_SOFT_SOFTMAX_AV = 10,  /* had_soft_softmax_av */
-    HAD_OP_SOFT_ATTENTION_FWD = 11 /* had_soft_attention_fwd */
+    HAD_OP_SOFT_ATTENTION_FWD = 11, /* had_soft_attention_fwd */
+    HAD_OP_ATTENTION_BWD = 12     /* had_attention_bwd */
 } had_op_t;
 
 /*
@@ -247,6 +248,35 @@ HAD_API had_status_t had_soft_attention_fwd(const void *Q, const void *K, const 
                                             int d, int N, float tau, float *out, void *ws,
                                             size_t ws_bytes, int32_t *dev_status,
                                             cudaStream_t stream);
+
+/*
+ * Backward pass of had_attention_fwd for the straight-through training stage
+ * ("Hamming Attention Distillation", pith.science review: a straight-through
+ * estimator finishes the binarization after the tanh stages).  The kept set
+ * is recomputed and held fixed; softmax and value product are
+ * differentiated exactly; the sign passes the gradient where
+ * |x / sigma| <= clip (clip = 1 is the usual choice, +inf passes it
+ * everywhere); the standardization contributes 1 / sigma and sigma gets no
+ * gradient.
+ *   Q, K, V, dt, sigma_q, sigma_k, N, tau   as had_attention_fwd
+ *   dout   [B,H,n,d] float (device): gradient of the loss w.r.t. the output
+ *   idx, logits  the forward's kept set ([B,H,n,N] int32 / int16, as
+ *          had_attention_fwd's debug outputs or had_hamming_topn give it),
+ *          or both NULL: then it is recomputed (one more launch)
+ *   clip   >= 0 (NaN rejected)
+ *   dq, dk, dv  [B,H,n,d] float out
+ *   ws     device workspace of had_workspace_bytes(HAD_OP_ATTENTION_BWD, ...)
+ *          bytes (about 4 + 26 N bytes per query row)
+ * The key-side sums (dk, dv) run over per-key lists that atomics fill, so
+ * their fp32 rounding is not reproducible bit for bit run to run.
+ */
+HAD_API had_status_t had_attention_bwd(const void *Q, const void *K, const void *V,
+                                       had_dtype_t dt, const float *sigma_q,
+                                       const float *sigma_k, const float *dout,
+                                       const int32_t *idx, const int16_t *logits, int B, int H,
+                                       int n, int d, int N, float tau, float clip, float *dq,
+                                       float *dk, float *dv, void *ws, size_t ws_bytes,
+                                       int32_t *dev_status, cudaStream_t stream);
 
 /*
  * Top-N mass retention diagnostic ("Hamming Attention Distillation",

@@ -15,6 +15,7 @@
 #include "had_fused.cuh"
 #include "had_mass.cuh"
 #include "had_soft.cuh"
+#include "had_bwd.cuh"
 
 namespace {
 
@@ -430,6 +431,81 @@ SoftWorkspace soft_layout(int B, int H, int n, int d, int N)
 
 bool finite_float(float x) { return x == x && x < 3.0e38f && x > -3.0e38f; }
 
+// Workspace of the straight-through backward: the forward's packed codes and
+// kept set, p and ds per kept pair, the per-key counts and offsets, and the
+// key-ordered lists.
+struct BwdWorkspace {
+    size_t qbits, kbits, idx, logits, P, DS, cnt, off, cursor, e_row, e_p, e_ds, total;
+};
+
+BwdWorkspace bwd_layout(int B, int H, int n, int d, int N)
+{
+    const size_t rows = (size_t)B * H * n, pairs = rows * (size_t)N;
+    BwdWorkspace w;
+    w.qbits = 0;
+    w.kbits = w.qbits + round_up(rows * (d / 8));
+    w.idx = w.kbits + round_up(rows * (d / 8));
+    w.logits = w.idx + round_up(pairs * 4);
+    w.P = w.logits + round_up(pairs * 2);
+    w.DS = w.P + round_up(pairs * 4);
+    w.cnt = w.DS + round_up(pairs * 4);
+    w.off = w.cnt + round_up(rows * 4);
+    w.cursor = w.off + round_up(rows * 8);
+    w.e_row = w.cursor + round_up(rows * 8);
+    w.e_p = w.e_row + round_up(pairs * 4);
+    w.e_ds = w.e_p + round_up(pairs * 4);
+    w.total = w.e_ds + round_up(pairs * 4);
+    return w;
+}
+
+template <typename T, int D>
+had_status_t launch_bwd_typed(const T *Q, const T *K, const T *V, const float *sq,
+                              const float *sk, const float *dout, const int32_t *kept_idx,
+                              const int16_t *kept_lg, int B, int H, int n, int N, float tau,
+                              float clip, float *dq, float *dk, float *dv,
+                              const BwdWorkspace &w, char *base, int32_t *status,
+                              cudaStream_t st)
+{
+    auto *qb = reinterpret_cast<uint32_t *>(base + w.qbits);
+    auto *kb = reinterpret_cast<uint32_t *>(base + w.kbits);
+    auto *idx = reinterpret_cast<int32_t *>(base + w.idx);
+    auto *lg = reinterpret_cast<int16_t *>(base + w.logits);
+    auto *P = reinterpret_cast<float *>(base + w.P);
+    auto *DS = reinterpret_cast<float *>(base + w.DS);
+    auto *cnt = reinterpret_cast<int32_t *>(base + w.cnt);
+    auto *off = reinterpret_cast<long long *>(base + w.off);
+    auto *cur = reinterpret_cast<long long *>(base + w.cursor);
+    auto *e_row = reinterpret_cast<int32_t *>(base + w.e_row);
+    auto *e_p = reinterpret_cast<float *>(base + w.e_p);
+    auto *e_ds = reinterpret_cast<float *>(base + w.e_ds);
+    const had_dtype_t dt = sizeof(T) == 2 ? HAD_BF16 : HAD_F32;
+    had_status_t s;
+    if ((s = launch_pack(Q, dt, sq, B, H, n, D, qb, status, st)) != HAD_OK) return s;
+    if ((s = launch_pack(K, dt, sk, B, H, n, D, kb, status, st)) != HAD_OK) return s;
+    if (kept_idx) {          // the forward's kept set, as given
+        idx = const_cast<int32_t *>(kept_idx);
+        lg = const_cast<int16_t *>(kept_lg);
+    } else if ((s = launch_topn(qb, kb, B, H, n, D, N, idx, lg, false, st)) != HAD_OK) {
+        return s;
+    }
+    const long long rows = (long long)B * H * n, pairs = rows * N;
+    const long long warp_blocks = (rows * 32 + 255) / 256;
+    if (warp_blocks > INT_MAX) return HAD_ERR_UNSUPPORTED;
+    had::bwd_rows_kernel<T, D><<<(unsigned)warp_blocks, 256, 0, st>>>(
+        idx, lg, V, dout, Q, sq, kb, H, n, N, tau, clip, rows, P, DS, dq, cnt, status);
+    if ((s = launched()) != HAD_OK) return s;
+    had::bwd_count_kernel<<<grid_for(pairs, 256), 256, 0, st>>>(idx, pairs, n, N, cnt);
+    if ((s = launched()) != HAD_OK) return s;
+    had::bwd_scan_kernel<<<(unsigned)(B * H), had::kScanThreads, 0, st>>>(cnt, n, N, off, cur);
+    if ((s = launched()) != HAD_OK) return s;
+    had::bwd_fill_kernel<<<grid_for(pairs, 256), 256, 0, st>>>(idx, P, DS, pairs, n, N, cur,
+                                                              e_row, e_p, e_ds);
+    if ((s = launched()) != HAD_OK) return s;
+    had::bwd_keys_kernel<T, D><<<(unsigned)warp_blocks, 256, 0, st>>>(
+        off, cnt, e_row, e_p, e_ds, dout, qb, K, sk, H, n, clip, rows, dk, dv);
+    return launched();
+}
+
 }  // namespace
 
 extern "C" {
@@ -721,6 +797,50 @@ had_status_t had_soft_attention_fwd(const void *Q, const void *K, const void *V,
     return launch_av(idx, lg, V, dt, B, H, n, d, N, tau, out, nullptr, dev_status, stream);
 }
 
+had_status_t had_attention_bwd(const void *Q, const void *K, const void *V, had_dtype_t dt,
+                               const float *sigma_q, const float *sigma_k, const float *dout,
+                               const int32_t *idx, const int16_t *logits, int B, int H, int n,
+                               int d, int N, float tau, float clip, float *dq, float *dk,
+                               float *dv, void *ws, size_t ws_bytes, int32_t *dev_status,
+                               cudaStream_t stream)
+{
+    had_status_t s = check_topn(B, H, n, d, N);
+    if (s != HAD_OK) return s;
+    if ((long long)B * H > INT_MAX) return HAD_ERR_UNSUPPORTED;
+    if (dt != HAD_BF16 && dt != HAD_F32) return HAD_ERR_INVALID_ARG;
+    if (!Q || !K || !V || !sigma_q || !sigma_k || !dout || !dq || !dk || !dv || !ws)
+        return HAD_ERR_INVALID_ARG;
+    if (!aligned16(Q) || !aligned16(K) || !aligned16(V) || !aligned16(dout) || !aligned16(dq) ||
+        !aligned16(dk) || !aligned16(dv) || !aligned16(ws))
+        return HAD_ERR_INVALID_ARG;
+    if (!finite_float(tau) || !(clip >= 0.0f)) return HAD_ERR_INVALID_ARG;
+    if ((idx == nullptr) != (logits == nullptr)) return HAD_ERR_INVALID_ARG;
+    if (idx && (!aligned16(idx) || !aligned16(logits))) return HAD_ERR_INVALID_ARG;
+    const BwdWorkspace w = bwd_layout(B, H, n, d, N);
+    if (ws_bytes < w.total) return HAD_ERR_WORKSPACE;
+    char *base = static_cast<char *>(ws);
+    if (dt == HAD_BF16) {
+        const auto *q = static_cast<const __nv_bfloat16 *>(Q);
+        const auto *k = static_cast<const __nv_bfloat16 *>(K);
+        const auto *v = static_cast<const __nv_bfloat16 *>(V);
+        return d == 64 ? launch_bwd_typed<__nv_bfloat16, 64>(q, k, v, sigma_q, sigma_k, dout, idx, logits, B,
+                                                              H, n, N, tau, clip, dq, dk, dv, w,
+                                                              base, dev_status, stream)
+                       : launch_bwd_typed<__nv_bfloat16, 128>(q, k, v, sigma_q, sigma_k, dout, idx, logits, B,
+                                                               H, n, N, tau, clip, dq, dk, dv, w,
+                                                               base, dev_status, stream);
+    }
+    const auto *q = static_cast<const float *>(Q);
+    const auto *k = static_cast<const float *>(K);
+    const auto *v = static_cast<const float *>(V);
+    return d == 64 ? launch_bwd_typed<float, 64>(q, k, v, sigma_q, sigma_k, dout, idx, logits, B, H, n, N,
+                                                 tau, clip, dq, dk, dv, w, base, dev_status,
+                                                 stream)
+                   : launch_bwd_typed<float, 128>(q, k, v, sigma_q, sigma_k, dout, idx, logits, B, H, n, N,
+                                                  tau, clip, dq, dk, dv, w, base, dev_status,
+                                                  stream);
+}
+
 size_t had_workspace_bytes(int op, int B, int H, int n, int d, int N)
 {
     switch (op) {
@@ -747,6 +867,9 @@ size_t had_workspace_bytes(int op, int B, int H, int n, int d, int N)
         return check_topn(B, H, n, d, N) == HAD_OK ? 0 : (size_t)-1;
     case HAD_OP_SOFT_ATTENTION_FWD:
         return check_soft(B, H, n, d, N) == HAD_OK ? soft_layout(B, H, n, d, N).total
+                                                   : (size_t)-1;
+    case HAD_OP_ATTENTION_BWD:
+        return check_topn(B, H, n, d, N) == HAD_OK ? bwd_layout(B, H, n, d, N).total
                                                    : (size_t)-1;
     default:
         return (size_t)-1;
@@ -779,6 +902,8 @@ int had_launch_count(int op, int B, int H, int n, int d, int N)
         return check_topn(B, H, n, d, N) == HAD_OK ? 1 : -1;
     case HAD_OP_SOFT_ATTENTION_FWD:
         return check_soft(B, H, n, d, N) == HAD_OK ? 3 + 2 * soft_passes(B, H, n) : -1;
+    case HAD_OP_ATTENTION_BWD:
+        return check_topn(B, H, n, d, N) == HAD_OK ? 8 : -1;
     default:
         return -1;
     }

@@ -39,6 +39,7 @@ HAD_OP_SOFT_BINARIZE = 8
 HAD_OP_SOFT_TOPN = 9
 HAD_OP_SOFT_SOFTMAX_AV = 10
 HAD_OP_SOFT_ATTENTION_FWD = 11
+HAD_OP_ATTENTION_BWD = 12
 
 
 class HadError(RuntimeError):
@@ -73,6 +74,8 @@ def _load():
         "had_soft_softmax_av": [vp, vp, vp, i32, i32, i32, i32, i32, i32, f32, vp, vp, vp, vp],
         "had_soft_attention_fwd": [vp, vp, vp, i32, vp, vp, f32, i32, i32, i32, i32, i32, f32,
                                    vp, vp, sz, vp, vp],
+        "had_attention_bwd": [vp, vp, vp, i32, vp, vp, vp, vp, vp, i32, i32, i32, i32, i32, f32,
+                              f32, vp, vp, vp, vp, sz, vp, vp],
     }
     for name, args in sig.items():
         fn = getattr(lib, name)
@@ -322,6 +325,45 @@ def had_soft_attention_fwd(Q, K, V, sigma_q, sigma_k, c, N, tau, out=None, ws=No
                                      _ptr(dev_status), _stream(stream))
     _check(st, "had_soft_attention_fwd")
     return out
+
+
+def had_attention_bwd(Q, K, V, sigma_q, sigma_k, dout, N, tau, clip=1.0, idx=None, logits=None,
+                      dq=None, dk=None, dv=None, ws=None, dev_status=None, stream=None):
+    """Straight-through backward of had_attention_fwd; returns (dq, dk, dv) float32.
+    idx/logits: the forward's kept set (e.g. had_attention_fwd's debug
+    outputs), or None to recompute it."""
+    _dev(Q, "Q")
+    B, H, n, d = _shape4(Q, "Q")
+    _dev(K, "K", Q.dtype, (B, H, n, d))
+    _dev(V, "V", Q.dtype, (B, H, n, d))
+    _dev(sigma_q, "sigma_q", torch.float32, (H,))
+    _dev(sigma_k, "sigma_k", torch.float32, (H,))
+    _dev(dout, "dout", torch.float32, (B, H, n, d))
+    if (idx is None) != (logits is None):
+        raise ValueError("give both idx and logits, or neither")
+    if idx is not None:
+        _dev(idx, "idx", torch.int32, (B, H, n, N))
+        _dev(logits, "logits", torch.int16, (B, H, n, N))
+    outs = []
+    for t, name in ((dq, "dq"), (dk, "dk"), (dv, "dv")):
+        if t is None:
+            t = torch.empty((B, H, n, d), dtype=torch.float32, device=Q.device)
+        _dev(t, name, torch.float32, (B, H, n, d))
+        outs.append(t)
+    need = had_workspace_bytes(HAD_OP_ATTENTION_BWD, B, H, n, d, N)
+    if need < 0:
+        raise HadError(HAD_ERR_UNSUPPORTED if d not in (64, 128) else HAD_ERR_INVALID_ARG,
+                       "had_attention_bwd")
+    if ws is None:
+        ws = torch.empty(need, dtype=torch.uint8, device=Q.device)
+    st = _lib.had_attention_bwd(_ptr(Q), _ptr(K), _ptr(V), _dtype_code(Q), _ptr(sigma_q),
+                                _ptr(sigma_k), _ptr(dout), _ptr(idx), _ptr(logits), B, H, n,
+                                d, N, ctypes.c_float(tau),
+                                ctypes.c_float(clip), _ptr(outs[0]), _ptr(outs[1]),
+                                _ptr(outs[2]), _ptr(ws), ws.numel(), _ptr(dev_status),
+                                _stream(stream))
+    _check(st, "had_attention_bwd")
+    return tuple(outs)
 
 
 def had_topn_mass(qbits, kbits, d, tau, p, nmin=None, dev_status=None, stream=None):

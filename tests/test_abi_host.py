@@ -172,3 +172,38 @@ def test_soft_argument_errors_return_before_any_cuda_call(lib):
     # ragged n: rows padded to a multiple of 4 floats
     assert lib.had_workspace_bytes(9, 1, 1, 130, 64, 5) >= 130 * 132 * 4
     assert lib.had_workspace_bytes(11, 1, 1, 130, 64, 5) >= 130 * (2 * 64 * 4 + 8 * 5) + 130 * 132 * 4
+
+
+def test_bwd_argument_errors_return_before_any_cuda_call(lib):
+    vp, i, sz, f = ctypes.c_void_p, ctypes.c_int, ctypes.c_size_t, ctypes.c_float
+    fake = vp(4096)        # never dereferenced: the checks fail first
+    b = lib.had_attention_bwd
+    b.argtypes = [vp, vp, vp, i, vp, vp, vp, vp, vp, i, i, i, i, i, f, f, vp, vp, vp, vp, sz,
+                  vp, vp]
+    b.restype = ctypes.c_int
+    ok = (fake, fake, fake, 0, fake, fake, fake, None, None, 1, 1, 8, 64, 2, 0.1, 1.0, fake,
+          fake, fake, fake, 1 << 30, None, None)
+
+    def call(**kw):
+        a = list(ok)
+        for pos, val in kw.items():
+            a[int(pos[1:])] = val
+        return b(*a)
+
+    assert call(a12=96) == 2                      # d
+    assert call(a13=9) == 1                       # N > n
+    assert call(a15=-1.0) == 1                    # clip < 0
+    assert call(a15=float("nan")) == 1            # clip NaN
+    assert call(a14=float("inf")) == 1            # tau
+    assert call(a6=None) == 1                     # no dout
+    assert call(a7=fake) == 1                     # idx without logits
+    assert call(a17=vp(4100)) == 1                # misaligned dk
+    assert call(a20=64) == 3                      # workspace
+    assert call(a15=float("inf"), a20=64) == 3    # clip = inf is allowed; fails on ws
+    assert call(a7=fake, a8=fake, a20=64) == 3    # a given kept set; fails on ws
+    lib.had_workspace_bytes.restype = ctypes.c_size_t
+    lib.had_workspace_bytes.argtypes = [ctypes.c_int] * 6
+    lib.had_launch_count.argtypes = [ctypes.c_int] * 6
+    # per query row: codes 16 B, per-key count and offsets 20 B, 26 B per kept pair
+    assert lib.had_workspace_bytes(12, 1, 1, 128, 64, 16) >= 128 * (16 + 20 + 26 * 16)
+    assert lib.had_launch_count(12, 4, 16, 4096, 64, 512) == 8

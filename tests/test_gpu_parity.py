@@ -537,3 +537,76 @@ def test_soft_long_workload_sampled(had):
     c = config_case("long")
     rows = synth.sample_rows(cfg, 192, seed=61)
     _check_soft(had, c.q, c.k, c.v, c.sgq, c.sgk, 1.0, cfg.N, cfg.tau, rows)
+
+
+# ------------------------------------------- straight-through backward
+
+
+def _bwd_inputs(B, H, n, d, seed, dtype=torch.bfloat16):
+    g = torch.Generator().manual_seed(seed)
+    q, k, v = (torch.randn(B, H, n, d, generator=g).to(dtype) for _ in range(3))
+    dout = torch.randn(B, H, n, d, generator=g)
+    return q, k, v, dout, synth.per_head_sigma(q), synth.per_head_sigma(k)
+
+
+def _check_bwd(had, q, k, v, dout, sgq, sgk, N, tau, clip, heads=None):
+    """GPU backward on the whole tensor; oracle on the listed (b, h) heads."""
+    dq, dk, dv = had.had_attention_bwd(q.cuda(), k.cuda(), v.cuda(), sgq.cuda(), sgk.cuda(),
+                                       dout.cuda(), N, tau, clip)
+    torch.cuda.synchronize()
+    B, H = q.shape[:2]
+    heads = heads if heads is not None else [(b, h) for b in range(B) for h in range(H)]
+    for b, h in heads:
+        sl = lambda t: t[b:b + 1, h:h + 1].contiguous()
+        oq, ok_, ov = oracle.attention_bwd(
+            synth.to_oracle_array(sl(q)), synth.to_oracle_array(sl(k)),
+            synth.to_oracle_array(sl(v)), sgq[h:h + 1].numpy(), sgk[h:h + 1].numpy(),
+            sl(dout).numpy(), tau, N, clip)
+        for got, want, name in ((dq, oq, "dq"), (dk, ok_, "dk"), (dv, ov, "dv")):
+            assert_close(got[b, h].cpu().numpy(), want[0, 0], f"{name} head {b},{h}")
+    return dq, dk, dv
+
+
+BWD_SMALL = [
+    # (B, H, n, d, N, seed, dtype, clip)
+    (1, 2, 300, 64, 40, 71, torch.bfloat16, 1.0),
+    (2, 1, 257, 128, 33, 72, torch.bfloat16, 1.0),
+    (1, 1, 1, 64, 1, 73, torch.bfloat16, 1.0),
+    (1, 2, 130, 64, 130, 74, torch.float32, float("inf")),   # N = n
+    (1, 3, 200, 64, 1, 75, torch.float32, 1.0),              # N = 1: dq = dk = 0
+    (1, 1, 700, 64, 90, 76, torch.bfloat16, 0.5),
+]
+
+
+@pytest.mark.parametrize("B,H,n,d,N,seed,dtype,clip", BWD_SMALL)
+def test_bwd_small_all_heads(had, B, H, n, d, N, seed, dtype, clip):
+    q, k, v, dout, sgq, sgk = _bwd_inputs(B, H, n, d, seed, dtype)
+    dq, dk, _ = _check_bwd(had, q, k, v, dout, sgq, sgk, N, 1 / math.sqrt(d), clip)
+    if N == 1:
+        assert not dq.any() and not dk.any()
+
+
+def test_bwd_with_the_forward_kept_set(had):
+    # the kept set from the fused forward's debug outputs gives the same dq
+    # (row gathers are deterministic) and the same dk, dv within rounding
+    q, k, v, dout, sgq, sgk = _bwd_inputs(1, 2, 520, 64, 78)
+    N, tau = 64, 0.125
+    g = [t.cuda() for t in (q, k, v, sgq, sgk)]
+    idx = torch.empty((1, 2, 520, N), dtype=torch.int32, device="cuda")
+    lg = torch.empty((1, 2, 520, N), dtype=torch.int16, device="cuda")
+    had.had_attention_fwd(*g, N, tau, dbg_idx=idx, dbg_logits=lg)
+    a = had.had_attention_bwd(*g, dout.cuda(), N, tau, idx=idx, logits=lg)
+    b = had.had_attention_bwd(*g, dout.cuda(), N, tau)
+    torch.cuda.synchronize()
+    assert torch.equal(a[0], b[0])
+    for x, y, name in zip(a[1:], b[1:], ("dk", "dv")):
+        assert_close(x.cpu().numpy(), y.cpu().numpy(), name)
+    _check_bwd(had, q, k, v, dout, sgq, sgk, N, tau, 1.0)
+
+
+def test_bwd_long_workload_two_heads(had):
+    cfg = synth.CONFIGS["long"]
+    c = config_case("long")
+    dout = torch.randn(c.q.shape, generator=torch.Generator().manual_seed(77))
+    _check_bwd(had, c.q, c.k, c.v, dout, c.sgq, c.sgk, cfg.N, cfg.tau, 1.0,
+               heads=[(0, 0), (cfg.B - 1, cfg.H - 1)])
