@@ -255,11 +255,13 @@ def run_reference(args, world, rank):
 
 
 def source_digest():
-    """sha256 of the fused kernel's sources (ties stored ncu counters to a build)."""
+    """sha256 of the fused path's sources: its kernels, the helpers they
+    include and its launch code (ties stored ncu counters to a build)."""
     import hashlib
     h = hashlib.sha256()
     csrc = os.path.join(ROOT, "sparse_attention_sigma_b200", "csrc")
-    for name in ("had_fused.cuh", "had_tc.cuh", "had_api.cu", "had_prep.cuh"):
+    for name in ("had_fused.cuh", "had_tc.cuh", "had_prep.cuh", "had_pack.cuh",
+                 "had_common.cuh", "had_fwd_launch.cuh"):
         with open(os.path.join(csrc, name), "rb") as f:
             h.update(f.read())
     return h.hexdigest()

@@ -5,48 +5,10 @@
 //
 // One warp per query row; the layout of the gather is described at the
 // kernel.  Accumulation is fp32; the result is divided by Z at the end.
-// VRow (a whole warp reading one V row, d/32 elements a lane) serves the
-// fused kernel's exact fix-up.
 #pragma once
 #include "had_common.cuh"
 
 namespace had {
-
-template <typename T, int PER>
-struct VRow;
-
-template <>
-struct VRow<__nv_bfloat16, 2> {
-    __device__ __forceinline__ static void load(const __nv_bfloat16 *p, float (&v)[2])
-    {
-        uint32_t u = __ldg(reinterpret_cast<const uint32_t *>(p));
-        v[0] = bf16_lo(u); v[1] = bf16_hi(u);
-    }
-};
-template <>
-struct VRow<__nv_bfloat16, 4> {
-    __device__ __forceinline__ static void load(const __nv_bfloat16 *p, float (&v)[4])
-    {
-        uint2 u = __ldg(reinterpret_cast<const uint2 *>(p));
-        v[0] = bf16_lo(u.x); v[1] = bf16_hi(u.x); v[2] = bf16_lo(u.y); v[3] = bf16_hi(u.y);
-    }
-};
-template <>
-struct VRow<float, 2> {
-    __device__ __forceinline__ static void load(const float *p, float (&v)[2])
-    {
-        float2 u = __ldg(reinterpret_cast<const float2 *>(p));
-        v[0] = u.x; v[1] = u.y;
-    }
-};
-template <>
-struct VRow<float, 4> {
-    __device__ __forceinline__ static void load(const float *p, float (&v)[4])
-    {
-        float4 u = __ldg(reinterpret_cast<const float4 *>(p));
-        v[0] = u.x; v[1] = u.y; v[2] = u.z; v[3] = u.w;
-    }
-};
 
 // Slice of one V row that a lane of an 8-lane group owns: d/8 consecutive
 // elements, loaded as 16-byte vectors and widened to fp32.

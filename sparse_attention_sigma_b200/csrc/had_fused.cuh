@@ -43,7 +43,6 @@
 #include <type_traits>
 
 #include "had_common.cuh"
-#include "had_av.cuh"
 #include "had_prep.cuh"
 #include "had_tc.cuh"
 
@@ -752,6 +751,43 @@ attention_fwd_kernel(const Params p)
 // miss counter (and its own done counter) for the next fused pass.
 constexpr int kFixSeg = 16384;
 constexpr int kFixList = 256;                     // kept keys a warp lists per round
+
+// A whole warp reads one V row, d/32 consecutive elements a lane.
+template <typename T, int PER>
+struct VRow;
+
+template <>
+struct VRow<__nv_bfloat16, 2> {
+    __device__ __forceinline__ static void load(const __nv_bfloat16 *p, float (&v)[2])
+    {
+        uint32_t u = __ldg(reinterpret_cast<const uint32_t *>(p));
+        v[0] = bf16_lo(u); v[1] = bf16_hi(u);
+    }
+};
+template <>
+struct VRow<__nv_bfloat16, 4> {
+    __device__ __forceinline__ static void load(const __nv_bfloat16 *p, float (&v)[4])
+    {
+        uint2 u = __ldg(reinterpret_cast<const uint2 *>(p));
+        v[0] = bf16_lo(u.x); v[1] = bf16_hi(u.x); v[2] = bf16_lo(u.y); v[3] = bf16_hi(u.y);
+    }
+};
+template <>
+struct VRow<float, 2> {
+    __device__ __forceinline__ static void load(const float *p, float (&v)[2])
+    {
+        float2 u = __ldg(reinterpret_cast<const float2 *>(p));
+        v[0] = u.x; v[1] = u.y;
+    }
+};
+template <>
+struct VRow<float, 4> {
+    __device__ __forceinline__ static void load(const float *p, float (&v)[4])
+    {
+        float4 u = __ldg(reinterpret_cast<const float4 *>(p));
+        v[0] = u.x; v[1] = u.y; v[2] = u.z; v[3] = u.w;
+    }
+};
 
 template <typename T, int D>
 __global__ void __launch_bounds__(256)

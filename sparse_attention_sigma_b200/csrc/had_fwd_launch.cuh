@@ -1,0 +1,156 @@
+// had_fwd_launch.cuh -- host side of the fused forward: the workspace
+// layout of had_attention_fwd / _prepare / _core and the launches of the
+// operand preparation, the fused kernel and its exact fix-up.  Kept apart
+// from the other entry points so that this file, with the kernels it
+// launches, is the whole of the fused path.
+#pragma once
+#include <climits>
+#include <cstddef>
+#include <cuda_runtime.h>
+
+#include "had.h"
+#include "had_common.cuh"
+#include "had_prep.cuh"
+#include "had_fused.cuh"
+
+namespace had {
+namespace fwdapi {
+
+inline size_t align256(size_t x) { return (x + 255) / 256 * 256; }
+
+inline had_status_t launch_status()
+{
+    return cudaGetLastError() == cudaSuccess ? HAD_OK : HAD_ERR_CUDA;
+}
+
+// Workspace of the fused forward: tensor-core operand tiles of Q, K and V^T
+// and the per-head V scale.
+struct FwdWorkspace {
+    size_t qop, qop2, kop, vop, qbits, kbits, vpart, miss, vexp, miss_rows, total;
+    int qtiles, ktiles, vchunks;
+};
+
+inline FwdWorkspace fwd_layout(int B, int H, int n, int d, int N)
+{
+    (void)N;
+    const size_t bh = (size_t)B * H;
+    FwdWorkspace w;
+    const int qt = d == 64 ? fused::Cfg<64>::QT : fused::Cfg<128>::QT;
+    w.qtiles = (n + fused::kRows - 1) / fused::kRows;
+    w.qtiles = (w.qtiles + qt - 1) / qt * qt;
+    w.ktiles = (n + fused::kKeys - 1) / fused::kKeys;
+    // V chunks of 8192 elements for the per-head maximum
+    w.vchunks = (int)(((size_t)n * d + 8191) / 8192);
+    w.qop = 0;
+    w.qop2 = w.qop + align256(bh * w.qtiles * fused::kRows * d);
+    w.kop = w.qop2 + align256(bh * w.qtiles * fused::kRows * d);
+    w.vop = w.kop + align256(bh * w.ktiles * fused::kKeys * d);
+    w.qbits = w.vop + align256(bh * w.ktiles * fused::kKeys * d * 2);
+    w.kbits = w.qbits + align256(bh * n * (d / 8));
+    w.vpart = w.kbits + align256(bh * n * (d / 8));
+    w.miss = w.vpart + align256(bh * w.vchunks * 4);
+    w.vexp = w.miss + align256(8);                      // miss counter, fix-up done counter
+    w.miss_rows = w.vexp + align256(bh * 4);
+    w.total = w.miss_rows + align256(bh * (size_t)w.qtiles * fused::kRows * 4);
+    return w;
+}
+
+// Operand preparation: Q/K signs as tensor-core tiles and packed bits and
+// the V chunk maxima in one launch, then V^T in fp16 with its per-head scale.
+template <typename T, int D>
+had_status_t prep_typed(const T *Q, const T *K, const T *V, const float *sq, const float *sk,
+                        int B, int H, int n, char *ws, const FwdWorkspace &w, int32_t *status,
+                        cudaStream_t st)
+{
+    const long long bh = (long long)B * H;
+    const long long blocks = bh * (w.qtiles + w.ktiles + w.vchunks);
+    if (blocks > INT_MAX || bh * w.ktiles > INT_MAX) return HAD_ERR_UNSUPPORTED;
+    auto *vpart = reinterpret_cast<float *>(ws + w.vpart);
+    // Q as +/-1 and +/-64, K as +/-4: the i8 MMA accumulates 4 s or 256 s
+    prep::operands_kernel<T, D><<<(unsigned)blocks, 256, 0, st>>>(
+        Q, K, V, sq, sk, H, n, (int)bh, w.qtiles, w.ktiles, w.vchunks,
+        reinterpret_cast<int8_t *>(ws + w.qop), reinterpret_cast<int8_t *>(ws + w.qop2),
+        reinterpret_cast<int8_t *>(ws + w.kop), reinterpret_cast<uint16_t *>(ws + w.qbits),
+        reinterpret_cast<uint16_t *>(ws + w.kbits), vpart, reinterpret_cast<int *>(ws + w.miss),
+        status);
+    prep::v_operand_kernel<T, D><<<(unsigned)(bh * w.ktiles), 256, 0, st>>>(
+        V, n, vpart, w.vchunks, reinterpret_cast<__half *>(ws + w.vop),
+        reinterpret_cast<int *>(ws + w.vexp));
+    return launch_status();
+}
+
+// The fused kernel on prepared operands, then the exact fix-up of the rows
+// whose threshold fell outside the sampled window.
+template <typename T, int D>
+had_status_t core_typed(const T *V, int B, int H, int n, int N, float tau, float *out,
+                        int32_t *dbg_idx, int16_t *dbg_lg, char *ws, const FwdWorkspace &w,
+                        int32_t *status, cudaStream_t st)
+{
+    using C = fused::Cfg<D>;
+    const long long bh = (long long)B * H;
+    const bool dbg = dbg_idx != nullptr || dbg_lg != nullptr;
+    auto kernel = dbg ? fused::attention_fwd_kernel<D, true>
+                      : fused::attention_fwd_kernel<D, false>;
+    // the CTA takes most of the unified L1 as shared memory
+    if (cudaFuncSetAttribute(kernel, cudaFuncAttributeMaxDynamicSharedMemorySize,
+                             C::SMEM_BYTES) != cudaSuccess ||
+        cudaFuncSetAttribute(kernel, cudaFuncAttributePreferredSharedMemoryCarveout,
+                             cudaSharedmemCarveoutMaxShared) != cudaSuccess)
+        return HAD_ERR_CUDA;
+    auto *qbits = reinterpret_cast<uint32_t *>(ws + w.qbits);
+    auto *kbits = reinterpret_cast<uint32_t *>(ws + w.kbits);
+    auto *miss_count = reinterpret_cast<int *>(ws + w.miss);
+    fused::Params p;
+    p.qop = reinterpret_cast<int8_t *>(ws + w.qop);
+    p.qop2 = reinterpret_cast<int8_t *>(ws + w.qop2);
+    p.kop = reinterpret_cast<int8_t *>(ws + w.kop);
+    p.vop = reinterpret_cast<__half *>(ws + w.vop);
+    p.vexp = reinterpret_cast<int *>(ws + w.vexp);
+    p.out = out;
+    p.dbg_idx = dbg_idx;
+    p.dbg_logits = dbg_lg;
+    p.status = status;
+    p.miss_count = miss_count;
+    p.miss_rows = reinterpret_cast<int *>(ws + w.miss_rows);
+    p.miss_cap = (long long)bh * w.qtiles * fused::kRows;
+    p.sample_tiles = w.ktiles / 16 > 4 ? w.ktiles / 16 : 4;
+    p.n = n;
+    p.N = N;
+    p.qtiles = w.qtiles;
+    p.ktiles = w.ktiles;
+    p.ctas_per_head = w.qtiles / C::QT;
+    p.c2 = tau * 1.4426950408889634f;
+    const long long blocks = bh * p.ctas_per_head;
+    kernel<<<(unsigned)blocks, C::THREADS, C::SMEM_BYTES, st>>>(p);
+    fused::fixup_rows_kernel<T, D><<<148 * 4, 256, 0, st>>>(
+        qbits, kbits, V, n, N, tau, miss_count, miss_count + 1, p.miss_rows, out, dbg_idx, dbg_lg);
+    return launch_status();
+}
+
+template <typename T, int D>
+had_status_t launch_fused_typed(const T *Q, const T *K, const T *V, const float *sq,
+                                const float *sk, int B, int H, int n, int N, float tau,
+                                float *out, int32_t *dbg_idx, int16_t *dbg_lg, char *ws,
+                                const FwdWorkspace &w, int32_t *status, cudaStream_t st)
+{
+    had_status_t s = prep_typed<T, D>(Q, K, V, sq, sk, B, H, n, ws, w, status, st);
+    if (s != HAD_OK) return s;
+    return core_typed<T, D>(V, B, H, n, N, tau, out, dbg_idx, dbg_lg, ws, w, status, st);
+}
+
+template <typename T>
+had_status_t launch_fused(const void *Q, const void *K, const void *V, const float *sq,
+                          const float *sk, int B, int H, int n, int d, int N, float tau,
+                          float *out, int32_t *dbg_idx, int16_t *dbg_lg, char *ws,
+                          const FwdWorkspace &w, int32_t *status, cudaStream_t st)
+{
+    const T *q = static_cast<const T *>(Q), *k = static_cast<const T *>(K),
+            *v = static_cast<const T *>(V);
+    return d == 64 ? launch_fused_typed<T, 64>(q, k, v, sq, sk, B, H, n, N, tau, out, dbg_idx,
+                                               dbg_lg, ws, w, status, st)
+                   : launch_fused_typed<T, 128>(q, k, v, sq, sk, B, H, n, N, tau, out, dbg_idx,
+                                                dbg_lg, ws, w, status, st);
+}
+
+}  // namespace fwdapi
+}  // namespace had
