@@ -513,15 +513,18 @@ def run_mass(args, world, rank, local):
 
 
 def run_causal(args, world, rank, local):
-    """The causal forward (had_attention_causal_fwd) on the workload: tokens per
-    second, issued as its three stages so that each has its own events.  The
-    dominant kernel is the causal top-N selection, bound by the popcount pipe:
-    d/32 popcounts per visible (query, key) pair, n (n + 1) / 2 pairs a head."""
+    """The causal forward: had_attention_causal_fwd (the fused tensor-core
+    path, each CTA streaming keys only up to its last row) timed as the
+    value, and the unfused composition (binarize, causal top-N, softmax-V)
+    timed stage by stage beside it.  Roofline as the non-causal call with the
+    causal work: n (n + 1) / 2 visible pairs a head, sum_i min(N, i + 1) kept
+    pairs."""
     from sparse_attention_sigma_b200 import had
     cfg = synth.CONFIGS[args.config]
     dev = torch.device("cuda", local)
     torch.cuda.set_device(dev)
     stream = torch.cuda.current_stream()
+    peaks = measured_peaks()
     q, k, v, sgq, sgk = synth.make_inputs(cfg)
     gq, gk, gv = q.to(dev), k.to(dev), v.to(dev)
     gsq, gsk = sgq.to(dev), sgk.to(dev)
@@ -531,7 +534,15 @@ def run_causal(args, world, rank, local):
     idx = torch.empty(shape + (cfg.N,), dtype=torch.int32, device=dev)
     lg = torch.empty(shape + (cfg.N,), dtype=torch.int16, device=dev)
     out = torch.empty(shape + (cfg.d,), dtype=torch.float32, device=dev)
+    out_u = torch.empty_like(out)
+    ws = torch.empty(had.had_workspace_bytes(had.HAD_OP_ATTENTION_CAUSAL, cfg.B, cfg.H, cfg.n,
+                                             cfg.d, cfg.N), dtype=torch.uint8, device=dev)
     flush = torch.empty(L2_FLUSH_BYTES // 4, dtype=torch.float32, device=dev)
+    launches = had.had_launch_count(had.HAD_OP_ATTENTION_CAUSAL, cfg.B, cfg.H, cfg.n, cfg.d,
+                                    cfg.N)
+
+    def fused():
+        had.had_attention_causal_fwd(gq, gk, gv, gsq, gsk, cfg.N, cfg.tau, out=out, ws=ws)
 
     def stages():
         had.had_binarize_pack(gq, gsq, bits=qb)
@@ -539,52 +550,73 @@ def run_causal(args, world, rank, local):
         yield
         had.had_hamming_topn_causal(qb, kb, cfg.d, cfg.N, idx=idx, logits=lg)
         yield
-        had.had_sparse_softmax_av(idx, lg, gv, cfg.tau, out=out)
+        had.had_sparse_softmax_av(idx, lg, gv, cfg.tau, out=out_u)
         yield
 
     for _ in range(max(3, args.warmup)):
+        fused()
         for _ in stages():
             pass
-    # the one-call entry point computes the same thing
-    ref = had.had_attention_causal_fwd(gq, gk, gv, gsq, gsk, cfg.N, cfg.tau)
     torch.cuda.synchronize()
-    if not torch.equal(ref, out):
-        raise RuntimeError("had_attention_causal_fwd differs from its three stages")
     clocks = ClockSampler(local)
     clocks.start()
-    ev = [[torch.cuda.Event(enable_timing=True) for _ in range(4)] for _ in range(args.steps)]
+    t_end = time.time() + 1.0                   # clocks settle under load first
+    while time.time() < t_end:
+        for _ in range(10):
+            fused()
+        torch.cuda.synchronize()
+    ev = [[torch.cuda.Event(enable_timing=True) for _ in range(2)] for _ in range(args.steps)]
     barrier(world)
     torch.cuda.synchronize()
     for i in range(args.steps):
         flush.fill_(float(i))
         ev[i][0].record(stream)
-        for j, _ in enumerate(stages()):
-            ev[i][j + 1].record(stream)
+        fused()
+        ev[i][1].record(stream)
     torch.cuda.synchronize()
     barrier(world)
     clock_info = clocks.stop()
-    stage_ms = [sum(e[j].elapsed_time(e[j + 1]) for e in ev) / args.steps for j in range(3)]
-    value, ms = aggregate(cfg.tokens, sum(stage_ms), world, dev)
-    topn_ms = max_over_ranks(stage_ms[1], world, dev)
-    popc = cfg.B * cfg.H * cfg.n * (cfg.n + 1) // 2 * (cfg.d // 32)
-    peak = SM_COUNT * 16 * 1.965e9
+    fused_local = sum(e[0].elapsed_time(e[1]) for e in ev) / args.steps
+    value, ms = aggregate(cfg.tokens, fused_local, world, dev)
+
+    usteps = max(1, min(args.steps, 5))
+    uev = [[torch.cuda.Event(enable_timing=True) for _ in range(4)] for _ in range(usteps)]
+    for i in range(usteps):
+        flush.fill_(float(i))
+        uev[i][0].record(stream)
+        for j, _ in enumerate(stages()):
+            uev[i][j + 1].record(stream)
+    torch.cuda.synchronize()
+    stage_ms = [sum(e[j].elapsed_time(e[j + 1]) for e in uev) / usteps for j in range(3)]
+
+    B, H, n, d, N = cfg.B, cfg.H, cfg.n, cfg.d, cfg.N
+    pairs = B * H * n * (n + 1) / 2
+    kept = B * H * (min(N, n) * (min(N, n) + 1) / 2 + max(n - N, 0) * N)
+    bf16 = peaks["bf16_tflops"] * 1e12
+    elt = 2 if cfg.dtype == "bf16" else 4
+    t_hbm = (3.0 * B * H * n * d * elt + B * H * n * d * 4) / (peaks["hbm_gbs"] * 1e9)
+    t_tc = 2.0 * pairs * d / (2 * bf16) + 2.0 * kept * d / bf16
+    t_alu = pairs / (SM_COUNT * 128 * peaks["sm_max_mhz"] * 1e6)
+    t_roof = max(t_hbm, t_tc, t_alu)
+    work = 2.0 * pairs * d + 2.0 * kept * d
     if rank != 0:
         return
     print(json.dumps({
         "metric": "HAD causal attention tokens/sec", "value": value, "unit": "tokens/s",
         "n_gpus": world, "steps": args.steps, "warmup": max(3, args.warmup), "ms_per_step": ms,
-        "higher_is_better": True, "scaling": "weak", "vs_baseline": None, "dtype": "bf16",
-        "data": "synthetic", "impl": "had_attention_causal_fwd",
+        "higher_is_better": True, "scaling": "weak", "vs_baseline": None, "dtype": cfg.dtype,
+        "data": "synthetic", "impl": "had_attention_causal_fwd (fused)",
         "config": {"workload": cfg.describe(), "causal": True,
                    "l2": "flushed between steps (256 MiB write outside the timed events)"},
-        "stage_ms": {"binarize_pack": stage_ms[0], "hamming_topn_causal": stage_ms[1],
-                     "sparse_softmax_av": stage_ms[2]},
-        "roofline": {"bound": "alu", "achieved": popc / (topn_ms * 1e-3) / 1e12,
-                     "peak": peak / 1e12, "unit": "Tpopc/s", "frac": popc / (topn_ms * 1e-3) / peak,
-                     "kernel": "topn_simt_kernel (causal)",
-                     "note": "popcount pipe, 16/clk/SM at 1.965 GHz; one popcount per 32 bits "
-                             "of each visible (query, key) pair"},
-        "gpu_launches": 4 * args.steps,
+        "unfused_stage_ms": {"binarize_pack": stage_ms[0], "hamming_topn_causal": stage_ms[1],
+                             "sparse_softmax_av": stage_ms[2]},
+        "roofline": {"bound": "tensor", "achieved": work / (ms * 1e-3) / 1e12,
+                     "peak": work / t_roof / 1e12, "unit": "TFLOP/s",
+                     "frac": t_roof / (ms * 1e-3), "traffic": None,
+                     "kernel": "whole call: prep + attention_fwd_kernel<causal> + fix-up",
+                     "t_roof_us": t_roof * 1e6, "t_hbm_us": t_hbm * 1e6, "t_tc_us": t_tc * 1e6,
+                     "t_alu_us": t_alu * 1e6, "peaks": peaks["source"]},
+        "gpu_launches": launches * args.steps,
         "clocks": clock_info,
     }), flush=True)
 

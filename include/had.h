@@ -182,18 +182,21 @@ HAD_API had_status_t had_hamming_topn_causal(const uint32_t *qbits, const uint32
                                              cudaStream_t stream);
 
 /*
- * Causal forward in one call: had_binarize_pack of Q and K, then
- * had_hamming_topn_causal, then had_sparse_softmax_av, inside a caller
- * workspace of had_workspace_bytes(HAD_OP_ATTENTION_CAUSAL, ...) bytes
- * (packed bits and the kept set: about B*H*n*(d/4 + 6 N) bytes).  Arguments
- * otherwise as had_attention_fwd (no debug outputs).
+ * Causal forward in one call, on the fused tensor-core path of
+ * had_attention_fwd: query i sees keys 0 .. i and keeps min(N, i + 1) of
+ * them (the rule of had_hamming_topn_causal).  Each CTA streams keys only up
+ * to its last query row, so the call does about half the work of the
+ * non-causal one.  Arguments, workspace (had_workspace_bytes(
+ * HAD_OP_ATTENTION_CAUSAL, ...) = that of HAD_OP_ATTENTION_FWD), launch
+ * count and errors as had_attention_fwd; dbg_idx / dbg_logits, when given,
+ * hold the kept set with empty slots as idx -1, logit 0.
  */
 HAD_API had_status_t had_attention_causal_fwd(const void *Q, const void *K, const void *V,
                                               had_dtype_t dt, const float *sigma_q,
                                               const float *sigma_k, int B, int H, int n, int d,
-                                              int N, float tau, float *out, void *ws,
-                                              size_t ws_bytes, int32_t *dev_status,
-                                              cudaStream_t stream);
+                                              int N, float tau, float *out, int32_t *dbg_idx,
+                                              int16_t *dbg_logits, void *ws, size_t ws_bytes,
+                                              int32_t *dev_status, cudaStream_t stream);
 
 /*
  * Soft codes for the tanh training stages ("Hamming Attention

@@ -104,23 +104,6 @@ had_status_t launch_topn(const uint32_t *qb, const uint32_t *kb, int B, int H, i
                    : launch_topn_dw<4, false>(qb, kb, B, H, n, N, idx, lg, st);
 }
 
-// Workspace of the causal forward: packed Q and K bits, then the kept set.
-struct CausalWorkspace {
-    size_t qbits, kbits, idx, logits, total;
-};
-
-CausalWorkspace causal_layout(int B, int H, int n, int d, int N)
-{
-    const size_t rows = (size_t)B * H * n;
-    CausalWorkspace w;
-    w.qbits = 0;
-    w.kbits = w.qbits + round_up(rows * (d / 8));
-    w.idx = w.kbits + round_up(rows * (d / 8));
-    w.logits = w.idx + round_up(rows * (size_t)N * 4);
-    w.total = w.logits + round_up(rows * (size_t)N * 2);
-    return w;
-}
-
 template <typename L>
 had_status_t launch_av(const int32_t *idx, const L *lg, const void *V, had_dtype_t dt,
                        int B, int H, int n, int d, int N, float tau, float *out, float *p,
@@ -430,27 +413,27 @@ had_status_t had_hamming_topn_causal(const uint32_t *qbits, const uint32_t *kbit
 had_status_t had_attention_causal_fwd(const void *Q, const void *K, const void *V,
                                       had_dtype_t dt, const float *sigma_q, const float *sigma_k,
                                       int B, int H, int n, int d, int N, float tau, float *out,
-                                      void *ws, size_t ws_bytes, int32_t *dev_status,
-                                      cudaStream_t stream)
+                                      int32_t *dbg_idx, int16_t *dbg_logits, void *ws,
+                                      size_t ws_bytes, int32_t *dev_status, cudaStream_t stream)
 {
     had_status_t s = check_topn(B, H, n, d, N);
     if (s != HAD_OK) return s;
     if (dt != HAD_BF16 && dt != HAD_F32) return HAD_ERR_INVALID_ARG;
-    if (!Q || !K || !V || !sigma_q || !sigma_k || !out || !ws) return HAD_ERR_INVALID_ARG;
-    if (!aligned16(Q) || !aligned16(K) || !aligned16(V) || !aligned16(out) || !aligned16(ws))
+    if (!Q || !K || !V || !sigma_q || !sigma_k || !out) return HAD_ERR_INVALID_ARG;
+    if (!aligned16(Q) || !aligned16(K) || !aligned16(V) || !aligned16(out) ||
+        (dbg_idx && !aligned16(dbg_idx)) || (dbg_logits && !aligned16(dbg_logits)))
         return HAD_ERR_INVALID_ARG;
-    if (!(tau == tau) || tau > 3.0e38f || tau < -3.0e38f) return HAD_ERR_INVALID_ARG;
-    const CausalWorkspace w = causal_layout(B, H, n, d, N);
-    if (ws_bytes < w.total) return HAD_ERR_WORKSPACE;
+    if (!(tau >= 0.0f) || tau > 3.0e38f) return HAD_ERR_INVALID_ARG;
+    const FwdWorkspace w = fwd_layout(B, H, n, d, N);
+    if (!ws || ws_bytes < w.total || !aligned16(ws)) return HAD_ERR_WORKSPACE;
+    if ((long long)B * H * w.qtiles > INT_MAX) return HAD_ERR_UNSUPPORTED;
     char *base = static_cast<char *>(ws);
-    auto *qb = reinterpret_cast<uint32_t *>(base + w.qbits);
-    auto *kb = reinterpret_cast<uint32_t *>(base + w.kbits);
-    auto *idx = reinterpret_cast<int32_t *>(base + w.idx);
-    auto *lg = reinterpret_cast<int16_t *>(base + w.logits);
-    if ((s = launch_pack(Q, dt, sigma_q, B, H, n, d, qb, dev_status, stream)) != HAD_OK) return s;
-    if ((s = launch_pack(K, dt, sigma_k, B, H, n, d, kb, dev_status, stream)) != HAD_OK) return s;
-    if ((s = launch_topn(qb, kb, B, H, n, d, N, idx, lg, true, stream)) != HAD_OK) return s;
-    return launch_av(idx, lg, V, dt, B, H, n, d, N, tau, out, nullptr, dev_status, stream);
+    if (dt == HAD_BF16)
+        return launch_fused<__nv_bfloat16>(Q, K, V, sigma_q, sigma_k, B, H, n, d, N, tau, out,
+                                           dbg_idx, dbg_logits, base, w, dev_status, stream,
+                                           true);
+    return launch_fused<float>(Q, K, V, sigma_q, sigma_k, B, H, n, d, N, tau, out, dbg_idx,
+                               dbg_logits, base, w, dev_status, stream, true);
 }
 
 had_status_t had_sparse_softmax_av(const int32_t *idx, const int16_t *logits, const void *V,
@@ -733,7 +716,7 @@ size_t had_workspace_bytes(int op, int B, int H, int n, int d, int N)
     case HAD_OP_TOPN_MASS:
         return check_shape(B, H, n, d) == HAD_OK ? 0 : (size_t)-1;
     case HAD_OP_ATTENTION_CAUSAL:
-        return check_topn(B, H, n, d, N) == HAD_OK ? causal_layout(B, H, n, d, N).total
+        return check_topn(B, H, n, d, N) == HAD_OK ? fwd_layout(B, H, n, d, N).total
                                                    : (size_t)-1;
     case HAD_OP_SOFT_BINARIZE:
         return check_shape(B, H, n, d) == HAD_OK ? 0 : (size_t)-1;

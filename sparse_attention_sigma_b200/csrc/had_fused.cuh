@@ -193,7 +193,7 @@ __device__ __forceinline__ uint32_t window_inc(int amount)
     return r;
 }
 
-template <int D, bool kDbg>
+template <int D, bool kDbg, bool kCausal = false>
 __global__ void __launch_bounds__(Cfg<D>::THREADS, 1)
 attention_fwd_kernel(const Params p)
 {
@@ -216,8 +216,13 @@ attention_fwd_kernel(const Params p)
     const int warp = threadIdx.x >> 5;
     const int lane = threadIdx.x & 31;
     const long long head = blockIdx.x / p.ctas_per_head;
-    const int qtile0 = (blockIdx.x % p.ctas_per_head) * QT;
-    const int T = p.ktiles;
+    // Causal: the CTAs of a head run from its last query tiles (the most
+    // keys) to its first, and each streams keys only up to its last row.
+    // Every role derives T from blockIdx alone, so all agree on it.
+    const int cta_in_head = blockIdx.x % p.ctas_per_head;
+    const int qtile0 = (kCausal ? p.ctas_per_head - 1 - cta_in_head : cta_in_head) * QT;
+    const int T = kCausal ? min(p.ktiles, ((qtile0 + QT) * kRows + kKeys - 1) / kKeys)
+                          : p.ktiles;
     const uint64_t deadline = tc::globaltimer_ns() + kWaitNs;
 
     if (threadIdx.x == 0) {
@@ -252,9 +257,9 @@ attention_fwd_kernel(const Params p)
         // ------------------------------------------------------------ producer
         if (lane == 0) {
             const int8_t *qsrc = p.qop + (head * p.qtiles + qtile0) * (long long)C::QBYTES;
-            const int8_t *ksrc = p.kop + head * (long long)T * C::KBYTES;
+            const int8_t *ksrc = p.kop + head * (long long)p.ktiles * C::KBYTES;
             const uint8_t *vsrc = reinterpret_cast<const uint8_t *>(p.vop) +
-                                  head * (long long)T * C::VBYTES;
+                                  head * (long long)p.ktiles * C::VBYTES;
             const int8_t *qsrc2 = p.qop2 + (head * p.qtiles + qtile0) * (long long)C::QBYTES;
             tc::mbar_expect_tx(b.q_full, 2 * QT * C::QBYTES);
             tc::bulk_g2s(smem + C::OFF_Q, qsrc, QT * C::QBYTES, b.q_full);
@@ -402,6 +407,10 @@ attention_fwd_kernel(const Params p)
         const int r = quarter * 32 + lane;            // row within the tile
         const int row = (qtile0 + g) * kRows + r;     // query index within the head
         const bool active = row < p.n;
+        // keys this row sees and keeps: all n and N, or (causal) keys 0..row
+        // and min(N, row + 1)
+        const int vis = kCausal ? min(p.n, row + 1) : p.n;
+        const int Nr = min(p.N, vis);
         const uint32_t lane_base = tmem + ((uint32_t)(quarter * 32) << 16) + g * C::GROUP_COLS;
         uint32_t *hist = reinterpret_cast<uint32_t *>(smem + C::OFF_HIST + g * C::HIST_BYTES);
         uint32_t *hcol = hist + r;                    // hist[bin][r] at hcol[bin * kRows]
@@ -439,7 +448,7 @@ attention_fwd_kernel(const Params p)
             __syncwarp();
             if (lane == 0) tc::mbar_arrive(b.s_empty(g, u % C::SBUF));
         };
-        auto half_valid = [&](int j, int h) { return min(32, p.n - j * kKeys - h * 32); };
+        auto half_valid = [&](int j, int h) { return min(32, vis - j * kKeys - h * 32); };
 
         // pass 1a: exact histogram of the first A key tiles
         auto hist_half = [&](const uint32_t (&rr)[32], auto full, int valid) {
@@ -471,8 +480,8 @@ attention_fwd_kernel(const Params p)
         // resolved exactly; the rest of the row updates four cumulative
         // counters f_k = #{level <= L0 - 1 + k}, k = 0..3.
         auto place_window = [&]() {
-            const int sampled = min(p.n, A * kKeys);
-            const int ns = max(1, (int)(((long long)p.N * sampled + p.n / 2) / p.n));
+            const int sampled = min(vis, A * kKeys);
+            const int ns = max(1, (int)(((long long)Nr * sampled + vis / 2) / vis));
             int cum = 0, est = C::BINS - 1;
             bool seen = false, found = false;
             for (int bin = 0; bin < C::BINS; ++bin) {
@@ -493,6 +502,9 @@ attention_fwd_kernel(const Params p)
                 if (valid >= 32) window_half(rr, BT{}, 32);
                 else window_half(rr, BF{}, valid);
             }
+            // causal: valid differs from lane to lane, so the lanes meet
+            // again before the next warp-wide TMEM access
+            if constexpr (kCausal) __syncwarp();
         };
         auto pass1_end_tile = [&](int j) {
             if (j == A - 1) place_window();
@@ -532,7 +544,7 @@ attention_fwd_kernel(const Params p)
             int below = 0;
             for (int bin = 0; bin < C::BINS; ++bin) {
                 const int c = (int)hcol[bin * kRows];
-                if (below + c >= p.N) { t = bin; quota = p.N - below; break; }
+                if (below + c >= Nr) { t = bin; quota = Nr - below; break; }
                 below += c;
             }
         } else {
@@ -544,10 +556,10 @@ attention_fwd_kernel(const Params p)
                 if (bin <= L0 + 1) f2 += c;
                 if (bin <= L0 + 2) f3 += c;
             }
-            if (f0 < p.N && f3 >= p.N) {
-                if (f1 >= p.N) { t = L0; quota = p.N - f0; }
-                else if (f2 >= p.N) { t = L0 + 1; quota = p.N - f1; }
-                else { t = L0 + 2; quota = p.N - f2; }
+            if (f0 < Nr && f3 >= Nr) {
+                if (f1 >= Nr) { t = L0; quota = Nr - f0; }
+                else if (f2 >= Nr) { t = L0 + 1; quota = Nr - f1; }
+                else { t = L0 + 2; quota = Nr - f2; }
             } else {
                 miss = true;
             }
@@ -558,6 +570,7 @@ attention_fwd_kernel(const Params p)
         // (the lowest indices) inside it, and none after it: from tile
         // zero_at on the weight table maps level t to 0.
         int zero_at = T, jstar = -1, kstar = 0;
+        __syncwarp();                                 // lanes left the threshold loops apart
         if (stash_ok && ok && A < T) {
             tc::tmem_wait_st();
             const bool want = t >= 0 && !miss;
@@ -665,6 +678,7 @@ attention_fwd_kernel(const Params p)
                 if (valid >= 32) slow_half(j * kKeys + h * 32, rr, pk, rl, BT{}, 32);
                 else slow_half(j * kKeys + h * 32, rr, pk, rl, BF{}, valid);
             }
+            if constexpr (kCausal) __syncwarp();      // slow differs from lane to lane
         };
         if (ok) ok = wait_s(T);
         if (ok) {
@@ -674,8 +688,15 @@ attention_fwd_kernel(const Params p)
         for (int j = 0; j < T && ok; ++j) {
             const int u = T + j;
             if (j == zero_at) hcol[t * kRows] = 0u;  // ties past the quota weigh nothing now
-            const bool slow = j < fast_from || half_valid(j, 1) < 32 ||
-                              __any_sync(kFullMask, j == jstar);
+            bool slow;
+            if constexpr (kCausal) {
+                // half_valid depends on the lane's row: the vote must not sit
+                // behind a short-circuit that some lanes take
+                const bool hit = __any_sync(kFullMask, j == jstar);
+                slow = j < fast_from || half_valid(j, 1) < 32 || hit;
+            } else {
+                slow = j < fast_from || half_valid(j, 1) < 32 || __any_sync(kFullMask, j == jstar);
+            }
             int rl = j < fast_from ? rem : (j == jstar ? kstar : kAll);
             uint32_t pk[16];
             const uint32_t pcol = lane_base + C::S_COL + (u % C::SBUF) * 64;   // P over S
@@ -699,6 +720,12 @@ attention_fwd_kernel(const Params p)
         }
         float Z = (zacc[0] + zacc[1]) + (zacc[2] + zacc[3]);
         if (!(Z > 0.0f)) Z = 1.0f;                    // missed or inactive rows only
+        // causal rows that see fewer than N keys: the unused slots are empty
+        if (kDbg && kCausal && active && !miss)
+            for (int k = kept; k < p.N; ++k) {
+                if (p.dbg_idx) p.dbg_idx[obase + k] = -1;
+                if (p.dbg_logits) p.dbg_logits[obase + k] = 0;
+            }
 
         // output: O / Z * 2^e_h
         if (ok) ok = __all_sync(kFullMask, wait_bar(b.o_full(g), 0, deadline, abort_flag, p.status));
@@ -789,7 +816,7 @@ struct VRow<float, 4> {
     }
 };
 
-template <typename T, int D>
+template <typename T, int D, bool kCausal = false>
 __global__ void __launch_bounds__(256)
 fixup_rows_kernel(const uint32_t *__restrict__ qbits, const uint32_t *__restrict__ kbits,
                   const T *__restrict__ V, int n, int N, float tau,
@@ -812,6 +839,9 @@ fixup_rows_kernel(const uint32_t *__restrict__ qbits, const uint32_t *__restrict
     for (int m = blockIdx.x; m < count; m += gridDim.x) {
         const int r = miss_rows[m];
         const long long head = r / n;
+        // keys the row sees and keeps (causal: keys 0 .. its position)
+        const int nv = kCausal ? (int)(r - head * n) + 1 : n;
+        const int Nr = min(N, nv);
         uint32_t q[DW];
 #pragma unroll
         for (int w = 0; w < DW; ++w) q[w] = qbits[(long long)r * DW + w];
@@ -839,8 +869,8 @@ fixup_rows_kernel(const uint32_t *__restrict__ qbits, const uint32_t *__restrict
         };
         for (int b = threadIdx.x; b < BINS; b += blockDim.x) hist[b] = 0;
         __syncthreads();
-        for (int s0 = 0; s0 < n; s0 += kFixSeg) {
-            const int s1 = min(n, s0 + kFixSeg);
+        for (int s0 = 0; s0 < nv; s0 += kFixSeg) {
+            const int s1 = min(nv, s0 + kFixSeg);
             fill(s0, s1);
             __syncthreads();
             for (int j = threadIdx.x; j < s1 - s0; j += blockDim.x) atomicAdd(&hist[dist[j]], 1);
@@ -853,7 +883,7 @@ fixup_rows_kernel(const uint32_t *__restrict__ qbits, const uint32_t *__restrict
                 const int c = hist[b];
                 if (!seen && c) { hmin = b; seen = true; }
                 if (!found) {
-                    if (below + c >= N) { t = b; quota = N - below; found = true; }
+                    if (below + c >= Nr) { t = b; quota = Nr - below; found = true; }
                     else below += c;
                 }
             }
@@ -867,9 +897,9 @@ fixup_rows_kernel(const uint32_t *__restrict__ qbits, const uint32_t *__restrict
         for (int e = 0; e < PER; ++e) acc[e] = 0.0f;
         float z = 0.0f;
         const T *vh = V + head * n * (long long)D;
-        for (int s0 = 0; s0 < n; s0 += kFixSeg) {
-            const int s1 = min(n, s0 + kFixSeg);
-            if (n > kFixSeg) {
+        for (int s0 = 0; s0 < nv; s0 += kFixSeg) {
+            const int s1 = min(nv, s0 + kFixSeg);
+            if (nv > kFixSeg) {
                 __syncthreads();
                 fill(s0, s1);
                 __syncthreads();
@@ -965,6 +995,12 @@ fixup_rows_kernel(const uint32_t *__restrict__ qbits, const uint32_t *__restrict
             for (int w = 0; w < NW; ++w) o += opart[w][c];
             out[(long long)r * D + c] = o / zt;
         }
+        if (kCausal)           // slots past the row's N_i keys are empty
+            for (int k = Nr + threadIdx.x; k < N; k += blockDim.x) {
+                const long long pos = (long long)r * N + k;
+                if (dbg_idx) dbg_idx[pos] = -1;
+                if (dbg_logits) dbg_logits[pos] = 0;
+            }
         __syncthreads();
     }
     if (threadIdx.x == 0) {

@@ -81,16 +81,19 @@ had_status_t prep_typed(const T *Q, const T *K, const T *V, const float *sq, con
 
 // The fused kernel on prepared operands, then the exact fix-up of the rows
 // whose threshold fell outside the sampled window.
+// causal: query i sees keys 0 .. i and keeps min(N, i + 1) of them.
 template <typename T, int D>
 had_status_t core_typed(const T *V, int B, int H, int n, int N, float tau, float *out,
                         int32_t *dbg_idx, int16_t *dbg_lg, char *ws, const FwdWorkspace &w,
-                        int32_t *status, cudaStream_t st)
+                        int32_t *status, cudaStream_t st, bool causal = false)
 {
     using C = fused::Cfg<D>;
     const long long bh = (long long)B * H;
     const bool dbg = dbg_idx != nullptr || dbg_lg != nullptr;
-    auto kernel = dbg ? fused::attention_fwd_kernel<D, true>
-                      : fused::attention_fwd_kernel<D, false>;
+    auto kernel = causal ? (dbg ? fused::attention_fwd_kernel<D, true, true>
+                                : fused::attention_fwd_kernel<D, false, true>)
+                         : (dbg ? fused::attention_fwd_kernel<D, true, false>
+                                : fused::attention_fwd_kernel<D, false, false>);
     // the CTA takes most of the unified L1 as shared memory
     if (cudaFuncSetAttribute(kernel, cudaFuncAttributeMaxDynamicSharedMemorySize,
                              C::SMEM_BYTES) != cudaSuccess ||
@@ -122,8 +125,9 @@ had_status_t core_typed(const T *V, int B, int H, int n, int N, float tau, float
     p.c2 = tau * 1.4426950408889634f;
     const long long blocks = bh * p.ctas_per_head;
     kernel<<<(unsigned)blocks, C::THREADS, C::SMEM_BYTES, st>>>(p);
-    fused::fixup_rows_kernel<T, D><<<148 * 4, 256, 0, st>>>(
-        qbits, kbits, V, n, N, tau, miss_count, miss_count + 1, p.miss_rows, out, dbg_idx, dbg_lg);
+    auto fixup = causal ? fused::fixup_rows_kernel<T, D, true> : fused::fixup_rows_kernel<T, D, false>;
+    fixup<<<148 * 4, 256, 0, st>>>(qbits, kbits, V, n, N, tau, miss_count, miss_count + 1,
+                                   p.miss_rows, out, dbg_idx, dbg_lg);
     return launch_status();
 }
 
@@ -131,25 +135,28 @@ template <typename T, int D>
 had_status_t launch_fused_typed(const T *Q, const T *K, const T *V, const float *sq,
                                 const float *sk, int B, int H, int n, int N, float tau,
                                 float *out, int32_t *dbg_idx, int16_t *dbg_lg, char *ws,
-                                const FwdWorkspace &w, int32_t *status, cudaStream_t st)
+                                const FwdWorkspace &w, int32_t *status, cudaStream_t st,
+                                bool causal)
 {
     had_status_t s = prep_typed<T, D>(Q, K, V, sq, sk, B, H, n, ws, w, status, st);
     if (s != HAD_OK) return s;
-    return core_typed<T, D>(V, B, H, n, N, tau, out, dbg_idx, dbg_lg, ws, w, status, st);
+    return core_typed<T, D>(V, B, H, n, N, tau, out, dbg_idx, dbg_lg, ws, w, status, st,
+                            causal);
 }
 
 template <typename T>
 had_status_t launch_fused(const void *Q, const void *K, const void *V, const float *sq,
                           const float *sk, int B, int H, int n, int d, int N, float tau,
                           float *out, int32_t *dbg_idx, int16_t *dbg_lg, char *ws,
-                          const FwdWorkspace &w, int32_t *status, cudaStream_t st)
+                          const FwdWorkspace &w, int32_t *status, cudaStream_t st,
+                          bool causal = false)
 {
     const T *q = static_cast<const T *>(Q), *k = static_cast<const T *>(K),
             *v = static_cast<const T *>(V);
     return d == 64 ? launch_fused_typed<T, 64>(q, k, v, sq, sk, B, H, n, N, tau, out, dbg_idx,
-                                               dbg_lg, ws, w, status, st)
+                                               dbg_lg, ws, w, status, st, causal)
                    : launch_fused_typed<T, 128>(q, k, v, sq, sk, B, H, n, N, tau, out, dbg_idx,
-                                                dbg_lg, ws, w, status, st);
+                                                dbg_lg, ws, w, status, st, causal);
 }
 
 }  // namespace fwdapi

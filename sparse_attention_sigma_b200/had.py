@@ -68,7 +68,7 @@ def _load():
         "had_topn_mass": [vp, vp, i32, i32, i32, i32, f32, vp, i32, vp, vp, vp],
         "had_hamming_topn_causal": [vp, vp, i32, i32, i32, i32, i32, vp, vp, vp, vp],
         "had_attention_causal_fwd": [vp, vp, vp, i32, vp, vp, i32, i32, i32, i32, i32, f32, vp,
-                                     vp, sz, vp, vp],
+                                     vp, vp, vp, sz, vp, vp],
         "had_soft_binarize": [vp, i32, vp, f32, i32, i32, i32, i32, vp, vp, vp],
         "had_soft_topn": [vp, vp, i32, i32, i32, i32, i32, vp, vp, vp, sz, vp, vp],
         "had_soft_softmax_av": [vp, vp, vp, i32, i32, i32, i32, i32, i32, f32, vp, vp, vp, vp],
@@ -213,9 +213,10 @@ def had_hamming_topn_causal(qbits, kbits, d, N, idx=None, logits=None, dev_statu
     return idx, logits
 
 
-def had_attention_causal_fwd(Q, K, V, sigma_q, sigma_k, N, tau, out=None, ws=None,
-                             dev_status=None, stream=None):
-    """Causal binarized top-N attention forward; returns out [B,H,n,d] float32."""
+def had_attention_causal_fwd(Q, K, V, sigma_q, sigma_k, N, tau, out=None, dbg_idx=None,
+                             dbg_logits=None, ws=None, dev_status=None, stream=None):
+    """Causal binarized top-N attention forward on the fused path (query i sees
+    keys 0..i, keeps min(N, i+1)); returns out [B,H,n,d] float32."""
     _dev(Q, "Q")
     B, H, n, d = _shape4(Q, "Q")
     _dev(K, "K", Q.dtype, (B, H, n, d))
@@ -225,6 +226,10 @@ def had_attention_causal_fwd(Q, K, V, sigma_q, sigma_k, N, tau, out=None, ws=Non
     if out is None:
         out = torch.empty((B, H, n, d), dtype=torch.float32, device=Q.device)
     _dev(out, "out", torch.float32, (B, H, n, d))
+    if dbg_idx is not None:
+        _dev(dbg_idx, "dbg_idx", torch.int32, (B, H, n, N))
+    if dbg_logits is not None:
+        _dev(dbg_logits, "dbg_logits", torch.int16, (B, H, n, N))
     need = had_workspace_bytes(HAD_OP_ATTENTION_CAUSAL, B, H, n, d, N)
     if need < 0:
         raise HadError(HAD_ERR_UNSUPPORTED if d not in (64, 128) else HAD_ERR_INVALID_ARG,
@@ -233,8 +238,8 @@ def had_attention_causal_fwd(Q, K, V, sigma_q, sigma_k, N, tau, out=None, ws=Non
         ws = torch.empty(need, dtype=torch.uint8, device=Q.device)
     st = _lib.had_attention_causal_fwd(_ptr(Q), _ptr(K), _ptr(V), _dtype_code(Q), _ptr(sigma_q),
                                        _ptr(sigma_k), B, H, n, d, N, ctypes.c_float(tau),
-                                       _ptr(out), _ptr(ws), ws.numel(), _ptr(dev_status),
-                                       _stream(stream))
+                                       _ptr(out), _ptr(dbg_idx), _ptr(dbg_logits), _ptr(ws),
+                                       ws.numel(), _ptr(dev_status), _stream(stream))
     _check(st, "had_attention_causal_fwd")
     return out
 

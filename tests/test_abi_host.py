@@ -110,19 +110,22 @@ def test_topn_mass_argument_errors_return_before_any_cuda_call(lib):
 def test_causal_argument_errors_return_before_any_cuda_call(lib):
     f = lib.had_attention_causal_fwd
     vp, i, sz = ctypes.c_void_p, ctypes.c_int, ctypes.c_size_t
-    f.argtypes = [vp, vp, vp, i, vp, vp, i, i, i, i, i, ctypes.c_float, vp, vp, sz, vp, vp]
+    f.argtypes = [vp, vp, vp, i, vp, vp, i, i, i, i, i, ctypes.c_float, vp, vp, vp, vp, sz, vp,
+                  vp]
     f.restype = ctypes.c_int
     fake = vp(4096)        # never dereferenced: the checks fail first
-    assert f(fake, fake, fake, 0, fake, fake, 1, 1, 8, 96, 2, 0.1, fake, fake, 1 << 20,
-             None, None) == 2                                                    # d
-    assert f(fake, fake, fake, 0, fake, fake, 1, 1, 8, 64, 9, 0.1, fake, fake, 1 << 20,
-             None, None) == 1                                                    # N > n
-    assert f(fake, fake, fake, 0, fake, fake, 1, 1, 8, 64, 2, 0.1, fake, None, 1 << 20,
-             None, None) == 1                                                    # no workspace
-    assert f(fake, fake, fake, 0, fake, fake, 1, 1, 8, 64, 2, 0.1, fake, fake, 16,
-             None, None) == 3                                                    # too small
-    assert f(fake, fake, fake, 0, fake, fake, 1, 1, 8, 64, 2, float("nan"), fake, fake,
-             1 << 20, None, None) == 1                                           # tau NaN
+    assert f(fake, fake, fake, 0, fake, fake, 1, 1, 8, 96, 2, 0.1, fake, None, None, fake,
+             1 << 20, None, None) == 2                                           # d
+    assert f(fake, fake, fake, 0, fake, fake, 1, 1, 8, 64, 9, 0.1, fake, None, None, fake,
+             1 << 20, None, None) == 1                                           # N > n
+    assert f(fake, fake, fake, 0, fake, fake, 1, 1, 8, 64, 2, 0.1, fake, None, None, None,
+             1 << 20, None, None) == 3                                           # no workspace
+    assert f(fake, fake, fake, 0, fake, fake, 1, 1, 8, 64, 2, 0.1, fake, None, None, fake,
+             16, None, None) == 3                                                # too small
+    assert f(fake, fake, fake, 0, fake, fake, 1, 1, 8, 64, 2, float("nan"), fake, None, None,
+             fake, 1 << 20, None, None) == 1                                     # tau NaN
+    assert f(fake, fake, fake, 0, fake, fake, 1, 1, 8, 64, 2, 0.1, fake, vp(4100), None, fake,
+             1 << 20, None, None) == 1                                           # misaligned
     g = lib.had_hamming_topn_causal
     g.argtypes = [vp, vp, i, i, i, i, i, vp, vp, vp, vp]
     g.restype = ctypes.c_int
@@ -132,10 +135,11 @@ def test_causal_argument_errors_return_before_any_cuda_call(lib):
     lib.had_workspace_bytes.restype = ctypes.c_size_t
     lib.had_workspace_bytes.argtypes = [ctypes.c_int] * 6
     lib.had_launch_count.argtypes = [ctypes.c_int] * 6
-    # packed Q and K bits (8 B per row at d = 64) plus idx and logits (6 B per slot)
-    assert lib.had_workspace_bytes(7, 1, 1, 128, 64, 16) >= 128 * (8 + 8 + 6 * 16)
+    # the causal call runs the fused path: same workspace and launches
+    for shape in ((1, 1, 128, 64, 16), (4, 16, 4096, 64, 512), (1, 32, 16384, 128, 2048)):
+        assert lib.had_workspace_bytes(7, *shape) == lib.had_workspace_bytes(2, *shape)
+        assert lib.had_launch_count(7, *shape) == 4
     assert lib.had_workspace_bytes(7, 1, 1, 128, 64, 129) == ctypes.c_size_t(-1).value
-    assert lib.had_launch_count(7, 1, 1, 128, 64, 16) == 4
 
 
 def test_soft_argument_errors_return_before_any_cuda_call(lib):

@@ -347,25 +347,63 @@ def _check_causal(had, c, rows):
     idx, lg = had.had_hamming_topn_causal(qb, kb, c.d, c.N)
     out, p = had.had_sparse_softmax_av(idx, lg, c.gv, c.tau, want_p=True)
     status = torch.zeros(1, dtype=torch.int32, device="cuda")
-    out1 = had.had_attention_causal_fwd(c.gq, c.gk, c.gv, c.gsq, c.gsk, c.N, c.tau,
-                                        dev_status=status)
+    dbg_idx = torch.empty((c.B, c.H, c.n, c.N), dtype=torch.int32, device="cuda")
+    dbg_lg = torch.empty((c.B, c.H, c.n, c.N), dtype=torch.int16, device="cuda")
+    fused = had.had_attention_causal_fwd(c.gq, c.gk, c.gv, c.gsq, c.gsk, c.N, c.tau,
+                                         dbg_idx=dbg_idx, dbg_logits=dbg_lg, dev_status=status)
+    plain = had.had_attention_causal_fwd(c.gq, c.gk, c.gv, c.gsq, c.gsk, c.N, c.tau,
+                                         dev_status=status)
     torch.cuda.synchronize()
     assert status.item() == 0
-    assert torch.equal(out, out1)
+    assert torch.equal(fused, plain)      # the debug outputs change nothing
     o_idx, o_lg, o_p, o_out = oracle.attention_causal_rows(c.sq, c.sk, c.v_or, c.tau, c.N, rows)
     flat = lambda t: t.reshape(-1, t.shape[-1]).cpu().numpy()[rows]
+    # unfused building blocks
     assert np.array_equal(flat(idx), o_idx)
     assert np.array_equal(flat(lg), o_lg)
     assert_close(flat(p), o_p, "causal p")
     assert_close(flat(out), o_out, "causal out")
+    # fused tensor-core path
+    assert np.array_equal(flat(dbg_idx), o_idx)
+    assert np.array_equal(flat(dbg_lg), o_lg)
+    assert_close(flat(fused), o_out, "causal fused out")
 
 
 @pytest.mark.parametrize("B,H,n,d,N,seed", [(1, 2, 300, 64, 40, 31), (2, 1, 257, 128, 33, 32),
                                             (1, 1, 1, 64, 1, 33), (1, 2, 130, 64, 130, 34),
-                                            (1, 3, 200, 64, 1, 35)])
+                                            (1, 3, 200, 64, 1, 35), (1, 2, 1100, 64, 200, 36),
+                                            (1, 1, 1000, 128, 100, 37)])
 def test_causal_small_all_rows(had, B, H, n, d, N, seed):
     c = random_case(B, H, n, d, N, seed)
     _check_causal(had, c, all_rows(c))
+
+
+def test_causal_window_misses_take_the_exact_fixup(had):
+    """As the non-causal case: the first 256 keys are far from every query,
+    so for rows past them the sampled window misses and the causal fix-up
+    recomputes the row on its visible keys."""
+    B, H, n, d, N = 1, 2, 1024, 64, 64
+    g = torch.Generator().manual_seed(79)
+    c = torch.randn(1, H, 1, d, generator=g)
+    q = (c + 0.3 * torch.randn(B, H, n, d, generator=g)).to(torch.bfloat16)
+    k = torch.randn(B, H, n, d, generator=g)
+    k[:, :, :256] = -c + 0.3 * torch.randn(B, H, 256, d, generator=g)
+    k = k.to(torch.bfloat16)
+    v = torch.randn(B, H, n, d, generator=g).to(torch.bfloat16)
+    case = Case(q, k, v, synth.per_head_sigma(q), synth.per_head_sigma(k), N, 1 / math.sqrt(d))
+    rows = all_rows(case)
+    # on the host, rows 768.. of the first head: the estimate from the first
+    # 256 keys misses the causal threshold level by more than one level
+    s = oracle.logits_rows(case.sq, case.sk, np.arange(768, 1024))
+    lev = (d - s) // 2
+    miss = 0
+    for t, i in enumerate(range(768, 1024)):
+        vis = lev[t, :i + 1]
+        thr = np.sort(vis)[N - 1]
+        est = np.sort(vis[:256])[max(1, round(N * 256 / (i + 1))) - 1]
+        miss += abs(int(thr) - int(est)) > 1
+    assert miss > 0.9 * 256
+    _check_causal(had, case, rows)
 
 
 def test_causal_long_workload_sampled(had):
