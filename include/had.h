@@ -269,7 +269,7 @@ HAD_API had_status_t had_soft_attention_fwd(const void *Q, const void *K, const 
  *   clip   >= 0 (NaN rejected)
  *   dq, dk, dv  [B,H,n,d] float out
  *   ws     device workspace of had_workspace_bytes(HAD_OP_ATTENTION_BWD, ...)
- *          bytes (about 4 + 26 N bytes per query row)
+ *          bytes (about 36 + 30 N bytes per query row)
  * The key-side sums (dk, dv) run over per-key lists that atomics fill, so
  * their fp32 rounding is not reproducible bit for bit run to run.
  */

@@ -294,7 +294,7 @@ bool finite_float(float x) { return x == x && x < 3.0e38f && x > -3.0e38f; }
 // kept set, p and ds per kept pair, the per-key counts and offsets, and the
 // key-ordered lists.
 struct BwdWorkspace {
-    size_t qbits, kbits, idx, logits, P, DS, cnt, off, cursor, e_row, e_p, e_ds, total;
+    size_t qbits, kbits, idx, logits, P, DS, cnt, off, cursor, rec, total;
 };
 
 BwdWorkspace bwd_layout(int B, int H, int n, int d, int N)
@@ -310,10 +310,8 @@ BwdWorkspace bwd_layout(int B, int H, int n, int d, int N)
     w.cnt = w.DS + round_up(pairs * 4);
     w.off = w.cnt + round_up(rows * 4);
     w.cursor = w.off + round_up(rows * 8);
-    w.e_row = w.cursor + round_up(rows * 8);
-    w.e_p = w.e_row + round_up(pairs * 4);
-    w.e_ds = w.e_p + round_up(pairs * 4);
-    w.total = w.e_ds + round_up(pairs * 4);
+    w.rec = w.cursor + round_up(rows * 4);
+    w.total = w.rec + round_up(pairs * 16);
     return w;
 }
 
@@ -333,10 +331,8 @@ had_status_t launch_bwd_typed(const T *Q, const T *K, const T *V, const float *s
     auto *DS = reinterpret_cast<float *>(base + w.DS);
     auto *cnt = reinterpret_cast<int32_t *>(base + w.cnt);
     auto *off = reinterpret_cast<long long *>(base + w.off);
-    auto *cur = reinterpret_cast<long long *>(base + w.cursor);
-    auto *e_row = reinterpret_cast<int32_t *>(base + w.e_row);
-    auto *e_p = reinterpret_cast<float *>(base + w.e_p);
-    auto *e_ds = reinterpret_cast<float *>(base + w.e_ds);
+    auto *cur = reinterpret_cast<uint32_t *>(base + w.cursor);
+    auto *rec = reinterpret_cast<int4 *>(base + w.rec);
     const had_dtype_t dt = sizeof(T) == 2 ? HAD_BF16 : HAD_F32;
     had_status_t s;
     if ((s = launch_pack(Q, dt, sq, B, H, n, D, qb, status, st)) != HAD_OK) return s;
@@ -357,11 +353,11 @@ had_status_t launch_bwd_typed(const T *Q, const T *K, const T *V, const float *s
     if ((s = launched()) != HAD_OK) return s;
     had::bwd_scan_kernel<<<(unsigned)(B * H), had::kScanThreads, 0, st>>>(cnt, n, N, off, cur);
     if ((s = launched()) != HAD_OK) return s;
-    had::bwd_fill_kernel<<<grid_for(pairs, 256), 256, 0, st>>>(idx, P, DS, pairs, n, N, cur,
-                                                              e_row, e_p, e_ds);
+    had::bwd_fill_kernel<<<grid_for(pairs, 256), 256, 0, st>>>(idx, P, DS, pairs, n, N, off,
+                                                              cur, rec);
     if ((s = launched()) != HAD_OK) return s;
     had::bwd_keys_kernel<T, D><<<(unsigned)warp_blocks, 256, 0, st>>>(
-        off, cnt, e_row, e_p, e_ds, dout, qb, K, sk, H, n, clip, rows, dk, dv);
+        off, cnt, rec, dout, qb, K, sk, H, n, clip, rows, dk, dv);
     return launched();
 }
 

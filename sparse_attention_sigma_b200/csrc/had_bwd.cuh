@@ -239,13 +239,13 @@ bwd_count_kernel(const int32_t *__restrict__ idx, long long pairs, int n, int N,
 }
 
 // One CTA per head: exclusive scan of the head's n counts, offset by the
-// head's first slot head n N.  off keeps the starts, cursor is the fill's
-// running copy.
+// head's first slot head n N, into off; the fill's per-key cursors (counts
+// from the key's start) are cleared.
 constexpr int kScanThreads = 1024;
 
 __global__ void __launch_bounds__(kScanThreads)
 bwd_scan_kernel(const int32_t *__restrict__ cnt, int n, int N, long long *__restrict__ off,
-                long long *__restrict__ cursor)
+                uint32_t *__restrict__ cursor)
 {
     __shared__ long long wsum[kScanThreads / 32];
     __shared__ long long carry;
@@ -269,7 +269,7 @@ bwd_scan_kernel(const int32_t *__restrict__ cnt, int n, int N, long long *__rest
         for (int w = 0; w < warp; ++w) before += wsum[w];
         if (j < n) {
             off[head * n + j] = before + incl - v;
-            cursor[head * n + j] = before + incl - v;
+            cursor[head * n + j] = 0u;
         }
         __syncthreads();
         if (tid == kScanThreads - 1) carry = before + incl;
@@ -277,12 +277,13 @@ bwd_scan_kernel(const int32_t *__restrict__ cnt, int n, int N, long long *__rest
     }
 }
 
-// Every kept pair to its key's list: (query row within the head, p, ds).
+// Every kept pair to its key's list as one 16-byte record (query row within
+// the head, p, ds, unused): one store per pair.
 __global__ void __launch_bounds__(256)
 bwd_fill_kernel(const int32_t *__restrict__ idx, const float *__restrict__ P,
                 const float *__restrict__ DS, long long pairs, int n, int N,
-                long long *__restrict__ cursor, int32_t *__restrict__ e_row,
-                float *__restrict__ e_p, float *__restrict__ e_ds)
+                const long long *__restrict__ off, uint32_t *__restrict__ cursor,
+                int4 *__restrict__ rec)
 {
     const long long stride = (long long)gridDim.x * blockDim.x;
     for (long long e = blockIdx.x * (long long)blockDim.x + threadIdx.x; e < pairs; e += stride) {
@@ -290,11 +291,10 @@ bwd_fill_kernel(const int32_t *__restrict__ idx, const float *__restrict__ P,
         if (j < 0 || j >= n) continue;
         const long long row = e / N;
         const long long head = row / n;
-        const long long pos = (long long)atomicAdd(
-            reinterpret_cast<unsigned long long *>(cursor + head * n + j), 1ull);
-        e_row[pos] = (int32_t)(row - head * n);
-        e_p[pos] = __ldg(P + e);
-        e_ds[pos] = __ldg(DS + e);
+        const long long key = head * n + j;
+        const long long pos = __ldg(off + key) + atomicAdd(cursor + key, 1u);
+        rec[pos] = make_int4((int)(row - head * n), __float_as_int(__ldg(P + e)),
+                             __float_as_int(__ldg(DS + e)), 0);
     }
 }
 
@@ -303,8 +303,7 @@ bwd_fill_kernel(const int32_t *__restrict__ idx, const float *__restrict__ P,
 template <typename T, int D>
 __global__ void __launch_bounds__(256)
 bwd_keys_kernel(const long long *__restrict__ off, const int32_t *__restrict__ cnt,
-                const int32_t *__restrict__ e_row, const float *__restrict__ e_p,
-                const float *__restrict__ e_ds, const float *__restrict__ dout,
+                const int4 *__restrict__ rec, const float *__restrict__ dout,
                 const uint32_t *__restrict__ qbits, const T *__restrict__ K,
                 const float *__restrict__ sigma_k, int H, int n, float clip, long long keys,
                 float *__restrict__ dk, float *__restrict__ dv)
@@ -332,9 +331,10 @@ bwd_keys_kernel(const long long *__restrict__ off, const int32_t *__restrict__ c
         int i = -1;
         float p = 0.0f, ds = 0.0f;
         if (k < c) {
-            i = __ldg(e_row + start + k);
-            p = __ldg(e_p + start + k);
-            ds = __ldg(e_ds + start + k);
+            const int4 e = __ldg(rec + start + k);
+            i = e.x;
+            p = __int_as_float(e.y);
+            ds = __int_as_float(e.z);
         }
 #pragma unroll
         for (int r = 0; r < 8; ++r) {

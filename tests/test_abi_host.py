@@ -208,6 +208,7 @@ def test_bwd_argument_errors_return_before_any_cuda_call(lib):
     lib.had_workspace_bytes.restype = ctypes.c_size_t
     lib.had_workspace_bytes.argtypes = [ctypes.c_int] * 6
     lib.had_launch_count.argtypes = [ctypes.c_int] * 6
-    # per query row: codes 16 B, per-key count and offsets 20 B, 26 B per kept pair
-    assert lib.had_workspace_bytes(12, 1, 1, 128, 64, 16) >= 128 * (16 + 20 + 26 * 16)
+    # per query row: codes 16 B, per-key count, offset and cursor 16 B; per kept
+    # pair: idx 4 B, logit 2 B, p and ds 8 B, a 16-byte key-list record
+    assert lib.had_workspace_bytes(12, 1, 1, 128, 64, 16) >= 128 * (16 + 16 + 30 * 16)
     assert lib.had_launch_count(12, 4, 16, 4096, 64, 512) == 8
