@@ -15,6 +15,18 @@
  *     O_i = sum_{j kept} p_ij V_j,   p_ij = exp(tau (s_ij - m_i)) / Z_i
  * with V kept in full precision and O returned as fp32.
  *
+ * Entry points
+ *   - the forward in one call (had_attention_fwd, _noalloc) or in two
+ *     stages (had_attention_prepare + had_attention_core), and its building
+ *     blocks had_binarize_pack, had_hamming_topn, had_sparse_softmax_av;
+ *   - the causal form (had_attention_causal_fwd; had_hamming_topn_causal);
+ *   - the top-N mass-retention diagnostic (had_topn_mass);
+ *   - the soft-code (tanh) forward of the training stages
+ *     (had_soft_attention_fwd; had_soft_binarize, had_soft_topn,
+ *     had_soft_softmax_av);
+ *   - the straight-through backward (had_attention_bwd);
+ *   - had_workspace_bytes, had_launch_count, had_status_string.
+ *
  * Conventions shared by every entry point
  *   - Tensors are dense, row-major, contiguous, in device memory, 16-byte
  *     aligned: Q, K, V and O are [B, H, n, d]; packed bits are
@@ -347,7 +359,8 @@ HAD_API const char *had_status_string(had_status_t status);
 /*
  * Number of kernels one call of `op` enqueues for these sizes (-1 for
  * unsupported or invalid sizes).  Lets a caller count launches without a
- * profiler.
+ * profiler.  HAD_OP_ATTENTION_BWD counts the recomputation of the kept set;
+ * a call given the forward's kept set enqueues one kernel fewer.
  */
 HAD_API int had_launch_count(int op, int B, int H, int n, int d, int N);
 
