@@ -4,7 +4,10 @@ silent CPU path, and the pairing rules of optional arguments hold."""
 import pytest
 import torch
 
-from sparse_attention_sigma_b200 import had
+from sparse_attention_sigma_b200 import build as _build
+
+_build.build()                      # the library loads without a GPU
+from sparse_attention_sigma_b200 import had  # noqa: E402
 
 x = torch.zeros(1, 1, 8, 64)
 bits = torch.zeros(1, 1, 8, 2, dtype=torch.int32)
