@@ -50,7 +50,9 @@ def parse():
     ap.add_argument("--no-cpu-baseline", action="store_true")
     ap.add_argument("--mode", choices=["attention", "mass", "causal", "soft", "bwd"],
                     default="attention",
-                    help="mass: time the top-N mass-retention diagnostic instead")
+                    help="attention: the forward (the default line); mass: the top-N "
+                         "mass-retention diagnostic; causal: the causal forward; soft: the "
+                         "soft-code (tanh) forward; bwd: forward + straight-through backward")
     return ap.parse_args()
 
 
