@@ -185,7 +185,7 @@ def test_golden_handworked(had):
     exp = case["expected"]
     kb = had.had_binarize_pack(c.gk, c.gsk).cpu().numpy().view(np.uint32)
     assert kb[0, 0].tolist() == exp["k_bits"]
-    for key in ("row0", "row1", "row3"):
+    for key in ("row0", "row1", "row2", "row3"):
         r = int(key[3:])
         assert dbg[0, 0, r].tolist() == exp[key]["idx"]
         want = np.zeros(case["d"])
@@ -193,6 +193,20 @@ def test_golden_handworked(had):
             want[int(col)] = _golden.closed_form(ex)
         # P enters the value product as fp16: within the output tolerance
         assert_close(out[0, 0, r].cpu().numpy(), want, f"golden {key}")
+    # the causal form of the fused kernel on the same hand-worked rows
+    dbg_c = torch.empty((1, 1, 4, 2), dtype=torch.int32, device="cuda")
+    lg_c = torch.empty((1, 1, 4, 2), dtype=torch.int16, device="cuda")
+    out_c = had.had_attention_causal_fwd(c.gq, c.gk, c.gv, c.gsq, c.gsk, c.N, c.tau,
+                                         dbg_idx=dbg_c, dbg_logits=lg_c)
+    torch.cuda.synchronize()
+    for key, e in case["expected_causal"].items():
+        r = int(key[3:])
+        assert dbg_c[0, 0, r].tolist() == e["idx"]
+        assert lg_c[0, 0, r].tolist() == e["logits"]
+        want = np.zeros(case["d"])
+        for col, ex in e["out_nonzero"].items():
+            want[int(col)] = _golden.closed_form(ex)
+        assert_close(out_c[0, 0, r].cpu().numpy(), want, f"golden causal {key}")
 
 
 def test_sign_edge_values_on_device(had):

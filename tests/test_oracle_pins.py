@@ -294,7 +294,7 @@ def test_golden_handworked():
     assert oracle.pack(sk)[0, 0].tolist() == exp["k_bits"]
     assert _head_logits(sq, sk, 0, 0)[0].tolist() == exp["logits_row0_all"]
     idx, lg, p, out = oracle.attention(sq, sk, v, case["tau"], case["N"])
-    for key in ("row0", "row1", "row3"):
+    for key in ("row0", "row1", "row2", "row3"):
         r = int(key[3:])
         e = exp[key]
         assert idx[0, 0, r].tolist() == e["idx"]
@@ -305,6 +305,23 @@ def test_golden_handworked():
         for c, ex in e["out_nonzero"].items():
             want[int(c)] = _golden.closed_form(ex)
         assert np.allclose(out[0, 0, r], want, rtol=1e-7, atol=1e-9)
+
+
+def test_golden_handworked_causal():
+    case = _golden.load()
+    q, k, v, sgq, sgk = _golden.tensors(case)
+    sq, sk = oracle.binarize(q, sgq), oracle.binarize(k, sgk)
+    idx, lg, p, out = oracle.attention_causal_rows(sq, sk, v, case["tau"], case["N"],
+                                                   np.arange(case["n"]))
+    for key, e in case["expected_causal"].items():
+        r = int(key[3:])
+        assert idx[r].tolist() == e["idx"]
+        assert lg[r].tolist() == e["logits"]
+        assert np.allclose(p[r], [_golden.closed_form(x) for x in e["p"]], rtol=1e-14, atol=0)
+        want = np.zeros(case["d"])
+        for c, ex in e["out_nonzero"].items():
+            want[int(c)] = _golden.closed_form(ex)
+        assert np.allclose(out[r], want, rtol=1e-7, atol=1e-9)
 
 
 # ----------------------------------------------------------------- plumbing
