@@ -661,3 +661,37 @@ def test_bwd_clip_masks_exactly():
     assert np.array_equal(b[0], np.where(np.abs(zq) <= 0.5, a[0], 0.0))
     assert np.array_equal(b[1], np.where(np.abs(zk) <= 0.5, a[1], 0.0))
     assert np.array_equal(b[2], a[2])
+
+
+def test_golden_handworked_soft():
+    """Soft codes at tanh's closed forms (3/5, 4/5, 1/2): logits, kept set,
+    weights and output of row 0 against the fixture's hand derivation."""
+    import json
+    import os
+    case = json.load(open(os.path.join(os.path.dirname(__file__), "golden",
+                                       "handworked_soft_n4_d64.json")))
+    n, d = case["n"], case["d"]
+    val = {"ln(2)": math.log(2.0), "ln(3)": math.log(3.0), "-ln(3)": -math.log(3.0),
+           "-ln(3)/2": -0.5 * math.log(3.0)}
+    q = np.zeros((1, 1, n, d), np.float32)
+    q[0, 0, 0] = val[case["q_row0"]]
+    k = np.zeros((1, 1, n, d), np.float32)
+    for r, spec in case["k_rows"].items():
+        row = []
+        for name, count in zip(spec[0::2], spec[1::2]):
+            row += [val[name]] * count
+        k[0, 0, int(r)] = row
+    v = np.eye(n, d, dtype=np.float32)[None, None]
+    sg = np.array(case["sigma"], np.float32)
+    tq, tk = oracle.soft_binarize(q, sg, case["c"]), oracle.soft_binarize(k, sg, case["c"])
+    exp = case["expected"]
+    s = oracle.soft_logits_rows(tq, tk, [0])[0]
+    assert np.allclose(s, [_golden.closed_form(e) for e in exp["logits_row0_all"]],
+                       rtol=0, atol=1e-4)
+    idx, lg, p, out = oracle.soft_attention_rows(tq, tk, v, case["tau"], case["N"], [0])
+    assert idx[0].tolist() == exp["idx"]
+    assert np.allclose(p[0], [_golden.closed_form(e) for e in exp["p"]], rtol=1e-5, atol=0)
+    want = np.zeros(d)
+    for col, e in exp["out_nonzero"].items():
+        want[int(col)] = _golden.closed_form(e)
+    assert np.allclose(out[0], want, rtol=1e-5, atol=1e-7)
