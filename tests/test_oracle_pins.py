@@ -695,3 +695,33 @@ def test_golden_handworked_soft():
     for col, e in exp["out_nonzero"].items():
         want[int(col)] = _golden.closed_form(e)
     assert np.allclose(out[0], want, rtol=1e-5, atol=1e-7)
+
+
+def test_golden_handworked_bwd():
+    """Straight-through backward of a two-key row worked by hand: the
+    gradients are closed forms in a = 1/(1+e^-2), b = e^-2/(1+e^-2)."""
+    import json
+    import os
+    case = json.load(open(os.path.join(os.path.dirname(__file__), "golden",
+                                       "handworked_bwd_n2_d64.json")))
+    n, d = case["n"], case["d"]
+    q = np.full((1, 1, n, d), 0.5, np.float32)
+    q[0, 0, :, 3] = 1.5                              # past the clip; the sign is still +1
+    k = np.full((1, 1, n, d), 0.5, np.float32)
+    k[0, 0, 1, :8] = -0.5
+    v = np.eye(n, d, dtype=np.float32)[None, None]
+    dout = np.zeros((1, 1, n, d), np.float32)
+    dout[0, 0, 0, 0] = 1.0
+    one = np.ones(1, np.float32)
+    dq, dk, dv = oracle.attention_bwd(q, k, v, one, one, dout, case["tau"], case["N"],
+                                      case["clip"])
+    e = {key: _golden.closed_form(x) for key, x in case["expected"].items()}
+    want_q = np.zeros((n, d))
+    want_q[0, :8] = e["dq_row0_first8_except3"]
+    want_q[0, 3] = 0.0
+    assert np.allclose(dq[0, 0], want_q, rtol=1e-12, atol=1e-15)
+    assert np.allclose(dk[0, 0, 0], e["dk_row0"], rtol=1e-12, atol=0)
+    assert np.allclose(dk[0, 0, 1], e["dk_row1"], rtol=1e-12, atol=0)
+    want_v = np.zeros((n, d))
+    want_v[0, 0], want_v[1, 0] = e["dv_row0_col0"], e["dv_row1_col0"]
+    assert np.allclose(dv[0, 0], want_v, rtol=1e-12, atol=1e-15)
