@@ -21,7 +21,9 @@ softmax, closed forms (all keys equal, N = 1), and a hand-worked example
 under ``tests/golden/``.  The soft (tanh) codes of the training stages are
 pinned by tanh closed forms (tanh(ln 2) = 3/5, tanh(ln 3) = 4/5, ...), their
 limits (signs at large c, the scaled dot product at small c), oddness, a
-numpy sort with exact ties, and a dense library softmax at N = n.  The
+numpy sort with exact ties, and a dense library softmax at N = n; their
+softmax over a GIVEN kept set by a library softmax and matrix product over
+that set, and by the selecting oracle on its own set.  The
 straight-through backward is pinned by torch autograd in float64 (the
 surrogate sign, the kept set as a fixed mask), by finite differences of the
 forward in V, and by closed forms (N = 1 and tau = 0 give dQ = dK = 0).  No
@@ -73,6 +75,10 @@ def _load():
             lp, lp, lp, c_int, c_long, c_long, c_long, c_long, c_long,
             ctypes.c_float, lp, c_long, lp, lp, lp, lp, c_int]
         lib.had_oracle_soft_attention_rows.restype = c_int
+        lib.had_oracle_soft_attention_given.argtypes = [
+            lp, lp, lp, c_int, c_long, c_long, c_long, c_long, c_long,
+            ctypes.c_float, lp, c_long, lp, lp, lp]
+        lib.had_oracle_soft_attention_given.restype = c_int
         lib.had_oracle_attention_bwd.argtypes = [
             lp, lp, lp, c_int, lp, lp, lp, c_long, c_long, c_long, c_long, c_long,
             ctypes.c_float, ctypes.c_float, lp, lp, lp, c_int]
@@ -275,6 +281,30 @@ def soft_attention_rows(tq, tk, v, tau, N, rows, threads=0):
     if rc != 0:
         raise ValueError("oracle rejected the arguments (N must be in [1, n])")
     return idx, lg, p, out
+
+
+def soft_attention_given(tq, tk, v, tau, idx, rows):
+    """Softmax and value product on the soft codes over a GIVEN kept set.
+
+    idx [R, N] int32 holds each listed row's kept keys; returns
+    (p [R, N] float64 in idx's order, out [R, d] float64)."""
+    tq = np.ascontiguousarray(tq, dtype=np.float32)
+    tk = np.ascontiguousarray(tk, dtype=np.float32)
+    v = np.ascontiguousarray(v)
+    B, H, n, d = tq.shape
+    assert tk.shape == tq.shape and v.shape == tq.shape
+    rows = _rows_array(rows, B * H * n)
+    idx = np.ascontiguousarray(idx, dtype=np.int32)
+    R, N = idx.shape
+    assert R == rows.size
+    p = np.empty((R, N), dtype=np.float64)
+    out = np.empty((R, d), dtype=np.float64)
+    rc = _load().had_oracle_soft_attention_given(
+        _ptr(tq), _ptr(tk), _ptr(v), _is_bf16(v), B, H, n, d, int(N),
+        ctypes.c_float(float(tau)), _ptr(rows), R, _ptr(idx), _ptr(p), _ptr(out))
+    if rc != 0:
+        raise ValueError("oracle rejected the arguments (indices must lie in [0, n))")
+    return p, out
 
 
 def attention_bwd(q, k, v, sigma_q, sigma_k, dout, tau, N, clip=1.0, threads=0):

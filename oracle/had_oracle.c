@@ -572,6 +572,72 @@ int had_oracle_soft_attention_rows(const float *tq, const float *tk,
 }
 
 /*
+ * Eq. 7 on the soft codes for a GIVEN kept set: for each listed row, the
+ * fp64 logits of its kept keys idx[t, 0..N-1] (any order, each in [0, n)),
+ * then the softmax over exactly those keys (temperature tau, reference the
+ * largest of them) and the value product, in fp64.  Lets a kept set chosen
+ * elsewhere be scored without the oracle's own selection.  p_out [R, N]
+ * (same order as idx) and o_out [R, d].  Returns 0, or -1 on a bad argument
+ * or an allocation failure.
+ */
+int had_oracle_soft_attention_given(const float *tq, const float *tk,
+                                    const void *v, int v_is_bf16, long B,
+                                    long H, long n, long d, long N, float tau,
+                                    const int64_t *rows, long nrows,
+                                    const int32_t *idx, double *p_out,
+                                    double *o_out)
+{
+    (void)B;
+    (void)H;
+    if (N < 1 || d < 1 || n < 1)
+        return -1;
+    for (long t = 0; t < nrows * N; ++t)
+        if (idx[t] < 0 || idx[t] >= n)
+            return -1;
+    double *s = (double *)malloc(sizeof(double) * (size_t)N);
+    double *e = (double *)malloc(sizeof(double) * (size_t)N);
+    if (!s || !e) {
+        free(s);
+        free(e);
+        return -1;
+    }
+    for (long t = 0; t < nrows; ++t) {
+        long r = (long)rows[t];
+        long head = r / n;
+        const float *qr = tq + r * d;
+        for (long k = 0; k < N; ++k) {
+            const float *kr = tk + (head * n + idx[t * N + k]) * d;
+            double acc = 0.0;
+            for (long c = 0; c < d; ++c)
+                acc += (double)qr[c] * (double)kr[c];
+            s[k] = acc;
+        }
+        double m = s[0];
+        for (long k = 1; k < N; ++k)
+            if (s[k] > m)
+                m = s[k];
+        double Z = 0.0;
+        for (long k = 0; k < N; ++k) {
+            e[k] = exp((double)tau * (s[k] - m));
+            Z += e[k];
+        }
+        for (long k = 0; k < N; ++k)
+            p_out[t * N + k] = e[k] / Z;
+        const long vbase = head * n * d;
+        for (long c = 0; c < d; ++c) {
+            double acc = 0.0;
+            for (long k = 0; k < N; ++k)
+                acc += (e[k] / Z) *
+                       (double)load_elem(v, v_is_bf16, vbase + (long)idx[t * N + k] * d + c);
+            o_out[t * d + c] = acc;
+        }
+    }
+    free(s);
+    free(e);
+    return 0;
+}
+
+/*
  * Backward pass of the binarized forward for the straight-through training
  * stage (pith.science review of arXiv 2502.01770: after the tanh stages a
  * straight-through estimator finishes the binarization).  Readings taken:

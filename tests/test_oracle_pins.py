@@ -561,6 +561,47 @@ def test_soft_N_equals_n_is_dense_softmax():
     assert np.allclose(out, ref, rtol=1e-6, atol=1e-6)
 
 
+def test_soft_given_set_is_a_softmax_over_exactly_those_keys():
+    # any kept set, in any order: a library softmax of tau * s over the set
+    # and a matrix product with the set's value rows
+    _, _, v, _, tq, tk = _soft_codes((1, 2, 50, 64), 1.1, seed=176)
+    g = np.random.default_rng(177)
+    rows = np.arange(100)
+    N = 11
+    idx = np.stack([g.permutation(50)[:N] for _ in rows]).astype(np.int32)
+    tau = float(np.float32(0.21))
+    p, out = oracle.soft_attention_given(tq, tk, v, tau, idx, rows)
+    s = oracle.soft_logits_rows(tq, tk, rows)
+    for t, r in enumerate(rows):
+        h = r // 50
+        sel = torch.tensor(s[t, idx[t]])
+        w = torch.softmax(tau * sel, dim=-1)
+        ref = w @ torch.tensor(v[0, h][idx[t]], dtype=torch.float64)
+        assert np.allclose(p[t], w.numpy(), rtol=1e-12, atol=1e-15)
+        assert np.allclose(out[t], ref.numpy(), rtol=1e-12, atol=1e-12)
+    # permuting a row's set permutes its weights and leaves its output
+    perm = g.permutation(N)
+    p2, out2 = oracle.soft_attention_given(tq, tk, v, tau, idx[:, perm], rows)
+    assert np.allclose(p2, p[:, perm], rtol=1e-13, atol=1e-16)
+    assert np.allclose(out2, out, rtol=1e-12, atol=1e-13)
+
+
+def test_soft_given_oracle_set_reproduces_the_selecting_oracle():
+    _, _, v, _, tq, tk = _soft_codes((1, 2, 90, 64), 0.9, seed=178, dup_keys=30)
+    rows = np.arange(180)
+    idx, _, p, out = oracle.soft_attention_rows(tq, tk, v, 0.125, 17, rows)
+    p2, out2 = oracle.soft_attention_given(tq, tk, v, 0.125, idx, rows)
+    assert np.array_equal(p2, p)
+    assert np.array_equal(out2.astype(np.float32), out)
+
+
+def test_soft_given_rejects_out_of_range_keys():
+    _, _, v, _, tq, tk = _soft_codes((1, 1, 20, 64), 1.0, seed=179)
+    bad = np.array([[0, 20]], np.int32)
+    with pytest.raises(ValueError):
+        oracle.soft_attention_given(tq, tk, v, 0.125, bad, np.arange(1))
+
+
 # ------------------------------------------- straight-through backward
 
 
