@@ -31,7 +31,6 @@ sys.path.insert(0, ROOT)
 import synth  # noqa: E402
 
 WORKLOAD = "long"
-METRIC = "HAD attention tokens/sec at n=4096,d=64,N=512; % of int8-TC/HBM roofline"
 L2_FLUSH_BYTES = 256 << 20
 SM_COUNT = 148
 ALU_LANES_PER_SM = 128
@@ -40,20 +39,27 @@ ALU_LANES_PER_SM = 128
 def parse():
     ap = argparse.ArgumentParser()
     ap.add_argument("--gpus", type=int, default=1)
-    ap.add_argument("--steps", type=int, default=20)
-    ap.add_argument("--warmup", type=int, default=5)
+    ap.add_argument("--steps", type=int, default=50)
+    ap.add_argument("--warmup", type=int, default=10)
     ap.add_argument("--impl", choices=["had", "reference"], default="had")
     ap.add_argument("--config", default=WORKLOAD, choices=sorted(synth.CONFIGS))
     ap.add_argument("--cpu-seconds", type=float, default=12.0,
                     help="target CPU time of the oracle baseline sample")
     ap.add_argument("--no-e2e", action="store_true")
     ap.add_argument("--no-cpu-baseline", action="store_true")
-    ap.add_argument("--mode", choices=["attention", "mass", "causal", "soft", "bwd"],
+    ap.add_argument("--mode", choices=["attention", "unfused", "mass", "causal", "soft", "bwd"],
                     default="attention",
-                    help="attention: the forward (the default line); mass: the top-N "
-                         "mass-retention diagnostic; causal: the causal forward; soft: the "
-                         "soft-code (tanh) forward; bwd: forward + straight-through backward")
+                    help="attention: the forward (the default line); unfused: the four-call "
+                         "composition (binarize, top-N, softmax-V) stage by stage; mass: the "
+                         "top-N mass-retention diagnostic; causal: the causal forward; soft: "
+                         "the soft-code (tanh) forward; bwd: forward + straight-through backward")
     return ap.parse_args()
+
+
+def metric_name(cfg):
+    """The headline metric, named for the workload it is measured on."""
+    return (f"HAD attention tokens/sec at n={cfg.n},d={cfg.d},N={cfg.N}; "
+            f"% of int8-TC/HBM roofline")
 
 
 # --------------------------------------------------------------------------- peaks
@@ -239,7 +245,7 @@ def run_reference(args, world, rank):
         oracle_baseline(cfg, per_step * 0.2, steps=1)
     value, info = oracle_baseline(cfg, per_step, steps=steps)
     line = {
-        "impl": "reference", "metric": METRIC, "value": value, "unit": "tokens/s",
+        "impl": "reference", "metric": metric_name(cfg), "value": value, "unit": "tokens/s",
         "n_gpus": args.gpus, "steps": steps, "warmup": args.warmup,
         "ms_per_step": info["seconds"] * 1e3 / steps, "higher_is_better": True,
         "scaling": "weak", "vs_baseline": None, "dtype": "int32+f64", "data": "synthetic",
@@ -359,6 +365,9 @@ def run_had(args, world, rank, local):
     achieved = model["work"] / (core_ms * 1e-3) / 1e12
     peak_eff = model["work"] / model["t_roof"] / 1e12
     traffic = stored_traffic(cfg)
+    misses = had.had_attention_window_misses(ws, cfg.B, cfg.H, cfg.n, cfg.d, cfg.N)
+    core_med = max_over_ranks(statistics.median(e[1].elapsed_time(e[2]) for e in ev), world, dev)
+    ms_med = max_over_ranks(statistics.median(e[0].elapsed_time(e[2]) for e in ev), world, dev)
 
     e2e = None
     if not args.no_e2e:
@@ -373,7 +382,7 @@ def run_had(args, world, rank, local):
     if rank != 0:
         return
     line = {
-        "metric": METRIC, "value": value, "unit": "tokens/s", "n_gpus": world,
+        "metric": metric_name(cfg), "value": value, "unit": "tokens/s", "n_gpus": world,
         "steps": args.steps, "warmup": max(3, args.warmup), "ms_per_step": ms,
         "higher_is_better": True, "scaling": "weak", "vs_baseline": None, "dtype": "bf16",
         "data": "synthetic",
@@ -384,11 +393,14 @@ def run_had(args, world, rank, local):
         "roofline": {"bound": "tensor", "achieved": achieved, "peak": peak_eff,
                      "unit": "TFLOP/s", "frac": achieved / peak_eff, "traffic": traffic,
                      "kernel": f"had_attention_core: {fused_kernel_name(cfg)} + fixup_rows_kernel",
-                     "core_ms": core_ms, "whole_call_frac": model["t_roof"] / (ms * 1e-3),
+                     "core_ms": core_ms, "core_ms_median": core_med, "ms_median": ms_med,
+                     "whole_call_frac": model["t_roof"] / (ms * 1e-3),
                      "t_roof_us": model["t_roof"] * 1e6, "t_hbm_us": model["t_hbm"] * 1e6,
                      "t_tc_us": model["t_tc"] * 1e6, "t_alu_us": model["t_alu"] * 1e6,
                      "peaks": peaks["source"]},
         "gpu_launches": launches * args.steps,
+        "window_misses": {"rows": misses, "of": cfg.B * cfg.H * cfg.n,
+                          "note": "rows the exact fix-up kernel recomputed in the last step"},
         "clocks": clock_info,
         "e2e": e2e,
         "cpu_baseline": cpu,
@@ -464,6 +476,100 @@ def end_to_end(had, cfg, q, k, v, gsq, gsk, ws, dev, steps, world):
             "h2d_bytes_per_step": h2d, "d2h_bytes_per_step": ho[0].numel() * 4,
             "ms_per_step": ms,
             "pipelining": "two buffer sets; upload, compute and download on three streams"}
+
+
+def run_unfused(args, world, rank, local):
+    """The four-call composition of the forward (had_binarize_pack on Q and
+    K, had_hamming_topn, had_sparse_softmax_av) timed stage by stage, each
+    against its own roofline:
+      pack   HBM: read Q and K, write their packed bits;
+      top-N  popcount pipe: two passes of d/32 popcounts per (query, key)
+             pair at 16 popcounts per clock per SM;
+      AV     HBM: read the kept set (6 B per kept pair) and V, write O.
+    The value is tokens per second of the three stages together."""
+    from sparse_attention_sigma_b200 import had
+    cfg = synth.CONFIGS[args.config]
+    dev = torch.device("cuda", local)
+    torch.cuda.set_device(dev)
+    stream = torch.cuda.current_stream()
+    peaks = measured_peaks()
+    q, k, v, sgq, sgk = synth.make_inputs(cfg)
+    gq, gk, gv = q.to(dev), k.to(dev), v.to(dev)
+    gsq, gsk = sgq.to(dev), sgk.to(dev)
+    shape = (cfg.B, cfg.H, cfg.n)
+    qb = torch.empty(shape + (cfg.d // 32,), dtype=torch.int32, device=dev)
+    kb = torch.empty_like(qb)
+    idx = torch.empty(shape + (cfg.N,), dtype=torch.int32, device=dev)
+    lg = torch.empty(shape + (cfg.N,), dtype=torch.int16, device=dev)
+    out = torch.empty(shape + (cfg.d,), dtype=torch.float32, device=dev)
+    flush = torch.empty(L2_FLUSH_BYTES // 4, dtype=torch.float32, device=dev)
+
+    def stages():
+        had.had_binarize_pack(gq, gsq, bits=qb)
+        had.had_binarize_pack(gk, gsk, bits=kb)
+        yield
+        had.had_hamming_topn(qb, kb, cfg.d, cfg.N, idx=idx, logits=lg)
+        yield
+        had.had_sparse_softmax_av(idx, lg, gv, cfg.tau, out=out)
+        yield
+
+    for _ in range(max(3, args.warmup)):
+        for _ in stages():
+            pass
+    torch.cuda.synchronize()
+    clocks = ClockSampler(local)
+    clocks.start()
+    ev = [[torch.cuda.Event(enable_timing=True) for _ in range(4)] for _ in range(args.steps)]
+    barrier(world)
+    torch.cuda.synchronize()
+    for i in range(args.steps):
+        flush.fill_(float(i))
+        ev[i][0].record(stream)
+        for j, _ in enumerate(stages()):
+            ev[i][j + 1].record(stream)
+    torch.cuda.synchronize()
+    barrier(world)
+    clock_info = clocks.stop()
+    per = [[e[j].elapsed_time(e[j + 1]) for e in ev] for j in range(3)]
+    stage_ms = [max_over_ranks(statistics.median(x), world, dev) for x in per]
+    value, ms = aggregate(cfg.tokens, sum(sum(x) for x in per) / args.steps, world, dev)
+    B, H, n, d, N = cfg.B, cfg.H, cfg.n, cfg.d, cfg.N
+    elt = 2 if cfg.dtype == "bf16" else 4
+    hbm = peaks["hbm_gbs"] * 1e9
+    pack_bytes = 2.0 * B * H * n * d * (elt + 1.0 / 8)
+    popc = 2.0 * B * H * n * n * (d // 32)
+    popc_peak = SM_COUNT * 16 * peaks["sm_max_mhz"] * 1e6
+    av_bytes = B * H * n * (6.0 * N + d * elt + d * 4)
+    frac = lambda work, t_ms, peak: work / (t_ms * 1e-3) / peak
+    if rank != 0:
+        return
+    print(json.dumps({
+        "metric": "HAD unfused forward (binarize, top-N, softmax-V) tokens/sec", "value": value,
+        "unit": "tokens/s", "n_gpus": world, "steps": args.steps,
+        "warmup": max(3, args.warmup), "ms_per_step": ms, "higher_is_better": True,
+        "scaling": "weak", "vs_baseline": None, "dtype": cfg.dtype, "data": "synthetic",
+        "impl": "had_binarize_pack x2 + had_hamming_topn + had_sparse_softmax_av",
+        "config": {"workload": cfg.describe(),
+                   "l2": "flushed between steps (256 MiB write outside the timed events)"},
+        "stage_ms_median": {"binarize_pack_qk": stage_ms[0], "hamming_topn": stage_ms[1],
+                            "sparse_softmax_av": stage_ms[2]},
+        "stage_roofline": {
+            "binarize_pack_qk": {"bound": "hbm", "bytes": pack_bytes, "unit": "GB/s",
+                                 "achieved": pack_bytes / (stage_ms[0] * 1e-3) / 1e9,
+                                 "peak": peaks["hbm_gbs"],
+                                 "frac": frac(pack_bytes, stage_ms[0], hbm)},
+            "hamming_topn": {"bound": "alu (popcount pipe)", "popc": popc, "unit": "Tpopc/s",
+                             "achieved": popc / (stage_ms[1] * 1e-3) / 1e12,
+                             "peak": popc_peak / 1e12,
+                             "frac": frac(popc, stage_ms[1], popc_peak)},
+            "sparse_softmax_av": {"bound": "hbm", "bytes": av_bytes, "unit": "GB/s",
+                                  "achieved": av_bytes / (stage_ms[2] * 1e-3) / 1e9,
+                                  "peak": peaks["hbm_gbs"],
+                                  "frac": frac(av_bytes, stage_ms[2], hbm)},
+            "peaks": peaks["source"]},
+        "gpu_launches": 4 * args.steps,
+        "clocks": clock_info,
+    }), flush=True)
 
 
 def run_mass(args, world, rank, local):
@@ -795,6 +901,8 @@ def main():
     try:
         if args.impl == "reference":
             run_reference(args, world, rank)
+        elif args.mode == "unfused":
+            run_unfused(args, world, rank, local)
         elif args.mode == "mass":
             run_mass(args, world, rank, local)
         elif args.mode == "causal":
