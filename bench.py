@@ -268,8 +268,8 @@ def source_digest():
     import hashlib
     h = hashlib.sha256()
     csrc = os.path.join(ROOT, "sparse_attention_sigma_b200", "csrc")
-    for name in ("had_fused.cuh", "had_tc.cuh", "had_prep.cuh", "had_pack.cuh",
-                 "had_common.cuh", "had_fwd_launch.cuh"):
+    for name in ("had_fwd_tc.cuh", "had_fused.cuh", "had_tc.cuh", "had_prep.cuh",
+                 "had_pack.cuh", "had_common.cuh", "had_fwd_launch.cuh"):
         with open(os.path.join(csrc, name), "rb") as f:
             h.update(f.read())
     return h.hexdigest()
@@ -277,7 +277,7 @@ def source_digest():
 
 def fused_kernel_name(cfg):
     """The fused kernel had_attention_core runs for this workload (no debug outputs)."""
-    return "attention_fwd_kernel"
+    return "attention_tc_kernel"
 
 
 def stored_traffic(cfg):

@@ -25,7 +25,8 @@
  *     (had_soft_attention_fwd; had_soft_binarize, had_soft_topn,
  *     had_soft_softmax_av);
  *   - the straight-through backward (had_attention_bwd);
- *   - had_workspace_bytes, had_launch_count, had_status_string.
+ *   - had_workspace_bytes, had_launch_count, had_status_string,
+ *     had_set_wait_limit_ns.
  *
  * Conventions shared by every entry point
  *   - Tensors are dense, row-major, contiguous, in device memory, 16-byte
@@ -38,8 +39,9 @@
  *   - sigma arrays are device float[H], one coefficient per head.
  *   - Supported: d in {64, 128}; 1 <= N <= n; n * N < 2^31; B, H, n >= 1.
  *   - Ownership: the caller allocates and frees every buffer, workspace
- *     included.  The library allocates nothing and keeps no state between
- *     calls.
+ *     included.  The library allocates nothing.  Its only state between
+ *     calls is the wait limit of had_set_wait_limit_ns and the device
+ *     address cache of had_attention_fwd_noalloc.
  *   - Calls are asynchronous on `stream` and never synchronize.  Argument
  *     errors are returned before anything is launched.  A launch failure
  *     returns HAD_ERR_CUDA.  Conditions only the device can see are OR-ed
@@ -179,6 +181,19 @@ HAD_API had_status_t had_attention_core(const void *V, had_dtype_t dt, int B, in
                                         int d, int N, float tau, float *out, int32_t *dbg_idx,
                                         int16_t *dbg_logits, void *ws, size_t ws_bytes,
                                         int32_t *dev_status, cudaStream_t stream);
+
+/*
+ * Diagnostic of the fused forward: how many query rows of the last
+ * had_attention_fwd / _core / had_attention_causal_fwd call on this
+ * workspace had their threshold level fall outside the window the fused
+ * kernel resolves exactly, and so were recomputed whole by the exact fix-up
+ * kernel (they get the same result; only the time differs).  Enqueues on
+ * `stream` a copy of that int32 count into *dst (device or host memory).
+ * ws, ws_bytes and the sizes as in that call.
+ */
+HAD_API had_status_t had_attention_window_misses(const void *ws, size_t ws_bytes, int B, int H,
+                                                 int n, int d, int N, int32_t *dst,
+                                                 cudaStream_t stream);
 
 /*
  * Causal variant.  The pages print no causal rule; this is the plain reading
@@ -328,9 +343,13 @@ HAD_API had_status_t had_topn_mass(const uint32_t *qbits, const uint32_t *kbits,
  *     d=64 N=512); larger sizes return HAD_ERR_WORKSPACE before any launch.
  *   - The array is part of the loaded module: every GPU that loads the
  *     library holds it until the process exits.
- *   - The first call on each device looks up the array's device address
- *     (cudaGetSymbolAddress, with that device current) and caches it; make
- *     that first call before any stream capture.
+ *   - The array's device address belongs to the CUDA context the module
+ *     was loaded in.  The first call in each context (the one current on
+ *     the calling thread: a device's primary context, or one the caller
+ *     created and made current) looks the address up with
+ *     cudaGetSymbolAddress and caches it under that context; later calls in
+ *     the same context reuse it.  Make that first call before any stream
+ *     capture.
  *   - Every call shares the one array per device and leaves its contents
  *     behind; the call re-initialises everything it reads.  Calls whose
  *     kernels overlap on the GPU (different streams, or host threads
@@ -346,6 +365,20 @@ HAD_API had_status_t had_attention_fwd_noalloc(const void *Q, const void *K, con
 
 /* Size in bytes of the fixed array had_attention_fwd_noalloc works in. */
 HAD_API size_t had_noalloc_scratch_bytes(void);
+
+/*
+ * Limit, in nanoseconds, of every on-chip wait of the fused forward kernels
+ * for another role of the same CTA (an operand copy, a tensor-core MMA, an
+ * epilogue warp).  A wait that runs out flags HAD_ERR_TIMEOUT in
+ * *dev_status; the CTA then lets its copies and MMAs in flight complete
+ * (those drain waits keep a limit of 0.5 s), frees its tensor memory and
+ * returns, so the context stays usable; the outputs of that call are
+ * unspecified.  Applies to non-causal calls of had_attention_fwd, _core and
+ * _noalloc launched afterwards, process-wide.  ns = 0 restores the default
+ * (2 s, far beyond any real wait).  Returns the previous limit.  Not a
+ * tuning knob: it exists so that the timeout path can be exercised.
+ */
+HAD_API unsigned long long had_set_wait_limit_ns(unsigned long long ns);
 
 /*
  * Workspace bytes an operation needs for these sizes (0 if none), or

@@ -4,6 +4,7 @@
 #include <climits>
 #include <cstdint>
 #include <mutex>
+#include <cuda.h>
 #include <cuda_runtime.h>
 
 #include "had.h"
@@ -66,15 +67,15 @@ int grid_for(long long work_items, int per_block)
 had_status_t launch_pack(const void *x, had_dtype_t dt, const float *sigma, int B, int H,
                          int n, int d, uint32_t *bits, int32_t *status, cudaStream_t st)
 {
-    const long long groups = (long long)B * H * n * d / 8;
+    const long long words = (long long)B * H * n * d / 32;
     const int threads = 256;
-    const int grid = grid_for(groups, threads);
+    const int grid = grid_for(words, threads);
     if (dt == HAD_BF16)
         had::pack_bits_kernel<__nv_bfloat16><<<grid, threads, 0, st>>>(
-            static_cast<const __nv_bfloat16 *>(x), sigma, H, n, d, groups, bits, status);
+            static_cast<const __nv_bfloat16 *>(x), sigma, H, n, d, words, bits, status);
     else
         had::pack_bits_kernel<float><<<grid, threads, 0, st>>>(
-            static_cast<const float *>(x), sigma, H, n, d, groups, bits, status);
+            static_cast<const float *>(x), sigma, H, n, d, words, bits, status);
     return launched();
 }
 
@@ -145,23 +146,56 @@ constexpr size_t kNoAllocScratchBytes = size_t(96) << 20;   // 96 MiB
 static __device__ __align__(256) unsigned char g_noalloc_scratch[kNoAllocScratchBytes];
 
 // In host code `g_noalloc_scratch` is only a stand-in symbol, never a device
-// address; the real address is looked up once per device, with that device
-// current, and cached here.
-constexpr int kMaxDevices = 64;
-void *g_noalloc_ptr[kMaxDevices] = {};
+// address.  Its device address belongs to the context the module was loaded
+// in, so it is looked up with cudaGetSymbolAddress in the context current on
+// the calling thread and cached under that context (a primary context and a
+// context the caller created on the same device hold different copies).
+using CtxGetCurrentFn = CUresult (*)(CUcontext *);
+
+CtxGetCurrentFn ctx_get_current()
+{
+    static CtxGetCurrentFn fn = []() -> CtxGetCurrentFn {
+        void *f = nullptr;
+        cudaDriverEntryPointQueryResult q;
+        if (cudaGetDriverEntryPoint("cuCtxGetCurrent", &f, cudaEnableDefault, &q) !=
+                cudaSuccess ||
+            q != cudaDriverEntryPointSuccess)
+            return nullptr;
+        return reinterpret_cast<CtxGetCurrentFn>(f);
+    }();
+    return fn;
+}
+
+constexpr int kMaxContexts = 64;
+struct NoallocEntry {
+    CUcontext ctx;
+    void *ptr;
+};
+NoallocEntry g_noalloc_cache[kMaxContexts] = {};
+int g_noalloc_entries = 0;
 std::mutex g_noalloc_mutex;
 
 had_status_t noalloc_scratch(void **ptr)
 {
-    int dev = 0;
-    if (cudaGetDevice(&dev) != cudaSuccess || dev < 0 || dev >= kMaxDevices) return HAD_ERR_CUDA;
+    CtxGetCurrentFn get = ctx_get_current();
+    if (!get) return HAD_ERR_CUDA;
+    CUcontext ctx = nullptr;
+    if (get(&ctx) != CUDA_SUCCESS) return HAD_ERR_CUDA;
     std::lock_guard<std::mutex> lock(g_noalloc_mutex);
-    if (!g_noalloc_ptr[dev]) {
-        void *p = nullptr;
-        if (cudaGetSymbolAddress(&p, g_noalloc_scratch) != cudaSuccess || !p) return HAD_ERR_CUDA;
-        g_noalloc_ptr[dev] = p;
-    }
-    *ptr = g_noalloc_ptr[dev];
+    if (ctx)
+        for (int i = 0; i < g_noalloc_entries; ++i)
+            if (g_noalloc_cache[i].ctx == ctx) {
+                *ptr = g_noalloc_cache[i].ptr;
+                return HAD_OK;
+            }
+    // First call in this context (or none current yet: the runtime makes the
+    // device's primary context current while looking the symbol up).
+    void *p = nullptr;
+    if (cudaGetSymbolAddress(&p, g_noalloc_scratch) != cudaSuccess || !p) return HAD_ERR_CUDA;
+    if (!ctx && get(&ctx) != CUDA_SUCCESS) return HAD_ERR_CUDA;
+    if (ctx && g_noalloc_entries < kMaxContexts)
+        g_noalloc_cache[g_noalloc_entries++] = NoallocEntry{ctx, p};
+    *ptr = p;
     return HAD_OK;
 }
 
@@ -559,7 +593,26 @@ had_status_t had_attention_fwd_noalloc(const void *Q, const void *K, const void 
                                nullptr, base, w, dev_status, stream);
 }
 
+had_status_t had_attention_window_misses(const void *ws, size_t ws_bytes, int B, int H, int n,
+                                         int d, int N, int32_t *dst, cudaStream_t stream)
+{
+    had_status_t s = check_topn(B, H, n, d, N);
+    if (s != HAD_OK) return s;
+    if (!dst) return HAD_ERR_INVALID_ARG;
+    const FwdWorkspace w = fwd_layout(B, H, n, d, N);
+    if (!ws || ws_bytes < w.total) return HAD_ERR_WORKSPACE;
+    const char *src = static_cast<const char *>(ws) + w.miss + 2 * sizeof(int32_t);
+    return cudaMemcpyAsync(dst, src, sizeof(int32_t), cudaMemcpyDefault, stream) == cudaSuccess
+               ? HAD_OK
+               : HAD_ERR_CUDA;
+}
+
 size_t had_noalloc_scratch_bytes(void) { return kNoAllocScratchBytes; }
+
+unsigned long long had_set_wait_limit_ns(unsigned long long ns)
+{
+    return had::fwdapi::wait_limit_ns().exchange(ns ? ns : had::fwdapi::kDefaultWaitNs);
+}
 
 had_status_t had_topn_mass(const uint32_t *qbits, const uint32_t *kbits, int B, int H, int n,
                            int d, float tau, const double *p, int np, int32_t *nmin,

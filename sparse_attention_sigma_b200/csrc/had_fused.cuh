@@ -5,8 +5,9 @@
 //
 // A CTA owns QT tiles of 128 query rows of one head (TMEM lane i = row i of
 // a tile) and streams the head's keys in tiles of 64, twice:
-//   pass 1  S = Q K^T on the tensor core (+/-4 x +/-1 int8 operands, so the
-//           s32 accumulator holds 4 s); each epilogue thread reads its row.
+//   pass 1  S = Q K^T on the tensor core (+/-4 x -/+1 int8 operands, Q
+//           negated, so the s32 accumulator holds -4 s); each epilogue
+//           thread reads its row.
 //           The first key tiles are counted exactly into a per-row histogram
 //           of the d+1 logit levels (shared memory); it places a window of
 //           three levels around the row's threshold, and the remaining tiles
@@ -103,7 +104,7 @@ struct Cfg {
 };
 
 struct Params {
-    const int8_t *qop;        // [BH][qtiles] 128 x D int8 tiles (+/-1)
+    const int8_t *qop;        // [BH][qtiles] 128 x D int8 tiles (-/+1: the negated signs)
     const int8_t *qop2;       // [BH][qtiles] 128 x D int8 tiles (+/-64)
     const int8_t *kop;        // [BH][ktiles] 64 x D int8 tiles (+/-4)
     const __half *vop;        // [BH][ktiles] D x 64 fp16 tiles (V^T, scaled)
@@ -118,7 +119,8 @@ struct Params {
     int sample_tiles;         // key tiles counted exactly before the window
     int n, N;
     int qtiles;               // query tiles per head in qop (a multiple of QT)
-    int ktiles;
+    int ktiles;               // 64-key tiles holding keys (ceil(n / 64))
+    int kstride;              // 64-key tiles per head in kop / vop (ktiles rounded up)
     int ctas_per_head;
     float c2;                 // tau * log2(e)
 };
@@ -257,9 +259,9 @@ attention_fwd_kernel(const Params p)
         // ------------------------------------------------------------ producer
         if (lane == 0) {
             const int8_t *qsrc = p.qop + (head * p.qtiles + qtile0) * (long long)C::QBYTES;
-            const int8_t *ksrc = p.kop + head * (long long)p.ktiles * C::KBYTES;
+            const int8_t *ksrc = p.kop + head * (long long)p.kstride * C::KBYTES;
             const uint8_t *vsrc = reinterpret_cast<const uint8_t *>(p.vop) +
-                                  head * (long long)p.ktiles * C::VBYTES;
+                                  head * (long long)p.kstride * C::VBYTES;
             const int8_t *qsrc2 = p.qop2 + (head * p.qtiles + qtile0) * (long long)C::QBYTES;
             tc::mbar_expect_tx(b.q_full, 2 * QT * C::QBYTES);
             tc::bulk_g2s(smem + C::OFF_Q, qsrc, QT * C::QBYTES, b.q_full);
@@ -415,9 +417,10 @@ attention_fwd_kernel(const Params p)
         uint32_t *hist = reinterpret_cast<uint32_t *>(smem + C::OFF_HIST + g * C::HIST_BYTES);
         uint32_t *hcol = hist + r;                    // hist[bin][r] at hcol[bin * kRows]
         for (int bin = 0; bin < C::BINS; ++bin) hcol[bin * kRows] = 0;
-        // The accumulator holds v = 4 s.  The level of a logit is its Hamming
-        // distance (D - s)/2; its histogram bin sits (D - s) * 256 bytes =
-        // 256 D - 64 v past this row's bin 0.
+        // The pass-1 accumulator holds v = -4 s.  The level of a logit is its
+        // Hamming distance (D - s)/2; its histogram bin sits (D - s) * 256
+        // bytes = 256 D + 64 v past this row's bin 0, and its counter shift
+        // is cshift + v.
         const uint32_t hbase = tc::smem_u32(hcol) + 256u * D;
         const int A = min(T, p.sample_tiles);         // tiles counted exactly
         // Pass 1 keeps one word of window counts per key tile in the TMEM
@@ -454,7 +457,7 @@ attention_fwd_kernel(const Params p)
         auto hist_half = [&](const uint32_t (&rr)[32], auto full, int valid) {
 #pragma unroll
             for (int c = 0; c < 32; ++c)
-                if (decltype(full)::value || c < valid) red_add1(hbase - (rr[c] << 6));
+                if (decltype(full)::value || c < valid) red_add1(hbase + (rr[c] << 6));
         };
         // pass 1b: four cumulative 8-bit window counters in one register;
         // four independent counter registers keep the adds off one chain
@@ -473,7 +476,7 @@ attention_fwd_kernel(const Params p)
 #pragma unroll
             for (int c = 0; c < 32; ++c)
                 if (decltype(full)::value || c < valid)
-                    acc[c & 3] += window_inc(cshift - (int)rr[c]);
+                    acc[c & 3] += window_inc(cshift + (int)rr[c]);
         };
         // Window from the sample: est = the level of the sample's
         // (N * sampled / n)-th best key.  Levels L0 = est - 1 .. est + 1 are
@@ -491,7 +494,7 @@ attention_fwd_kernel(const Params p)
                 if (!found && cum >= ns) { est = bin; found = true; }
             }
             L0 = est - 1;
-            cshift = 4 * D - 8 * L0 + 8;              // 8 * (level - L0 + 1) = cshift - v
+            cshift = 4 * D - 8 * L0 + 8;              // 8 * (level - L0 + 1) = cshift + v
         };
         auto pass1_half = [&](int j, int h, const uint32_t (&rr)[32]) {
             const int valid = half_valid(j, h);
@@ -774,8 +777,9 @@ attention_fwd_kernel(const Params p)
 //      D/32 columns, so each row is one coalesced read), accumulating fp32;
 //      the partial sums meet in shared memory.
 // For n <= kFixSeg the distances of step 1 are kept for step 2; longer rows
-// recompute each segment's distances.  The last CTA to finish zeroes the
-// miss counter (and its own done counter) for the next fused pass.
+// recompute each segment's distances.  The last CTA to finish copies the
+// miss count to miss_count[2] (the diagnostic's copy) and zeroes the miss
+// counter and its own done counter for the next fused pass.
 constexpr int kFixSeg = 16384;
 constexpr int kFixList = 256;                     // kept keys a warp lists per round
 
@@ -1006,6 +1010,7 @@ fixup_rows_kernel(const uint32_t *__restrict__ qbits, const uint32_t *__restrict
     if (threadIdx.x == 0) {
         __threadfence();
         if (atomicAdd(done_count, 1) == (int)gridDim.x - 1) {
+            miss_count[2] = *miss_count;          // kept for had_attention_window_misses
             *miss_count = 0;
             *done_count = 0;
             __threadfence();

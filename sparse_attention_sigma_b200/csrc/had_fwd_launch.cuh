@@ -1,10 +1,12 @@
 // had_fwd_launch.cuh -- host side of the fused forward: the workspace
 // layout of had_attention_fwd / _prepare / _core and the launches of the
-// operand preparation, the fused kernel and its exact fix-up.  Kept apart
+// operand preparation, the fused kernels and their exact fix-up.  Kept apart
 // from the other entry points so that this file, with the kernels it
 // launches, is the whole of the fused path.
 #pragma once
+#include <atomic>
 #include <climits>
+#include <cmath>
 #include <cstddef>
 #include <cuda_runtime.h>
 
@@ -12,6 +14,7 @@
 #include "had_common.cuh"
 #include "had_prep.cuh"
 #include "had_fused.cuh"
+#include "had_fwd_tc.cuh"
 
 namespace had {
 namespace fwdapi {
@@ -23,11 +26,21 @@ inline had_status_t launch_status()
     return cudaGetLastError() == cudaSuccess ? HAD_OK : HAD_ERR_CUDA;
 }
 
-// Workspace of the fused forward: tensor-core operand tiles of Q, K and V^T
-// and the per-head V scale.
+// Limit of every wait of the fused kernels for another role of the same CTA
+// (a copy, an MMA, an epilogue warp).  Far beyond any real wait by default.
+constexpr unsigned long long kDefaultWaitNs = 2000000000ull;
+inline std::atomic<unsigned long long> &wait_limit_ns()
+{
+    static std::atomic<unsigned long long> ns{kDefaultWaitNs};
+    return ns;
+}
+
+// Workspace of the fused forward: tensor-core operand tiles of Q, K and V^T,
+// packed signs, per-head V scale and key column sums, and the list of rows
+// the fix-up kernel recomputes.
 struct FwdWorkspace {
-    size_t qop, qop2, kop, vop, qbits, kbits, vpart, miss, vexp, miss_rows, total;
-    int qtiles, ktiles, vchunks;
+    size_t qop, qop2, kop, vop, qbits, kbits, vpart, miss, vexp, kpart, ksum, miss_rows, total;
+    int qtiles, ktiles, kstride, vchunks;
 };
 
 inline FwdWorkspace fwd_layout(int B, int H, int n, int d, int N)
@@ -39,70 +52,134 @@ inline FwdWorkspace fwd_layout(int B, int H, int n, int d, int N)
     w.qtiles = (n + fused::kRows - 1) / fused::kRows;
     w.qtiles = (w.qtiles + qt - 1) / qt * qt;
     w.ktiles = (n + fused::kKeys - 1) / fused::kKeys;
+    w.kstride = (w.ktiles + 1) / 2 * 2;                 // whole 128-key pairs
     // V chunks of 8192 elements for the per-head maximum
     w.vchunks = (int)(((size_t)n * d + 8191) / 8192);
     w.qop = 0;
     w.qop2 = w.qop + align256(bh * w.qtiles * fused::kRows * d);
     w.kop = w.qop2 + align256(bh * w.qtiles * fused::kRows * d);
-    w.vop = w.kop + align256(bh * w.ktiles * fused::kKeys * d);
-    w.qbits = w.vop + align256(bh * w.ktiles * fused::kKeys * d * 2);
+    w.vop = w.kop + align256(bh * w.kstride * fused::kKeys * d);
+    w.qbits = w.vop + align256(bh * w.kstride * fused::kKeys * d * 2);
     w.kbits = w.qbits + align256(bh * n * (d / 8));
     w.vpart = w.kbits + align256(bh * n * (d / 8));
     w.miss = w.vpart + align256(bh * w.vchunks * 4);
     w.vexp = w.miss + align256(8);                      // miss counter, fix-up done counter
-    w.miss_rows = w.vexp + align256(bh * 4);
+    w.kpart = w.vexp + align256(bh * 4);
+    w.ksum = w.kpart + align256(bh * w.kstride * d);
+    w.miss_rows = w.ksum + align256(bh * d * 4);
     w.total = w.miss_rows + align256(bh * (size_t)w.qtiles * fused::kRows * 4);
     return w;
 }
 
-// Operand preparation: Q/K signs as tensor-core tiles and packed bits and
-// the V chunk maxima in one launch, then V^T in fp16 with its per-head scale.
+// Operand preparation: Q/K signs as tensor-core tiles and packed bits, the
+// key column sums and the V chunk maxima in one launch, then V^T in fp16 with
+// its per-head scale (and the per-head key sums).
 template <typename T, int D>
 had_status_t prep_typed(const T *Q, const T *K, const T *V, const float *sq, const float *sk,
                         int B, int H, int n, char *ws, const FwdWorkspace &w, int32_t *status,
                         cudaStream_t st)
 {
     const long long bh = (long long)B * H;
-    const long long blocks = bh * (w.qtiles + w.ktiles + w.vchunks);
-    if (blocks > INT_MAX || bh * w.ktiles > INT_MAX) return HAD_ERR_UNSUPPORTED;
+    const long long blocks = bh * (w.qtiles + w.kstride + w.vchunks);
+    if (blocks > INT_MAX || bh * w.kstride > INT_MAX) return HAD_ERR_UNSUPPORTED;
     auto *vpart = reinterpret_cast<float *>(ws + w.vpart);
     // Q as +/-1 and +/-64, K as +/-4: the i8 MMA accumulates 4 s or 256 s
     prep::operands_kernel<T, D><<<(unsigned)blocks, 256, 0, st>>>(
-        Q, K, V, sq, sk, H, n, (int)bh, w.qtiles, w.ktiles, w.vchunks,
+        Q, K, V, sq, sk, H, n, (int)bh, w.qtiles, w.kstride, w.vchunks,
         reinterpret_cast<int8_t *>(ws + w.qop), reinterpret_cast<int8_t *>(ws + w.qop2),
         reinterpret_cast<int8_t *>(ws + w.kop), reinterpret_cast<uint16_t *>(ws + w.qbits),
-        reinterpret_cast<uint16_t *>(ws + w.kbits), vpart, reinterpret_cast<int *>(ws + w.miss),
-        status);
-    prep::v_operand_kernel<T, D><<<(unsigned)(bh * w.ktiles), 256, 0, st>>>(
-        V, n, vpart, w.vchunks, reinterpret_cast<__half *>(ws + w.vop),
-        reinterpret_cast<int *>(ws + w.vexp));
+        reinterpret_cast<uint16_t *>(ws + w.kbits), reinterpret_cast<int8_t *>(ws + w.kpart),
+        vpart, reinterpret_cast<int *>(ws + w.miss), status);
+    prep::v_operand_kernel<T, D><<<(unsigned)(bh * w.kstride), 256, 0, st>>>(
+        V, n, w.kstride, vpart, w.vchunks, reinterpret_cast<__half *>(ws + w.vop),
+        reinterpret_cast<int *>(ws + w.vexp), reinterpret_cast<const int8_t *>(ws + w.kpart),
+        reinterpret_cast<int *>(ws + w.ksum));
     return launch_status();
 }
 
-// The fused kernel on prepared operands, then the exact fix-up of the rows
-// whose threshold fell outside the sampled window.
-// causal: query i sees keys 0 .. i and keeps min(N, i + 1) of them.
-template <typename T, int D>
-had_status_t core_typed(const T *V, int B, int H, int n, int N, float tau, float *out,
-                        int32_t *dbg_idx, int16_t *dbg_lg, char *ws, const FwdWorkspace &w,
-                        int32_t *status, cudaStream_t st, bool causal = false)
+// Standard normal quantile Phi^-1(p) by bisection on erfc (host, once per
+// call); it only places the fused kernel's threshold window.
+inline float normal_quantile(double p)
+{
+    p = std::fmin(std::fmax(p, 1e-9), 1.0 - 1e-9);
+    double lo = -40.0, hi = 40.0;
+    for (int i = 0; i < 100; ++i) {
+        const double mid = 0.5 * (lo + hi);
+        if (0.5 * std::erfc(-mid / std::sqrt(2.0)) < p) lo = mid;
+        else hi = mid;
+    }
+    return (float)(0.5 * (lo + hi));
+}
+
+inline int sm_count()
+{
+    int dev = 0, sms = 0;
+    if (cudaGetDevice(&dev) != cudaSuccess ||
+        cudaDeviceGetAttribute(&sms, cudaDevAttrMultiProcessorCount, dev) != cudaSuccess ||
+        sms < 1)
+        return 148;
+    return sms;
+}
+
+// Non-causal core: the 128-key tensor-core kernel.
+template <int D>
+had_status_t core_tc(int B, int H, int n, int N, float tau, float *out, int32_t *dbg_idx,
+                     int16_t *dbg_lg, char *ws, const FwdWorkspace &w, int32_t *status,
+                     cudaStream_t st)
+{
+    using C = tcfwd::Cfg<D>;
+    const long long bh = (long long)B * H;
+    const bool dbg = dbg_idx != nullptr || dbg_lg != nullptr;
+    auto kernel = dbg ? tcfwd::attention_tc_kernel<D, true> : tcfwd::attention_tc_kernel<D, false>;
+    if (cudaFuncSetAttribute(kernel, cudaFuncAttributeMaxDynamicSharedMemorySize,
+                             C::SMEM_BYTES) != cudaSuccess ||
+        cudaFuncSetAttribute(kernel, cudaFuncAttributePreferredSharedMemoryCarveout,
+                             cudaSharedmemCarveoutMaxShared) != cudaSuccess)
+        return HAD_ERR_CUDA;
+    tcfwd::Params p;
+    p.qop = reinterpret_cast<int8_t *>(ws + w.qop);
+    p.kop = reinterpret_cast<int8_t *>(ws + w.kop);
+    p.vop = reinterpret_cast<__half *>(ws + w.vop);
+    p.vexp = reinterpret_cast<int *>(ws + w.vexp);
+    p.qbits = reinterpret_cast<uint32_t *>(ws + w.qbits);
+    p.ksum = reinterpret_cast<int *>(ws + w.ksum);
+    p.out = out;
+    p.dbg_idx = dbg_idx;
+    p.dbg_logits = dbg_lg;
+    p.status = status;
+    p.miss_count = reinterpret_cast<int *>(ws + w.miss);
+    p.miss_rows = reinterpret_cast<int *>(ws + w.miss_rows);
+    p.miss_cap = (long long)bh * w.qtiles * fused::kRows;
+    p.n = n;
+    p.N = N;
+    p.qtiles = w.qtiles;
+    p.kstride = w.kstride;
+    p.ctas_per_head = w.qtiles / C::QT;
+    p.c2 = tau * 1.4426950408889634f;
+    p.z = normal_quantile((double)N / (double)n);
+    p.wait_ns = wait_limit_ns().load();
+    const long long blocks = bh * p.ctas_per_head;
+    kernel<<<(unsigned)blocks, C::THREADS, C::SMEM_BYTES, st>>>(p);
+    return launch_status();
+}
+
+// Causal core: the 64-key fused kernel in its causal form.
+template <int D>
+had_status_t core_causal(int B, int H, int n, int N, float tau, float *out, int32_t *dbg_idx,
+                         int16_t *dbg_lg, char *ws, const FwdWorkspace &w, int32_t *status,
+                         cudaStream_t st)
 {
     using C = fused::Cfg<D>;
     const long long bh = (long long)B * H;
     const bool dbg = dbg_idx != nullptr || dbg_lg != nullptr;
-    auto kernel = causal ? (dbg ? fused::attention_fwd_kernel<D, true, true>
-                                : fused::attention_fwd_kernel<D, false, true>)
-                         : (dbg ? fused::attention_fwd_kernel<D, true, false>
-                                : fused::attention_fwd_kernel<D, false, false>);
+    auto kernel = dbg ? fused::attention_fwd_kernel<D, true, true>
+                      : fused::attention_fwd_kernel<D, false, true>;
     // the CTA takes most of the unified L1 as shared memory
     if (cudaFuncSetAttribute(kernel, cudaFuncAttributeMaxDynamicSharedMemorySize,
                              C::SMEM_BYTES) != cudaSuccess ||
         cudaFuncSetAttribute(kernel, cudaFuncAttributePreferredSharedMemoryCarveout,
                              cudaSharedmemCarveoutMaxShared) != cudaSuccess)
         return HAD_ERR_CUDA;
-    auto *qbits = reinterpret_cast<uint32_t *>(ws + w.qbits);
-    auto *kbits = reinterpret_cast<uint32_t *>(ws + w.kbits);
-    auto *miss_count = reinterpret_cast<int *>(ws + w.miss);
     fused::Params p;
     p.qop = reinterpret_cast<int8_t *>(ws + w.qop);
     p.qop2 = reinterpret_cast<int8_t *>(ws + w.qop2);
@@ -113,7 +190,7 @@ had_status_t core_typed(const T *V, int B, int H, int n, int N, float tau, float
     p.dbg_idx = dbg_idx;
     p.dbg_logits = dbg_lg;
     p.status = status;
-    p.miss_count = miss_count;
+    p.miss_count = reinterpret_cast<int *>(ws + w.miss);
     p.miss_rows = reinterpret_cast<int *>(ws + w.miss_rows);
     p.miss_cap = (long long)bh * w.qtiles * fused::kRows;
     p.sample_tiles = w.ktiles / 16 > 4 ? w.ktiles / 16 : 4;
@@ -121,13 +198,34 @@ had_status_t core_typed(const T *V, int B, int H, int n, int N, float tau, float
     p.N = N;
     p.qtiles = w.qtiles;
     p.ktiles = w.ktiles;
+    p.kstride = w.kstride;
     p.ctas_per_head = w.qtiles / C::QT;
     p.c2 = tau * 1.4426950408889634f;
     const long long blocks = bh * p.ctas_per_head;
     kernel<<<(unsigned)blocks, C::THREADS, C::SMEM_BYTES, st>>>(p);
+    return launch_status();
+}
+
+// The fused kernel on prepared operands, then the exact fix-up of the rows
+// whose threshold fell outside their window.
+// causal: query i sees keys 0 .. i and keeps min(N, i + 1) of them.
+template <typename T, int D>
+had_status_t core_typed(const T *V, int B, int H, int n, int N, float tau, float *out,
+                        int32_t *dbg_idx, int16_t *dbg_lg, char *ws, const FwdWorkspace &w,
+                        int32_t *status, cudaStream_t st, bool causal = false)
+{
+    had_status_t s = causal ? core_causal<D>(B, H, n, N, tau, out, dbg_idx, dbg_lg, ws, w,
+                                             status, st)
+                            : core_tc<D>(B, H, n, N, tau, out, dbg_idx, dbg_lg, ws, w, status,
+                                         st);
+    if (s != HAD_OK) return s;
+    auto *qbits = reinterpret_cast<uint32_t *>(ws + w.qbits);
+    auto *kbits = reinterpret_cast<uint32_t *>(ws + w.kbits);
+    auto *miss_count = reinterpret_cast<int *>(ws + w.miss);
+    auto *miss_rows = reinterpret_cast<int *>(ws + w.miss_rows);
     auto fixup = causal ? fused::fixup_rows_kernel<T, D, true> : fused::fixup_rows_kernel<T, D, false>;
-    fixup<<<148 * 4, 256, 0, st>>>(qbits, kbits, V, n, N, tau, miss_count, miss_count + 1,
-                                   p.miss_rows, out, dbg_idx, dbg_lg);
+    fixup<<<sm_count() * 4, 256, 0, st>>>(qbits, kbits, V, n, N, tau, miss_count, miss_count + 1,
+                                          miss_rows, out, dbg_idx, dbg_lg);
     return launch_status();
 }
 

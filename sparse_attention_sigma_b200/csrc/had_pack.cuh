@@ -3,9 +3,7 @@
 // "What carries the argument").
 //
 // HBM-bound: every element is read once (16-byte vector loads) and 1 bit per
-// element is written.  A thread turns 8 consecutive elements into one byte;
-// four neighbouring lanes merge their bytes into a 32-bit word with two warp
-// shuffles, so stores are whole words.  Word w of a row holds elements
+// element is written, as whole 32-bit words.  Word w of a row holds elements
 // 32w..32w+31 with element 32w+k in bit k; bit = 1 means sign -1.
 #pragma once
 #include "had_common.cuh"
@@ -38,33 +36,46 @@ struct Load8<float> {
     }
 };
 
-// groups = B*H*n*d/8 (a multiple of 4 because d is a multiple of 32).
+// One thread per output word: 32 consecutive elements of a row (16-byte
+// vector loads) give the 32 bits of one uint32.  With a normal sigma an
+// element at or below -sigma * 2^-100 is surely negative after the division
+// and one at or above zero surely not, so the sign is a comparison; only a
+// word holding an element strictly between (possible, never seen in
+// practice) takes the exact IEEE division, for all 32 elements.
+// words = B*H*n*d/32; word w covers elements 32w .. 32w+31 of the tensor.
 template <typename T>
 __global__ void __launch_bounds__(256)
-pack_bits_kernel(const T *__restrict__ x, const float *__restrict__ sigma, int H,
-                 int n, int d, long long groups, uint32_t *__restrict__ bits,
-                 int32_t *status)
+pack_bits_kernel(const T *__restrict__ x, const float *__restrict__ sigma, int H, int n, int d,
+                 long long words, uint32_t *__restrict__ bits, int32_t *status)
 {
-    const int lane = threadIdx.x & 31;
-    const long long warp0 = (blockIdx.x * (long long)blockDim.x + threadIdx.x) >> 5;
-    const long long nwarps = ((long long)gridDim.x * blockDim.x) >> 5;
-    const int groups_per_row = d >> 3;
-    for (long long base = warp0 * 32; base < groups; base += nwarps * 32) {
-        const long long g = base + lane;
-        uint32_t byte = 0;
-        if (g < groups) {
-            const long long row = g / groups_per_row;
-            const int head = (int)((row / n) % H);
-            const SignRule r = sign_rule(__ldg(sigma + head));
-            if (r.bad) flag(status, HAD_ERR_BAD_SIGMA);
-            float v[8];
-            Load8<T>::run(x + g * 8, v);
-#pragma unroll
-            for (int k = 0; k < 8; ++k) byte |= negative_bit(v[k], r) << k;
+    const long long stride = (long long)gridDim.x * blockDim.x;
+    const int words_per_row = d >> 5;
+    int cached = -1;
+    SignRule rule = sign_rule(1.0f);
+    for (long long w = blockIdx.x * (long long)blockDim.x + threadIdx.x; w < words; w += stride) {
+        const int head = (int)((w / words_per_row / n) % H);
+        if (head != cached) {
+            cached = head;
+            rule = sign_rule(__ldg(sigma + head));
+            if (rule.bad) flag(status, HAD_ERR_BAD_SIGMA);
         }
-        uint32_t pair = byte | (__shfl_down_sync(kFullMask, byte, 1) << 8);
-        uint32_t word = pair | (__shfl_down_sync(kFullMask, pair, 2) << 16);
-        if ((lane & 3) == 0 && g < groups) bits[g >> 2] = word;
+        float v[32];
+#pragma unroll
+        for (int c = 0; c < 4; ++c)
+            Load8<T>::run(x + w * 32 + 8 * c, *reinterpret_cast<float(*)[8]>(v + 8 * c));
+        uint32_t word = 0;
+        bool unsure = !rule.fast;
+#pragma unroll
+        for (int i = 0; i < 32; ++i) {
+            word |= (uint32_t)(v[i] <= -rule.thr) << i;
+            unsure |= (v[i] < 0.0f) && (v[i] > -rule.thr);
+        }
+        if (unsure) {
+            word = 0;
+#pragma unroll
+            for (int i = 0; i < 32; ++i) word |= negative_bit(v[i], rule) << i;
+        }
+        bits[w] = word;
     }
 }
 

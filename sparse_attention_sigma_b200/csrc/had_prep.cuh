@@ -7,16 +7,22 @@
 // 128 bytes apart, row groups (8 rows) (K bytes / 16) * 128 bytes apart.
 // Tiles are stored contiguously so the kernel moves each with one bulk copy.
 //
-//   Qop1, Qop2 [BH][qtiles] tiles of 128 rows x d int8: the signs as +/-1
-//                    and as +/-64 (0 padding; qtiles >= ceil(n/128), the
-//                    extra tiles all padding)
-//   Kop [BH][ceil(n/64)] tiles of 64 keys x d int8 (+4 / -4, 0 padding)
+//   Qop1, Qop2 [BH][qtiles] tiles of 128 rows x d int8: the signs negated,
+//                    as -/+1, and as +/-64 (0 padding; qtiles >= ceil(n/128),
+//                    the extra tiles all padding)
+//   Kop [BH][kstride] tiles of 64 keys x d int8 (+4 / -4, 0 padding); kstride
+//                    = ceil(n/64) rounded up to even, so that pairs of tiles
+//                    (128 keys) always move as one whole copy
 //   Qbits, Kbits [BH][n][d/32] the same signs bit-packed (1 = -1)
-// With K as +/-4 the s32 accumulator holds 4 s against Qop1 (the counter
-// shifts of the fused kernel's first pass are one integer add away) and
-// 256 s against Qop2 (the byte offset of the logit's level in its per-row
-// tables, again one integer add away).
-//   Vop [BH][ceil(n/64)]  tiles of V^T: d rows x 64 keys fp16, scaled by
+//   Kpart [BH][kstride][d] int8  per 64-key tile: sum over its keys of the
+//                    +/-1 code of each dimension; Ksum [BH][d] int32 their
+//                    sum over the head (the exact mean logit of a query row is
+//                    q . Ksum / n)
+// With K as +/-4 the s32 accumulator holds -4 s against Qop1 (so that a
+// per-row bias added by the tensor core turns it into the counter shift of
+// the fused kernel's first pass) and 256 s against Qop2 (the byte offset of
+// the logit's level in its per-row tables, one integer add away).
+//   Vop [BH][kstride]     tiles of V^T: d rows x 64 keys fp16, scaled by
 //                         2^-e_h so the head's largest |v| lies in
 //                         [2^14, 2^15) (bf16 -> fp16 then loses no bits for
 //                         any value within 2^39 of the head maximum)
@@ -95,7 +101,7 @@ __device__ __forceinline__ uint4 recode(const uint32_t (&w)[4], uint32_t pos, ui
 
 // All operand preparation that needs only the inputs, in one launch.  Block
 // b of the grid takes, in this order:
-//   b <  BH*qtiles            one 128-row Q tile -> Qop1 (+/-1), Qop2 (+/-64), Qbits
+//   b <  BH*qtiles            one 128-row Q tile -> Qop1 (-/+1), Qop2 (+/-64), Qbits
 //   b <  BH*(qtiles+ktiles)   one 64-key K tile  -> Kop (+/-4), Kbits
 //   otherwise                 one chunk of V     -> the chunk's largest |v|
 // Rows past n are written as zero padding.  A thread handles 16 consecutive
@@ -111,9 +117,11 @@ operands_kernel(const T *__restrict__ Q, const T *__restrict__ K, const T *__res
                 int bh, int qtiles, int ktiles, int vchunks, int8_t *__restrict__ qop,
                 int8_t *__restrict__ qop2, int8_t *__restrict__ kop,
                 uint16_t *__restrict__ qbits, uint16_t *__restrict__ kbits,
-                float *__restrict__ vpart, int *__restrict__ miss_count, int32_t *status)
+                int8_t *__restrict__ kpart, float *__restrict__ vpart,
+                int *__restrict__ miss_count, int32_t *status)
 {
     constexpr int CPR = D / 16;                                // 16-element chunks per row
+    __shared__ uint16_t sbits[kKeys][CPR];                     // K tile signs, for column sums
     const int b = blockIdx.x;
     if (b == 0 && threadIdx.x < 2) miss_count[threadIdx.x] = 0;   // miss and fix-up done counters
     const int nq = bh * qtiles, nk = bh * ktiles;
@@ -130,21 +138,35 @@ operands_kernel(const T *__restrict__ Q, const T *__restrict__ K, const T *__res
         int8_t *tile = (isq ? qop : kop) + (size_t)bb * rows * D;
         int8_t *tile2 = qop2 + (size_t)bb * rows * D;
         uint16_t *bits = isq ? qbits : kbits;
-        const uint32_t pos = isq ? 0x01u : 0x04u, neg = isq ? 0xFFu : 0xFCu;
+        // Q as -1 / +1 for sign + / - (the pass-1 accumulator then holds -4 s),
+        // K as +4 / -4
+        const uint32_t pos = isq ? 0xFFu : 0x04u, neg = isq ? 0x01u : 0xFCu;
         for (int c = threadIdx.x; c < rows * CPR; c += blockDim.x) {
             const int r = c / CPR, kc = c % CPR;
             const int row = t * rows + r;
             uint32_t w[4] = {0u, 0u, 0u, 0u};
+            uint32_t packed = 0u;
             if (row < n) {
                 const size_t e = ((size_t)head * n + row) * D + kc * 16;
-                const uint32_t packed = sign16<T>(x + e, rule, pos, neg, w);
+                packed = sign16<T>(x + e, rule, pos, neg, w);
                 bits[e / 16] = (uint16_t)packed;
             }
+            if (!isq) sbits[r][kc] = (uint16_t)packed;
             const uint32_t off = core_offset(r, kc * 16, D);
             *reinterpret_cast<uint4 *>(tile + off) = make_uint4(w[0], w[1], w[2], w[3]);
             if (isq)
                 *reinterpret_cast<uint4 *>(tile2 + off) =
-                    row < n ? recode(w, 0x01u, 0x40u, 0xC0u) : make_uint4(0u, 0u, 0u, 0u);
+                    row < n ? recode(w, 0xFFu, 0x40u, 0xC0u) : make_uint4(0u, 0u, 0u, 0u);
+        }
+        if (!isq) {
+            // column sums of the tile's codes: valid keys minus twice the negatives
+            __syncthreads();
+            const int valid = max(0, min(kKeys, n - t * kKeys));
+            for (int a = threadIdx.x; a < D; a += blockDim.x) {
+                int neg_count = 0;
+                for (int rr = 0; rr < valid; ++rr) neg_count += (sbits[rr][a >> 4] >> (a & 15)) & 1;
+                kpart[(size_t)bb * D + a] = (int8_t)(valid - 2 * neg_count);
+            }
         }
         return;
     }
@@ -186,16 +208,16 @@ __device__ __forceinline__ int vscale_exp(float m)
 
 // One CTA per (head, 64-key tile): the head's largest |v| from the chunk
 // maxima of operands_kernel, then the tile transposed through shared memory
-// and written as V^T fp16 core matrices.  Writes e_h for every head (by the
-// CTA of tile 0).
+// and written as V^T fp16 core matrices (tiles past n are zeros).  The CTA of
+// tile 0 writes the head's e_h and reduces its key column sums to Ksum.
 template <typename T, int D>
 __global__ void __launch_bounds__(256)
-v_operand_kernel(const T *__restrict__ v, int n, const float *__restrict__ vpart, int vchunks,
-                 __half *__restrict__ op, int *__restrict__ vexp)
+v_operand_kernel(const T *__restrict__ v, int n, int tiles, const float *__restrict__ vpart,
+                 int vchunks, __half *__restrict__ op, int *__restrict__ vexp,
+                 const int8_t *__restrict__ kpart, int *__restrict__ ksum)
 {
     __shared__ float tile[kKeys][D + 1];
     __shared__ float head_max;
-    const int tiles = (n + kKeys - 1) / kKeys;
     const long long head = blockIdx.x / tiles;
     const int t = blockIdx.x % tiles;
     if (threadIdx.x < 32) {
@@ -209,6 +231,12 @@ v_operand_kernel(const T *__restrict__ v, int n, const float *__restrict__ vpart
     const int e = vscale_exp(head_max);
     const float scale = ldexpf(1.0f, -e);
     if (t == 0 && threadIdx.x == 0) vexp[head] = e;
+    if (t == 0)
+        for (int a = threadIdx.x; a < D; a += blockDim.x) {
+            int sum = 0;
+            for (int k = 0; k < tiles; ++k) sum += kpart[((size_t)head * tiles + k) * D + a];
+            ksum[head * D + a] = sum;
+        }
     // load 64 keys x D values (coalesced, 8 elements per thread-iteration)
     constexpr int G = kKeys * D / 8;
     for (int g = threadIdx.x; g < G; g += blockDim.x) {

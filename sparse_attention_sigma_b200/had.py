@@ -85,6 +85,10 @@ def _load():
     lib.had_workspace_bytes.restype = ctypes.c_size_t
     lib.had_launch_count.argtypes = [i32] * 6
     lib.had_launch_count.restype = ctypes.c_int
+    lib.had_attention_window_misses.argtypes = [vp, sz, i32, i32, i32, i32, i32, vp, vp]
+    lib.had_attention_window_misses.restype = ctypes.c_int
+    lib.had_set_wait_limit_ns.argtypes = [ctypes.c_ulonglong]
+    lib.had_set_wait_limit_ns.restype = ctypes.c_ulonglong
     lib.had_noalloc_scratch_bytes.argtypes = []
     lib.had_noalloc_scratch_bytes.restype = ctypes.c_size_t
     lib.had_status_string.argtypes = [ctypes.c_int]
@@ -505,6 +509,24 @@ def had_attention_fwd_noalloc(Q, K, V, sigma_q, sigma_k, N, tau, out, dev_status
 
 def had_noalloc_scratch_bytes() -> int:
     return int(_lib.had_noalloc_scratch_bytes())
+
+
+def had_attention_window_misses(ws, B, H, n, d, N, stream=None) -> int:
+    """Rows of the last fused call on ``ws`` that the exact fix-up kernel
+    recomputed (their threshold fell outside the fused kernel's window).
+    Synchronizes the stream to read the count."""
+    _dev(ws, "ws", torch.uint8)
+    dst = torch.zeros(1, dtype=torch.int32, device=ws.device)
+    st = _lib.had_attention_window_misses(_ptr(ws), ws.numel(), B, H, n, d, N, _ptr(dst),
+                                          _stream(stream))
+    _check(st, "had_attention_window_misses")
+    return int(dst.item())
+
+
+def had_set_wait_limit_ns(ns: int) -> int:
+    """Limit of the fused kernels' on-chip waits (0 = the 2 s default);
+    returns the previous limit."""
+    return int(_lib.had_set_wait_limit_ns(int(ns)))
 
 
 def workspace(B, H, n, d, N, device="cuda"):

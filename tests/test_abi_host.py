@@ -62,6 +62,15 @@ def test_workspace_and_launch_counts(lib):
     assert lib.had_launch_count(2, 1, 1, 8, 64, 0) == -1
 
 
+def test_wait_limit_setter_swaps_and_restores_the_default(lib):
+    lib.had_set_wait_limit_ns.restype = ctypes.c_ulonglong
+    lib.had_set_wait_limit_ns.argtypes = [ctypes.c_ulonglong]
+    default = 2_000_000_000
+    assert lib.had_set_wait_limit_ns(1000) == default
+    assert lib.had_set_wait_limit_ns(0) == 1000          # 0 restores the default
+    assert lib.had_set_wait_limit_ns(0) == default
+
+
 def test_argument_errors_return_before_any_cuda_call(lib):
     f = lib.had_attention_fwd
     vp, i, sz = ctypes.c_void_p, ctypes.c_int, ctypes.c_size_t

@@ -43,7 +43,8 @@ def test_host_tensors_are_refused(name):
 # fused path's argument checks)
 HELPERS = {"had_status_string", "had_workspace_bytes", "had_launch_count",
            "had_noalloc_scratch_bytes", "had_attention_prepare", "had_attention_core",
-           "had_attention_fwd_noalloc"}
+           "had_attention_fwd_noalloc", "had_set_wait_limit_ns",
+           "had_attention_window_misses"}
 
 
 def test_every_wrapper_is_covered():

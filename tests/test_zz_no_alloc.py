@@ -4,9 +4,11 @@ had_attention_fwd_noalloc serves callers that cannot call cudaMalloc (code
 running under another runtime's allocator, plugins handed only their input
 and output buffers, processes whose device memory is reserved up front): it
 runs the same kernels as had_attention_fwd but in a fixed device array
-inside the library.  This file is collected last so that a run stopping at
-the first failure has already run every other test; it also passes alone in
-a fresh process.
+inside the library.  The kernels are deterministic, so its output must equal
+the workspace entry point's bit for bit, call after call; and after its first
+call on a device its calls must not change the device's free memory.  This
+file is collected last so that a run stopping at the first failure has
+already run every other test; it also passes alone in a fresh process.
 """
 import ctypes
 import math
@@ -48,12 +50,19 @@ def test_noalloc_matches_workspace_entry_point_twice(B, H, n, d, N, dtype):
     tau = 1 / math.sqrt(d)
     ref = had.had_attention_fwd(q, k, v, sq, sk, N, tau)
     status = torch.zeros(1, dtype=torch.int32, device="cuda")
-    for _ in range(2):
-        out = torch.full((B, H, n, d), float("nan"), device="cuda")
+    outs = [torch.full((B, H, n, d), float("nan"), device="cuda") for _ in range(3)]
+    # the first call looks the array's address up; later calls allocate nothing
+    had.had_attention_fwd_noalloc(q, k, v, sq, sk, N, tau, outs[0], dev_status=status)
+    torch.cuda.synchronize()
+    free0 = torch.cuda.mem_get_info()[0]
+    for out in outs[1:]:
         had.had_attention_fwd_noalloc(q, k, v, sq, sk, N, tau, out, dev_status=status)
-        torch.cuda.synchronize()
-        assert status.item() == 0
+    torch.cuda.synchronize()
+    assert torch.cuda.mem_get_info()[0] == free0
+    assert status.item() == 0
+    for out in outs:
         _close(out, ref)
+        assert torch.equal(out, ref)
 
 
 def test_noalloc_long_workload_fits_and_matches():
@@ -68,6 +77,7 @@ def test_noalloc_long_workload_fits_and_matches():
         had.had_attention_fwd_noalloc(q, k, v, sq, sk, cfg.N, cfg.tau, out)
         torch.cuda.synchronize()
         _close(out, ref)
+        assert torch.equal(out, ref)
 
 
 def test_noalloc_rejects_sizes_beyond_its_array():
