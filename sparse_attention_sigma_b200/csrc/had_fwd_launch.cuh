@@ -73,20 +73,23 @@ inline FwdWorkspace fwd_layout(int B, int H, int n, int d, int N)
 
 // Operand preparation: Q/K signs as tensor-core tiles and packed bits, the
 // key column sums and the V chunk maxima in one launch, then V^T in fp16 with
-// its per-head scale (and the per-head key sums).
+// its per-head scale (and the per-head key sums).  The +/-64 copy of Q is
+// written only for the causal kernel (causal = true), which reads it.
 template <typename T, int D>
 had_status_t prep_typed(const T *Q, const T *K, const T *V, const float *sq, const float *sk,
                         int B, int H, int n, char *ws, const FwdWorkspace &w, int32_t *status,
-                        cudaStream_t st)
+                        cudaStream_t st, bool causal = false)
 {
     const long long bh = (long long)B * H;
     const long long blocks = bh * (w.qtiles + w.kstride + w.vchunks);
     if (blocks > INT_MAX || bh * w.kstride > INT_MAX) return HAD_ERR_UNSUPPORTED;
     auto *vpart = reinterpret_cast<float *>(ws + w.vpart);
-    // Q as +/-1 and +/-64, K as +/-4: the i8 MMA accumulates 4 s or 256 s
+    // Q as the negated signs (and, for the causal kernel, +/-64), K as +/-4:
+    // the i8 MMA accumulates -4 s (or 256 s)
     prep::operands_kernel<T, D><<<(unsigned)blocks, 256, 0, st>>>(
         Q, K, V, sq, sk, H, n, (int)bh, w.qtiles, w.kstride, w.vchunks,
-        reinterpret_cast<int8_t *>(ws + w.qop), reinterpret_cast<int8_t *>(ws + w.qop2),
+        reinterpret_cast<int8_t *>(ws + w.qop),
+        causal ? reinterpret_cast<int8_t *>(ws + w.qop2) : nullptr,
         reinterpret_cast<int8_t *>(ws + w.kop), reinterpret_cast<uint16_t *>(ws + w.qbits),
         reinterpret_cast<uint16_t *>(ws + w.kbits), reinterpret_cast<int8_t *>(ws + w.kpart),
         vpart, reinterpret_cast<int *>(ws + w.miss), status);
@@ -236,7 +239,7 @@ had_status_t launch_fused_typed(const T *Q, const T *K, const T *V, const float 
                                 const FwdWorkspace &w, int32_t *status, cudaStream_t st,
                                 bool causal)
 {
-    had_status_t s = prep_typed<T, D>(Q, K, V, sq, sk, B, H, n, ws, w, status, st);
+    had_status_t s = prep_typed<T, D>(Q, K, V, sq, sk, B, H, n, ws, w, status, st, causal);
     if (s != HAD_OK) return s;
     return core_typed<T, D>(V, B, H, n, N, tau, out, dbg_idx, dbg_lg, ws, w, status, st,
                             causal);

@@ -325,13 +325,17 @@ attention_tc_kernel(const Params p)
             // S tile kidx = S = Q_g K_u^T into slot kidx % 3; G is the K stream
             // entry that holds key tile u (the stage is waited for at g = 0 and
             // released after the last query tile's MMAs).
-            // bias: 0 none, 1 the pass-1 window offset, 2 the pass-2 table offset
-            auto qk = [&](int kidx, int g, int G, int bias) -> bool {
+            // bias: 0 none, 1 the pass-1 window offset, 2 the pass-2 table offset.
+            // synced: a barrier that epilogue threads arrive on was just waited
+            // for, so their prior TMEM and shared-memory work must be ordered
+            // before these MMAs (a fence); the copy barriers (async proxy, like
+            // the MMA) and the in-order reuse of a slot after its P V need none.
+            auto qk = [&](int kidx, int g, int G, int bias, bool synced) -> bool {
                 const int ks = G % C::KSTAGES;
                 if (g == 0 &&
                     !wait_bar(k_full + ks, (G / C::KSTAGES) & 1, deadline, abort_flag, p.status))
                     return false;
-                tc::fence_after_sync();
+                if (synced) tc::fence_after_sync();
                 const uint64_t dqa = dq + (uint64_t)((g * C::QBYTES) >> 4);
                 const uint64_t dkb = dk + (uint64_t)((ks * C::KBYTES) >> 4);
                 const uint32_t dcol = tmem + (kidx % kSlots) * kKeys;
@@ -360,8 +364,8 @@ attention_tc_kernel(const Params p)
                     ok = false;
                     break;
                 }
-                if (kidx == QT) tc::fence_after_sync();
-                ok = qk(kidx, kidx % QT, kidx / QT, kidx >= QT ? 1 : 0);
+                ok = qk(kidx, kidx % QT, kidx / QT, kidx >= QT ? 1 : 0,
+                        kidx >= kSlots || kidx == QT);
             }
             // pass 2: tile j of the pass is stream tile J + j
             auto qk2 = [&](int j) -> bool {
@@ -369,11 +373,12 @@ attention_tc_kernel(const Params p)
                 if (u == 0 && !wait_bar(q2_ready + g, 0, deadline, abort_flag, p.status))
                     return false;
                 // the slot last held pass-1 tile kidx - 3 (if any): wait until read
-                if (kidx >= kSlots && kidx - kSlots < J &&
+                const bool after_pass1 = kidx >= kSlots && kidx - kSlots < J;
+                if (after_pass1 &&
                     !wait_bar(s_free + kidx % kSlots, ((kidx - kSlots) / kSlots) & 1, deadline,
                               abort_flag, p.status))
                     return false;
-                return qk(kidx, g, T + u, 2);
+                return qk(kidx, g, T + u, 2, u == 0 || after_pass1);
             };
             for (int j = 0; j < min(kSlots, J) && ok; ++j) ok = qk2(j);
             for (int j = 0; j < J && ok; ++j) {

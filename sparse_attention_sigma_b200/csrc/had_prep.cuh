@@ -101,7 +101,8 @@ __device__ __forceinline__ uint4 recode(const uint32_t (&w)[4], uint32_t pos, ui
 
 // All operand preparation that needs only the inputs, in one launch.  Block
 // b of the grid takes, in this order:
-//   b <  BH*qtiles            one 128-row Q tile -> Qop1 (-/+1), Qop2 (+/-64), Qbits
+//   b <  BH*qtiles            one 128-row Q tile -> Qop1 (-/+1), Qop2 (+/-64, when
+//                             qop2 is given: only the causal kernel reads it), Qbits
 //   b <  BH*(qtiles+ktiles)   one 64-key K tile  -> Kop (+/-4), Kbits
 //   otherwise                 one chunk of V     -> the chunk's largest |v|
 // Rows past n are written as zero padding.  A thread handles 16 consecutive
@@ -136,7 +137,7 @@ operands_kernel(const T *__restrict__ Q, const T *__restrict__ K, const T *__res
         const SignRule rule = sign_rule(__ldg((isq ? sq : sk) + head % H));
         if (rule.bad && threadIdx.x == 0) flag(status, HAD_ERR_BAD_SIGMA);
         int8_t *tile = (isq ? qop : kop) + (size_t)bb * rows * D;
-        int8_t *tile2 = qop2 + (size_t)bb * rows * D;
+        int8_t *tile2 = qop2 ? qop2 + (size_t)bb * rows * D : nullptr;
         uint16_t *bits = isq ? qbits : kbits;
         // Q as -1 / +1 for sign + / - (the pass-1 accumulator then holds -4 s),
         // K as +4 / -4
@@ -154,7 +155,7 @@ operands_kernel(const T *__restrict__ Q, const T *__restrict__ K, const T *__res
             if (!isq) sbits[r][kc] = (uint16_t)packed;
             const uint32_t off = core_offset(r, kc * 16, D);
             *reinterpret_cast<uint4 *>(tile + off) = make_uint4(w[0], w[1], w[2], w[3]);
-            if (isq)
+            if (isq && qop2)
                 *reinterpret_cast<uint4 *>(tile2 + off) =
                     row < n ? recode(w, 0xFFu, 0x40u, 0xC0u) : make_uint4(0u, 0u, 0u, 0u);
         }
