@@ -126,9 +126,9 @@ inline int sm_count()
 
 // Non-causal core: the 128-key tensor-core kernel.
 template <int D>
-had_status_t core_tc(int B, int H, int n, int N, float tau, float *out, int32_t *dbg_idx,
-                     int16_t *dbg_lg, char *ws, const FwdWorkspace &w, int32_t *status,
-                     cudaStream_t st)
+had_status_t core_tc(const void *V, bool v_f32, int B, int H, int n, int N, float tau,
+                     float *out, int32_t *dbg_idx, int16_t *dbg_lg, char *ws,
+                     const FwdWorkspace &w, int32_t *status, cudaStream_t st)
 {
     using C = tcfwd::Cfg<D>;
     const long long bh = (long long)B * H;
@@ -145,6 +145,9 @@ had_status_t core_tc(int B, int H, int n, int N, float tau, float *out, int32_t 
     p.vop = reinterpret_cast<__half *>(ws + w.vop);
     p.vexp = reinterpret_cast<int *>(ws + w.vexp);
     p.qbits = reinterpret_cast<uint32_t *>(ws + w.qbits);
+    p.kbits = reinterpret_cast<uint32_t *>(ws + w.kbits);
+    p.v = V;
+    p.v_f32 = v_f32 ? 1 : 0;
     p.ksum = reinterpret_cast<int *>(ws + w.ksum);
     p.out = out;
     p.dbg_idx = dbg_idx;
@@ -219,8 +222,8 @@ had_status_t core_typed(const T *V, int B, int H, int n, int N, float tau, float
 {
     had_status_t s = causal ? core_causal<D>(B, H, n, N, tau, out, dbg_idx, dbg_lg, ws, w,
                                              status, st)
-                            : core_tc<D>(B, H, n, N, tau, out, dbg_idx, dbg_lg, ws, w, status,
-                                         st);
+                            : core_tc<D>(V, sizeof(T) == 4, B, H, n, N, tau, out, dbg_idx,
+                                         dbg_lg, ws, w, status, st);
     if (s != HAD_OK) return s;
     auto *qbits = reinterpret_cast<uint32_t *>(ws + w.qbits);
     auto *kbits = reinterpret_cast<uint32_t *>(ws + w.kbits);

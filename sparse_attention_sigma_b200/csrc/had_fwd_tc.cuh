@@ -13,39 +13,39 @@
 //           over the first key tile, as mean + z sd with z the standard normal
 //           quantile at N/n.  Levels est-1 .. est+1 form the row's window.
 //   pass 1  S = Q K^T (-/+1 x +/-4 int8: Q negated, the s32 accumulator holds
-//           -4 s) plus, from the second key tile on, a third MMA step that
-//           adds each row's bias (its window offset spread over 32 int8
-//           columns, times a tile of ones), so that the accumulator is
-//           directly the logit's shift in a thermometer of four 8-bit counters
-//           of one register (level <= L0-1, L0, L0+1, L0+2).  One word of
-//           counts per tile and row is kept in TMEM.  At the end the summed
-//           counters give the exact threshold level t and the number q of
-//           keys kept at it whenever t falls inside the window; rows where it
-//           does not are listed and recomputed exactly by the fix-up kernel.
-//           The tile words give the one tile where the row's tie quota runs
-//           out.
-//   regroup the CTA's rows are sorted by that tile (a counting sort in shared
-//           memory) and the Q tiles are rewritten in that order, so that the
-//           32 rows of a warp share few such tiles: they are the only tiles
-//           that count ties key by key.
+//           -4 s).  Adding the row's window offset to it (one fused add-max
+//           per logit) gives the logit's shift in a thermometer of four 8-bit
+//           counters of one register (level <= L0-1, L0, L0+1, L0+2).  One
+//           word of counts per tile and row is kept in TMEM.  At the end the
+//           summed counters give the exact threshold level t and the number q
+//           of keys kept at it whenever t falls inside the window; rows where
+//           it does not are listed and recomputed exactly by the fix-up
+//           kernel.  The tile words give the one tile where the row's tie
+//           quota runs out.
 //   pass 2  S again, with Q as -64 times the signs and a bias step that adds
 //           the offset of the thread's weight-table column, so that the
 //           accumulator is directly the byte offset of the logit's weight:
 //           exp2(c2 (s_l - ref)) for levels <= t, 0 beyond.  One shared load
-//           per logit gives it; ties at level t are kept or zeroed through the
-//           table, except in the quota tile, which keeps the first of them in
-//           key order (the lower index wins).  P is packed to fp16 pairs over
+//           per logit gives it.  Ties at level t weigh w_t before the quota
+//           tile and 0 from it on (the table entry is cleared there), so every
+//           full tile takes the same path.  P is packed to fp16 pairs over
 //           the first half of its own S in TMEM and the tensor core
 //           accumulates O += P V (fp16 x fp16 -> f32).
+//   quota   the kept ties of the quota tile (the first of them in key order:
+//           the lower index wins) are found after pass 2 from the packed sign
+//           bits (Hamming distance = level) and added to O and Z by the row's
+//           thread.
 // The n x n logits never leave the SM.
 //
 // Warp roles: warp 0 bulk-copies the Q tiles once and streams K (twice) and
-// V^T (pass 2) through shared-memory rings; warp 1 issues every MMA from one
-// thread, in order, over a ring of three 128-column S slots shared by the
-// query tiles (S tile k of the stream sits in slot k % 3; tile k + 3 is issued
-// into it once the epilogue has released it in pass 1, or right after the
-// P V that reads it in pass 2, since tcgen05 operations of one thread run in
-// issue order); warps 2 .. 1 + 4 QT are the epilogue, four per query tile.
+// V^T (pass 2) through shared-memory rings.  One thread of warp 1 issues the
+// Q K^T MMAs and one of warp 2 the P V MMAs (a thread can issue a tcgen05 MMA
+// only every few tens of cycles, so the two streams go out in parallel).  S
+// tiles use a ring of three 128-column TMEM slots shared by the query tiles
+// (S tile k of the stream sits in slot k % 3); tile k + 3 is issued into a
+// slot once the epilogue has released it (pass 1) or once the P V that reads
+// it has completed (pass 2).  Warps 3 .. 2 + 4 QT are the epilogue, four per
+// query tile.
 // Every wait is bounded by a caller-set limit: a CTA that hits it flags
 // HAD_ERR_TIMEOUT, lets its copies and MMAs drain, frees its TMEM and returns.
 #pragma once
@@ -71,7 +71,8 @@ template <int D>
 struct Cfg {
     static constexpr int QT = D == 64 ? HAD_TC_QT64 : 1;   // query tiles per CTA
     static constexpr int EPI_WARPS = 4 * QT;
-    static constexpr int THREADS = 32 * (2 + EPI_WARPS);
+    static constexpr int EPI_WARP0 = 3;                // producer, QK issuer, PV issuer
+    static constexpr int THREADS = 32 * (EPI_WARP0 + EPI_WARPS);
     static constexpr int QBYTES = kRows * D;            // int8 Q tile
     static constexpr int KBYTES = kKeys * D;            // int8 K tile (two workspace tiles)
     static constexpr int VSUB = D * kSub * 2;           // fp16 V^T workspace tile
@@ -89,24 +90,15 @@ struct Cfg {
     static constexpr int OFF_K = OFF_Q + QT * QBYTES;
     static constexpr int OFF_V = OFF_K + KSTAGES * KBYTES;
     static constexpr int OFF_TAB = OFF_V + VSTAGES * VBYTES;
-    // pass-1 bias step: per query tile 128 rows x 32 int8 (one K=32 step),
-    // and a 128-key x 32 tile of ones
+    // pass-2 bias step: per query tile 128 rows x 32 int8 (one K=32 step),
+    // and per key 16 bytes of 127 then 16 bytes of 1, so that a row's bias
+    // bytes (x0..x15, y0..y15) add 127 sum x + sum y
     static constexpr int BIAS_BYTES = kRows * 32;
     static constexpr int ONES_BYTES = kKeys * 32;
     static constexpr int OFF_BIAS = OFF_TAB + QT * TAB_BYTES;
-    static constexpr int OFF_ONES = OFF_BIAS + QT * BIAS_BYTES;
-    // pass-2 bias step: per key 16 bytes of 127 then 16 bytes of 1, so that
-    // a row's bias bytes (x0..x15, y0..y15) add 127 sum x + sum y
-    static constexpr int OFF_ONES2 = OFF_ONES + ONES_BYTES;
-    // between the passes the CTA's rows are regrouped by the key tile where
-    // their tie quota runs out: per-row state at the new position, and the
-    // bucket counts of the counting sort
-    static constexpr int ROWS = QT * kRows;
-    static constexpr int OFF_STATE = OFF_ONES2 + ONES_BYTES;
-    static constexpr int OFF_SORT = OFF_STATE + ROWS * 32;
-    static constexpr int SORT_BUCKETS = STASH_CAP + 2;
-    static constexpr int OFF_BAR = OFF_SORT + ((SORT_BUCKETS * 4 + 15) / 16) * 16;
-    static constexpr int NBARS = 1 + 2 * KSTAGES + 2 * VSTAGES + 3 * kSlots + 2 * QT + 2;
+    static constexpr int OFF_ONES2 = OFF_BIAS + QT * BIAS_BYTES;
+    static constexpr int OFF_BAR = OFF_ONES2 + ONES_BYTES;
+    static constexpr int NBARS = 1 + 2 * KSTAGES + 2 * VSTAGES + 4 * kSlots + 2 * QT + 2;
     static constexpr int OFF_MISC = OFF_BAR + NBARS * 8;
     static constexpr int SMEM_BYTES = OFF_MISC + 16 + 1024;   // + alignment slack
     static_assert(SMEM_BYTES <= 227 * 1024, "shared memory budget");
@@ -120,6 +112,9 @@ struct Params {
     const __half *vop;        // [BH][kstride] D x 64 fp16 tiles (V^T, scaled)
     const int *vexp;          // [BH] power of two of the V scale
     const uint32_t *qbits;    // [BH][n][D/32] packed query signs (1 = -1)
+    const uint32_t *kbits;    // [BH][n][D/32] packed key signs (1 = -1)
+    const void *v;            // [BH][n][D] the values as given (bf16 or f32)
+    int v_f32;                // 1: v is f32, 0: bf16
     const int *ksum;          // [BH][D] sum over the head's keys of the +/-1 codes
     float *out;               // [BH][n][D]
     int32_t *dbg_idx;         // [BH][n][N] or null
@@ -138,13 +133,15 @@ struct Params {
 };
 
 // Bounded wait: false if the deadline passed or another role aborted.  The
-// deadline is checked after the first failed try and every 256 after it.
+// abort flag and the deadline are checked every 32 failed tries (each try
+// may suspend the thread for a while); reading the global timer on every
+// failed try measurably slowed the issuing threads.
 __device__ __forceinline__ bool wait_bar(uint64_t *bar, uint32_t parity, uint64_t deadline,
                                          volatile int *abort_flag, int32_t *status)
 {
     uint32_t spins = 0;
     while (!tc::mbar_try_wait(bar, parity)) {
-        if ((spins++ & 255u) == 0) {
+        if ((++spins & 31u) == 0) {
             if (*abort_flag) return false;
             if (tc::globaltimer_ns() > deadline) {
                 *abort_flag = 1;
@@ -164,30 +161,13 @@ __device__ __forceinline__ float ex2(float x)
 }
 
 // Thermometer increment of the four 8-bit window counters for a logit whose
-// first counter is 8 * amount bits up (amount <= 0: all four counters;
-// >= 32: none): the high word of 0x01010101:0 shifted left by the amount,
-// clamped at 32.
-__device__ __forceinline__ uint32_t window_inc(int amount)
+// first counter is 8 * amount bits up, amount = v + shift (amount <= 0: all
+// four counters; >= 32: none): the high word of 0x01010101:0 shifted left by
+// the amount, clamped at 32 (the add and the clamp at 0 are one instruction).
+__device__ __forceinline__ uint32_t window_inc(int v, int shift)
 {
-    return __funnelshift_lc(0u, 0x01010101u, (uint32_t)max(amount, 0));
+    return __funnelshift_lc(0u, 0x01010101u, (uint32_t)__viaddmax_s32(v, shift, 0));
 }
-
-// Barrier of the epilogue warps only (named barrier 1).
-__device__ __forceinline__ void epi_sync(int nthreads)
-{
-    asm volatile("bar.sync 1, %0;" ::"r"(nthreads) : "memory");
-}
-
-// Per-row state handed from pass 1 to pass 2 at the row's new position.
-struct RowState {
-    int row;          // query index within the head
-    int t;            // threshold level (-1: the fix-up kernel recomputes the row)
-    int zero_at;      // key tile from which level t weighs nothing
-    int jstar;        // key tile where the tie quota runs out (-1: none)
-    int kstar;        // ties kept inside it
-    int quota;        // ties kept in all (for the key-by-key mode)
-    int pad[2];
-};
 
 // Make this thread's generic-proxy shared-memory writes visible to the
 // tensor core (async proxy).
@@ -216,10 +196,10 @@ attention_tc_kernel(const Params p)
     uint64_t *const s_full = v_empty + C::VSTAGES;     // [kSlots] S tile in the slot
     uint64_t *const s_free = s_full + kSlots;          // [kSlots] pass-1 slot read
     uint64_t *const p_full = s_free + kSlots;          // [kSlots] pass-2 P in the slot
-    uint64_t *const q2_ready = p_full + kSlots;        // [QT] Q tile rewritten for pass 2
+    uint64_t *const pv_done = p_full + kSlots;         // [kSlots] the P V reading it done
+    uint64_t *const q2_ready = pv_done + kSlots;       // [QT] Q tile rewritten for pass 2
     uint64_t *const o_full = q2_ready + QT;            // [QT] last P V of the tile done
-    uint64_t *const drain = o_full + QT;
-    uint64_t *const bias_ready = drain + 1;            // bias rows and ones tile written
+    uint64_t *const drain = o_full + QT;               // [2] each issuer's MMAs done
     uint32_t *tmem_holder = reinterpret_cast<uint32_t *>(smem + C::OFF_MISC);
     volatile int *abort_flag = reinterpret_cast<volatile int *>(smem + C::OFF_MISC + 4);
 
@@ -246,15 +226,14 @@ attention_tc_kernel(const Params p)
             tc::mbar_init(s_full + s, 1);
             tc::mbar_init(s_free + s, 4);               // the four warps of the tile
             tc::mbar_init(p_full + s, 4);
+            tc::mbar_init(pv_done + s, 1);
         }
         for (int g = 0; g < QT; ++g) {
             tc::mbar_init(q2_ready + g, 4);
             tc::mbar_init(o_full + g, 1);
         }
         tc::mbar_init(drain, 1);
-        tc::mbar_init(bias_ready, C::EPI_WARPS);
-        int *buckets = reinterpret_cast<int *>(smem + C::OFF_SORT);
-        for (int b = 0; b < C::SORT_BUCKETS; ++b) buckets[b] = 0;
+        tc::mbar_init(drain + 1, 1);
         *abort_flag = 0;
         tc::fence_mbar_init();
     }
@@ -309,116 +288,162 @@ attention_tc_kernel(const Params p)
             }
         }
     } else if (warp == 1) {
-        // ------------------------------------------------------------ MMA issuer
+        // ------------------------------------------------------------ Q K^T issuer
+        // The loop keeps every ring position and phase in counters and every
+        // descriptor precomputed: this thread shares its scheduler with
+        // epilogue warps, so each instruction between two MMAs costs.
         if (lane == 0) {
-            // Descriptors are built once; a tile, stage or K step moves only
-            // the start-address field (16-byte units).
-            const uint64_t dq = tc::smem_desc(tc::smem_u32(smem + C::OFF_Q), 128, D * 8);
-            const uint64_t dk = tc::smem_desc(tc::smem_u32(smem + C::OFF_K), 128, D * 8);
-            const uint64_t dv = tc::smem_desc(tc::smem_u32(smem + C::OFF_V), 128, 8 * 128);
-            // the bias step: K extent 32 bytes (two core matrices), rows 256 B apart
-            const uint64_t dbias = tc::smem_desc(tc::smem_u32(smem + C::OFF_BIAS), 128, 256);
-            const uint64_t dones = tc::smem_desc(tc::smem_u32(smem + C::OFF_ONES), 128, 256);
+            uint64_t dq[QT], dbias[QT];
+#pragma unroll
+            for (int g = 0; g < QT; ++g) {
+                dq[g] = tc::smem_desc(tc::smem_u32(smem + C::OFF_Q + g * C::QBYTES), 128, D * 8);
+                // the bias step: K extent 32 bytes (two core matrices), rows 256 B apart
+                dbias[g] = tc::smem_desc(tc::smem_u32(smem + C::OFF_BIAS + g * C::BIAS_BYTES),
+                                         128, 256);
+            }
+            const uint64_t dk0 = tc::smem_desc(tc::smem_u32(smem + C::OFF_K), 128, D * 8);
+            uint64_t dk = dk0;          // descriptor of the current K stage
             const uint64_t dones2 = tc::smem_desc(tc::smem_u32(smem + C::OFF_ONES2), 128, 256);
             bool ok = wait_bar(q_full, 0, deadline, abort_flag, p.status);
             tc::fence_after_sync();
-            // S tile kidx = S = Q_g K_u^T into slot kidx % 3; G is the K stream
-            // entry that holds key tile u (the stage is waited for at g = 0 and
-            // released after the last query tile's MMAs).
-            // bias: 0 none, 1 the pass-1 window offset, 2 the pass-2 table offset.
-            // synced: a barrier that epilogue threads arrive on was just waited
-            // for, so their prior TMEM and shared-memory work must be ordered
-            // before these MMAs (a fence); the copy barriers (async proxy, like
-            // the MMA) and the in-order reuse of a slot after its P V need none.
-            auto qk = [&](int kidx, int g, int G, int bias, bool synced) -> bool {
-                const int ks = G % C::KSTAGES;
-                if (g == 0 &&
-                    !wait_bar(k_full + ks, (G / C::KSTAGES) & 1, deadline, abort_flag, p.status))
-                    return false;
-                if (synced) tc::fence_after_sync();
-                const uint64_t dqa = dq + (uint64_t)((g * C::QBYTES) >> 4);
-                const uint64_t dkb = dk + (uint64_t)((ks * C::KBYTES) >> 4);
-                const uint32_t dcol = tmem + (kidx % kSlots) * kKeys;
+            int ks = 0;                 // K stage of the current key tile
+            uint32_t kph = 0;           // its fill phase
+            int sl = 0;                 // S slot of tile kidx (kidx % 3)
+            int wrap = 0;               // kidx / 3
+            int kidx = 0;
+            // S tile kidx = Q_g K^T of the current stage into slot sl; every
+            // wait before it is on a barrier that other threads arrive on, so
+            // a fence orders their prior TMEM and shared-memory work first.
+            auto issue = [&](int g, bool bias) {
+                tc::fence_after_sync();
+                const uint32_t dcol = tmem + sl * kKeys;
 #pragma unroll
                 for (int kk = 0; kk < D / 32; ++kk)
-                    tc::mma_i8_ss(dcol, dqa + (uint64_t)(kk * 16), dkb + (uint64_t)(kk * 16),
+                    tc::mma_i8_ss(dcol, dq[g] + (uint64_t)(kk * 16), dk + (uint64_t)(kk * 16),
                                   C::IDESC_QK, kk > 0 ? 1u : 0u);
-                if (bias)
-                    tc::mma_i8_ss(dcol, dbias + (uint64_t)((g * C::BIAS_BYTES) >> 4),
-                                  bias == 1 ? dones : dones2, C::IDESC_QK, 1u);
-                tc::mma_commit(s_full + kidx % kSlots);
-                if (g == QT - 1) tc::mma_commit(k_empty + ks);
-                return true;
+                if (bias) tc::mma_i8_ss(dcol, dbias[g], dones2, C::IDESC_QK, 1u);
+                tc::mma_commit(s_full + sl);
+                ++kidx;
+                if (++sl == kSlots) {
+                    sl = 0;
+                    ++wrap;
+                }
             };
-            // pass 1: slot reuse waits for the epilogue to have read tile kidx - 3;
-            // key tiles after the first add the rows' bias (written once the
-            // first tile has placed each row's window)
-            for (int kidx = 0; kidx < J && ok; ++kidx) {
-                if (kidx >= kSlots &&
-                    !wait_bar(s_free + kidx % kSlots, ((kidx - kSlots) / kSlots) & 1, deadline,
-                              abort_flag, p.status)) {
-                    ok = false;
-                    break;
-                }
-                if (kidx == QT && !wait_bar(bias_ready, 0, deadline, abort_flag, p.status)) {
-                    ok = false;
-                    break;
-                }
-                ok = qk(kidx, kidx % QT, kidx / QT, kidx >= QT ? 1 : 0,
-                        kidx >= kSlots || kidx == QT);
-            }
-            // pass 2: tile j of the pass is stream tile J + j
-            auto qk2 = [&](int j) -> bool {
-                const int kidx = J + j, u = j / QT, g = j % QT;
-                if (u == 0 && !wait_bar(q2_ready + g, 0, deadline, abort_flag, p.status))
-                    return false;
-                // the slot last held pass-1 tile kidx - 3 (if any): wait until read
-                const bool after_pass1 = kidx >= kSlots && kidx - kSlots < J;
-                if (after_pass1 &&
-                    !wait_bar(s_free + kidx % kSlots, ((kidx - kSlots) / kSlots) & 1, deadline,
-                              abort_flag, p.status))
-                    return false;
-                return qk(kidx, g, T + u, 2, u == 0 || after_pass1);
-            };
-            for (int j = 0; j < min(kSlots, J) && ok; ++j) ok = qk2(j);
-            for (int j = 0; j < J && ok; ++j) {
-                const int kidx = J + j, u = j / QT, g = j % QT;
-                const int vs = u % C::VSTAGES;
-                if (g == 0 &&
-                    !wait_bar(v_full + vs, (u / C::VSTAGES) & 1, deadline, abort_flag, p.status)) {
-                    ok = false;
-                    break;
-                }
-                if (!wait_bar(p_full + kidx % kSlots, (j / kSlots) & 1, deadline, abort_flag,
-                              p.status)) {
-                    ok = false;
-                    break;
-                }
-                tc::fence_after_sync();
-                const uint32_t pcol = tmem + (kidx % kSlots) * kKeys;   // P over S
-                const uint32_t ocol = tmem + C::O_COL + g * D;
-                const uint64_t dvs = dv + (uint64_t)((vs * C::VBYTES) >> 4);
+            // pass 1: slot reuse waits for the epilogue to have read tile kidx - 3
+            for (int u = 0; u < T && ok; ++u) {
+                ok = wait_bar(k_full + ks, kph, deadline, abort_flag, p.status);
 #pragma unroll
-                for (int c = 0; c < kKeys / 16; ++c) {
-                    const uint32_t boff = (uint32_t)((c >> 2) * C::VSUB + (c & 3) * 256);
-                    tc::mma_f16_ts(ocol, pcol + c * 8, dvs + (uint64_t)(boff >> 4), C::IDESC_PV,
-                                   (u > 0 || c > 0) ? 1u : 0u);
+                for (int g = 0; g < QT; ++g) {
+                    if (ok && kidx >= kSlots)
+                        ok = wait_bar(s_free + sl, (wrap - 1) & 1, deadline, abort_flag,
+                                      p.status);
+                    if (ok) issue(g, false);
                 }
-                if (g == QT - 1) tc::mma_commit(v_empty + vs);
-                if (u == T - 1) tc::mma_commit(o_full + g);
-                if (j + kSlots < J) ok = qk2(j + kSlots);
+                if (!ok) break;
+                tc::mma_commit(k_empty + ks);
+                dk += (uint64_t)(C::KBYTES >> 4);
+                if (++ks == C::KSTAGES) {
+                    ks = 0;
+                    kph ^= 1u;
+                    dk = dk0;
+                }
+            }
+            // before the first pass-2 MMA: every query tile's rewritten Q and
+            // bias rows, and the ones tile that all epilogue warps wrote
+            for (int g = 0; g < QT && ok; ++g)
+                ok = wait_bar(q2_ready + g, 0, deadline, abort_flag, p.status);
+            // pass 2 (tile j of the pass is stream tile J + j): the slot last
+            // held pass-1 tile J + j - 3 (read by the epilogue) or pass-2 tile
+            // j - 3 (read by its P V; pv_done of a slot completes once per
+            // pass-2 tile in it, the n-th time for tile 3 n + j % 3)
+            int j = 0, jw = 0, j3 = 0;  // j / 3 and j % 3
+            for (int u = 0; u < T && ok; ++u) {
+                ok = wait_bar(k_full + ks, kph, deadline, abort_flag, p.status);
+#pragma unroll
+                for (int g = 0; g < QT; ++g) {
+                    if (ok) {
+                        if (j >= kSlots)
+                            ok = wait_bar(pv_done + sl, (jw - 1) & 1, deadline, abort_flag,
+                                          p.status);
+                        else if (kidx >= kSlots)
+                            ok = wait_bar(s_free + sl, (wrap - 1) & 1, deadline, abort_flag,
+                                          p.status);
+                    }
+                    if (ok) issue(g, true);
+                    ++j;
+                    if (++j3 == kSlots) {
+                        j3 = 0;
+                        ++jw;
+                    }
+                }
+                if (!ok) break;
+                tc::mma_commit(k_empty + ks);
+                dk += (uint64_t)(C::KBYTES >> 4);
+                if (++ks == C::KSTAGES) {
+                    ks = 0;
+                    kph ^= 1u;
+                    dk = dk0;
+                }
             }
             // drain: wait until every MMA this thread issued has completed
             tc::mma_commit(drain);
             volatile int never = 0;
             wait_bar(drain, 0, tc::globaltimer_ns() + kDrainNs, &never, p.status);
         }
+    } else if (warp == 2) {
+        // ------------------------------------------------------------ P V issuer
+        if (lane == 0) {
+            const uint64_t dv0 = tc::smem_desc(tc::smem_u32(smem + C::OFF_V), 128, 8 * 128);
+            uint64_t dv = dv0;          // descriptor of the current V stage
+            bool ok = true;
+            int vs = 0;                 // V stage of the current key tile
+            uint32_t vph = 0;           // its fill phase
+            int sl = J % kSlots;        // slot of pass-2 tile j
+            int jw = 0, j3 = 0;         // j / 3 and j % 3: p_full of the slot completes the
+                                        // (j / 3)-th time for tile j
+            for (int u = 0; u < T && ok; ++u) {
+                ok = wait_bar(v_full + vs, vph, deadline, abort_flag, p.status);
+#pragma unroll
+                for (int g = 0; g < QT; ++g) {
+                    if (ok) ok = wait_bar(p_full + sl, jw & 1, deadline, abort_flag, p.status);
+                    if (ok) {
+                        tc::fence_after_sync();
+                        const uint32_t pcol = tmem + sl * kKeys;   // P over S
+                        const uint32_t ocol = tmem + C::O_COL + g * D;
+#pragma unroll
+                        for (int c = 0; c < kKeys / 16; ++c) {
+                            const uint32_t boff = (uint32_t)((c >> 2) * C::VSUB + (c & 3) * 256);
+                            tc::mma_f16_ts(ocol, pcol + c * 8, dv + (uint64_t)(boff >> 4),
+                                           C::IDESC_PV, (u > 0 || c > 0) ? 1u : 0u);
+                        }
+                        tc::mma_commit(pv_done + sl);
+                        if (u == T - 1) tc::mma_commit(o_full + g);
+                    }
+                    if (++sl == kSlots) sl = 0;
+                    if (++j3 == kSlots) {
+                        j3 = 0;
+                        ++jw;
+                    }
+                }
+                if (!ok) break;
+                tc::mma_commit(v_empty + vs);
+                dv += (uint64_t)(C::VBYTES >> 4);
+                if (++vs == C::VSTAGES) {
+                    vs = 0;
+                    vph ^= 1u;
+                    dv = dv0;
+                }
+            }
+            tc::mma_commit(drain + 1);
+            volatile int never = 0;
+            wait_bar(drain + 1, 0, tc::globaltimer_ns() + kDrainNs, &never, p.status);
+        }
     } else {
         // ------------------------------------------------------------ epilogue
         using BT = std::integral_constant<bool, true>;
         using BF = std::integral_constant<bool, false>;
         constexpr int NT = C::EPI_WARPS * 32;
-        const int g = (warp - 2) >> 2;                // query tile of this warp
+        const int g = (warp - C::EPI_WARP0) >> 2;     // query tile of this warp
         const int quarter = warp & 3;                 // TMEM lanes 32*quarter ...
         const int r = quarter * 32 + lane;            // row (TMEM lane) within the tile
         const int f = g * kRows + r;                  // position among the CTA's rows
@@ -470,8 +495,7 @@ attention_tc_kernel(const Params p)
         // ---------------------------------------------------------- window
         // Spread of the first key tile's logits (v = -4 s) -> estimated
         // threshold level est; counters cover levels L0 - 1 .. L0 + 2 with
-        // L0 = est - 1, and a logit's counter shift is cshift + v: the bias
-        // step adds cshift on the tensor core from the second key tile on.
+        // L0 = est - 1, and a logit's counter shift is cshift + v.
         int cshift = 0, L0 = 0;
         if (ok) ok = wait_s(g);
         if (ok) {
@@ -502,50 +526,23 @@ attention_tc_kernel(const Params p)
             L0 = est - 1;
             cshift = 4 * D - 8 * L0 + 8;              // 8 (level - L0 + 1) = cshift + v
         }
-        {
-            // this row's bias: 32 int8 values summing to cshift (each within
-            // one of cshift / 32), in the K-major layout of the bias step
-            const int qb = cshift / 32, rem = cshift - 32 * qb;
-            const int sgn = rem < 0 ? -1 : 1, nrem = rem < 0 ? -rem : rem;
-            uint32_t wb[8];
-#pragma unroll
-            for (int i = 0; i < 8; ++i) {
-                uint32_t word = 0;
-#pragma unroll
-                for (int b = 0; b < 4; ++b) {
-                    const int m = 4 * i + b;
-                    word |= (uint32_t)(uint8_t)(int8_t)(qb + (m < nrem ? sgn : 0)) << (8 * b);
-                }
-                wb[i] = word;
-            }
-            uint8_t *bt = smem + C::OFF_BIAS + g * C::BIAS_BYTES;
-#pragma unroll
-            for (int h = 0; h < 2; ++h)
-                *reinterpret_cast<uint4 *>(bt + ((r >> 3) * 2 + h) * 128 + (r & 7) * 16) =
-                    make_uint4(wb[4 * h], wb[4 * h + 1], wb[4 * h + 2], wb[4 * h + 3]);
-            // the constant tiles of the bias steps, shared by the query tiles:
-            // all ones (pass 1); per key 16 x 127 then 16 x 1 (pass 2), which
-            // in the K-major layout is core matrices of 127 then of 1
-            for (int i = f; i < C::ONES_BYTES / 16; i += NT) {
-                reinterpret_cast<uint4 *>(smem + C::OFF_ONES)[i] =
-                    make_uint4(0x01010101u, 0x01010101u, 0x01010101u, 0x01010101u);
-                const uint32_t x = ((i >> 3) & 1) ? 0x01010101u : 0x7F7F7F7Fu;
-                reinterpret_cast<uint4 *>(smem + C::OFF_ONES2)[i] = make_uint4(x, x, x, x);
-            }
-            fence_async_smem();
-            __syncwarp();
-            if (lane == 0) tc::mbar_arrive(bias_ready);
+        // the constant tile of the pass-2 bias step, shared by the query
+        // tiles: per key 16 x 127 then 16 x 1, which in the K-major layout is
+        // core matrices of 127 then of 1 (made visible to the tensor core by
+        // the fence before the pass-2 Q tiles are released)
+        for (int i = f; i < C::ONES_BYTES / 16; i += NT) {
+            const uint32_t x = ((i >> 3) & 1) ? 0x01010101u : 0x7F7F7F7Fu;
+            reinterpret_cast<uint4 *>(smem + C::OFF_ONES2)[i] = make_uint4(x, x, x, x);
         }
 
         // ---------------------------------------------------------- pass 1
         uint32_t acc[4] = {0u, 0u, 0u, 0u};
         int tot[4] = {0, 0, 0, 0};                    // the four counters over all tiles
-        // off = cshift for the first key tile (no bias step), 0 after it
-        auto therm = [&](const uint32_t (&rr)[32], int valid, int off, auto masked) {
+        auto therm = [&](const uint32_t (&rr)[32], int valid, auto masked) {
 #pragma unroll
             for (int c = 0; c < 32; ++c)
                 if (!decltype(masked)::value || c < valid)
-                    acc[c & 3] += window_inc(off + (int)rr[c]);
+                    acc[c & 3] += window_inc((int)rr[c], cshift);
         };
         auto end_tile1 = [&](int u) {
             const uint32_t w = (acc[0] + acc[1]) + (acc[2] + acc[3]);   // fields <= 128
@@ -555,18 +552,17 @@ attention_tc_kernel(const Params p)
             if (stash_ok) tc::tmem_st1(stash + u, w);
         };
         // one key tile; chunk 0 is in ra on entry, the next tile's chunk 0
-        // on exit; first: no bias step (add cshift); masked: padding keys
-        auto p1_tile = [&](int u, auto first, auto masked) {
+        // on exit; masked: padding keys
+        auto p1_tile = [&](int u, auto masked) {
             const int kidx = u * QT + g;
-            const int off = decltype(first)::value ? cshift : 0;
             ld(kidx, 1, rb);
-            therm(ra, chunk_valid(u, 0), off, masked);
+            therm(ra, chunk_valid(u, 0), masked);
             tc::tmem_wait_ld(rb);
             ld(kidx, 2, ra);
-            therm(rb, chunk_valid(u, 1), off, masked);
+            therm(rb, chunk_valid(u, 1), masked);
             tc::tmem_wait_ld(ra);
             ld(kidx, 3, rb);
-            therm(ra, chunk_valid(u, 2), off, masked);
+            therm(ra, chunk_valid(u, 2), masked);
             tc::tmem_wait_ld(rb);
             release_s(kidx);
             const bool more = u + 1 < T;
@@ -574,18 +570,18 @@ attention_tc_kernel(const Params p)
                 ok = wait_s(kidx + QT);
                 if (ok) ld(kidx + QT, 0, ra);
             }
-            therm(rb, chunk_valid(u, 3), off, masked);
+            therm(rb, chunk_valid(u, 3), masked);
             end_tile1(u);
             if (more && ok) tc::tmem_wait_ld(ra);
         };
         if (ok) {
             ld(g, 0, ra);
             tc::tmem_wait_ld(ra);
-            p1_tile(0, BT{}, BT{});
+            p1_tile(0, BT{});
         }
 #pragma unroll 1
-        for (int u = 1; u < T_full && ok; ++u) p1_tile(u, BF{}, BF{});
-        if (ok && T > T_full && T_full >= 1) p1_tile(T - 1, BF{}, BT{});
+        for (int u = 1; u < T_full && ok; ++u) p1_tile(u, BF{});
+        if (ok && T > T_full && T_full >= 1) p1_tile(T - 1, BT{});
 
         // threshold level t and the number q of keys kept at it
         const int f0 = tot[0], f1 = tot[1], f2 = tot[2], f3 = tot[3];
@@ -599,8 +595,10 @@ attention_tc_kernel(const Params p)
             miss = true;
         }
         // Where the tie quota runs out: ties are kept in full before tile
-        // jstar, kstar of them (the lowest indices) inside it, none after it;
-        // from tile zero_at on the weight table maps level t to 0.
+        // jstar, kstar of them (the lowest indices) inside it, none after it.
+        // From tile zero_at on the weight table maps level t to 0: the quota
+        // tile itself when the quota ends inside one (its kept ties are added
+        // after pass 2), else the tile after the last one kept in full.
         int zero_at = T, jstar = -1, kstar = 0;
         if (stash_ok && ok) {
             tc::tmem_wait_st();
@@ -621,7 +619,11 @@ attention_tc_kernel(const Params p)
                         if (cum + cnt >= quota) {
                             found = true;
                             zero_at = jj + 1;
-                            if (quota - cum < cnt) { jstar = jj; kstar = quota - cum; }
+                            if (quota - cum < cnt) {
+                                jstar = jj;
+                                kstar = quota - cum;
+                                zero_at = jj;
+                            }
                         }
                         cum += cnt;
                     }
@@ -636,63 +638,29 @@ attention_tc_kernel(const Params p)
         // missed rows keep nothing here; the fix-up kernel rewrites them
         if (miss) { t = -1; quota = 0; zero_at = T; jstar = -1; }
 
-        // ---------------------------------------------------------- regroup
-        // Rows move to new positions sorted by jstar, so that the 32 rows of
-        // a warp share few quota tiles (the only tiles that count ties key by
-        // key).  Every pass-1 MMA has completed: each warp has seen its
-        // tile's last pass-1 S before the first barrier.
-        RowState *state = reinterpret_cast<RowState *>(smem + C::OFF_STATE);
-        int *buckets = reinterpret_cast<int *>(smem + C::OFF_SORT);
-        const int key = (stash_ok && active1 && jstar >= 0) ? jstar + 1 : 0;
-        const int rank = atomicAdd(buckets + key, 1);
-        uint4 qrow[D / 16];                           // this row's pass-1 Q bytes
+        // ---------------------------------------------------------- Q for pass 2
+        // Every pass-1 MMA of this query tile has completed (this warp has
+        // seen its last S), so the tile's Q rows can be rewritten in place as
+        // -64 times the signs (64 times the negated signs): bytes 0xFF -> 0xC0,
+        // 0x01 -> 0x40.
         {
-            const uint8_t *qt = smem + C::OFF_Q + g * C::QBYTES;
-#pragma unroll
-            for (int kc = 0; kc < D / 16; ++kc)
-                qrow[kc] = *reinterpret_cast<const uint4 *>(
-                    qt + ((r >> 3) * (D / 16) + kc) * 128 + (r & 7) * 16);
-        }
-        epi_sync(NT);
-        if (f == 0) {                                 // exclusive prefix over the buckets
-            int run = 0;
-            for (int b = 0; b < C::SORT_BUCKETS; ++b) {
-                const int c = buckets[b];
-                buckets[b] = run;
-                run += c;
-            }
-        }
-        epi_sync(NT);
-        const int fnew = buckets[key] + rank;
-        {
-            RowState st;
-            st.row = row1;
-            st.t = t;
-            st.zero_at = zero_at;
-            st.jstar = jstar;
-            st.kstar = kstar;
-            st.quota = quota;
-            st.pad[0] = st.pad[1] = 0;
-            state[fnew] = st;
-            // the row's Q at its new position as -64 times the signs (64
-            // times the negated signs): bytes 0xFF -> 0xC0, 0x01 -> 0x40
-            const int gn = fnew / kRows, rn = fnew % kRows;
-            uint8_t *qt = smem + C::OFF_Q + gn * C::QBYTES;
+            uint8_t *qt = smem + C::OFF_Q + g * C::QBYTES;
 #pragma unroll
             for (int kc = 0; kc < D / 16; ++kc) {
-                uint4 x = qrow[kc];
+                uint4 *q4 = reinterpret_cast<uint4 *>(qt + ((r >> 3) * (D / 16) + kc) * 128 +
+                                                      (r & 7) * 16);
+                uint4 x = *q4;
                 x.x = (x.x << 6) & 0xC0C0C0C0u;
                 x.y = (x.y << 6) & 0xC0C0C0C0u;
                 x.z = (x.z << 6) & 0xC0C0C0C0u;
                 x.w = (x.w << 6) & 0xC0C0C0C0u;
-                *reinterpret_cast<uint4 *>(qt + ((rn >> 3) * (D / 16) + kc) * 128 +
-                                           (rn & 7) * 16) = x;
+                *q4 = x;
             }
         }
         {
-            // pass-2 bias of this thread's position: the byte offset of its
-            // table column's level 0 plus 256 D, as 127 * X + Y with X spread
-            // over the first 16 bias bytes and Y over the last 16
+            // pass-2 bias of this row: the byte offset of its table column's
+            // level 0 plus 256 D, as 127 * X + Y with X spread over the first
+            // 16 bias bytes and Y over the last 16
             const int hbv = g * C::TAB_BYTES + r * 4 + 256 * D;
             const int X = hbv / 127, Y = hbv - 127 * X;
             uint32_t wb[8];
@@ -714,33 +682,23 @@ attention_tc_kernel(const Params p)
                     make_uint4(wb[4 * h], wb[4 * h + 1], wb[4 * h + 2], wb[4 * h + 3]);
         }
         fence_async_smem();
-        epi_sync(NT);                                 // every row of every tile rewritten
         tc::fence_before_sync();
         __syncwarp();
         if (lane == 0) tc::mbar_arrive(q2_ready + g);
 
-        // this thread's pass-2 row: the one now at position f
-        const RowState st = state[f];
-        const int row = st.row;
-        const bool active = row < p.n;
-        t = st.t;
-        zero_at = st.zero_at;
-        jstar = st.jstar;
-        kstar = st.kstar;
+        const int row = row1;
+        const bool active = active1;
         // Weight table of the row, in this thread's own column (so the lanes
         // of a warp read distinct banks): level l holds exp2(c2 (s_l - ref))
         // for l <= t and 0 beyond.  ref is the threshold logit, raised where
         // needed so that no weight can exceed the fp16 range (s <= D).
         const int tab_off = g * C::TAB_BYTES + r * 4;
         float *tcol = reinterpret_cast<float *>(smem + C::OFF_TAB + tab_off);
-        {
-            const int headroom =
-                p.c2 > 1.0e-6f ? (int)fminf(floorf(15.99f / p.c2), 1.0e6f) : 1000000;
-            const int ref = max(D - 2 * max(t, 0), D - headroom);
-            for (int bin = 0; bin < C::BINS; ++bin)
-                tcol[bin * kRows] =
-                    bin <= t ? ex2(p.c2 * (float)(D - 2 * bin - ref)) : 0.0f;
-        }
+        const int headroom =
+            p.c2 > 1.0e-6f ? (int)fminf(floorf(15.99f / p.c2), 1.0e6f) : 1000000;
+        const int ref = max(D - 2 * max(t, 0), D - headroom);
+        for (int bin = 0; bin < C::BINS; ++bin)
+            tcol[bin * kRows] = bin <= t ? ex2(p.c2 * (float)(D - 2 * bin - ref)) : 0.0f;
         // The pass-2 accumulator holds a = hb - 256 s (the bias step adds
         // hb): level l = (D - s) / 2 sits l * 512 bytes past the column's
         // level 0, so a is the byte offset of the logit's weight in the tables.
@@ -749,7 +707,7 @@ attention_tc_kernel(const Params p)
         auto weight = [&](uint32_t a) { return *reinterpret_cast<const float *>(tab + a); };
 
         const uint32_t vt = (uint32_t)(hb - 256 * (D - 2 * t));   // accumulator of the threshold
-        int rem = st.quota;                           // ties still to keep (key-by-key mode)
+        int rem = quota;                              // ties still to keep (key-by-key mode)
         int kept = 0;
         float zacc[4] = {0.0f, 0.0f, 0.0f, 0.0f};
         const long long obase = ((head * p.n) + row) * (long long)p.N;
@@ -808,8 +766,11 @@ attention_tc_kernel(const Params p)
         auto p2_tile = [&](int u, bool masked) {
             const int kidx = J + u * QT + g;
             if (u == zero_at) tcol[t * kRows] = 0.0f;   // ties past the quota weigh nothing now
-            const bool slow = masked || !stash_ok || __any_sync(kFullMask, u == jstar);
-            int rl = !stash_ok ? rem : (u == jstar ? kstar : kAll);
+            // key by key only on the ragged last tile (keys past n) and in
+            // the mode without tile words; ties there follow the table (and,
+            // without tile words, the running quota)
+            const bool slow = masked || !stash_ok;
+            int rl = !stash_ok ? rem : kAll;
             uint32_t pk[16];
             const uint32_t pcol = lane_base + (kidx % kSlots) * kKeys;   // P over S
             ld(kidx, 1, rb);
@@ -824,10 +785,17 @@ attention_tc_kernel(const Params p)
             chunk2(u, 2, slow, ra, pk, rl);
             tc::tmem_st16(pcol + 32, pk);
             tc::tmem_wait_ld(rb);
+            // The next tile's first chunk is loaded here only if its S is
+            // already in, else after this P is released: releasing P never
+            // waits for the next S (whose slot may wait on the P V of the
+            // other query tile's last P).
             const bool more = u + 1 < T;
-            if (more) {
-                ok = wait_s(kidx + QT);
-                if (ok) ld(kidx + QT, 0, ra);
+            const bool early = more && __all_sync(kFullMask, tc::mbar_test_wait(
+                                                                 s_full + (kidx + QT) % kSlots,
+                                                                 ((kidx + QT) / kSlots) & 1));
+            if (early) {
+                tc::fence_after_sync();
+                ld(kidx + QT, 0, ra);
             }
             chunk2(u, 3, slow, rb, pk, rl);
             if (!stash_ok) rem = rl;
@@ -835,7 +803,11 @@ attention_tc_kernel(const Params p)
             tc::tmem_wait_st();
             tc::fence_before_sync();
             __syncwarp();
-            if (ok && lane == 0) tc::mbar_arrive(p_full + kidx % kSlots);
+            if (lane == 0) tc::mbar_arrive(p_full + kidx % kSlots);
+            if (more && !early) {
+                ok = wait_s(kidx + QT);
+                if (ok) ld(kidx + QT, 0, ra);
+            }
             if (more && ok) tc::tmem_wait_ld(ra);
         };
         if (ok) ok = wait_s(J + g);
@@ -847,27 +819,203 @@ attention_tc_kernel(const Params p)
         for (int u = 0; u < T_full && ok; ++u) p2_tile(u, false);
         if (ok && T > T_full) p2_tile(T - 1, true);
         float Z = (zacc[0] + zacc[1]) + (zacc[2] + zacc[3]);
-        if (!(Z > 0.0f)) Z = 1.0f;                    // missed or inactive rows only
 
-        // output: O / Z * 2^e_h
-        if (ok)
-            ok = __all_sync(kFullMask, wait_bar(o_full + g, 0, deadline, abort_flag, p.status));
-        if (ok) {
-            tc::fence_after_sync();
-            const float scale = ldexpf(1.0f, p.vexp[head]) / Z;
-            float *orow = p.out + ((head * p.n) + row) * (long long)D;
+        // ---------------------------------------------------------- quota tile
+        // The kstar kept ties of tile jstar are its first keys at level t in
+        // key order (level = Hamming distance of the packed signs); they add
+        // w_t V_j to the output and w_t each to Z.  The 32 rows of a warp are
+        // served together so that every global load is coalesced: the sign
+        // words of one row's quota tile (lane = key within a 32-key word),
+        // then one value row per kept key (lane = column pair).
+        const bool has_quota = ok && jstar >= 0 && active;
+        const float wq = has_quota ? ex2(p.c2 * (float)(D - 2 * t - ref)) : 0.0f;
+        if (has_quota) Z += wq * (float)kstar;
+        if (!(Z > 0.0f)) Z = 1.0f;                    // missed or inactive rows only
+        constexpr int DW = D / 32;                    // sign words per key
+        uint32_t keep[4] = {0u, 0u, 0u, 0u};          // bit i of word c: key 32 c + i of tile jstar
+        const uint32_t qlanes = __ballot_sync(kFullMask, has_quota);
+        if (qlanes) {
+            uint32_t qw[DW];
 #pragma unroll
-            for (int c0 = 0; c0 < D; c0 += 32) {
+            for (int w = 0; w < DW; ++w)
+                qw[w] = has_quota ? __ldg(p.qbits + ((head * p.n) + row) * DW + w) : 0u;
+            const uint32_t *kbh = p.kbits + head * p.n * (long long)DW;
+            constexpr int LPR = D == 64 ? 8 : 4;      // rows per round, their loads in flight together
+            uint32_t todo = qlanes;
+            while (todo) {                            // warp-uniform
+                int Ls[LPR];
+#pragma unroll
+                for (int e = 0; e < LPR; ++e) {
+                    Ls[e] = todo ? __ffs(todo) - 1 : -1;
+                    todo &= todo - 1u;
+                }
+                uint32_t kw[LPR][4][DW];
+#pragma unroll
+                for (int e = 0; e < LPR; ++e) {
+                    const int jl = __shfl_sync(kFullMask, jstar, max(Ls[e], 0));
+#pragma unroll
+                    for (int k = 0; k < 4; ++k) {
+                        const long long key = min(jl * kKeys + 32 * k + lane, p.n - 1);
+                        if (DW == 2) {
+                            const uint2 x = __ldg(reinterpret_cast<const uint2 *>(kbh + key * DW));
+                            kw[e][k][0] = x.x;
+                            kw[e][k][DW - 1] = x.y;
+                        } else {
+                            const uint4 x = __ldg(reinterpret_cast<const uint4 *>(kbh + key * DW));
+                            kw[e][k][0] = x.x;
+                            kw[e][k][1 % DW] = x.y;
+                            kw[e][k][2 % DW] = x.z;
+                            kw[e][k][3 % DW] = x.w;
+                        }
+                    }
+                }
+#pragma unroll
+                for (int e = 0; e < LPR; ++e) {
+                    const int L = Ls[e];
+                    if (L < 0) break;
+                    const int jl = __shfl_sync(kFullMask, jstar, L);
+                    const int tl = __shfl_sync(kFullMask, t, L);
+                    uint32_t ql[DW];
+#pragma unroll
+                    for (int w = 0; w < DW; ++w) ql[w] = __shfl_sync(kFullMask, qw[w], L);
+#pragma unroll
+                    for (int k = 0; k < 4; ++k) {
+                        int ham = 0;
+#pragma unroll
+                        for (int w = 0; w < DW; ++w) ham += __popc(ql[w] ^ kw[e][k][w]);
+                        const bool tie = ham == tl && jl * kKeys + 32 * k + lane < p.n;
+                        const uint32_t bits = __ballot_sync(kFullMask, tie);
+                        if (lane == L) keep[k] = bits;
+                    }
+                }
+            }
+            // the first kstar of the ties
+            int need = has_quota ? kstar : 0;
+#pragma unroll
+            for (int k = 0; k < 4; ++k) {
+                const int cnt = __popc(keep[k]);
+                if (need <= 0) {
+                    keep[k] = 0u;
+                } else if (cnt > need) {
+                    const int cut = __fns(keep[k], 0, need + 1);   // position of tie need + 1
+                    keep[k] &= (1u << cut) - 1u;
+                    need = 0;
+                } else {
+                    need -= cnt;
+                }
+            }
+        }
+
+        // output: (O 2^e_h + w_t sum of the quota tile's kept V) / Z, in
+        // halves of 64 columns.  The kept-V sums are gathered per round (each
+        // row with kept keys left gives its next one; lane i loads columns
+        // 2i, 2i+1 of the half from each of those value rows) and transposed
+        // through this warp's own bytes of the weight table, which pass 2 no
+        // longer reads: row L, pair p sits in bin 2L + p / 16 at pair slot
+        // (p ^ L) mod 16, so that both the writes and the reads spread over
+        // the banks.
+        const float scale = ok ? ldexpf(1.0f, p.vexp[head]) / Z : 0.0f;
+        const float qscale = wq / Z;
+        float *orow = p.out + ((head * p.n) + row) * (long long)D;
+        uint8_t *vt_base = smem + C::OFF_TAB + g * C::TAB_BYTES + quarter * 128;
+        auto vslot = [&](int L, int pr) -> float2 * {
+            return reinterpret_cast<float2 *>(vt_base + (2 * L + pr / 16) * (kRows * 4) +
+                                              ((pr ^ L) & 15) * 8);
+        };
+#pragma unroll 1
+        for (int h = 0; h < D / 64 && ok; ++h) {
+            float vq[64];
+#pragma unroll
+            for (int c = 0; c < 64; ++c) vq[c] = 0.0f;
+            if (qlanes) {
+                float2 acc[32];
+#pragma unroll
+                for (int L = 0; L < 32; ++L) acc[L] = make_float2(0.0f, 0.0f);
+                uint32_t m[4] = {keep[0], keep[1], keep[2], keep[3]};
+                const long long col = 64 * h + 2 * lane;
+                while (__any_sync(kFullMask, (m[0] | m[1] | m[2] | m[3]) != 0u)) {
+                    int mykey = -1;
+#pragma unroll
+                    for (int k = 0; k < 4; ++k) {
+                        if (mykey < 0 && m[k] != 0u) {
+                            mykey = jstar * kKeys + 32 * k + __ffs(m[k]) - 1;
+                            m[k] &= m[k] - 1u;
+                        }
+                    }
+                    // all sixteen loads of a batch are issued before any is used
+                    // (a key of -1 loads row 0 and adds nothing)
+                    if (p.v_f32) {
+                        const float *vb = static_cast<const float *>(p.v) + col;
+#pragma unroll
+                        for (int L0 = 0; L0 < 32; L0 += 16) {
+                            int key[16];
+                            float2 x[16];
+#pragma unroll
+                            for (int e = 0; e < 16; ++e) {
+                                key[e] = __shfl_sync(kFullMask, mykey, L0 + e);
+                                x[e] = __ldg(reinterpret_cast<const float2 *>(
+                                    vb + ((head * p.n) + max(key[e], 0)) * (long long)D));
+                            }
+#pragma unroll
+                            for (int e = 0; e < 16; ++e)
+                                if (key[e] >= 0) {
+                                    acc[L0 + e].x += x[e].x;
+                                    acc[L0 + e].y += x[e].y;
+                                }
+                        }
+                    } else {
+                        const uint16_t *vb = static_cast<const uint16_t *>(p.v) + col;
+#pragma unroll
+                        for (int L0 = 0; L0 < 32; L0 += 16) {
+                            int key[16];
+                            uint32_t x[16];
+#pragma unroll
+                            for (int e = 0; e < 16; ++e) {
+                                key[e] = __shfl_sync(kFullMask, mykey, L0 + e);
+                                x[e] = __ldg(reinterpret_cast<const uint32_t *>(
+                                    vb + ((head * p.n) + max(key[e], 0)) * (long long)D));
+                            }
+#pragma unroll
+                            for (int e = 0; e < 16; ++e)
+                                if (key[e] >= 0) {
+                                    acc[L0 + e].x += __uint_as_float(x[e] << 16);
+                                    acc[L0 + e].y += __uint_as_float(x[e] & 0xFFFF0000u);
+                                }
+                        }
+                    }
+                }
+                __syncwarp();
+#pragma unroll
+                for (int L = 0; L < 32; ++L) *vslot(L, lane) = acc[L];
+                __syncwarp();
+#pragma unroll
+                for (int pr = 0; pr < 32; ++pr) {
+                    const float2 v2 = *vslot(lane, pr);
+                    vq[2 * pr] = v2.x;
+                    vq[2 * pr + 1] = v2.y;
+                }
+                __syncwarp();
+            }
+            if (h == 0) {
+                ok = __all_sync(kFullMask,
+                                wait_bar(o_full + g, 0, deadline, abort_flag, p.status));
+                if (!ok) break;
+                tc::fence_after_sync();
+            }
+#pragma unroll
+            for (int c1 = 0; c1 < 64; c1 += 32) {
+                const int c0 = 64 * h + c1;
                 uint32_t o[32];
                 tc::tmem_ld32(lane_base + C::O_COL + g * D + c0, o);
                 tc::tmem_wait_ld(o);
                 if (active) {
 #pragma unroll
                     for (int c = 0; c < 32; c += 4) {
-                        float4 v = make_float4(__uint_as_float(o[c]) * scale,
-                                               __uint_as_float(o[c + 1]) * scale,
-                                               __uint_as_float(o[c + 2]) * scale,
-                                               __uint_as_float(o[c + 3]) * scale);
+                        float4 v = make_float4(
+                            fmaf(__uint_as_float(o[c]), scale, vq[c1 + c] * qscale),
+                            fmaf(__uint_as_float(o[c + 1]), scale, vq[c1 + c + 1] * qscale),
+                            fmaf(__uint_as_float(o[c + 2]), scale, vq[c1 + c + 2] * qscale),
+                            fmaf(__uint_as_float(o[c + 3]), scale, vq[c1 + c + 3] * qscale));
                         *reinterpret_cast<float4 *>(orow + c0 + c) = v;
                     }
                 }

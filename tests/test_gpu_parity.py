@@ -124,12 +124,15 @@ def _check_fused(had, c, rows):
     flat = lambda t: t.reshape(-1, t.shape[-1])[sel].cpu().numpy()
     assert np.array_equal(flat(dbg_idx), o_idx)
     assert np.array_equal(flat(dbg_lg), o_lg)
-    got = flat(out)
-    assert_close(got, o_out, "fused out")
-    # without the debug outputs the result is the same
+    assert_close(flat(out), o_out, "fused out (debug outputs on)")
+    # Without the debug outputs every full key tile takes the table path and
+    # the kept ties of a row's quota tile are added afterwards in fp32, so the
+    # rounding differs from the key-by-key debug path: both must match the
+    # oracle on their own.
     out2 = had.had_attention_fwd(c.gq, c.gk, c.gv, c.gsq, c.gsk, c.N, c.tau)
     torch.cuda.synchronize()
-    assert torch.equal(out, out2)
+    got = flat(out2)
+    assert_close(got, o_out, "fused out")
     err = np.abs(got.astype(np.float64) - o_out)
     rel = np.linalg.norm(got.astype(np.float64) - o_out) / max(np.linalg.norm(o_out), 1e-30)
     return float(err.max()), float(rel)
