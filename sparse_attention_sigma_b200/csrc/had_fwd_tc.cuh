@@ -39,13 +39,14 @@
 //
 // Warp roles: warp 0 bulk-copies the Q tiles once and streams K (twice) and
 // V^T (pass 2) through shared-memory rings.  One thread of warp 1 issues the
-// Q K^T MMAs and one of warp 2 the P V MMAs (a thread can issue a tcgen05 MMA
-// only every few tens of cycles, so the two streams go out in parallel).  S
+// Q K^T MMAs and one thread of warp 2 + g the P V MMAs of query tile g (a
+// thread that shares its scheduler with epilogue warps issues a tcgen05
+// instruction only every ~100 cycles, so the streams go out in parallel).  S
 // tiles use a ring of three 128-column TMEM slots shared by the query tiles
 // (S tile k of the stream sits in slot k % 3); tile k + 3 is issued into a
 // slot once the epilogue has released it (pass 1) or once the P V that reads
-// it has completed (pass 2).  Warps 3 .. 2 + 4 QT are the epilogue, four per
-// query tile.
+// it has completed (pass 2).  Warps 2 + QT .. 1 + 5 QT are the epilogue,
+// four per query tile.
 // Every wait is bounded by a caller-set limit: a CTA that hits it flags
 // HAD_ERR_TIMEOUT, lets its copies and MMAs drain, frees its TMEM and returns.
 #pragma once
@@ -71,7 +72,7 @@ template <int D>
 struct Cfg {
     static constexpr int QT = D == 64 ? HAD_TC_QT64 : 1;   // query tiles per CTA
     static constexpr int EPI_WARPS = 4 * QT;
-    static constexpr int EPI_WARP0 = 3;                // producer, QK issuer, PV issuer
+    static constexpr int EPI_WARP0 = 2 + QT;           // producer, Q K^T issuer, a P V issuer per query tile
     static constexpr int THREADS = 32 * (EPI_WARP0 + EPI_WARPS);
     static constexpr int QBYTES = kRows * D;            // int8 Q tile
     static constexpr int KBYTES = kKeys * D;            // int8 K tile (two workspace tiles)
@@ -98,7 +99,12 @@ struct Cfg {
     static constexpr int OFF_BIAS = OFF_TAB + QT * TAB_BYTES;
     static constexpr int OFF_ONES2 = OFF_BIAS + QT * BIAS_BYTES;
     static constexpr int OFF_BAR = OFF_ONES2 + ONES_BYTES;
-    static constexpr int NBARS = 1 + 2 * KSTAGES + 2 * VSTAGES + 4 * kSlots + 2 * QT + 2;
+    // the pass-2 bias (a shared address of the tables + 256 D, with up to 1 KB
+    // of alignment and a small window base below it) is 127 X + Y with
+    // X, Y <= 16 * 127
+    static_assert(OFF_TAB + QT * TAB_BYTES + 256 * D + 4096 < 127 * (16 * 127 + 1),
+                  "pass-2 bias range");
+    static constexpr int NBARS = 1 + 2 * KSTAGES + 2 * VSTAGES + (3 + QT) * kSlots + 3 * QT + 1;
     static constexpr int OFF_MISC = OFF_BAR + NBARS * 8;
     static constexpr int SMEM_BYTES = OFF_MISC + 16 + 1024;   // + alignment slack
     static_assert(SMEM_BYTES <= 227 * 1024, "shared memory budget");
@@ -195,11 +201,14 @@ attention_tc_kernel(const Params p)
     uint64_t *const v_empty = v_full + C::VSTAGES;
     uint64_t *const s_full = v_empty + C::VSTAGES;     // [kSlots] S tile in the slot
     uint64_t *const s_free = s_full + kSlots;          // [kSlots] pass-1 slot read
-    uint64_t *const p_full = s_free + kSlots;          // [kSlots] pass-2 P in the slot
-    uint64_t *const pv_done = p_full + kSlots;         // [kSlots] the P V reading it done
+    // [QT][kSlots] pass-2 P of query tile g in the slot: one barrier per
+    // (tile, slot), so that the P V issuer of a tile, which skips the other
+    // tile's S tiles, never waits on a phase more than one ahead
+    uint64_t *const p_full = s_free + kSlots;
+    uint64_t *const pv_done = p_full + QT * kSlots;    // [kSlots] the P V reading it done
     uint64_t *const q2_ready = pv_done + kSlots;       // [QT] Q tile rewritten for pass 2
     uint64_t *const o_full = q2_ready + QT;            // [QT] last P V of the tile done
-    uint64_t *const drain = o_full + QT;               // [2] each issuer's MMAs done
+    uint64_t *const drain = o_full + QT;               // [1 + QT] each issuer's MMAs done
     uint32_t *tmem_holder = reinterpret_cast<uint32_t *>(smem + C::OFF_MISC);
     volatile int *abort_flag = reinterpret_cast<volatile int *>(smem + C::OFF_MISC + 4);
 
@@ -220,20 +229,19 @@ attention_tc_kernel(const Params p)
         }
         for (int s = 0; s < C::VSTAGES; ++s) {
             tc::mbar_init(v_full + s, 1);
-            tc::mbar_init(v_empty + s, 1);
+            tc::mbar_init(v_empty + s, QT);             // the P V issuer of every query tile
         }
         for (int s = 0; s < kSlots; ++s) {
             tc::mbar_init(s_full + s, 1);
             tc::mbar_init(s_free + s, 4);               // the four warps of the tile
-            tc::mbar_init(p_full + s, 4);
             tc::mbar_init(pv_done + s, 1);
         }
+        for (int s = 0; s < QT * kSlots; ++s) tc::mbar_init(p_full + s, 4);
         for (int g = 0; g < QT; ++g) {
             tc::mbar_init(q2_ready + g, 4);
             tc::mbar_init(o_full + g, 1);
         }
-        tc::mbar_init(drain, 1);
-        tc::mbar_init(drain + 1, 1);
+        for (int i = 0; i < 1 + QT; ++i) tc::mbar_init(drain + i, 1);
         *abort_flag = 0;
         tc::fence_mbar_init();
     }
@@ -390,43 +398,39 @@ attention_tc_kernel(const Params p)
             volatile int never = 0;
             wait_bar(drain, 0, tc::globaltimer_ns() + kDrainNs, &never, p.status);
         }
-    } else if (warp == 2) {
-        // ------------------------------------------------------------ P V issuer
+    } else if (warp < C::EPI_WARP0) {
+        // ------------------------------------------------------------ P V issuers
+        // one per query tile: O_g += P V for the tile's pass-2 S tiles
+        // (stream tiles J + u QT + g), so that the two streams of eight MMAs
+        // per key tile go out in parallel
         if (lane == 0) {
+            const int g = warp - 2;
             const uint64_t dv0 = tc::smem_desc(tc::smem_u32(smem + C::OFF_V), 128, 8 * 128);
             uint64_t dv = dv0;          // descriptor of the current V stage
+            const uint32_t ocol = tmem + C::O_COL + g * D;
             bool ok = true;
             int vs = 0;                 // V stage of the current key tile
             uint32_t vph = 0;           // its fill phase
-            int sl = J % kSlots;        // slot of pass-2 tile j
-            int jw = 0, j3 = 0;         // j / 3 and j % 3: p_full of the slot completes the
-                                        // (j / 3)-th time for tile j
-            for (int u = 0; u < T && ok; ++u) {
-                ok = wait_bar(v_full + vs, vph, deadline, abort_flag, p.status);
-#pragma unroll
-                for (int g = 0; g < QT; ++g) {
-                    if (ok) ok = wait_bar(p_full + sl, jw & 1, deadline, abort_flag, p.status);
-                    if (ok) {
-                        tc::fence_after_sync();
-                        const uint32_t pcol = tmem + sl * kKeys;   // P over S
-                        const uint32_t ocol = tmem + C::O_COL + g * D;
-#pragma unroll
-                        for (int c = 0; c < kKeys / 16; ++c) {
-                            const uint32_t boff = (uint32_t)((c >> 2) * C::VSUB + (c & 3) * 256);
-                            tc::mma_f16_ts(ocol, pcol + c * 8, dv + (uint64_t)(boff >> 4),
-                                           C::IDESC_PV, (u > 0 || c > 0) ? 1u : 0u);
-                        }
-                        tc::mma_commit(pv_done + sl);
-                        if (u == T - 1) tc::mma_commit(o_full + g);
-                    }
-                    if (++sl == kSlots) sl = 0;
-                    if (++j3 == kSlots) {
-                        j3 = 0;
-                        ++jw;
-                    }
-                }
+            int j = g;                  // pass-2 tile index
+            for (int u = 0; u < T && ok; ++u, j += QT) {
+                const int sl = (J + j) % kSlots;
+                // this tile's p_full of the slot completes the (u / 3)-th time
+                // for key tile u (its S tiles visit the three slots in turn)
+                ok = wait_bar(v_full + vs, vph, deadline, abort_flag, p.status) &&
+                     wait_bar(p_full + g * kSlots + sl, (u / kSlots) & 1, deadline, abort_flag,
+                              p.status);
                 if (!ok) break;
+                tc::fence_after_sync();
+                const uint32_t pcol = tmem + sl * kKeys;           // P over S
+#pragma unroll
+                for (int c = 0; c < kKeys / 16; ++c) {
+                    const uint32_t boff = (uint32_t)((c >> 2) * C::VSUB + (c & 3) * 256);
+                    tc::mma_f16_ts(ocol, pcol + c * 8, dv + (uint64_t)(boff >> 4), C::IDESC_PV,
+                                   (u > 0 || c > 0) ? 1u : 0u);
+                }
+                tc::mma_commit(pv_done + sl);
                 tc::mma_commit(v_empty + vs);
+                if (u == T - 1) tc::mma_commit(o_full + g);
                 dv += (uint64_t)(C::VBYTES >> 4);
                 if (++vs == C::VSTAGES) {
                     vs = 0;
@@ -434,9 +438,9 @@ attention_tc_kernel(const Params p)
                     dv = dv0;
                 }
             }
-            tc::mma_commit(drain + 1);
+            tc::mma_commit(drain + 1 + g);
             volatile int never = 0;
-            wait_bar(drain + 1, 0, tc::globaltimer_ns() + kDrainNs, &never, p.status);
+            wait_bar(drain + 1 + g, 0, tc::globaltimer_ns() + kDrainNs, &never, p.status);
         }
     } else {
         // ------------------------------------------------------------ epilogue
@@ -658,10 +662,10 @@ attention_tc_kernel(const Params p)
             }
         }
         {
-            // pass-2 bias of this row: the byte offset of its table column's
-            // level 0 plus 256 D, as 127 * X + Y with X spread over the first
-            // 16 bias bytes and Y over the last 16
-            const int hbv = g * C::TAB_BYTES + r * 4 + 256 * D;
+            // pass-2 bias of this row: the shared-memory address of its table
+            // column's level 0 plus 256 D, as 127 * X + Y with X spread over
+            // the first 16 bias bytes and Y over the last 16
+            const int hbv = (int)tc::smem_u32(smem + C::OFF_TAB) + g * C::TAB_BYTES + r * 4 + 256 * D;
             const int X = hbv / 127, Y = hbv - 127 * X;
             uint32_t wb[8];
 #pragma unroll
@@ -701,15 +705,18 @@ attention_tc_kernel(const Params p)
             tcol[bin * kRows] = bin <= t ? ex2(p.c2 * (float)(D - 2 * bin - ref)) : 0.0f;
         // The pass-2 accumulator holds a = hb - 256 s (the bias step adds
         // hb): level l = (D - s) / 2 sits l * 512 bytes past the column's
-        // level 0, so a is the byte offset of the logit's weight in the tables.
-        const uint8_t *tab = smem + C::OFF_TAB;
-        const int hb = tab_off + 256 * D;
-        auto weight = [&](uint32_t a) { return *reinterpret_cast<const float *>(tab + a); };
+        // level 0, so a is the shared-memory address of the logit's weight.
+        const int hb = (int)tc::smem_u32(smem + C::OFF_TAB) + tab_off + 256 * D;
+        const uint32_t sbase = tc::smem_u32(smem_raw);
+        auto weight = [&](uint32_t a) {
+            return *reinterpret_cast<const float *>(smem_raw + (a - sbase));
+        };
 
         const uint32_t vt = (uint32_t)(hb - 256 * (D - 2 * t));   // accumulator of the threshold
         int rem = quota;                              // ties still to keep (key-by-key mode)
         int kept = 0;
-        float zacc[4] = {0.0f, 0.0f, 0.0f, 0.0f};
+        float zacc[4] = {0.0f, 0.0f, 0.0f, 0.0f};      // key-by-key chunks
+        uint64_t zpair[2] = {0ull, 0ull};              // table chunks: pairs of f32 sums
         const long long obase = ((head * p.n) + row) * (long long)p.N;
         constexpr int kAll = 1 << 30;
 
@@ -719,8 +726,11 @@ attention_tc_kernel(const Params p)
             for (int c = 0; c < 32; c += 2) {
                 const float w0 = weight(rr[c]);
                 const float w1 = weight(rr[c + 1]);
-                zacc[c & 2] += w0;
-                zacc[(c & 2) + 1] += w1;
+                // both weights into one pair of sums with one packed add
+                asm("{\n\t.reg .b64 t;\n\tmov.b64 t, {%1, %2};\n\t"
+                    "add.rn.f32x2 %0, %0, t;\n\t}"
+                    : "+l"(zpair[(c >> 1) & 1])
+                    : "f"(w0), "f"(w1));
                 __half2 h2 = __floats2half2_rn(w0, w1);
                 pk[c >> 1] = *reinterpret_cast<uint32_t *>(&h2);
             }
@@ -803,7 +813,7 @@ attention_tc_kernel(const Params p)
             tc::tmem_wait_st();
             tc::fence_before_sync();
             __syncwarp();
-            if (lane == 0) tc::mbar_arrive(p_full + kidx % kSlots);
+            if (lane == 0) tc::mbar_arrive(p_full + g * kSlots + kidx % kSlots);
             if (more && !early) {
                 ok = wait_s(kidx + QT);
                 if (ok) ld(kidx + QT, 0, ra);
@@ -819,6 +829,9 @@ attention_tc_kernel(const Params p)
         for (int u = 0; u < T_full && ok; ++u) p2_tile(u, false);
         if (ok && T > T_full) p2_tile(T - 1, true);
         float Z = (zacc[0] + zacc[1]) + (zacc[2] + zacc[3]);
+#pragma unroll
+        for (int i = 0; i < 2; ++i)
+            Z += __uint_as_float((uint32_t)zpair[i]) + __uint_as_float((uint32_t)(zpair[i] >> 32));
 
         // ---------------------------------------------------------- quota tile
         // The kstar kept ties of tile jstar are its first keys at level t in
@@ -907,11 +920,10 @@ attention_tc_kernel(const Params p)
         }
 
         // output: (O 2^e_h + w_t sum of the quota tile's kept V) / Z, in
-        // halves of 64 columns.  The kept-V sums are gathered per round (each
-        // row with kept keys left gives its next one; lane i loads columns
-        // 2i, 2i+1 of the half from each of those value rows) and transposed
-        // through this warp's own bytes of the weight table, which pass 2 no
-        // longer reads: row L, pair p sits in bin 2L + p / 16 at pair slot
+        // halves of 64 columns.  Lane i loads columns 2i, 2i+1 of the half
+        // from each kept value row and adds them to that row's sums, kept in
+        // this warp's own bytes of the weight table (which pass 2 no longer
+        // reads): row L, pair p sits in bin 2L + p / 16 at pair slot
         // (p ^ L) mod 16, so that both the writes and the reads spread over
         // the banks.
         const float scale = ok ? ldexpf(1.0f, p.vexp[head]) / Z : 0.0f;
@@ -922,71 +934,75 @@ attention_tc_kernel(const Params p)
             return reinterpret_cast<float2 *>(vt_base + (2 * L + pr / 16) * (kRows * 4) +
                                               ((pr ^ L) & 15) * 8);
         };
+        // The warp's kept (row, key) pairs, numbered in lane order (lane L's
+        // are off_L .. off_L + kstar_L - 1, in key order), are listed in this
+        // warp's bytes of its query tile's Q (free once pass 2's Q K^T MMAs
+        // are done) and gathered sixteen value rows at a time.
+        const int nkeep = __popc(keep[0]) + __popc(keep[1]) + __popc(keep[2]) + __popc(keep[3]);
+        int off = nkeep;
+#pragma unroll
+        for (int dd = 1; dd < 32; dd <<= 1) {
+            const int y = __shfl_up_sync(kFullMask, off, dd);
+            if (lane >= dd) off += y;
+        }
+        const int total = __shfl_sync(kFullMask, off, 31);
+        off -= nkeep;
+        constexpr int kListCap = 8 * D;               // 32 rows x D bytes of Q
+        uint32_t *list = reinterpret_cast<uint32_t *>(smem + C::OFF_Q + g * C::QBYTES +
+                                                      quarter * 32 * D);
 #pragma unroll 1
         for (int h = 0; h < D / 64 && ok; ++h) {
             float vq[64];
 #pragma unroll
             for (int c = 0; c < 64; ++c) vq[c] = 0.0f;
-            if (qlanes) {
-                float2 acc[32];
+            if (total > 0) {
 #pragma unroll
-                for (int L = 0; L < 32; ++L) acc[L] = make_float2(0.0f, 0.0f);
-                uint32_t m[4] = {keep[0], keep[1], keep[2], keep[3]};
+                for (int L = 0; L < 32; ++L) *vslot(L, lane) = make_float2(0.0f, 0.0f);
                 const long long col = 64 * h + 2 * lane;
-                while (__any_sync(kFullMask, (m[0] | m[1] | m[2] | m[3]) != 0u)) {
-                    int mykey = -1;
+                for (int w0 = 0; w0 < total; w0 += kListCap) {
+                    const int w1 = min(total, w0 + kListCap);
+                    // this lane's pairs in the window, in key order
+                    __syncwarp();
+                    int idx = off;
 #pragma unroll
                     for (int k = 0; k < 4; ++k) {
-                        if (mykey < 0 && m[k] != 0u) {
-                            mykey = jstar * kKeys + 32 * k + __ffs(m[k]) - 1;
-                            m[k] &= m[k] - 1u;
-                        }
+                        for (uint32_t m = keep[k]; m != 0u && idx < w1; m &= m - 1u, ++idx)
+                            if (idx >= w0)
+                                list[idx - w0] = ((uint32_t)lane << 24) |
+                                                 (uint32_t)(jstar * kKeys + 32 * k + __ffs(m) - 1);
                     }
-                    // all sixteen loads of a batch are issued before any is used
-                    // (a key of -1 loads row 0 and adds nothing)
-                    if (p.v_f32) {
-                        const float *vb = static_cast<const float *>(p.v) + col;
+                    __syncwarp();
+                    // sixteen value rows per step, all loads issued before any is used
+                    for (int b0 = w0; b0 < w1; b0 += 16) {
+                        uint32_t ent[16];
+                        float2 x[16];
 #pragma unroll
-                        for (int L0 = 0; L0 < 32; L0 += 16) {
-                            int key[16];
-                            float2 x[16];
-#pragma unroll
-                            for (int e = 0; e < 16; ++e) {
-                                key[e] = __shfl_sync(kFullMask, mykey, L0 + e);
+                        for (int e = 0; e < 16; ++e) {
+                            ent[e] = b0 + e < w1 ? list[b0 + e - w0] : 0xFFFFFFFFu;
+                            const long long vr =
+                                ((head * p.n) + (b0 + e < w1 ? (ent[e] & 0xFFFFFFu) : 0u)) *
+                                    (long long)D + col;
+                            if (p.v_f32) {
                                 x[e] = __ldg(reinterpret_cast<const float2 *>(
-                                    vb + ((head * p.n) + max(key[e], 0)) * (long long)D));
+                                    static_cast<const float *>(p.v) + vr));
+                            } else {
+                                const uint32_t b2 = __ldg(reinterpret_cast<const uint32_t *>(
+                                    static_cast<const uint16_t *>(p.v) + vr));
+                                x[e] = make_float2(__uint_as_float(b2 << 16),
+                                                   __uint_as_float(b2 & 0xFFFF0000u));
                             }
-#pragma unroll
-                            for (int e = 0; e < 16; ++e)
-                                if (key[e] >= 0) {
-                                    acc[L0 + e].x += x[e].x;
-                                    acc[L0 + e].y += x[e].y;
-                                }
                         }
-                    } else {
-                        const uint16_t *vb = static_cast<const uint16_t *>(p.v) + col;
 #pragma unroll
-                        for (int L0 = 0; L0 < 32; L0 += 16) {
-                            int key[16];
-                            uint32_t x[16];
-#pragma unroll
-                            for (int e = 0; e < 16; ++e) {
-                                key[e] = __shfl_sync(kFullMask, mykey, L0 + e);
-                                x[e] = __ldg(reinterpret_cast<const uint32_t *>(
-                                    vb + ((head * p.n) + max(key[e], 0)) * (long long)D));
+                        for (int e = 0; e < 16; ++e)
+                            if (b0 + e < w1) {
+                                float2 *sl = vslot((int)(ent[e] >> 24), lane);
+                                float2 y = *sl;
+                                y.x += x[e].x;
+                                y.y += x[e].y;
+                                *sl = y;
                             }
-#pragma unroll
-                            for (int e = 0; e < 16; ++e)
-                                if (key[e] >= 0) {
-                                    acc[L0 + e].x += __uint_as_float(x[e] << 16);
-                                    acc[L0 + e].y += __uint_as_float(x[e] & 0xFFFF0000u);
-                                }
-                        }
                     }
                 }
-                __syncwarp();
-#pragma unroll
-                for (int L = 0; L < 32; ++L) *vslot(L, lane) = acc[L];
                 __syncwarp();
 #pragma unroll
                 for (int pr = 0; pr < 32; ++pr) {
