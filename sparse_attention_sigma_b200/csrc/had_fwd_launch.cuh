@@ -133,7 +133,13 @@ had_status_t core_tc(const void *V, bool v_f32, int B, int H, int n, int N, floa
     using C = tcfwd::Cfg<D>;
     const long long bh = (long long)B * H;
     const bool dbg = dbg_idx != nullptr || dbg_lg != nullptr;
-    auto kernel = dbg ? tcfwd::attention_tc_kernel<D, true> : tcfwd::attention_tc_kernel<D, false>;
+    // The quota tile's kept ties: with few key tiles a per-chunk mask in
+    // pass 2 costs less than gathering them after it (a fixed latency per
+    // CTA); with many, the other way round (measured crossover near 12).
+    const bool q2 = (n + tcfwd::kKeys - 1) / tcfwd::kKeys <= 12;
+    auto kernel = dbg  ? tcfwd::attention_tc_kernel<D, true, false>
+                  : q2 ? tcfwd::attention_tc_kernel<D, false, true>
+                       : tcfwd::attention_tc_kernel<D, false, false>;
     if (cudaFuncSetAttribute(kernel, cudaFuncAttributeMaxDynamicSharedMemorySize,
                              C::SMEM_BYTES) != cudaSuccess ||
         cudaFuncSetAttribute(kernel, cudaFuncAttributePreferredSharedMemoryCarveout,
@@ -148,6 +154,7 @@ had_status_t core_tc(const void *V, bool v_f32, int B, int H, int n, int N, floa
     p.kbits = reinterpret_cast<uint32_t *>(ws + w.kbits);
     p.v = V;
     p.v_f32 = v_f32 ? 1 : 0;
+
     p.ksum = reinterpret_cast<int *>(ws + w.ksum);
     p.out = out;
     p.dbg_idx = dbg_idx;

@@ -182,7 +182,9 @@ __device__ __forceinline__ void fence_async_smem()
     asm volatile("fence.proxy.async.shared::cta;" ::: "memory");
 }
 
-template <int D, bool kDbg>
+// kQ2: the quota tile's kept ties are masked in pass 2 (cheaper with few key
+// tiles) rather than gathered after it (cheaper with many).
+template <int D, bool kDbg, bool kQ2>
 __global__ void __launch_bounds__(Cfg<D>::THREADS, 1)
 attention_tc_kernel(const Params p)
 {
@@ -600,9 +602,9 @@ attention_tc_kernel(const Params p)
         }
         // Where the tie quota runs out: ties are kept in full before tile
         // jstar, kstar of them (the lowest indices) inside it, none after it.
-        // From tile zero_at on the weight table maps level t to 0: the quota
-        // tile itself when the quota ends inside one (its kept ties are added
-        // after pass 2), else the tile after the last one kept in full.
+        // From tile zero_at on the weight table maps level t to 0: the tile
+        // after the last one with kept ties, or, when the quota tile's kept
+        // ties are added after pass 2, the quota tile itself.
         int zero_at = T, jstar = -1, kstar = 0;
         if (stash_ok && ok) {
             tc::tmem_wait_st();
@@ -626,7 +628,7 @@ attention_tc_kernel(const Params p)
                             if (quota - cum < cnt) {
                                 jstar = jj;
                                 kstar = quota - cum;
-                                zero_at = jj;
+                                if (!kQ2) zero_at = jj;
                             }
                         }
                         cum += cnt;
@@ -713,6 +715,8 @@ attention_tc_kernel(const Params p)
         };
 
         const uint32_t vt = (uint32_t)(hb - 256 * (D - 2 * t));   // accumulator of the threshold
+        const float wt_tab = t >= 0 ? tcol[t * kRows] : 0.0f;       // the table's weight of level t
+        float zdrop = 0.0f;                           // weights of ties dropped after the table
         int rem = quota;                              // ties still to keep (key-by-key mode)
         int kept = 0;
         float zacc[4] = {0.0f, 0.0f, 0.0f, 0.0f};      // key-by-key chunks
@@ -772,6 +776,28 @@ attention_tc_kernel(const Params p)
             if (!slow) fast_chunk(rr, pk);
             else slow_chunk(u * kKeys + ch * 32, rr, pk, rl, chunk_valid(u, ch));
         };
+        // Quota tile: rl ties of this chunk may still be kept (the lowest
+        // indices); the table gave every tie its weight, so the ones past rl
+        // are set to 0 in P and taken out of Z.  No per-key dependency: the
+        // chunk's ties form a mask, the cut is the (rl+1)-th set bit.
+        auto drop_ties = [&](const uint32_t (&rr)[32], uint32_t (&pk)[16], int &rl) {
+            uint32_t m = 0;
+#pragma unroll
+            for (int c = 0; c < 32; ++c) m |= rr[c] == vt ? (1u << c) : 0u;
+            const int cnt = __popc(m);
+            uint32_t drop = 0;
+            if (rl <= 0) drop = m;
+            else if (rl < cnt) drop = m & ~((1u << __fns(m, 0, rl + 1)) - 1u);
+            rl = max(rl - cnt, 0);
+            if (__any_sync(kFullMask, drop != 0u)) {
+#pragma unroll
+                for (int i = 0; i < 16; ++i) {
+                    const uint32_t b = (drop >> (2 * i)) & 3u;
+                    pk[i] &= ~(((b & 1u) ? 0x0000FFFFu : 0u) | ((b & 2u) ? 0xFFFF0000u : 0u));
+                }
+                zdrop += wt_tab * (float)__popc(drop);
+            }
+        };
         // one key tile; chunk 0 is in ra on entry, the next tile's in ra on exit
         auto p2_tile = [&](int u, bool masked) {
             const int kidx = J + u * QT + g;
@@ -780,19 +806,26 @@ attention_tc_kernel(const Params p)
             // the mode without tile words; ties there follow the table (and,
             // without tile words, the running quota)
             const bool slow = masked || !stash_ok;
-            int rl = !stash_ok ? rem : kAll;
+            int rl = !stash_ok ? rem : (kQ2 && u == jstar ? kstar : kAll);
+            // some row of the warp has its quota tile here (pass-2 mode):
+            // every chunk also drops that row's ties past its quota
+            const bool quota_tile =
+                !slow && kQ2 && __any_sync(kFullMask, u == jstar);
             uint32_t pk[16];
             const uint32_t pcol = lane_base + (kidx % kSlots) * kKeys;   // P over S
             ld(kidx, 1, rb);
             chunk2(u, 0, slow, ra, pk, rl);
+            if (quota_tile) drop_ties(ra, pk, rl);
             tc::tmem_st16(pcol, pk);                  // S columns 0-15 are already read
             tc::tmem_wait_ld(rb);
             ld(kidx, 2, ra);
             chunk2(u, 1, slow, rb, pk, rl);
+            if (quota_tile) drop_ties(rb, pk, rl);
             tc::tmem_st16(pcol + 16, pk);
             tc::tmem_wait_ld(ra);
             ld(kidx, 3, rb);
             chunk2(u, 2, slow, ra, pk, rl);
+            if (quota_tile) drop_ties(ra, pk, rl);
             tc::tmem_st16(pcol + 32, pk);
             tc::tmem_wait_ld(rb);
             // The next tile's first chunk is loaded here only if its S is
@@ -808,6 +841,7 @@ attention_tc_kernel(const Params p)
                 ld(kidx + QT, 0, ra);
             }
             chunk2(u, 3, slow, rb, pk, rl);
+            if (quota_tile) drop_ties(rb, pk, rl);
             if (!stash_ok) rem = rl;
             tc::tmem_st16(pcol + 48, pk);
             tc::tmem_wait_st();
@@ -833,14 +867,17 @@ attention_tc_kernel(const Params p)
         for (int i = 0; i < 2; ++i)
             Z += __uint_as_float((uint32_t)zpair[i]) + __uint_as_float((uint32_t)(zpair[i] >> 32));
 
+        Z -= zdrop;                                   // ties the pass-2 quota masks dropped
+
         // ---------------------------------------------------------- quota tile
-        // The kstar kept ties of tile jstar are its first keys at level t in
-        // key order (level = Hamming distance of the packed signs); they add
-        // w_t V_j to the output and w_t each to Z.  The 32 rows of a warp are
-        // served together so that every global load is coalesced: the sign
-        // words of one row's quota tile (lane = key within a 32-key word),
-        // then one value row per kept key (lane = column pair).
-        const bool has_quota = ok && jstar >= 0 && active;
+        // (mode for many key tiles) The kstar kept ties of tile jstar are its
+        // first keys at level t in key order (level = Hamming distance of the
+        // packed signs); they add w_t V_j to the output and w_t each to Z.
+        // The 32 rows of a warp are served together so that every global load
+        // is coalesced: the sign words of one row's quota tile (lane = key
+        // within a 32-key word), then one value row per kept key (lane =
+        // column pair).
+        const bool has_quota = ok && jstar >= 0 && active && !kQ2;
         const float wq = has_quota ? ex2(p.c2 * (float)(D - 2 * t - ref)) : 0.0f;
         if (has_quota) Z += wq * (float)kstar;
         if (!(Z > 0.0f)) Z = 1.0f;                    // missed or inactive rows only
