@@ -47,6 +47,10 @@ def parse():
                     help="target CPU time of the oracle baseline sample")
     ap.add_argument("--no-e2e", action="store_true")
     ap.add_argument("--no-cpu-baseline", action="store_true")
+    ap.add_argument("--no-settle", action="store_true",
+                    help="skip the timed-loop warm-up of the clocks (for profiler captures, "
+                         "whose launch counts must be fixed; numbers taken under a profiler "
+                         "are not reported)")
     ap.add_argument("--mode", choices=["attention", "unfused", "mass", "causal", "soft", "bwd"],
                     default="attention",
                     help="attention: the forward (the default line); unfused: the four-call "
@@ -335,7 +339,7 @@ def run_had(args, world, rank, local):
 
     clocks = ClockSampler(local)
     clocks.start()
-    t_end = time.time() + 1.5                   # clocks settle under load first
+    t_end = time.time() + (0.0 if args.no_settle else 1.5)   # clocks settle under load first
     while time.time() < t_end:
         for _ in range(20):
             prepare()
@@ -668,7 +672,7 @@ def run_causal(args, world, rank, local):
     torch.cuda.synchronize()
     clocks = ClockSampler(local)
     clocks.start()
-    t_end = time.time() + 1.0                   # clocks settle under load first
+    t_end = time.time() + (0.0 if args.no_settle else 1.0)   # clocks settle under load first
     while time.time() < t_end:
         for _ in range(10):
             fused()

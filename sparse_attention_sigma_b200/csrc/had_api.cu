@@ -67,15 +67,19 @@ int grid_for(long long work_items, int per_block)
 had_status_t launch_pack(const void *x, had_dtype_t dt, const float *sigma, int B, int H,
                          int n, int d, uint32_t *bits, int32_t *status, cudaStream_t st)
 {
-    const long long words = (long long)B * H * n * d / 32;
+    // one block row per (b, h) slab; one 1024-element step per warp
+    const long long slab = (long long)n * d, bh = (long long)B * H;
     const int threads = 256;
-    const int grid = grid_for(words, threads);
+    const long long quads = (slab + 1023) / 1024;   // a warp's 1024-element steps
+    const long long bx = (quads + 8 - 1) / 8;
+    const dim3 grid((unsigned)(bx < 1 ? 1 : bx > 65535 ? 65535 : bx),
+                    (unsigned)(bh > 65535 ? 65535 : bh));
     if (dt == HAD_BF16)
         had::pack_bits_kernel<__nv_bfloat16><<<grid, threads, 0, st>>>(
-            static_cast<const __nv_bfloat16 *>(x), sigma, H, n, d, words, bits, status);
+            static_cast<const __nv_bfloat16 *>(x), sigma, H, slab, bh, bits, status);
     else
         had::pack_bits_kernel<float><<<grid, threads, 0, st>>>(
-            static_cast<const float *>(x), sigma, H, n, d, words, bits, status);
+            static_cast<const float *>(x), sigma, H, slab, bh, bits, status);
     return launched();
 }
 

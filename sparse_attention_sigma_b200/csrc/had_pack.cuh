@@ -2,9 +2,9 @@
 // coefficients of "Hamming Attention Distillation", pith.science review,
 // "What carries the argument").
 //
-// HBM-bound: every element is read once (16-byte vector loads) and 1 bit per
-// element is written, as whole 32-bit words.  Word w of a row holds elements
-// 32w..32w+31 with element 32w+k in bit k; bit = 1 means sign -1.
+// HBM-bound: every element is read once (coalesced 16-byte vector loads) and
+// 1 bit per element is written, as whole 32-bit words.  Word w of a row holds
+// elements 32w..32w+31 with element 32w+k in bit k; bit = 1 means sign -1.
 #pragma once
 #include "had_common.cuh"
 
@@ -36,46 +36,66 @@ struct Load8<float> {
     }
 };
 
-// One thread per output word: 32 consecutive elements of a row (16-byte
-// vector loads) give the 32 bits of one uint32.  With a normal sigma an
-// element at or below -sigma * 2^-100 is surely negative after the division
-// and one at or above zero surely not, so the sign is a comparison; only a
-// word holding an element strictly between (possible, never seen in
-// practice) takes the exact IEEE division, for all 32 elements.
-// words = B*H*n*d/32; word w covers elements 32w .. 32w+31 of the tensor.
+// One (b, h) slab per blockIdx.y (striding over slabs beyond the grid), so
+// sigma is read once per block and slab.  A warp streams 1024 consecutive
+// elements per step in four 256-element chunks whose loads are in flight
+// together: in a chunk lane L takes elements 8L..8L+7 (one 16-byte load for
+// bf16, so the warp reads 512 contiguous bytes), forms their 8 bits, and the
+// four lanes of a 32-element word join their bytes with two shuffles; every
+// fourth lane stores the word.  With a normal
+// sigma an element at or below -sigma * 2^-100 is surely negative after the
+// division and one at or above zero surely not, so the sign is a
+// comparison; only a lane holding an element strictly between (possible,
+// never seen in practice) takes the exact IEEE division, for its 8 elements.
+// slab = n*d elements (a multiple of 32, so a word never straddles slabs).
 template <typename T>
 __global__ void __launch_bounds__(256)
-pack_bits_kernel(const T *__restrict__ x, const float *__restrict__ sigma, int H, int n, int d,
-                 long long words, uint32_t *__restrict__ bits, int32_t *status)
+pack_bits_kernel(const T *__restrict__ x, const float *__restrict__ sigma, int H, long long slab,
+                 long long slabs, uint32_t *__restrict__ bits, int32_t *status)
 {
-    const long long stride = (long long)gridDim.x * blockDim.x;
-    const int words_per_row = d >> 5;
-    int cached = -1;
-    SignRule rule = sign_rule(1.0f);
-    for (long long w = blockIdx.x * (long long)blockDim.x + threadIdx.x; w < words; w += stride) {
-        const int head = (int)((w / words_per_row / n) % H);
-        if (head != cached) {
-            cached = head;
-            rule = sign_rule(__ldg(sigma + head));
-            if (rule.bad) flag(status, HAD_ERR_BAD_SIGMA);
-        }
-        float v[32];
+    for (long long bh = blockIdx.y; bh < slabs; bh += gridDim.y) {
+        const SignRule rule = sign_rule(__ldg(sigma + bh % H));
+        if (rule.bad && blockIdx.x == 0 && threadIdx.x == 0) flag(status, HAD_ERR_BAD_SIGMA);
+        const T *xs = x + bh * slab;
+        uint32_t *bs = bits + bh * (slab / 32);
+        const int lane = threadIdx.x & 31;
+        // four 256-element chunks per warp step, their loads in flight together
+        const long long quads = (slab + 1023) / 1024;
+        const long long step = (long long)gridDim.x * (blockDim.x / 32);
+        const long long q0 = blockIdx.x * (long long)(blockDim.x / 32) + (threadIdx.x >> 5);
+        for (long long q = q0; q < quads; q += step) {
+            float v[4][8];
 #pragma unroll
-        for (int c = 0; c < 4; ++c)
-            Load8<T>::run(x + w * 32 + 8 * c, *reinterpret_cast<float(*)[8]>(v + 8 * c));
-        uint32_t word = 0;
-        bool unsure = !rule.fast;
+            for (int k = 0; k < 4; ++k) {
+                const long long e0 = q * 1024 + k * 256 + 8 * lane;
+                if (e0 < slab) {                      // all 8 or none: slab is a multiple of 32
+                    Load8<T>::run(xs + e0, v[k]);
+                } else {
 #pragma unroll
-        for (int i = 0; i < 32; ++i) {
-            word |= (uint32_t)(v[i] <= -rule.thr) << i;
-            unsure |= (v[i] < 0.0f) && (v[i] > -rule.thr);
-        }
-        if (unsure) {
-            word = 0;
+                    for (int i = 0; i < 8; ++i) v[k][i] = 0.0f;
+                }
+            }
 #pragma unroll
-            for (int i = 0; i < 32; ++i) word |= negative_bit(v[i], rule) << i;
+            for (int k = 0; k < 4; ++k) {
+                const long long e0 = q * 1024 + k * 256 + 8 * lane;
+                uint32_t byte = 0;
+                bool unsure = !rule.fast;
+#pragma unroll
+                for (int i = 0; i < 8; ++i) {
+                    byte |= (uint32_t)(v[k][i] <= -rule.thr) << i;
+                    unsure |= (v[k][i] < 0.0f) && (v[k][i] > -rule.thr);
+                }
+                if (unsure) {
+                    byte = 0;
+#pragma unroll
+                    for (int i = 0; i < 8; ++i) byte |= negative_bit(v[k][i], rule) << i;
+                }
+                uint32_t word = byte << (8 * (lane & 3));
+                word |= __shfl_xor_sync(kFullMask, word, 1);
+                word |= __shfl_xor_sync(kFullMask, word, 2);
+                if (e0 < slab && (lane & 3) == 0) bs[e0 >> 5] = word;
+            }
         }
-        bits[w] = word;
     }
 }
 
