@@ -16,12 +16,12 @@
 //           -4 s).  Adding the row's window offset to it (one fused add-max
 //           per logit) gives the logit's shift in a thermometer of four 8-bit
 //           counters of one register (level <= L0-1, L0, L0+1, L0+2).  One
-//           word of counts per tile and row is kept in TMEM.  At the end the
-//           summed counters give the exact threshold level t and the number q
-//           of keys kept at it whenever t falls inside the window; rows where
-//           it does not are listed and recomputed exactly by the fix-up
-//           kernel.  The tile words give the one tile where the row's tie
-//           quota runs out.
+//           word of counts per tile and row is kept in shared memory.  At the
+//           end the summed counters give the exact threshold level t and the
+//           number q of keys kept at it whenever t falls inside the window;
+//           rows where it does not are listed and recomputed exactly by the
+//           fix-up kernel.  The tile words give the one tile where the row's
+//           tie quota runs out.
 //   pass 2  S again, with Q as -64 times the signs and a bias step that adds
 //           the offset of the thread's weight-table column, so that the
 //           accumulator is directly the byte offset of the logit's weight:
@@ -41,12 +41,13 @@
 // V^T (pass 2) through shared-memory rings.  One thread of warp 1 issues the
 // Q K^T MMAs and one thread of warp 2 + g the P V MMAs of query tile g (a
 // thread that shares its scheduler with epilogue warps issues a tcgen05
-// instruction only every ~100 cycles, so the streams go out in parallel).  S
-// tiles use a ring of three 128-column TMEM slots shared by the query tiles
-// (S tile k of the stream sits in slot k % 3); tile k + 3 is issued into a
-// slot once the epilogue has released it (pass 1) or once the P V that reads
-// it has completed (pass 2).  Warps 2 + QT .. 1 + 5 QT are the epilogue,
-// four per query tile.
+// instruction only every ~100 cycles, so the streams go out in parallel).
+// Pass 1 uses all four 128-column TMEM slots: key tile u's S tiles (one per
+// query tile) go to stage u % (4 / QT), reused once every epilogue warp has
+// read it; the row's tile words go to its weight-table column in shared
+// memory.  Pass 2 uses three slots and O: S tile j (= u QT + g) goes to slot
+// j % 3 once the P V of tile j - 3 has completed.  Warps 2 + QT .. 1 + 5 QT
+// are the epilogue, four per query tile.
 // Every wait is bounded by a caller-set limit: a CTA that hits it flags
 // HAD_ERR_TIMEOUT, lets its copies and MMAs drain, frees its TMEM and returns.
 #pragma once
@@ -84,7 +85,10 @@ struct Cfg {
     static constexpr int TAB_BYTES = BINS * kRows * 4;  // per query tile: [level][row] f32
     static constexpr uint32_t TMEM_COLS = 512;
     static constexpr uint32_t O_COL = kSlots * kKeys;   // query tile g's O at O_COL + g D
-    static constexpr int STASH_CAP = D;                 // tile words per row (in O's columns)
+    // pass 1 uses all four 128-column slots (O's columns are free then):
+    // stage st of key tile u (u % P1_STAGES) holds the QT S tiles of u
+    static constexpr int P1_STAGES = 4 / QT;
+    static constexpr int STASH_CAP = D;                 // tile words per row (its table column)
     static_assert(O_COL + QT * D <= TMEM_COLS, "TMEM budget");
     // shared memory layout (offsets from a 1024-aligned base)
     static constexpr int OFF_Q = 0;
@@ -104,7 +108,8 @@ struct Cfg {
     // X, Y <= 16 * 127
     static_assert(OFF_TAB + QT * TAB_BYTES + 256 * D + 4096 < 127 * (16 * 127 + 1),
                   "pass-2 bias range");
-    static constexpr int NBARS = 1 + 2 * KSTAGES + 2 * VSTAGES + (3 + QT) * kSlots + 3 * QT + 1;
+    static constexpr int NBARS = 1 + 2 * KSTAGES + 2 * VSTAGES + (2 + QT) * kSlots +
+                                 2 * P1_STAGES + 3 * QT + 1;
     static constexpr int OFF_MISC = OFF_BAR + NBARS * 8;
     static constexpr int SMEM_BYTES = OFF_MISC + 16 + 1024;   // + alignment slack
     static_assert(SMEM_BYTES <= 227 * 1024, "shared memory budget");
@@ -201,16 +206,17 @@ attention_tc_kernel(const Params p)
     uint64_t *const k_empty = k_full + C::KSTAGES;
     uint64_t *const v_full = k_empty + C::KSTAGES;
     uint64_t *const v_empty = v_full + C::VSTAGES;
-    uint64_t *const s_full = v_empty + C::VSTAGES;     // [kSlots] S tile in the slot
-    uint64_t *const s_free = s_full + kSlots;          // [kSlots] pass-1 slot read
+    uint64_t *const s_full = v_empty + C::VSTAGES;     // [kSlots] pass-2 S tile in the slot
     // [QT][kSlots] pass-2 P of query tile g in the slot: one barrier per
     // (tile, slot), so that the P V issuer of a tile, which skips the other
     // tile's S tiles, never waits on a phase more than one ahead
-    uint64_t *const p_full = s_free + kSlots;
+    uint64_t *const p_full = s_full + kSlots;
     uint64_t *const pv_done = p_full + QT * kSlots;    // [kSlots] the P V reading it done
     uint64_t *const q2_ready = pv_done + kSlots;       // [QT] Q tile rewritten for pass 2
     uint64_t *const o_full = q2_ready + QT;            // [QT] last P V of the tile done
     uint64_t *const drain = o_full + QT;               // [1 + QT] each issuer's MMAs done
+    uint64_t *const s1_full = drain + 1 + QT;          // [P1_STAGES] pass-1 S tiles of a key tile
+    uint64_t *const s1_free = s1_full + C::P1_STAGES;  // [P1_STAGES] ... read by every epilogue warp
     uint32_t *tmem_holder = reinterpret_cast<uint32_t *>(smem + C::OFF_MISC);
     volatile int *abort_flag = reinterpret_cast<volatile int *>(smem + C::OFF_MISC + 4);
 
@@ -219,7 +225,6 @@ attention_tc_kernel(const Params p)
     const long long head = blockIdx.x / p.ctas_per_head;
     const int qtile0 = (blockIdx.x % p.ctas_per_head) * QT;
     const int T = (p.n + kKeys - 1) / kKeys;            // 128-key tiles
-    const int J = T * QT;                               // S tiles per pass
     const uint64_t deadline = tc::globaltimer_ns() + p.wait_ns;
     constexpr uint64_t kDrainNs = 500000000ull;         // drains keep a long limit
 
@@ -235,7 +240,6 @@ attention_tc_kernel(const Params p)
         }
         for (int s = 0; s < kSlots; ++s) {
             tc::mbar_init(s_full + s, 1);
-            tc::mbar_init(s_free + s, 4);               // the four warps of the tile
             tc::mbar_init(pv_done + s, 1);
         }
         for (int s = 0; s < QT * kSlots; ++s) tc::mbar_init(p_full + s, 4);
@@ -244,6 +248,10 @@ attention_tc_kernel(const Params p)
             tc::mbar_init(o_full + g, 1);
         }
         for (int i = 0; i < 1 + QT; ++i) tc::mbar_init(drain + i, 1);
+        for (int st = 0; st < C::P1_STAGES; ++st) {
+            tc::mbar_init(s1_full + st, 1);
+            tc::mbar_init(s1_free + st, C::EPI_WARPS);
+        }
         *abort_flag = 0;
         tc::fence_mbar_init();
     }
@@ -318,38 +326,16 @@ attention_tc_kernel(const Params p)
             tc::fence_after_sync();
             int ks = 0;                 // K stage of the current key tile
             uint32_t kph = 0;           // its fill phase
-            int sl = 0;                 // S slot of tile kidx (kidx % 3)
-            int wrap = 0;               // kidx / 3
-            int kidx = 0;
-            // S tile kidx = Q_g K^T of the current stage into slot sl; every
-            // wait before it is on a barrier that other threads arrive on, so
-            // a fence orders their prior TMEM and shared-memory work first.
-            auto issue = [&](int g, bool bias) {
-                tc::fence_after_sync();
-                const uint32_t dcol = tmem + sl * kKeys;
+            // the D/32 (and, in pass 2, the bias) MMA steps of S = Q_g K^T into
+            // the TMEM columns at dcol
+            auto qk = [&](uint32_t dcol, int g, bool bias) {
 #pragma unroll
                 for (int kk = 0; kk < D / 32; ++kk)
                     tc::mma_i8_ss(dcol, dq[g] + (uint64_t)(kk * 16), dk + (uint64_t)(kk * 16),
                                   C::IDESC_QK, kk > 0 ? 1u : 0u);
                 if (bias) tc::mma_i8_ss(dcol, dbias[g], dones2, C::IDESC_QK, 1u);
-                tc::mma_commit(s_full + sl);
-                ++kidx;
-                if (++sl == kSlots) {
-                    sl = 0;
-                    ++wrap;
-                }
             };
-            // pass 1: slot reuse waits for the epilogue to have read tile kidx - 3
-            for (int u = 0; u < T && ok; ++u) {
-                ok = wait_bar(k_full + ks, kph, deadline, abort_flag, p.status);
-#pragma unroll
-                for (int g = 0; g < QT; ++g) {
-                    if (ok && kidx >= kSlots)
-                        ok = wait_bar(s_free + sl, (wrap - 1) & 1, deadline, abort_flag,
-                                      p.status);
-                    if (ok) issue(g, false);
-                }
-                if (!ok) break;
+            auto next_k = [&]() {
                 tc::mma_commit(k_empty + ks);
                 dk += (uint64_t)(C::KBYTES >> 4);
                 if (++ks == C::KSTAGES) {
@@ -357,43 +343,52 @@ attention_tc_kernel(const Params p)
                     kph ^= 1u;
                     dk = dk0;
                 }
+            };
+            // Pass 1: key tile u's S tiles (all query tiles) go to stage
+            // u % P1_STAGES, which is reused once every epilogue warp has read
+            // it.  Every wait before the MMAs is on a barrier that other threads
+            // arrive on, so a fence orders their prior TMEM and shared-memory
+            // work first.
+            for (int u = 0; u < T && ok; ++u) {
+                const int st = u % C::P1_STAGES;
+                if (u >= C::P1_STAGES)
+                    ok = wait_bar(s1_free + st, ((u / C::P1_STAGES) - 1) & 1, deadline, abort_flag,
+                                  p.status);
+                ok = ok && wait_bar(k_full + ks, kph, deadline, abort_flag, p.status);
+                if (!ok) break;
+                tc::fence_after_sync();
+#pragma unroll
+                for (int g = 0; g < QT; ++g) qk(tmem + (st * QT + g) * kKeys, g, false);
+                tc::mma_commit(s1_full + st);
+                next_k();
             }
             // before the first pass-2 MMA: every query tile's rewritten Q and
-            // bias rows, and the ones tile that all epilogue warps wrote
+            // bias rows, and the ones tile that all epilogue warps wrote; every
+            // epilogue warp has then also read all of its pass-1 S tiles
             for (int g = 0; g < QT && ok; ++g)
                 ok = wait_bar(q2_ready + g, 0, deadline, abort_flag, p.status);
-            // pass 2 (tile j of the pass is stream tile J + j): the slot last
-            // held pass-1 tile J + j - 3 (read by the epilogue) or pass-2 tile
-            // j - 3 (read by its P V; pv_done of a slot completes once per
-            // pass-2 tile in it, the n-th time for tile 3 n + j % 3)
-            int j = 0, jw = 0, j3 = 0;  // j / 3 and j % 3
-            for (int u = 0; u < T && ok; ++u) {
+            // Pass 2: tile j = u QT + g goes to slot j % 3, once the P V of
+            // tile j - 3 (pv_done of the slot, its (j / 3 - 1)-th completion)
+            // has read it.
+            int sl = 0, jw = 0;         // j % 3 and j / 3
+            for (int u = 0, j = 0; u < T && ok; ++u) {
                 ok = wait_bar(k_full + ks, kph, deadline, abort_flag, p.status);
 #pragma unroll
-                for (int g = 0; g < QT; ++g) {
+                for (int g = 0; g < QT; ++g, ++j) {
+                    if (ok && j >= kSlots)
+                        ok = wait_bar(pv_done + sl, (jw - 1) & 1, deadline, abort_flag, p.status);
                     if (ok) {
-                        if (j >= kSlots)
-                            ok = wait_bar(pv_done + sl, (jw - 1) & 1, deadline, abort_flag,
-                                          p.status);
-                        else if (kidx >= kSlots)
-                            ok = wait_bar(s_free + sl, (wrap - 1) & 1, deadline, abort_flag,
-                                          p.status);
+                        tc::fence_after_sync();
+                        qk(tmem + sl * kKeys, g, true);
+                        tc::mma_commit(s_full + sl);
                     }
-                    if (ok) issue(g, true);
-                    ++j;
-                    if (++j3 == kSlots) {
-                        j3 = 0;
+                    if (++sl == kSlots) {
+                        sl = 0;
                         ++jw;
                     }
                 }
                 if (!ok) break;
-                tc::mma_commit(k_empty + ks);
-                dk += (uint64_t)(C::KBYTES >> 4);
-                if (++ks == C::KSTAGES) {
-                    ks = 0;
-                    kph ^= 1u;
-                    dk = dk0;
-                }
+                next_k();
             }
             // drain: wait until every MMA this thread issued has completed
             tc::mma_commit(drain);
@@ -403,7 +398,7 @@ attention_tc_kernel(const Params p)
     } else if (warp < C::EPI_WARP0) {
         // ------------------------------------------------------------ P V issuers
         // one per query tile: O_g += P V for the tile's pass-2 S tiles
-        // (stream tiles J + u QT + g), so that the two streams of eight MMAs
+        // (pass-2 tiles u QT + g), so that the two streams of eight MMAs
         // per key tile go out in parallel
         if (lane == 0) {
             const int g = warp - 2;
@@ -415,7 +410,7 @@ attention_tc_kernel(const Params p)
             uint32_t vph = 0;           // its fill phase
             int j = g;                  // pass-2 tile index
             for (int u = 0; u < T && ok; ++u, j += QT) {
-                const int sl = (J + j) % kSlots;
+                const int sl = j % kSlots;
                 // this tile's p_full of the slot completes the (u / 3)-th time
                 // for key tile u (its S tiles visit the three slots in turn)
                 ok = wait_bar(v_full + vs, vph, deadline, abort_flag, p.status) &&
@@ -457,7 +452,11 @@ attention_tc_kernel(const Params p)
         const bool active1 = row1 < p.n;
         const int Nr = p.N;
         const uint32_t lane_base = tmem + ((uint32_t)(quarter * 32) << 16);
-        const uint32_t stash = lane_base + C::O_COL + g * D;
+        // this thread's column of the weight table: in pass 1 it holds the
+        // row's tile words (word u at u * kRows), later the weights
+        const int tab_off = g * C::TAB_BYTES + r * 4;
+        float *tcol = reinterpret_cast<float *>(smem + C::OFF_TAB + tab_off);
+        uint32_t *stash = reinterpret_cast<uint32_t *>(tcol);
         const bool stash_ok = !kDbg && T <= C::STASH_CAP;
         const int T_full = p.n / kKeys;               // key tiles without padding keys
         bool ok = true;
@@ -481,20 +480,31 @@ attention_tc_kernel(const Params p)
         }
 
         uint32_t ra[32], rb[32];
-        auto ld = [&](int kidx, int ch, uint32_t (&rr)[32]) {
-            tc::tmem_ld32(lane_base + (kidx % kSlots) * kKeys + ch * 32, rr);
+        // pass-2 S tile j (= u QT + g) sits in slot j % 3
+        auto ld = [&](int j, int ch, uint32_t (&rr)[32]) {
+            tc::tmem_ld32(lane_base + (j % kSlots) * kKeys + ch * 32, rr);
         };
-        auto wait_s = [&](int kidx) -> bool {
-            const bool w = __all_sync(kFullMask, wait_bar(s_full + kidx % kSlots,
-                                                          (kidx / kSlots) & 1, deadline,
+        auto wait_s = [&](int j) -> bool {
+            const bool w = __all_sync(kFullMask, wait_bar(s_full + j % kSlots, (j / kSlots) & 1,
+                                                          deadline, abort_flag, p.status));
+            tc::fence_after_sync();
+            return w;
+        };
+        // pass-1 key tile u sits in stage u % P1_STAGES, slot stage * QT + g
+        auto ld1 = [&](int u, int ch, uint32_t (&rr)[32]) {
+            tc::tmem_ld32(lane_base + ((u % C::P1_STAGES) * QT + g) * kKeys + ch * 32, rr);
+        };
+        auto wait_s1 = [&](int u) -> bool {
+            const bool w = __all_sync(kFullMask, wait_bar(s1_full + u % C::P1_STAGES,
+                                                          (u / C::P1_STAGES) & 1, deadline,
                                                           abort_flag, p.status));
             tc::fence_after_sync();
             return w;
         };
-        auto release_s = [&](int kidx) {
+        auto release_s1 = [&](int u) {
             tc::fence_before_sync();
             __syncwarp();
-            if (lane == 0) tc::mbar_arrive(s_free + kidx % kSlots);
+            if (lane == 0) tc::mbar_arrive(s1_free + u % C::P1_STAGES);
         };
         auto chunk_valid = [&](int u, int ch) { return min(32, p.n - u * kKeys - ch * 32); };
 
@@ -503,13 +513,13 @@ attention_tc_kernel(const Params p)
         // threshold level est; counters cover levels L0 - 1 .. L0 + 2 with
         // L0 = est - 1, and a logit's counter shift is cshift + v.
         int cshift = 0, L0 = 0;
-        if (ok) ok = wait_s(g);
+        if (ok) ok = wait_s1(0);
         if (ok) {
             long long sv = 0, sv2 = 0;
             const int cnt = min(kKeys, p.n);
 #pragma unroll 1
             for (int ch = 0; ch < 4; ++ch) {
-                ld(g, ch, ra);
+                ld1(0, ch, ra);
                 tc::tmem_wait_ld(ra);
                 const int valid = chunk_valid(0, ch);
                 int s1 = 0, s2 = 0;
@@ -555,33 +565,32 @@ attention_tc_kernel(const Params p)
             acc[0] = acc[1] = acc[2] = acc[3] = 0u;
 #pragma unroll
             for (int k = 0; k < 4; ++k) tot[k] += (int)((w >> (8 * k)) & 0xFFu);
-            if (stash_ok) tc::tmem_st1(stash + u, w);
+            if (stash_ok) stash[u * kRows] = w;
         };
         // one key tile; chunk 0 is in ra on entry, the next tile's chunk 0
         // on exit; masked: padding keys
         auto p1_tile = [&](int u, auto masked) {
-            const int kidx = u * QT + g;
-            ld(kidx, 1, rb);
+            ld1(u, 1, rb);
             therm(ra, chunk_valid(u, 0), masked);
             tc::tmem_wait_ld(rb);
-            ld(kidx, 2, ra);
+            ld1(u, 2, ra);
             therm(rb, chunk_valid(u, 1), masked);
             tc::tmem_wait_ld(ra);
-            ld(kidx, 3, rb);
+            ld1(u, 3, rb);
             therm(ra, chunk_valid(u, 2), masked);
             tc::tmem_wait_ld(rb);
-            release_s(kidx);
+            release_s1(u);
             const bool more = u + 1 < T;
             if (more) {
-                ok = wait_s(kidx + QT);
-                if (ok) ld(kidx + QT, 0, ra);
+                ok = wait_s1(u + 1);
+                if (ok) ld1(u + 1, 0, ra);
             }
             therm(rb, chunk_valid(u, 3), masked);
             end_tile1(u);
             if (more && ok) tc::tmem_wait_ld(ra);
         };
         if (ok) {
-            ld(g, 0, ra);
+            ld1(0, 0, ra);
             tc::tmem_wait_ld(ra);
             p1_tile(0, BT{});
         }
@@ -607,21 +616,18 @@ attention_tc_kernel(const Params p)
         // ties are added after pass 2, the quota tile itself.
         int zero_at = T, jstar = -1, kstar = 0;
         if (stash_ok && ok) {
-            tc::tmem_wait_st();
             const bool want = t >= 0 && !miss;
             const int ts = t - L0 + 1;                // 1..3: field of level t in a tile word
             bool found = !want;
             int cum = 0;
             for (int c0 = 0; c0 < T; c0 += 32) {
-                uint32_t w[32];
-                tc::tmem_ld32(stash + c0, w);
-                tc::tmem_wait_ld(w);
-#pragma unroll
+#pragma unroll 8
                 for (int i = 0; i < 32; ++i) {
                     const int jj = c0 + i;
                     if (!found && jj < T) {
-                        const int cnt = (int)((w[i] >> (8 * ts)) & 0xFFu) -
-                                        (int)((w[i] >> (8 * ts - 8)) & 0xFFu);
+                        const uint32_t w = stash[jj * kRows];
+                        const int cnt = (int)((w >> (8 * ts)) & 0xFFu) -
+                                        (int)((w >> (8 * ts - 8)) & 0xFFu);
                         if (cum + cnt >= quota) {
                             found = true;
                             zero_at = jj + 1;
@@ -695,11 +701,10 @@ attention_tc_kernel(const Params p)
         const int row = row1;
         const bool active = active1;
         // Weight table of the row, in this thread's own column (so the lanes
-        // of a warp read distinct banks): level l holds exp2(c2 (s_l - ref))
-        // for l <= t and 0 beyond.  ref is the threshold logit, raised where
-        // needed so that no weight can exceed the fp16 range (s <= D).
-        const int tab_off = g * C::TAB_BYTES + r * 4;
-        float *tcol = reinterpret_cast<float *>(smem + C::OFF_TAB + tab_off);
+        // of a warp read distinct banks; its tile words are no longer needed):
+        // level l holds exp2(c2 (s_l - ref)) for l <= t and 0 beyond.  ref is
+        // the threshold logit, raised where needed so that no weight can
+        // exceed the fp16 range (s <= D).
         const int headroom =
             p.c2 > 1.0e-6f ? (int)fminf(floorf(15.99f / p.c2), 1.0e6f) : 1000000;
         const int ref = max(D - 2 * max(t, 0), D - headroom);
@@ -800,7 +805,7 @@ attention_tc_kernel(const Params p)
         };
         // one key tile; chunk 0 is in ra on entry, the next tile's in ra on exit
         auto p2_tile = [&](int u, bool masked) {
-            const int kidx = J + u * QT + g;
+            const int kidx = u * QT + g;               // pass-2 S tile index
             if (u == zero_at) tcol[t * kRows] = 0.0f;   // ties past the quota weigh nothing now
             // key by key only on the ragged last tile (keys past n) and in
             // the mode without tile words; ties there follow the table (and,
@@ -854,9 +859,9 @@ attention_tc_kernel(const Params p)
             }
             if (more && ok) tc::tmem_wait_ld(ra);
         };
-        if (ok) ok = wait_s(J + g);
+        if (ok) ok = wait_s(g);
         if (ok) {
-            ld(J + g, 0, ra);
+            ld(g, 0, ra);
             tc::tmem_wait_ld(ra);
         }
 #pragma unroll 1
