@@ -1014,28 +1014,12 @@ attention_tc_kernel(const Params p)
                                                  (uint32_t)(jstar * kKeys + 32 * k + __ffs(m) - 1);
                     }
                     __syncwarp();
-                    // sixteen value rows per step, all loads issued before any is used
-                    for (int b0 = w0; b0 < w1; b0 += 16) {
-                        uint32_t ent[16];
-                        float2 x[16];
+                    // KV value rows per step, all loads issued before any is used
+                    // (the entries past the list load row 0 and add nothing)
+                    constexpr int KV = 32;
+                    auto add = [&](const uint32_t (&ent)[KV], const float2 (&x)[KV], int b0) {
 #pragma unroll
-                        for (int e = 0; e < 16; ++e) {
-                            ent[e] = b0 + e < w1 ? list[b0 + e - w0] : 0xFFFFFFFFu;
-                            const long long vr =
-                                ((head * p.n) + (b0 + e < w1 ? (ent[e] & 0xFFFFFFu) : 0u)) *
-                                    (long long)D + col;
-                            if (p.v_f32) {
-                                x[e] = __ldg(reinterpret_cast<const float2 *>(
-                                    static_cast<const float *>(p.v) + vr));
-                            } else {
-                                const uint32_t b2 = __ldg(reinterpret_cast<const uint32_t *>(
-                                    static_cast<const uint16_t *>(p.v) + vr));
-                                x[e] = make_float2(__uint_as_float(b2 << 16),
-                                                   __uint_as_float(b2 & 0xFFFF0000u));
-                            }
-                        }
-#pragma unroll
-                        for (int e = 0; e < 16; ++e)
+                        for (int e = 0; e < KV; ++e)
                             if (b0 + e < w1) {
                                 float2 *sl = vslot((int)(ent[e] >> 24), lane);
                                 float2 y = *sl;
@@ -1043,6 +1027,32 @@ attention_tc_kernel(const Params p)
                                 y.y += x[e].y;
                                 *sl = y;
                             }
+                    };
+                    for (int b0 = w0; b0 < w1; b0 += KV) {
+                        uint32_t ent[KV];
+                        float2 x[KV];
+#pragma unroll
+                        for (int e = 0; e < KV; ++e)
+                            ent[e] = b0 + e < w1 ? list[b0 + e - w0] : 0u;
+                        if (p.v_f32) {
+                            const float *vb = static_cast<const float *>(p.v) + col;
+#pragma unroll
+                            for (int e = 0; e < KV; ++e)
+                                x[e] = __ldg(reinterpret_cast<const float2 *>(
+                                    vb + ((head * p.n) + (ent[e] & 0xFFFFFFu)) * (long long)D));
+                        } else {
+                            const uint16_t *vb = static_cast<const uint16_t *>(p.v) + col;
+                            uint32_t b2[KV];
+#pragma unroll
+                            for (int e = 0; e < KV; ++e)
+                                b2[e] = __ldg(reinterpret_cast<const uint32_t *>(
+                                    vb + ((head * p.n) + (ent[e] & 0xFFFFFFu)) * (long long)D));
+#pragma unroll
+                            for (int e = 0; e < KV; ++e)
+                                x[e] = make_float2(__uint_as_float(b2[e] << 16),
+                                                   __uint_as_float(b2[e] & 0xFFFF0000u));
+                        }
+                        add(ent, x, b0);
                     }
                 }
                 __syncwarp();
