@@ -232,12 +232,23 @@ v_operand_kernel(const T *__restrict__ v, int n, int tiles, const float *__restr
     const int e = vscale_exp(head_max);
     const float scale = ldexpf(1.0f, -e);
     if (t == 0 && threadIdx.x == 0) vexp[head] = e;
-    if (t == 0)
-        for (int a = threadIdx.x; a < D; a += blockDim.x) {
-            int sum = 0;
-            for (int k = 0; k < tiles; ++k) sum += kpart[((size_t)head * tiles + k) * D + a];
+    if (t == 0) {
+        // column sums over the head's key tiles: each of the blockDim / D
+        // thread groups sums a strided share of the tiles (independent loads
+        // in flight), then the groups' partial sums meet in shared memory
+        static_assert(256 % D == 0, "thread groups of D columns");
+        __shared__ int kpsum[256];
+        const int a = threadIdx.x % D, grp = threadIdx.x / D, ngrp = blockDim.x / D;
+        int sum = 0;
+#pragma unroll 4
+        for (int k = grp; k < tiles; k += ngrp) sum += kpart[((size_t)head * tiles + k) * D + a];
+        kpsum[threadIdx.x] = sum;
+        __syncthreads();
+        if (grp == 0) {
+            for (int g2 = 1; g2 < ngrp; ++g2) sum += kpsum[g2 * D + a];
             ksum[head * D + a] = sum;
         }
+    }
     // load 64 keys x D values (coalesced, 8 elements per thread-iteration)
     constexpr int G = kKeys * D / 8;
     for (int g = threadIdx.x; g < G; g += blockDim.x) {
