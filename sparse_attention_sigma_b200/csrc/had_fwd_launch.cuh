@@ -133,15 +133,23 @@ had_status_t core_tc(const void *V, bool v_f32, int B, int H, int n, int N, floa
     using C = tcfwd::Cfg<D>;
     const long long bh = (long long)B * H;
     const bool dbg = dbg_idx != nullptr || dbg_lg != nullptr;
-    // The quota tile's kept ties: with few key tiles a per-chunk mask in
-    // pass 2 costs less than gathering them after it (a fixed latency per
-    // CTA); with many, the other way round (measured crossover near 12).
-    const bool q2 = (n + tcfwd::kKeys - 1) / tcfwd::kKeys <= 12;
-    auto kernel = dbg  ? tcfwd::attention_tc_kernel<D, true, false>
-                  : q2 ? tcfwd::attention_tc_kernel<D, false, true>
-                       : tcfwd::attention_tc_kernel<D, false, false>;
+    // The quota tile's kept ties: found by a scan of the head's key signs in
+    // shared memory where they fit (mode 2, measured fastest at 4 and at 32
+    // key tiles); else, with few key tiles, a per-chunk mask in pass 2
+    // (mode 1) costs less than gathering them after it (mode 0, a fixed
+    // latency per CTA; measured crossover near 12 tiles).
+    const int T = (n + tcfwd::kKeys - 1) / tcfwd::kKeys;
+    const long long kb_bytes = (long long)n * (D / 8);
+    const bool kb = !dbg && kb_bytes <= C::KB_CAP && kb_bytes % 16 == 0 && T <= C::STASH_CAP &&
+                    (reinterpret_cast<uintptr_t>(ws + w.kbits) & 15u) == 0;
+    const bool q2 = T <= 12;
+    auto kernel = dbg  ? tcfwd::attention_tc_kernel<D, true, 0>
+                  : kb ? tcfwd::attention_tc_kernel<D, false, 2>
+                  : q2 ? tcfwd::attention_tc_kernel<D, false, 1>
+                       : tcfwd::attention_tc_kernel<D, false, 0>;
+    const int smem_bytes = kb ? C::SMEM_BYTES_KB : C::SMEM_BYTES;
     if (cudaFuncSetAttribute(kernel, cudaFuncAttributeMaxDynamicSharedMemorySize,
-                             C::SMEM_BYTES) != cudaSuccess ||
+                             smem_bytes) != cudaSuccess ||
         cudaFuncSetAttribute(kernel, cudaFuncAttributePreferredSharedMemoryCarveout,
                              cudaSharedmemCarveoutMaxShared) != cudaSuccess)
         return HAD_ERR_CUDA;
@@ -172,7 +180,7 @@ had_status_t core_tc(const void *V, bool v_f32, int B, int H, int n, int N, floa
     p.z = normal_quantile((double)N / (double)n);
     p.wait_ns = wait_limit_ns().load();
     const long long blocks = bh * p.ctas_per_head;
-    kernel<<<(unsigned)blocks, C::THREADS, C::SMEM_BYTES, st>>>(p);
+    kernel<<<(unsigned)blocks, C::THREADS, smem_bytes, st>>>(p);
     return launch_status();
 }
 

@@ -109,10 +109,17 @@ struct Cfg {
     static_assert(OFF_TAB + QT * TAB_BYTES + 256 * D + 4096 < 127 * (16 * 127 + 1),
                   "pass-2 bias range");
     static constexpr int NBARS = 1 + 2 * KSTAGES + 2 * VSTAGES + (2 + QT) * kSlots +
-                                 2 * P1_STAGES + 3 * QT + 1;
+                                 2 * P1_STAGES + 3 * QT + 2;
     static constexpr int OFF_MISC = OFF_BAR + NBARS * 8;
     static constexpr int SMEM_BYTES = OFF_MISC + 16 + 1024;   // + alignment slack
     static_assert(SMEM_BYTES <= 227 * 1024, "shared memory budget");
+    // mode with the head's packed key signs in shared memory (n D / 8 bytes,
+    // at most KB_CAP), after the rest of the layout
+    static constexpr int KB_CAP = D == 64 ? 32768 : 16384;
+    static constexpr int OFF_KB = (OFF_MISC + 16 + 127) / 128 * 128;   // 16-byte aligned for the bulk copy
+    static constexpr int OFF_KM = OFF_KB + KB_CAP;      // per row its 128-bit kept-tie mask
+    static constexpr int SMEM_BYTES_KB = OFF_KM + QT * kRows * 16 + 1024;
+    static_assert(SMEM_BYTES_KB <= 227 * 1024, "shared memory budget (key signs)");
     static constexpr uint32_t IDESC_QK = tc::idesc(2, 1, 1, kRows, kKeys);   // s32 <- s8 x s8
     static constexpr uint32_t IDESC_PV = tc::idesc(1, 0, 0, kRows, D);       // f32 <- f16 x f16
 };
@@ -187,13 +194,22 @@ __device__ __forceinline__ void fence_async_smem()
     asm volatile("fence.proxy.async.shared::cta;" ::: "memory");
 }
 
-// kQ2: the quota tile's kept ties are masked in pass 2 (cheaper with few key
-// tiles) rather than gathered after it (cheaper with many).
-template <int D, bool kDbg, bool kQ2>
+// The quota tile's kept ties (its first kstar keys at level t), by kMode:
+//   0: left out of pass 2 and gathered after it from global memory (a fixed
+//      latency per CTA; the mode for any size);
+//   1: every tie given its weight in pass 2, those past the quota masked out
+//      by a per-chunk tie mask of the S values (cheaper with few key tiles);
+//   2: found before pass 2 by a scan of the head's packed key signs, copied
+//      to shared memory at the start, and set in P by pass 2 (heads whose
+//      signs fit in KB_CAP bytes).
+template <int D, bool kDbg, int kMode>
 __global__ void __launch_bounds__(Cfg<D>::THREADS, 1)
 attention_tc_kernel(const Params p)
 {
     using C = Cfg<D>;
+    constexpr bool kQ2 = kMode == 1;
+    constexpr bool kKB = kMode == 2;
+    static_assert(!(kDbg && kMode != 0), "the diagnostic outputs run in mode 0");
     constexpr int QT = C::QT;
     // 1024-aligned base, as an offset from the shared array (so that the
     // compiler keeps shared-memory addressing for every access through it);
@@ -217,6 +233,7 @@ attention_tc_kernel(const Params p)
     uint64_t *const drain = o_full + QT;               // [1 + QT] each issuer's MMAs done
     uint64_t *const s1_full = drain + 1 + QT;          // [P1_STAGES] pass-1 S tiles of a key tile
     uint64_t *const s1_free = s1_full + C::P1_STAGES;  // [P1_STAGES] ... read by every epilogue warp
+    uint64_t *const kb_full = s1_free + C::P1_STAGES;  // the head's key signs (kMode 2)
     uint32_t *tmem_holder = reinterpret_cast<uint32_t *>(smem + C::OFF_MISC);
     volatile int *abort_flag = reinterpret_cast<volatile int *>(smem + C::OFF_MISC + 4);
 
@@ -252,6 +269,7 @@ attention_tc_kernel(const Params p)
             tc::mbar_init(s1_full + st, 1);
             tc::mbar_init(s1_free + st, C::EPI_WARPS);
         }
+        tc::mbar_init(kb_full, 1);
         *abort_flag = 0;
         tc::fence_mbar_init();
     }
@@ -270,6 +288,13 @@ attention_tc_kernel(const Params p)
                                   head * (long long)p.kstride * C::VSUB;
             tc::mbar_expect_tx(q_full, QT * C::QBYTES);
             tc::bulk_g2s(smem + C::OFF_Q, qsrc, QT * C::QBYTES, q_full);
+            if (kKB) {
+                // the head's packed key signs, for the quota-tile scan
+                const uint32_t kb_bytes = (uint32_t)p.n * (D / 8);
+                tc::mbar_expect_tx(kb_full, kb_bytes);
+                tc::bulk_g2s(smem + C::OFF_KB, p.kbits + head * p.n * (long long)(D / 32),
+                             kb_bytes, kb_full);
+            }
             // K stream G = 0 .. 2T-1 (key tile G % T); V tile H follows K
             // stream entry T + H.
             int issued_k = 0, issued_v = 0;
@@ -303,6 +328,12 @@ attention_tc_kernel(const Params p)
                     wait_bar(k_full + G % C::KSTAGES, (G / C::KSTAGES) & 1, dl, &never, p.status);
                 for (int H = max(0, issued_v - C::VSTAGES); H < issued_v; ++H)
                     wait_bar(v_full + H % C::VSTAGES, (H / C::VSTAGES) & 1, dl, &never, p.status);
+            }
+            if (kKB) {
+                // the key-sign copy lands before the CTA exits, whether or not
+                // an epilogue warp got as far as waiting for it
+                volatile int never = 0;
+                wait_bar(kb_full, 0, tc::globaltimer_ns() + kDrainNs, &never, p.status);
             }
         }
     } else if (warp == 1) {
@@ -598,6 +629,13 @@ attention_tc_kernel(const Params p)
         for (int u = 1; u < T_full && ok; ++u) p1_tile(u, BF{});
         if (ok && T > T_full && T_full >= 1) p1_tile(T - 1, BT{});
 
+        // (kMode 2) the row's packed signs for the quota-tile scan, loaded
+        // while the threshold and the pass-2 tables are set up
+        uint32_t qw[D / 32];
+#pragma unroll
+        for (int w = 0; w < D / 32; ++w)
+            qw[w] = kKB && active1 ? __ldg(p.qbits + ((head * p.n) + row1) * (D / 32) + w) : 0u;
+
         // threshold level t and the number q of keys kept at it
         const int f0 = tot[0], f1 = tot[1], f2 = tot[2], f3 = tot[3];
         int t = -1, quota = 0;
@@ -721,6 +759,85 @@ attention_tc_kernel(const Params p)
 
         const uint32_t vt = (uint32_t)(hb - 256 * (D - 2 * t));   // accumulator of the threshold
         const float wt_tab = t >= 0 ? tcol[t * kRows] : 0.0f;       // the table's weight of level t
+
+        // (kMode 2) The kept ties of the quota tile, before pass 2: bit i of
+        // word c is key 32 c + i of tile jstar.  The warp's rows go LPR at a
+        // time with lane = key within a 32-key chunk (a chunk's sign words
+        // are 32 consecutive entries of shared memory), all loads of a round
+        // issued before any is used; lane L keeps the tie ballots of its own
+        // row and then cuts them to the first kstar by itself.
+        if constexpr (kKB) {
+            constexpr int DW = D / 32, LPR = D == 64 ? 4 : 2;
+            const bool hq = ok && active && jstar >= 0 && kstar > 0;
+            ok = __all_sync(kFullMask, wait_bar(kb_full, 0, deadline, abort_flag, p.status));
+            const uint32_t *kbs = reinterpret_cast<const uint32_t *>(smem + C::OFF_KB);
+            uint32_t tw[4] = {0u, 0u, 0u, 0u};
+            uint32_t todo = ok ? __ballot_sync(kFullMask, hq) : 0u;
+            while (todo) {                            // warp-uniform
+                int Ls[LPR], jl[LPR], tl[LPR];
+                uint32_t ql[LPR][DW];
+#pragma unroll
+                for (int e = 0; e < LPR; ++e) {
+                    Ls[e] = todo ? __ffs(todo) - 1 : -1;
+                    todo &= todo - 1u;
+                    const int Lc = max(Ls[e], 0);
+                    jl[e] = max(__shfl_sync(kFullMask, jstar, Lc), 0);
+                    tl[e] = Ls[e] >= 0 ? __shfl_sync(kFullMask, t, Lc) : -1;   // -1: no tie
+#pragma unroll
+                    for (int w = 0; w < DW; ++w) ql[e][w] = __shfl_sync(kFullMask, qw[w], Lc);
+                }
+                uint32_t kx[LPR][4][DW];
+#pragma unroll
+                for (int e = 0; e < LPR; ++e)
+#pragma unroll
+                    for (int c = 0; c < 4; ++c) {
+                        const int key = min(jl[e] * kKeys + 32 * c + lane, p.n - 1);
+                        if (DW == 2) {
+                            const uint2 x = *reinterpret_cast<const uint2 *>(kbs + key * 2);
+                            kx[e][c][0] = x.x;
+                            kx[e][c][DW - 1] = x.y;
+                        } else {
+                            const uint4 x = *reinterpret_cast<const uint4 *>(kbs + key * 4);
+                            kx[e][c][0] = x.x;
+                            kx[e][c][1 % DW] = x.y;
+                            kx[e][c][2 % DW] = x.z;
+                            kx[e][c][3 % DW] = x.w;
+                        }
+                    }
+#pragma unroll
+                for (int e = 0; e < LPR; ++e)
+#pragma unroll
+                    for (int c = 0; c < 4; ++c) {
+                        int ham = 0;
+#pragma unroll
+                        for (int w = 0; w < DW; ++w) ham += __popc(ql[e][w] ^ kx[e][c][w]);
+                        const bool tie = ham == tl[e] && jl[e] * kKeys + 32 * c + lane < p.n;
+                        const uint32_t b = __ballot_sync(kFullMask, tie);
+                        tw[c] = lane == Ls[e] ? b : tw[c];
+                    }
+            }
+            // this row's cut: its first kstar ties
+            int need = hq ? kstar : 0;
+#pragma unroll
+            for (int c = 0; c < 4; ++c) {
+                const int cnt = __popc(tw[c]);
+                if (need <= 0) {
+                    tw[c] = 0u;
+                } else if (cnt > need) {
+                    tw[c] &= (1u << __fns(tw[c], 0, need + 1)) - 1u;
+                    need = 0;
+                } else {
+                    need -= cnt;
+                }
+            }
+            // kept in shared memory through pass 2, read on the quota tile
+            *reinterpret_cast<uint4 *>(smem + C::OFF_KM + f * 16) = make_uint4(tw[0], tw[1], tw[2], tw[3]);
+        }
+        uint32_t wt_h2;                                // the tie weight as a pair of fp16
+        {
+            __half2 h2 = __floats2half2_rn(wt_tab, wt_tab);
+            wt_h2 = *reinterpret_cast<uint32_t *>(&h2);
+        }
         float zdrop = 0.0f;                           // weights of ties dropped after the table
         int rem = quota;                              // ties still to keep (key-by-key mode)
         int kept = 0;
@@ -803,6 +920,25 @@ attention_tc_kernel(const Params p)
                 zdrop += wt_tab * (float)__popc(drop);
             }
         };
+        // (kMode 2) the chunk's kept ties of the quota tile (mask m, bit i =
+        // column i) take the tie weight in P, where the table gave them 0 (so
+        // an OR sets them).  Four mask bits are spread to the sign bits of
+        // four bytes (bit b to bit 8 b + 7: the shifted copies of the
+        // multiply do not overlap), and a sign-replicating byte permute
+        // widens them to half-word masks.
+        auto set_kept = [&](uint32_t m, uint32_t (&pk)[16]) {
+            if (__any_sync(kFullMask, m != 0u)) {
+#pragma unroll
+                for (int i = 0; i < 8; ++i) {
+                    const uint32_t sp = ((m >> (4 * i)) & 15u) * 0x10204080u;
+                    uint32_t lo, hi;
+                    asm("prmt.b32 %0, %1, 0, 0x9988;" : "=r"(lo) : "r"(sp));
+                    asm("prmt.b32 %0, %1, 0, 0xBBAA;" : "=r"(hi) : "r"(sp));
+                    pk[2 * i] |= wt_h2 & lo;
+                    pk[2 * i + 1] |= wt_h2 & hi;
+                }
+            }
+        };
         // one key tile; chunk 0 is in ra on entry, the next tile's in ra on exit
         auto p2_tile = [&](int u, bool masked) {
             const int kidx = u * QT + g;               // pass-2 S tile index
@@ -818,19 +954,24 @@ attention_tc_kernel(const Params p)
                 !slow && kQ2 && __any_sync(kFullMask, u == jstar);
             uint32_t pk[16];
             const uint32_t pcol = lane_base + (kidx % kSlots) * kKeys;   // P over S
+            uint4 km = make_uint4(0u, 0u, 0u, 0u);    // (kMode 2) kept ties, quota tile only
+            if (kKB && u == jstar) km = *reinterpret_cast<const uint4 *>(smem + C::OFF_KM + f * 16);
             ld(kidx, 1, rb);
             chunk2(u, 0, slow, ra, pk, rl);
             if (quota_tile) drop_ties(ra, pk, rl);
+            if (kKB) set_kept(km.x, pk);
             tc::tmem_st16(pcol, pk);                  // S columns 0-15 are already read
             tc::tmem_wait_ld(rb);
             ld(kidx, 2, ra);
             chunk2(u, 1, slow, rb, pk, rl);
             if (quota_tile) drop_ties(rb, pk, rl);
+            if (kKB) set_kept(km.y, pk);
             tc::tmem_st16(pcol + 16, pk);
             tc::tmem_wait_ld(ra);
             ld(kidx, 3, rb);
             chunk2(u, 2, slow, ra, pk, rl);
             if (quota_tile) drop_ties(ra, pk, rl);
+            if (kKB) set_kept(km.z, pk);
             tc::tmem_st16(pcol + 32, pk);
             tc::tmem_wait_ld(rb);
             // The next tile's first chunk is loaded here only if its S is
@@ -847,6 +988,7 @@ attention_tc_kernel(const Params p)
             }
             chunk2(u, 3, slow, rb, pk, rl);
             if (quota_tile) drop_ties(rb, pk, rl);
+            if (kKB) set_kept(km.w, pk);
             if (!stash_ok) rem = rl;
             tc::tmem_st16(pcol + 48, pk);
             tc::tmem_wait_st();
@@ -888,7 +1030,7 @@ attention_tc_kernel(const Params p)
         if (!(Z > 0.0f)) Z = 1.0f;                    // missed or inactive rows only
         constexpr int DW = D / 32;                    // sign words per key
         uint32_t keep[4] = {0u, 0u, 0u, 0u};          // bit i of word c: key 32 c + i of tile jstar
-        const uint32_t qlanes = __ballot_sync(kFullMask, has_quota);
+        const uint32_t qlanes = kKB ? 0u : __ballot_sync(kFullMask, has_quota);   // kMode 2: set in P
         if (qlanes) {
             uint32_t qw[DW];
 #pragma unroll

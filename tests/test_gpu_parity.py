@@ -87,6 +87,12 @@ SMALL = [
     (2, 1, 129, 128, 129, 5, torch.float32),        # N = n: dense softmax
     (1, 1, 1, 64, 1, 6, torch.bfloat16),            # a single row and key
     (1, 3, 97, 64, 1, 7, torch.bfloat16),           # N = 1
+    # more than 12 key tiles, ragged last tile: the quota tile's kept ties
+    # found from the key signs in shared memory (n d / 8 a multiple of 16),
+    # then gathered after pass 2 (odd n; d 128 beyond 16 KB of key signs)
+    (1, 2, 2000, 64, 300, 8, torch.bfloat16),
+    (1, 1, 1999, 64, 250, 9, torch.float32),
+    (1, 1, 1700, 128, 200, 10, torch.bfloat16),
 ]
 
 
@@ -219,6 +225,21 @@ def test_all_keys_equal(had):
     torch.cuda.synchronize()
     assert (dbg.cpu() == torch.arange(17, dtype=torch.int32)).all()
     mean = c.v[:, :, :17].double().mean(dim=2, keepdim=True).expand(-1, -1, 300, -1)
+    assert_close(out.cpu().numpy(), mean.numpy(), "mean of first N")
+
+
+@pytest.mark.parametrize("n", [2048, 2047])
+def test_all_keys_equal_many_tiles(had, n):
+    """Every key a tie at the threshold, over 16 key tiles: the quota tile
+    is the third (keys 256 .. 383) and keeps its first 44 keys, on the
+    production path (key-sign scan for even n, gather for odd n)."""
+    N = 300
+    c = random_case(1, 2, n, 64, N, 13)
+    c.k[:] = c.k[:, :, :1]
+    c = Case(c.q, c.k, c.v, c.sgq, synth.per_head_sigma(c.k), c.N, c.tau)
+    out = had.had_attention_fwd(c.gq, c.gk, c.gv, c.gsq, c.gsk, c.N, c.tau)
+    torch.cuda.synchronize()
+    mean = c.v[:, :, :N].double().mean(dim=2, keepdim=True).expand(-1, -1, n, -1)
     assert_close(out.cpu().numpy(), mean.numpy(), "mean of first N")
 
 
