@@ -766,6 +766,12 @@ attention_tc_kernel(const Params p)
         // are 32 consecutive entries of shared memory), all loads of a round
         // issued before any is used; lane L keeps the tie ballots of its own
         // row and then cuts them to the first kstar by itself.
+        int zq = kstar;                                // ties of tile jstar that Z gains at the end
+        uint32_t wt_x;                                 // (kMode 2) what P's changed ties become:
+        {                                              // the tie weight as a pair of fp16, or 0
+            __half2 h2 = __floats2half2_rn(wt_tab, wt_tab);
+            wt_x = *reinterpret_cast<uint32_t *>(&h2);
+        }
         if constexpr (kKB) {
             constexpr int DW = D / 32, LPR = D == 64 ? 4 : 2;
             const bool hq = ok && active && jstar >= 0 && kstar > 0;
@@ -816,27 +822,39 @@ attention_tc_kernel(const Params p)
                         tw[c] = lane == Ls[e] ? b : tw[c];
                     }
             }
-            // this row's cut: its first kstar ties
-            int need = hq ? kstar : 0;
+            // this row's cut: its first kstar ties are kept, the rest dropped.
+            // The smaller set is the one pass 2 changes in P: the kept ties,
+            // set over the table's 0 (the table zeroes level t from tile
+            // jstar on), or the dropped ties, cleared from the table's tie
+            // weight (then level t keeps its weight through tile jstar).
+            int need = hq ? kstar : 0, nkeep = 0, ndrop = 0;
+            uint32_t kept[4];
 #pragma unroll
             for (int c = 0; c < 4; ++c) {
                 const int cnt = __popc(tw[c]);
+                kept[c] = tw[c];
                 if (need <= 0) {
-                    tw[c] = 0u;
+                    kept[c] = 0u;
                 } else if (cnt > need) {
-                    tw[c] &= (1u << __fns(tw[c], 0, need + 1)) - 1u;
+                    kept[c] &= (1u << __fns(tw[c], 0, need + 1)) - 1u;
                     need = 0;
                 } else {
                     need -= cnt;
                 }
+                nkeep += __popc(kept[c]);
+                ndrop += cnt - __popc(kept[c]);
             }
-            // kept in shared memory through pass 2, read on the quota tile
-            *reinterpret_cast<uint4 *>(smem + C::OFF_KM + f * 16) = make_uint4(tw[0], tw[1], tw[2], tw[3]);
-        }
-        uint32_t wt_h2;                                // the tie weight as a pair of fp16
-        {
-            __half2 h2 = __floats2half2_rn(wt_tab, wt_tab);
-            wt_h2 = *reinterpret_cast<uint32_t *>(&h2);
+            const bool drop_mode = hq && ndrop < nkeep;
+            if (drop_mode) {
+                zero_at = jstar + 1;
+                zq = -ndrop;
+            }
+            // in shared memory through pass 2, read on the quota tile
+            *reinterpret_cast<uint4 *>(smem + C::OFF_KM + f * 16) =
+                drop_mode ? make_uint4(tw[0] & ~kept[0], tw[1] & ~kept[1], tw[2] & ~kept[2],
+                                       tw[3] & ~kept[3])
+                          : make_uint4(kept[0], kept[1], kept[2], kept[3]);
+            if (drop_mode) wt_x = 0u;
         }
         float zdrop = 0.0f;                           // weights of ties dropped after the table
         int rem = quota;                              // ties still to keep (key-by-key mode)
@@ -920,12 +938,13 @@ attention_tc_kernel(const Params p)
                 zdrop += wt_tab * (float)__popc(drop);
             }
         };
-        // (kMode 2) the chunk's kept ties of the quota tile (mask m, bit i =
-        // column i) take the tie weight in P, where the table gave them 0 (so
-        // an OR sets them).  Four mask bits are spread to the sign bits of
-        // four bytes (bit b to bit 8 b + 7: the shifted copies of the
-        // multiply do not overlap), and a sign-replicating byte permute
-        // widens them to half-word masks.
+        // (kMode 2) the chunk's changed ties of the quota tile (mask m, bit i
+        // = column i) become wt_x in P: the tie weight (kept ties, which the
+        // table gave 0) or 0 (dropped ties, which it gave the tie weight).
+        // Four mask bits are spread to the sign bits of four bytes (bit b to
+        // bit 8 b + 7: the shifted copies of the multiply do not overlap), a
+        // sign-replicating byte permute widens them to half-word masks, and
+        // one three-input logic op selects.
         auto set_kept = [&](uint32_t m, uint32_t (&pk)[16]) {
             if (__any_sync(kFullMask, m != 0u)) {
 #pragma unroll
@@ -934,8 +953,8 @@ attention_tc_kernel(const Params p)
                     uint32_t lo, hi;
                     asm("prmt.b32 %0, %1, 0, 0x9988;" : "=r"(lo) : "r"(sp));
                     asm("prmt.b32 %0, %1, 0, 0xBBAA;" : "=r"(hi) : "r"(sp));
-                    pk[2 * i] |= wt_h2 & lo;
-                    pk[2 * i + 1] |= wt_h2 & hi;
+                    pk[2 * i] = (pk[2 * i] & ~lo) | (wt_x & lo);
+                    pk[2 * i + 1] = (pk[2 * i + 1] & ~hi) | (wt_x & hi);
                 }
             }
         };
@@ -1026,7 +1045,7 @@ attention_tc_kernel(const Params p)
         // column pair).
         const bool has_quota = ok && jstar >= 0 && active && !kQ2;
         const float wq = has_quota ? ex2(p.c2 * (float)(D - 2 * t - ref)) : 0.0f;
-        if (has_quota) Z += wq * (float)kstar;
+        if (has_quota) Z += wq * (float)zq;
         if (!(Z > 0.0f)) Z = 1.0f;                    // missed or inactive rows only
         constexpr int DW = D / 32;                    // sign words per key
         uint32_t keep[4] = {0u, 0u, 0u, 0u};          // bit i of word c: key 32 c + i of tile jstar
