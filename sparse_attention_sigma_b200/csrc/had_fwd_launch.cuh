@@ -93,8 +93,9 @@ had_status_t prep_typed(const T *Q, const T *K, const T *V, const float *sq, con
         reinterpret_cast<int8_t *>(ws + w.kop), reinterpret_cast<uint16_t *>(ws + w.qbits),
         reinterpret_cast<uint16_t *>(ws + w.kbits), reinterpret_cast<int8_t *>(ws + w.kpart),
         vpart, reinterpret_cast<int *>(ws + w.miss), status);
-    prep::v_operand_kernel<T, D><<<(unsigned)(bh * w.kstride), 256, 0, st>>>(
-        V, n, w.kstride, vpart, w.vchunks, reinterpret_cast<__half *>(ws + w.vop),
+    const int ctiles = (w.kstride + 256 / D - 1) / (256 / D);   // CTAs per head, 256 / D tiles each
+    prep::v_operand_kernel<T, D><<<(unsigned)(bh * ctiles), 256, 0, st>>>(
+        V, n, w.kstride, ctiles, vpart, w.vchunks, reinterpret_cast<__half *>(ws + w.vop),
         reinterpret_cast<int *>(ws + w.vexp), reinterpret_cast<const int8_t *>(ws + w.kpart),
         reinterpret_cast<int *>(ws + w.ksum));
     return launch_status();

@@ -160,12 +160,20 @@ operands_kernel(const T *__restrict__ Q, const T *__restrict__ K, const T *__res
                     row < n ? recode(w, 0xFFu, 0x40u, 0xC0u) : make_uint4(0u, 0u, 0u, 0u);
         }
         if (!isq) {
-            // column sums of the tile's codes: valid keys minus twice the negatives
+            // column sums of the tile's codes: valid keys minus twice the
+            // negatives, each of the blockDim / D thread groups counting a
+            // strided share of the rows
+            static_assert(256 % D == 0, "thread groups of D columns");
+            __shared__ int negp[256];
             __syncthreads();
             const int valid = max(0, min(kKeys, n - t * kKeys));
-            for (int a = threadIdx.x; a < D; a += blockDim.x) {
-                int neg_count = 0;
-                for (int rr = 0; rr < valid; ++rr) neg_count += (sbits[rr][a >> 4] >> (a & 15)) & 1;
+            const int a = threadIdx.x % D, grp = threadIdx.x / D, ngrp = blockDim.x / D;
+            int neg_count = 0;
+            for (int rr = grp; rr < valid; rr += ngrp) neg_count += (sbits[rr][a >> 4] >> (a & 15)) & 1;
+            negp[threadIdx.x] = neg_count;
+            __syncthreads();
+            if (grp == 0) {
+                for (int g2 = 1; g2 < ngrp; ++g2) neg_count += negp[g2 * D + a];
                 kpart[(size_t)bb * D + a] = (int8_t)(valid - 2 * neg_count);
             }
         }
@@ -207,20 +215,24 @@ __device__ __forceinline__ int vscale_exp(float m)
     return e - 15;            // m * 2^-(e-15) in [2^14, 2^15)
 }
 
-// One CTA per (head, 64-key tile): the head's largest |v| from the chunk
-// maxima of operands_kernel, then the tile transposed through shared memory
-// and written as V^T fp16 core matrices (tiles past n are zeros).  The CTA of
-// tile 0 writes the head's e_h and reduces its key column sums to Ksum.
+// The head's largest |v| from the chunk maxima of operands_kernel, then V^T
+// as fp16 core matrices scaled by 2^-e_h (tiles past n are zeros).  A CTA
+// takes 256 / D consecutive 64-key tiles of one head (ctiles per head);
+// each thread one block of 8 keys x 8 dims: eight 16-byte rows of V in,
+// transposed in registers, eight 16-byte core-matrix rows (8 keys of one
+// dim) out.  The head's first CTA also writes e_h and reduces its key
+// column sums to Ksum.
 template <typename T, int D>
 __global__ void __launch_bounds__(256)
-v_operand_kernel(const T *__restrict__ v, int n, int tiles, const float *__restrict__ vpart,
+v_operand_kernel(const T *__restrict__ v, int n, int tiles, int ctiles, const float *__restrict__ vpart,
                  int vchunks, __half *__restrict__ op, int *__restrict__ vexp,
                  const int8_t *__restrict__ kpart, int *__restrict__ ksum)
 {
-    __shared__ float tile[kKeys][D + 1];
+    static_assert(256 % D == 0, "thread groups of D columns / blocks");
+    constexpr int TPC = 256 / D;                   // tiles per CTA (D threads per tile)
     __shared__ float head_max;
-    const long long head = blockIdx.x / tiles;
-    const int t = blockIdx.x % tiles;
+    const long long head = blockIdx.x / ctiles;
+    const int ct = blockIdx.x % ctiles;
     if (threadIdx.x < 32) {
         float m = 0.0f;
         for (int c = threadIdx.x; c < vchunks; c += 32) m = fmaxf(m, vpart[head * vchunks + c]);
@@ -231,12 +243,11 @@ v_operand_kernel(const T *__restrict__ v, int n, int tiles, const float *__restr
     __syncthreads();
     const int e = vscale_exp(head_max);
     const float scale = ldexpf(1.0f, -e);
-    if (t == 0 && threadIdx.x == 0) vexp[head] = e;
-    if (t == 0) {
+    if (ct == 0 && threadIdx.x == 0) vexp[head] = e;
+    if (ct == 0) {
         // column sums over the head's key tiles: each of the blockDim / D
         // thread groups sums a strided share of the tiles (independent loads
         // in flight), then the groups' partial sums meet in shared memory
-        static_assert(256 % D == 0, "thread groups of D columns");
         __shared__ int kpsum[256];
         const int a = threadIdx.x % D, grp = threadIdx.x / D, ngrp = blockDim.x / D;
         int sum = 0;
@@ -249,35 +260,35 @@ v_operand_kernel(const T *__restrict__ v, int n, int tiles, const float *__restr
             ksum[head * D + a] = sum;
         }
     }
-    // load 64 keys x D values (coalesced, 8 elements per thread-iteration)
-    constexpr int G = kKeys * D / 8;
-    for (int g = threadIdx.x; g < G; g += blockDim.x) {
-        const int key = g / (D / 8);
-        const int c0 = (g % (D / 8)) * 8;
-        const int j = t * kKeys + key;
-        float e8[8];
+    const int t = ct * TPC + (int)threadIdx.x / D;  // this thread's tile
+    if (t >= tiles) return;
+    const int local = threadIdx.x % D;
+    const int db = local % (D / 8), kb = local / (D / 8);   // dims 8 db.., keys 8 kb..
+    // rows: keys 8 kb + r of the tile, dims 8 db .. 8 db + 7 (a warp's lanes
+    // read D / 8 consecutive 16-byte pieces of each of 32 / (D / 8) rows)
+    float x[8][8];
+#pragma unroll
+    for (int r = 0; r < 8; ++r) {
+        const int j = t * kKeys + kb * 8 + r;
         if (j < n) {
-            Load8<T>::run(v + ((head * n + j) * (long long)D + c0), e8);
+            Load8<T>::run(v + ((head * n + j) * (long long)D + db * 8), x[r]);
         } else {
 #pragma unroll
-            for (int k = 0; k < 8; ++k) e8[k] = 0.0f;
+            for (int c = 0; c < 8; ++c) x[r][c] = 0.0f;
         }
-#pragma unroll
-        for (int k = 0; k < 8; ++k) tile[key][c0 + k] = e8[k] * scale;
     }
-    __syncthreads();
-    // write D rows x 64 keys: one thread per 16-byte chunk (8 keys of a dim)
-    __half *dst = op + (head * tiles + t) * (long long)D * kKeys;
-    constexpr int CH = D * (kKeys / 8);
-    for (int c = threadIdx.x; c < CH; c += blockDim.x) {
-        const int dim = c / (kKeys / 8);
-        const int k0 = (c % (kKeys / 8)) * 8;
-        __align__(16) __half h[8];
+    char *dst = reinterpret_cast<char *>(op + (head * tiles + t) * (long long)D * kKeys);
 #pragma unroll
-        for (int k = 0; k < 8; ++k) h[k] = __float2half_rn(tile[k0 + k][dim]);
-        const uint32_t off = core_offset(dim, k0 * 2, kKeys * 2);
-        *reinterpret_cast<uint4 *>(reinterpret_cast<char *>(dst) + off) =
-            *reinterpret_cast<const uint4 *>(h);
+    for (int c = 0; c < 8; ++c) {
+        uint32_t h2[4];
+#pragma unroll
+        for (int r = 0; r < 8; r += 2) {
+            __half2 h = __halves2half2(__float2half_rn(x[r][c] * scale),
+                                       __float2half_rn(x[r + 1][c] * scale));
+            h2[r / 2] = *reinterpret_cast<uint32_t *>(&h);
+        }
+        const uint32_t off = core_offset(db * 8 + c, kb * 16, kKeys * 2);
+        *reinterpret_cast<uint4 *>(dst + off) = make_uint4(h2[0], h2[1], h2[2], h2[3]);
     }
 }
 
