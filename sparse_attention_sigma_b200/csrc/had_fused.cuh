@@ -964,19 +964,21 @@ fixup_rows_kernel(const uint32_t *__restrict__ qbits, const uint32_t *__restrict
                 }
                 kept_before += cnt;
                 __syncwarp();
-                // gather the listed V rows, eight loads in flight per lane
-                for (int i0 = 0; i0 < cnt; i0 += 8) {
-                    float v[8][PER];
-                    float ww[8];
+                // gather the listed V rows, GU loads in flight per lane (at d
+                // 128, 16 rows cost more in occupancy than they save in latency)
+                constexpr int GU = D == 64 ? 16 : 8;
+                for (int i0 = 0; i0 < cnt; i0 += GU) {
+                    float v[GU][PER];
+                    float ww[GU];
 #pragma unroll
-                    for (int u = 0; u < 8; ++u) {
+                    for (int u = 0; u < GU; ++u) {
                         const bool has = i0 + u < cnt;
                         const int jj = has ? lidx[warp][i0 + u] : 0;
                         ww[u] = has ? lw[warp][i0 + u] : 0.0f;
                         VRow<T, PER>::load(vh + (long long)jj * D + lane * PER, v[u]);
                     }
 #pragma unroll
-                    for (int u = 0; u < 8; ++u) {
+                    for (int u = 0; u < GU; ++u) {
 #pragma unroll
                         for (int e = 0; e < PER; ++e) acc[e] = fmaf(ww[u], v[u][e], acc[e]);
                         z += ww[u];

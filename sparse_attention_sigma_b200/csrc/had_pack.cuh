@@ -6,6 +6,8 @@
 // 1 bit per element is written, as whole 32-bit words.  Word w of a row holds
 // elements 32w..32w+31 with element 32w+k in bit k; bit = 1 means sign -1.
 #pragma once
+#include <type_traits>
+
 #include "had_common.cuh"
 
 namespace had {
@@ -45,8 +47,10 @@ struct Load8<float> {
 // fourth lane stores the word.  With a normal
 // sigma an element at or below -sigma * 2^-100 is surely negative after the
 // division and one at or above zero surely not, so the sign is a
-// comparison; only a lane holding an element strictly between (possible,
-// never seen in practice) takes the exact IEEE division, for its 8 elements.
+// comparison (for bf16 one on the raw bits, four values per few integer
+// instructions: bf16_signs4); only a lane holding an element strictly
+// between (possible, never seen in practice: -0, tiny values, -inf, NaN)
+// takes the exact IEEE division, for its 8 elements.
 // slab = n*d elements (a multiple of 32, so a word never straddles slabs).
 template <typename T>
 __global__ void __launch_bounds__(256)
@@ -55,6 +59,7 @@ pack_bits_kernel(const T *__restrict__ x, const float *__restrict__ sigma, int H
 {
     for (long long bh = blockIdx.y; bh < slabs; bh += gridDim.y) {
         const SignRule rule = sign_rule(__ldg(sigma + bh % H));
+        const uint32_t kge = bf16_kge(rule);
         if (rule.bad && blockIdx.x == 0 && threadIdx.x == 0) flag(status, HAD_ERR_BAD_SIGMA);
         const T *xs = x + bh * slab;
         uint32_t *bs = bits + bh * (slab / 32);
@@ -64,11 +69,16 @@ pack_bits_kernel(const T *__restrict__ x, const float *__restrict__ sigma, int H
         const long long step = (long long)gridDim.x * (blockDim.x / 32);
         const long long q0 = blockIdx.x * (long long)(blockDim.x / 32) + (threadIdx.x >> 5);
         for (long long q = q0; q < quads; q += step) {
-            float v[4][8];
+            constexpr bool kBf16 = std::is_same<T, __nv_bfloat16>::value;
+            uint4 raw[4];                             // bf16: the 8 values' bits
+            float v[4][8];                            // f32: the values
 #pragma unroll
             for (int k = 0; k < 4; ++k) {
                 const long long e0 = q * 1024 + k * 256 + 8 * lane;
-                if (e0 < slab) {                      // all 8 or none: slab is a multiple of 32
+                const bool in = e0 < slab;            // all 8 or none: slab is a multiple of 32
+                if constexpr (kBf16) {
+                    raw[k] = in ? __ldg(reinterpret_cast<const uint4 *>(xs + e0)) : make_uint4(0u, 0u, 0u, 0u);
+                } else if (in) {
                     Load8<T>::run(xs + e0, v[k]);
                 } else {
 #pragma unroll
@@ -80,10 +90,24 @@ pack_bits_kernel(const T *__restrict__ x, const float *__restrict__ sigma, int H
                 const long long e0 = q * 1024 + k * 256 + 8 * lane;
                 uint32_t byte = 0;
                 bool unsure = !rule.fast;
+                if constexpr (kBf16) {
+                    uint32_t n0, u0, n1, u1;
+                    bf16_signs4(raw[k].x, raw[k].y, kge, n0, u0);
+                    bf16_signs4(raw[k].z, raw[k].w, kge, n1, u1);
+                    byte = flags4(n0) | flags4(n1) << 4;
+                    unsure |= (u0 | u1) != 0u;
+                    if (unsure) {
+                        v[k][0] = bf16_lo(raw[k].x); v[k][1] = bf16_hi(raw[k].x);
+                        v[k][2] = bf16_lo(raw[k].y); v[k][3] = bf16_hi(raw[k].y);
+                        v[k][4] = bf16_lo(raw[k].z); v[k][5] = bf16_hi(raw[k].z);
+                        v[k][6] = bf16_lo(raw[k].w); v[k][7] = bf16_hi(raw[k].w);
+                    }
+                } else {
 #pragma unroll
-                for (int i = 0; i < 8; ++i) {
-                    byte |= (uint32_t)(v[k][i] <= -rule.thr) << i;
-                    unsure |= (v[k][i] < 0.0f) && (v[k][i] > -rule.thr);
+                    for (int i = 0; i < 8; ++i) {
+                        byte |= (uint32_t)(v[k][i] <= -rule.thr) << i;
+                        unsure |= (v[k][i] < 0.0f) && (v[k][i] > -rule.thr);
+                    }
                 }
                 if (unsure) {
                     byte = 0;

@@ -31,6 +31,7 @@
 // x / sigma_h < 0 in IEEE fp32.
 #pragma once
 #include <cuda_fp16.h>
+#include <type_traits>
 
 #include "had_common.cuh"
 #include "had_pack.cuh"
@@ -56,6 +57,32 @@ template <typename T>
 __device__ __forceinline__ uint32_t sign16(const T *src, const SignRule &rule, uint32_t pos,
                                            uint32_t neg, uint32_t (&w)[4])
 {
+    if constexpr (std::is_same<T, __nv_bfloat16>::value) {
+        // on the raw bits: four values per bf16_signs4; a negative value's
+        // byte flag, sign-replicated over its byte, selects the neg code
+        if (rule.fast) {
+            const uint4 a = __ldg(reinterpret_cast<const uint4 *>(src));
+            const uint4 b = __ldg(reinterpret_cast<const uint4 *>(src + 8));
+            const uint32_t kge = bf16_kge(rule);
+            uint32_t n[4], u[4];
+            bf16_signs4(a.x, a.y, kge, n[0], u[0]);
+            bf16_signs4(a.z, a.w, kge, n[1], u[1]);
+            bf16_signs4(b.x, b.y, kge, n[2], u[2]);
+            bf16_signs4(b.z, b.w, kge, n[3], u[3]);
+            if (((u[0] | u[1]) | (u[2] | u[3])) == 0u) {
+                const uint32_t pos4 = pos * 0x01010101u, flip4 = ((pos ^ neg) & 0xFFu) * 0x01010101u;
+                uint32_t packed = 0;
+#pragma unroll
+                for (int q = 0; q < 4; ++q) {
+                    uint32_t m;
+                    asm("prmt.b32 %0, %1, 0, 0xBA98;" : "=r"(m) : "r"(n[q]));   // 0xFF per negative byte
+                    w[q] = pos4 ^ (m & flip4);
+                    packed |= flags4(n[q]) << (4 * q);
+                }
+                return packed;
+            }
+        }
+    }
     float v[16];
     Load8<T>::run(src, *reinterpret_cast<float(*)[8]>(v));
     Load8<T>::run(src + 8, *reinterpret_cast<float(*)[8]>(v + 8));

@@ -289,6 +289,44 @@ def test_sign_edge_values_on_device(had):
     assert np.array_equal(got, ref)
 
 
+# Values whose sign after the fp32 division is decided at an edge: -0, the
+# tiny magnitudes (bf16 keeps the fp32 exponent range, down to 2^-133) whose
+# quotient rounds to -0 under a large sigma, infinities and NaN.
+BF16_SIGN_VALS = [0.0, -0.0, float("nan"), float("inf"), float("-inf"), -9.2e-41, 9.2e-41,
+                  -1.1754944e-38, -1e-37, -1e-30, -1e-22, -1e-20, -1e-10, 3.0, -3.0]
+BF16_SIGMAS = [1.0, 3.0, 1e9, 1e30, 1e-30]
+
+
+def test_sign_edge_values_on_device_bf16(had):
+    """bf16 signs on their raw bits (pack kernel), edges against the oracle."""
+    H = len(BF16_SIGMAS)
+    x = (torch.randn(1, H, 2, 64, generator=torch.Generator().manual_seed(21)) * 1e-21)
+    for i, v in enumerate(BF16_SIGN_VALS):
+        x[0, :, 0, i] = v
+    x = x.to(torch.bfloat16)
+    sigma = torch.tensor(BF16_SIGMAS)
+    got = had.had_binarize_pack(x.cuda(), sigma.cuda()).cpu().numpy().view(np.uint32)
+    ref = oracle.pack(oracle.binarize(synth.to_oracle_array(x), sigma.numpy()))
+    assert np.array_equal(got, ref)
+
+
+def test_fused_sign_edge_values_bf16(had):
+    """The same edges in Q and K through the fused path's operand
+    preparation: indices and logits must equal the oracle's exactly."""
+    H, n, d, N = len(BF16_SIGMAS), 130, 64, 20
+    g = torch.Generator().manual_seed(22)
+    q = torch.randn(1, H, n, d, generator=g)
+    k = torch.randn(1, H, n, d, generator=g)
+    v = torch.randn(1, H, n, d, generator=g).to(torch.bfloat16)
+    for t in (q, k):
+        for i, val in enumerate(BF16_SIGN_VALS):
+            t[0, :, (7 * i) % n, (5 * i) % d] = val
+            t[0, :, (11 * i + 3) % n, :: 9] = val * (1 if i % 2 else 1e-25)
+    sigma = torch.tensor(BF16_SIGMAS)
+    case = Case(q.to(torch.bfloat16), k.to(torch.bfloat16), v, sigma, sigma, N, 0.125)
+    _check_fused(had, case, all_rows(case))
+
+
 def test_bad_sigma_is_flagged(had):
     c = random_case(1, 2, 64, 64, 8, 12)
     status = torch.zeros(1, dtype=torch.int32, device="cuda")
