@@ -135,13 +135,17 @@ had_status_t core_tc(const void *V, bool v_f32, int B, int H, int n, int N, floa
     const long long bh = (long long)B * H;
     const bool dbg = dbg_idx != nullptr || dbg_lg != nullptr;
     // The quota tile's kept ties: found by a scan of the head's key signs in
-    // shared memory where they fit (mode 2, measured fastest at 4 and at 32
-    // key tiles); else, with few key tiles, a per-chunk mask in pass 2
+    // shared memory where they fit and there are 4 key tiles or more (mode
+    // 2, measured fastest at 4 and at 32 tiles; at 2 the scan costs more
+    // than the mask); else, with few key tiles, a per-chunk mask in pass 2
     // (mode 1) costs less than gathering them after it (mode 0, a fixed
     // latency per CTA; measured crossover near 12 tiles).
     const int T = (n + tcfwd::kKeys - 1) / tcfwd::kKeys;
     const long long kb_bytes = (long long)n * (D / 8);
-    const bool kb = !dbg && kb_bytes <= C::KB_CAP && kb_bytes % 16 == 0 && T <= C::STASH_CAP &&
+    // a head's signs start on a 16-byte boundary when their size is a
+    // multiple of 16; otherwise the copy widens them by up to 30 bytes
+    const long long kb_copy = kb_bytes % 16 == 0 ? kb_bytes : kb_bytes + 32;
+    const bool kb = !dbg && T >= 4 && kb_copy <= C::KB_CAP && T <= C::STASH_CAP &&
                     (reinterpret_cast<uintptr_t>(ws + w.kbits) & 15u) == 0;
     const bool q2 = T <= 12;
     auto kernel = dbg  ? tcfwd::attention_tc_kernel<D, true, 0>

@@ -32,9 +32,12 @@
 //           the first half of its own S in TMEM and the tensor core
 //           accumulates O += P V (fp16 x fp16 -> f32).
 //   quota   the kept ties of the quota tile (the first of them in key order:
-//           the lower index wins) are found after pass 2 from the packed sign
-//           bits (Hamming distance = level) and added to O and Z by the row's
-//           thread.
+//           the lower index wins), by one of three modes (kMode): found
+//           between the passes by a scan of the head's packed key signs in
+//           shared memory (Hamming distance = level) and set in P in pass 2;
+//           masked in P from the S values in pass 2; or found after pass 2
+//           from the key signs in global memory and added to O and Z by the
+//           row's thread.
 // The n x n logits never leave the SM.
 //
 // Warp roles: warp 0 bulk-copies the Q tiles once and streams K (twice) and
@@ -113,8 +116,9 @@ struct Cfg {
     static constexpr int OFF_MISC = OFF_BAR + NBARS * 8;
     static constexpr int SMEM_BYTES = OFF_MISC + 16 + 1024;   // + alignment slack
     static_assert(SMEM_BYTES <= 227 * 1024, "shared memory budget");
-    // mode with the head's packed key signs in shared memory (n D / 8 bytes,
-    // at most KB_CAP), after the rest of the layout
+    // mode with the head's packed key signs in shared memory (n D / 8 bytes
+    // widened to 16-byte boundaries, at most KB_CAP), after the rest of the
+    // layout
     static constexpr int KB_CAP = D == 64 ? 32768 : 16384;
     static constexpr int OFF_KB = (OFF_MISC + 16 + 127) / 128 * 128;   // 16-byte aligned for the bulk copy
     static constexpr int OFF_KM = OFF_KB + KB_CAP;      // per row its 128-bit kept-tie mask
@@ -201,7 +205,7 @@ __device__ __forceinline__ void fence_async_smem()
 //      by a per-chunk tie mask of the S values (cheaper with few key tiles);
 //   2: found before pass 2 by a scan of the head's packed key signs, copied
 //      to shared memory at the start, and set in P by pass 2 (heads whose
-//      signs fit in KB_CAP bytes).
+//      signs, widened to 16-byte boundaries, fit in KB_CAP bytes).
 template <int D, bool kDbg, int kMode>
 __global__ void __launch_bounds__(Cfg<D>::THREADS, 1)
 attention_tc_kernel(const Params p)
@@ -289,11 +293,15 @@ attention_tc_kernel(const Params p)
             tc::mbar_expect_tx(q_full, QT * C::QBYTES);
             tc::bulk_g2s(smem + C::OFF_Q, qsrc, QT * C::QBYTES, q_full);
             if (kKB) {
-                // the head's packed key signs, for the quota-tile scan
-                const uint32_t kb_bytes = (uint32_t)p.n * (D / 8);
-                tc::mbar_expect_tx(kb_full, kb_bytes);
-                tc::bulk_g2s(smem + C::OFF_KB, p.kbits + head * p.n * (long long)(D / 32),
-                             kb_bytes, kb_full);
+                // the head's packed key signs, for the quota-tile scan: from
+                // the 16-byte boundary at or below their start, rounded up to
+                // a whole 16 bytes (at most 30 bytes of the neighbouring heads
+                // or of the workspace's padding come along)
+                const long long b0 = head * p.n * (long long)(D / 8);
+                const long long a0 = b0 & ~15ll, a1 = (b0 + p.n * (long long)(D / 8) + 15) & ~15ll;
+                tc::mbar_expect_tx(kb_full, (uint32_t)(a1 - a0));
+                tc::bulk_g2s(smem + C::OFF_KB, reinterpret_cast<const uint8_t *>(p.kbits) + a0,
+                             (uint32_t)(a1 - a0), kb_full);
             }
             // K stream G = 0 .. 2T-1 (key tile G % T); V tile H follows K
             // stream entry T + H.
@@ -776,7 +784,10 @@ attention_tc_kernel(const Params p)
             constexpr int DW = D / 32, LPR = D == 64 ? 4 : 2;
             const bool hq = ok && active && jstar >= 0 && kstar > 0;
             ok = __all_sync(kFullMask, wait_bar(kb_full, 0, deadline, abort_flag, p.status));
-            const uint32_t *kbs = reinterpret_cast<const uint32_t *>(smem + C::OFF_KB);
+            // key j's sign words: (D / 32) words from byte (head n + j) D / 8 of
+            // the packed signs, copied from the 16-byte boundary below the head
+            const uint32_t *kbs = reinterpret_cast<const uint32_t *>(
+                smem + C::OFF_KB + ((head * p.n * (long long)(D / 8)) & 15));
             uint32_t tw[4] = {0u, 0u, 0u, 0u};
             uint32_t todo = ok ? __ballot_sync(kFullMask, hq) : 0u;
             while (todo) {                            // warp-uniform

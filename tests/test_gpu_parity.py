@@ -87,11 +87,14 @@ SMALL = [
     (2, 1, 129, 128, 129, 5, torch.float32),        # N = n: dense softmax
     (1, 1, 1, 64, 1, 6, torch.bfloat16),            # a single row and key
     (1, 3, 97, 64, 1, 7, torch.bfloat16),           # N = 1
-    # more than 12 key tiles, ragged last tile: the quota tile's kept ties
-    # found from the key signs in shared memory (n d / 8 a multiple of 16),
-    # then gathered after pass 2 (odd n; d 128 beyond 16 KB of key signs)
+    # ragged last tiles in each way of finding the quota tile's kept ties:
+    # from the key signs in shared memory (4 .. 32 key tiles at d 64, odd n
+    # too), masked from S in pass 2 (fewer key tiles, or d 128 with more than
+    # 16 KB of key signs and at most 12 tiles), gathered after pass 2 (d 128,
+    # more key tiles)
     (1, 2, 2000, 64, 300, 8, torch.bfloat16),
     (1, 1, 1999, 64, 250, 9, torch.float32),
+    (1, 1, 1100, 128, 150, 11, torch.bfloat16),
     (1, 1, 1700, 128, 200, 10, torch.bfloat16),
 ]
 
