@@ -231,12 +231,12 @@ def test_all_keys_equal(had):
     assert_close(out.cpu().numpy(), mean.numpy(), "mean of first N")
 
 
-@pytest.mark.parametrize("n", [2048, 2047])
-def test_all_keys_equal_many_tiles(had, n):
-    """Every key a tie at the threshold, over 16 key tiles: the quota tile
-    is the third (keys 256 .. 383) and keeps its first 44 keys, on the
-    production path (key-sign scan for even n, gather for odd n)."""
-    N = 300
+@pytest.mark.parametrize("n,N", [(2048, 300), (2047, 300), (2048, 356), (1700, 356)])
+def test_all_keys_equal_many_tiles(had, n, N):
+    """Every key a tie at the threshold, over 14-16 key tiles: the quota
+    tile is the third (keys 256 .. 383) and keeps its first N - 256 keys, on
+    the production path (the key-sign scan).  44 kept of 128 ties: the kept
+    ones are set in P; 100 kept: the 28 dropped ones are cleared instead."""
     c = random_case(1, 2, n, 64, N, 13)
     c.k[:] = c.k[:, :, :1]
     c = Case(c.q, c.k, c.v, c.sgq, synth.per_head_sigma(c.k), c.N, c.tau)
