@@ -783,7 +783,9 @@ attention_tc_kernel(const Params p)
         if constexpr (kKB) {
             constexpr int DW = D / 32, LPR = D == 64 ? 4 : 2;
             const bool hq = ok && active && jstar >= 0 && kstar > 0;
-            ok = __all_sync(kFullMask, wait_bar(kb_full, 0, deadline, abort_flag, p.status));
+            // (a CTA that has already aborted stays aborted)
+            const bool kb_in = wait_bar(kb_full, 0, deadline, abort_flag, p.status);
+            ok = __all_sync(kFullMask, ok && kb_in);
             // key j's sign words: (D / 32) words from byte (head n + j) D / 8 of
             // the packed signs, copied from the 16-byte boundary below the head
             const uint32_t *kbs = reinterpret_cast<const uint32_t *>(
