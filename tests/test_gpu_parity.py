@@ -134,6 +134,17 @@ def _check_fused(had, c, rows):
     assert np.array_equal(flat(dbg_idx), o_idx)
     assert np.array_equal(flat(dbg_lg), o_lg)
     assert_close(flat(out), o_out, "fused out (debug outputs on)")
+    # the same through the split calls, whose core writes the kept set from
+    # the 128-key kernel (had_attention_fwd takes the 64-key one for it)
+    ws = had.workspace(c.B, c.H, c.n, c.d, c.N)
+    had.had_attention_prepare(c.gq, c.gk, c.gv, c.gsq, c.gsk, c.N, ws)
+    dbg_idx.fill_(-7)
+    dbg_lg.fill_(-7)
+    out_s = had.had_attention_core(c.gv, c.N, c.tau, ws, dbg_idx=dbg_idx, dbg_logits=dbg_lg)
+    torch.cuda.synchronize()
+    assert np.array_equal(flat(dbg_idx), o_idx)
+    assert np.array_equal(flat(dbg_lg), o_lg)
+    assert_close(flat(out_s), o_out, "fused out (split calls, debug outputs on)")
     # Without the debug outputs every full key tile takes the table path and
     # the kept ties of a row's quota tile are added afterwards in fp32, so the
     # rounding differs from the key-by-key debug path: both must match the
@@ -203,9 +214,11 @@ def test_workload_fused(had, name):
 
 @pytest.mark.parametrize("name", ["bert", "vit", "long"])
 def test_workload_fused_equals_unfused_on_every_row(had, name):
-    """Every row, on the GPU: the fused kernel's kept set (its debug outputs)
-    is bit-identical to the unfused top-N kernel's, whichever path (window or
-    exact fix-up) the row took."""
+    """Every row, on the GPU: the fused kernels' kept sets (their debug
+    outputs) are bit-identical to the unfused top-N kernel's, whichever path
+    (window or exact fix-up) the row took.  had_attention_fwd writes the kept
+    set from the 64-key kernel, had_attention_core from the 128-key one (its
+    window, threshold and fix-up logic, shared with the production call)."""
     c = config_case(name)
     qb = had.had_binarize_pack(c.gq, c.gsq)
     kb = had.had_binarize_pack(c.gk, c.gsk)
@@ -214,6 +227,14 @@ def test_workload_fused_equals_unfused_on_every_row(had, name):
     dbg_lg = torch.empty_like(lg)
     had.had_attention_fwd(c.gq, c.gk, c.gv, c.gsq, c.gsk, c.N, c.tau,
                           dbg_idx=dbg_idx, dbg_logits=dbg_lg)
+    torch.cuda.synchronize()
+    assert torch.equal(dbg_idx, idx)
+    assert torch.equal(dbg_lg, lg)
+    ws = had.workspace(c.B, c.H, c.n, c.d, c.N)
+    had.had_attention_prepare(c.gq, c.gk, c.gv, c.gsq, c.gsk, c.N, ws)
+    dbg_idx.fill_(-7)
+    dbg_lg.fill_(-7)
+    had.had_attention_core(c.gv, c.N, c.tau, ws, dbg_idx=dbg_idx, dbg_logits=dbg_lg)
     torch.cuda.synchronize()
     assert torch.equal(dbg_idx, idx)
     assert torch.equal(dbg_lg, lg)
